@@ -1,0 +1,379 @@
+"""Benchmark of the routed-MoE layer (route + expert FFNs + combine) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step = moe_route + moe_forward over one batch of synthetic tokens (every hot-path
+step).  The default workload is the 1-token decode layer (hidden 7168, 256 routed
+experts, top-8, one shared 3-bit expert, 2-bit routed experts), a fresh token per
+step.  Device time comes from CUDA events on the launching stream; the L2 cache is
+flushed (a 512 MiB write) between timed steps, outside the events, so every step
+reads its experts from HBM.  For N > 1 (torchrun) each rank runs an independent
+replica on its own token stream (the layer is data-parallel: no collective on the
+data path) and the time is the max over ranks.
+
+--impl reference times the CPU oracle (the only reference that exists for this
+layer) on the same workload, a bounded sample per step, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B200)"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GATEUP_KERNEL = "ffn_mma_kernel<0>"
+KERNEL_SOURCES = ["bit_routed_expert_fp32_b200/csrc/expert_mma.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(cfg_name: str):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary, if
+    it was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(cfg_name)
+    if not rec or rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec
+
+
+def gu_bytes(cfg, fmt: int) -> int:
+    """Packed bytes of one expert's fused gate/up matrix (codes + scales [+ third bits])."""
+    K, rows = cfg.H, 2 * cfg.I
+    b = rows * (K // 4 + K // 32)
+    if fmt == synth.FMT_Q3:
+        b += rows * 4 * 4 * ((K + 127) // 128)
+    return b
+
+
+def dn_bytes(cfg, fmt: int) -> int:
+    K, rows = cfg.I, cfg.H
+    b = rows * (K // 4 + K // 32)
+    if fmt == synth.FMT_Q3:
+        b += rows * 4 * 4 * ((K + 127) // 128)
+    return b
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# --------------------------------------------------------------------------- oracle
+def oracle_tokens_per_s(cfg, layer, xs, budget_s: float, max_tokens: int):
+    """Times the CPU oracle (routing + experts + combine) on whole tokens until
+    budget_s has elapsed; returns (tokens/s, tokens, seconds, threads)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    done, t0 = 0, time.perf_counter()
+    while done < max_tokens and time.perf_counter() - t0 < budget_s:
+        x = xs[done % len(xs)]
+        L = oracle.logits(x, layer.router_w, threads)
+        ids, gates = oracle.select(L, layer.router_b, cfg.k)
+        oracle.forward_tokens(layer, x, ids, gates, range(x.shape[0]), threads)
+        done += x.shape[0]
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt, min(threads, 9 * max(1, xs[0].shape[0]))
+
+
+def run_reference(args, cfg):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    layer = synth.Layer(cfg, 0)
+    per_step = max(1, min(cfg.T, 4))           # bounded sample of tokens per step
+    xs = [synth.tokens(cfg, 0, s, per_step) for s in range(args.warmup + args.steps)]
+    for s in range(args.warmup):
+        oracle_tokens_per_s(cfg, layer, [xs[s]], 0.0, per_step)
+    t0 = time.perf_counter()
+    tok, threads = 0, 1
+    for s in range(args.steps):
+        _, n, _, threads = oracle_tokens_per_s(cfg, layer, [xs[args.warmup + s]], 0.0, per_step)
+        tok += n
+    dt = time.perf_counter() - t0
+    value = tok / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(cfg, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{per_step} token(s) of the workload per step, routed and run through "
+                                       f"all selected experts and the shared expert in fp64"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(cfg, world):
+    return {"workload": cfg.name, "tokens_per_step": cfg.T, "hidden": cfg.H, "experts": cfg.E, "top_k": cfg.k,
+            "ffn": cfg.I, "shared": cfg.S, "formats": cfg.formats, "layers": cfg.layers,
+            "l2": "flushed between timed steps (512 MiB write)", "parallelism": f"replicas x{world}"}
+
+
+# --------------------------------------------------------------------------- ours
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import bit_routed_expert_fp32_b200 as moe
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    T = cfg.T
+    n_layers = cfg.layers
+    layers, fmts = [], []
+    for li in range(n_layers):
+        L = synth.Layer(cfg, li)
+        buf = np.zeros(moe.moe_packed_size(cfg, L.fmt), dtype=np.uint8)
+        from concurrent.futures import ThreadPoolExecutor
+
+        def job(e, L=L, buf=buf):
+            moe.moe_pack_experts(cfg, L.fmt, e, [L.expert(e)], buf)
+
+        with ThreadPoolExecutor(os.cpu_count() or 1) as ex:
+            list(ex.map(job, range(cfg.E + cfg.S)))
+        layers.append(moe.MoeLayer(cfg, buf, L.router_w, L.router_b, T, device=dev))
+        fmts.append(L.fmt)
+        del buf
+    total = args.warmup + args.steps
+    # fresh tokens per step; each rank draws its own stream (seeded by rank)
+    xs_host = np.stack([synth.tokens(cfg, 0, 1000 * rank + s, T) for s in range(total)])
+    x_dev = moe.bf16_to_device(xs_host.reshape(total * T, cfg.H), dev).view(total, T, cfg.H)
+    y = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    ids_log = torch.empty((total, T, cfg.k), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(total)]
+
+    def step(s, record=True):
+        lay = layers[s % n_layers]
+        e = ev[s]
+        e[0].record(stream)
+        lay.route(x_dev[s])
+        lay.forward(x_dev[s], y, events=e[1:5] if record else None)
+        e[5].record(stream)
+        ids_log[s].copy_(lay.rt["topk_ids"][:T])
+
+    for s in range(args.warmup):
+        flush.zero_()
+        step(s)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = Clocks(local)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    wall0 = time.perf_counter()
+    for s in range(args.warmup, total):
+        flush.zero_()
+        step(s)
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    ck = clocks.stop()
+    step_ms = [ev[s][0].elapsed_time(ev[s][5]) for s in range(args.warmup, total)]
+    gu_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.warmup, total)]
+    dn_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(args.warmup, total)]
+    rt_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.warmup, total)]
+    my_ms = float(sum(step_ms))
+    t = torch.tensor([my_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = world * T * args.steps / (max_ms / 1e3)
+
+    # algorithmic bytes of the gate/up launches from the routing each step produced
+    ids_h = ids_log.cpu().numpy()
+    gu_alg, dn_alg = [], []
+    for s in range(args.warmup, total):
+        f = fmts[s % n_layers]
+        distinct = np.unique(ids_h[s])
+        gb = sum(gu_bytes(cfg, int(f[e])) for e in distinct) + sum(gu_bytes(cfg, int(f[cfg.E + j]))
+                                                                   for j in range(cfg.S))
+        db = sum(dn_bytes(cfg, int(f[e])) for e in distinct) + sum(dn_bytes(cfg, int(f[cfg.E + j]))
+                                                                   for j in range(cfg.S))
+        gu_alg.append(gb)
+        dn_alg.append(db)
+    pk, pk_kind = peaks()
+    gu_gbs = (sum(gu_alg) / 1e9) / (sum(gu_ms) / 1e3)
+    dn_gbs = (sum(dn_alg) / 1e9) / (sum(dn_ms) / 1e3)
+    layer_gbs = ((sum(gu_alg) + sum(dn_alg)) / 1e9) / (my_ms / 1e3)
+    tr = traffic_record(cfg.name)
+    roofline = {"bound": "hbm", "kernel": GATEUP_KERNEL, "achieved": gu_gbs, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": gu_gbs / pk["hbm_gbs"],
+                "traffic": None if tr is None else tr["dram_bytes_per_launch"],
+                "algorithmic_bytes_per_launch": float(np.mean(gu_alg)),
+                "peak_source": f"{pk_kind} (MEASURED_PEAKS.json hbm_gbs)" if pk_kind == "measured" else "fallback",
+                "avg_launch_us": 1e3 * float(np.mean(gu_ms))}
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    x_pin = torch.from_numpy(xs_host.view(np.int16)).pin_memory()
+    y_pin = torch.empty((total, T, cfg.H), dtype=torch.int16).pin_memory()
+    x_stage = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    e2e_ms = []
+    for s in range(total):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x_stage.view(torch.int16).copy_(x_pin[s], non_blocking=True)
+        lay = layers[s % n_layers]
+        lay.route(x_stage)
+        lay.forward(x_stage, y)
+        y_pin[s].copy_(y.view(torch.int16), non_blocking=True)
+        b.record(stream)
+        if s >= args.warmup:
+            e2e_ms.append((a, b))
+    torch.cuda.synchronize(dev)
+    e2e_total = sum(a.elapsed_time(b) for a, b in e2e_ms)
+    t2 = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_value = world * T * args.steps / (float(t2.item()) / 1e3)
+    st, det = moe.moe_get_error(layers[0].ws)
+    if st != 0:
+        raise RuntimeError(f"device error {moe.STATUS[st]} {det:#x}")
+
+    line = None
+    if rank == 0:
+        launches_per_step = (1 if T <= 64 else 3) + 2
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_dict(cfg, world),
+                "roofline": roofline,
+                "layer_weight_stream_gbs": layer_gbs,
+                "kernel_us": {"route": 1e3 * float(np.mean(rt_ms)), "gate_up": 1e3 * float(np.mean(gu_ms)),
+                              "down_combine": 1e3 * float(np.mean(dn_ms)),
+                              "down_gbs": dn_gbs},
+                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.H * 2,
+                        "d2h_bytes_per_step": T * cfg.H * 2},
+                "gpu_launches": launches_per_step * args.steps,
+                "wall_s_timed_region": wall,
+                "clocks": ck}
+        if world == 1 and not args.no_cpu_baseline:
+            L0 = synth.Layer(cfg, 0)
+            sample = [xs_host[i][: max(1, min(T, 4))] for i in range(4)]
+            v, n, dt, cores = oracle_tokens_per_s(cfg, L0, sample, args.cpu_budget, 64)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"{n} token(s) of this workload ({dt:.1f} s), routed and run "
+                                              f"through every selected expert and the shared expert in fp64"}
+        print(json.dumps(line), flush=True)
+    for lay in layers:
+        del lay
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

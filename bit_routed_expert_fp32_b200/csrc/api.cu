@@ -1,0 +1,201 @@
+// C ABI of the routed-MoE layer (include/moe.h): argument checks, workspace
+// layout and kernel launches.  Nothing here allocates memory or synchronises,
+// except moe_get_error, which is documented to.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "kernels.h"
+#include "moe.h"
+
+namespace {
+
+using namespace moe;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool shape_ok(const moe_shape* s) {
+    return s && s->hidden > 0 && s->inter > 0 && s->hidden % 64 == 0 && s->inter % 64 == 0 &&
+           s->n_experts >= 1 && s->n_experts <= 256 && s->top_k >= 1 && s->top_k <= 16 &&
+           s->top_k <= s->n_experts && (s->n_shared == 0 || s->n_shared == 1);
+}
+
+// Workspace layout.  The control block, tile counters and the active-expert list
+// sit at fixed offsets (independent of T) so that their cleared state survives
+// calls with different token counts; the token-sized arrays follow.
+struct Ws {
+    size_t ctrl, tile_ctr, active, logits, hist, h, ypart, total;
+};
+
+Ws ws_layout(const moe_shape* s, int64_t T) {
+    Ws w;
+    const int64_t E = s->n_experts, S = s->n_shared, k = s->top_k, H = s->hidden, I = s->inter;
+    size_t off = 0;
+    w.ctrl = off;
+    off += 4096;
+    w.tile_ctr = off;
+    off = align256(off + 4 * (size_t)(H / 16));
+    w.active = off;
+    off = align256(off + 4 * (size_t)(E + S));
+    w.logits = off;
+    off = align256(off + 4 * (size_t)(T * E));
+    w.hist = off;
+    off = align256(off + 4 * (size_t)(((T + kChunk - 1) / kChunk) * E));
+    w.h = off;
+    off = align256(off + 2 * (size_t)(T * (k + S) * I));
+    w.ypart = off;
+    off = align256(off + 4 * (size_t)(T * (k + S) * H));
+    w.total = off;
+    return w;
+}
+
+size_t ws_fixed_prefix(const moe_shape* s) { return ws_layout(s, 0).active; }
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+bool routing_ok(const moe_routing* r) {
+    return r && r->topk_ids && r->topk_w && r->counts && r->offsets && r->perm && r->inv_perm;
+}
+
+moe_status check_common(const moe_shape* shape, int32_t T, const void* d_ws, size_t ws_bytes) {
+    if (!shape_ok(shape) || T < 0) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * shape->top_k > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    if (!d_ws) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(shape, T).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_WORKSPACE: return "workspace or destination buffer too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+        case MOE_ERR_DEVICE_CHECK: return "device-side data check failed";
+    }
+    return "unknown status";
+}
+
+moe_status moe_workspace_size(const moe_shape* shape, int32_t max_tokens, size_t* bytes) {
+    if (!shape_ok(shape) || max_tokens < 0 || !bytes) return MOE_ERR_INVALID_ARG;
+    *bytes = ws_layout(shape, max_tokens).total;
+    return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* d_ws, size_t ws_bytes, void* stream) {
+    if (!d_ws || ws_bytes < 4096) return MOE_ERR_INVALID_ARG;
+    // Clears the control block and every counter that can follow it (up to H = 256K).
+    const size_t n = ws_bytes < 4096 + 65536 ? ws_bytes : 4096 + 65536;
+    if (cudaMemsetAsync(d_ws, 0, n, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x, const float* d_router_w,
+                     const float* d_router_b, const moe_routing* out, void* d_ws, size_t ws_bytes, void* stream) {
+    moe_status st = check_common(shape, T, d_ws, ws_bytes);
+    if (st != MOE_OK) return st;
+    if (!d_x || !d_router_w || !routing_ok(out)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (ws_fixed_prefix(shape) > 4096 + 65536) return MOE_ERR_UNSUPPORTED;
+    const Ws w = ws_layout(shape, T);
+    uint8_t* ws = static_cast<uint8_t*>(d_ws);
+    RouteArgs a;
+    a.T = T;
+    a.H = shape->hidden;
+    a.E = shape->n_experts;
+    a.k = shape->top_k;
+    a.S = shape->n_shared;
+    a.x = d_x;
+    a.Wr = d_router_w;
+    a.bias = d_router_b;
+    a.logits = reinterpret_cast<float*>(ws + w.logits);
+    a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
+    a.active = reinterpret_cast<int32_t*>(ws + w.active);
+    a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
+    a.r = *out;
+    if (launch_route(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_packed, const uint16_t* d_x,
+                             const moe_routing* r, uint16_t* d_y, moe_path path, void* d_ws, size_t ws_bytes,
+                             void* stream, void* const* events, int32_t n_events) {
+    moe_status st = check_common(shape, T, d_ws, ws_bytes);
+    if (st != MOE_OK) return st;
+    if (!d_packed || !d_x || !d_y || !routing_ok(r)) return MOE_ERR_INVALID_ARG;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+    if (events && n_events < 4) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Ws w = ws_layout(shape, T);
+    uint8_t* ws = static_cast<uint8_t*>(d_ws);
+    FfnArgs a;
+    a.T = T;
+    a.H = shape->hidden;
+    a.I = shape->inter;
+    a.E = shape->n_experts;
+    a.k = shape->top_k;
+    a.S = shape->n_shared;
+    a.packed = static_cast<const uint8_t*>(d_packed);
+    a.x = d_x;
+    a.perm = r->perm;
+    a.inv_perm = r->inv_perm;
+    a.counts = r->counts;
+    a.offsets = r->offsets;
+    a.topk_w = r->topk_w;
+    a.active = reinterpret_cast<const int32_t*>(ws + w.active);
+    a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
+    a.h = reinterpret_cast<uint16_t*>(ws + w.h);
+    a.ypart = reinterpret_cast<float*>(ws + w.ypart);
+    a.tile_ctr = reinterpret_cast<uint32_t*>(ws + w.tile_ctr);
+    a.y = d_y;
+    a.num_ctas = sm_count();
+    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+    if (events)
+        for (int i = 0; i < 4; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
+    if (ev[0] && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t err = launch_ffn_mma(a, s, ev[1]);
+    if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+    if (ev[2] && cudaEventRecord(ev[2], s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (ev[3] && cudaEventRecord(ev[3], s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_forward(const moe_shape* shape, int32_t T, const void* d_packed, const uint16_t* d_x,
+                       const moe_routing* r, uint16_t* d_y, moe_path path, void* d_ws, size_t ws_bytes,
+                       void* stream) {
+    return moe_forward_timed(shape, T, d_packed, d_x, r, d_y, path, d_ws, ws_bytes, stream, nullptr, 0);
+}
+
+moe_status moe_get_error(void* d_ws, size_t ws_bytes, void* stream, uint32_t* detail) {
+    if (!d_ws || ws_bytes < sizeof(Ctrl)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t word[2] = {0, 0};
+    if (cudaMemcpy(word, d_ws, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemset(d_ws, 0, sizeof word) != cudaSuccess) return MOE_ERR_CUDA;
+    if (detail) *detail = word[1];
+    if (word[0] == MOE_ERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+    if (word[0] != 0) return MOE_ERR_DEVICE_CHECK;
+    return MOE_OK;
+}
+
+}  // extern "C"

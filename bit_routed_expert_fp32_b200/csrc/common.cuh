@@ -1,0 +1,199 @@
+// Device helpers shared by the kernels: packed-table access, PTX wrappers for
+// mbarriers and bulk (TMA) copies, bounded waits and the workspace error word.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// ---- packed format v1 (see include/moe.h) ----------------------------------
+constexpr uint32_t kMagic = 0x50454F4Du;
+constexpr int kGroup = 64;
+constexpr int kInterleave = 8;
+constexpr int kHeaderBytes = 256;
+constexpr int kEntryBytes = 64;
+
+struct __align__(16) PackedEntry {
+    uint32_t fmt;
+    uint32_t zero;
+    uint64_t gu_scales, gu_codes, gu_hi;
+    uint64_t dn_scales, dn_codes, dn_hi;
+    uint64_t zero2;
+};
+static_assert(sizeof(PackedEntry) == kEntryBytes, "entry layout");
+
+__host__ __device__ inline int hi_words(int K) { return 4 * ((K + 127) / 128); }
+
+// ---- workspace control block --------------------------------------------------
+// The first 4 KiB of the workspace; zeroed by moe_workspace_init.
+struct Ctrl {
+    uint32_t err_code;      // 0 = ok, else moe_status
+    uint32_t err_detail;    // kernel-specific detail (where a wait gave up, ...)
+    uint32_t route_ticket;  // last-block counters (self-resetting)
+    uint32_t topk_ticket;
+    int32_t n_active;       // experts with tokens + shared experts, written by moe_route
+    int32_t routed_T;       // T of the last moe_route
+    uint32_t pad[58];
+};
+
+// error detail codes
+enum : uint32_t {
+    kDetWaitFull = 0x100,
+    kDetWaitEmpty = 0x200,
+    kDetDrain = 0x300,
+    kDetHeader = 0x400,
+};
+
+__device__ inline void report_error(Ctrl* c, uint32_t code, uint32_t detail) {
+    if (atomicCAS(&c->err_code, 0u, code) == 0u) atomicExch(&c->err_detail, detail);
+}
+
+// ---- PTX wrappers -----------------------------------------------------------------
+__device__ inline uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ inline void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ inline void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after `limit` clock cycles and returns false.
+__device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ inline void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ inline void bulk_g2s_evict_first(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+        "%4;" ::"r"(smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ inline uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ inline void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ inline uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
+    return r;
+}
+
+__device__ inline uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ inline void mma_bf16_16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1,
+                                      uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ inline uint32_t f16x2_sub(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ inline void mma_f16_16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1,
+                                     uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ inline uint4 ldg_nc_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ inline float ldcg_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+__device__ inline float silu_f(float a) { return a / (1.0f + expf(-a)); }
+
+__device__ inline uint16_t f32_to_bf16_bits(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ inline uint16_t f32_to_f16_bits(float f) { return __half_as_ushort(__float2half_rn(f)); }
+
+__host__ __device__ inline uint32_t f16x2_bits_of(float v) {
+    // exact for the small dequantiser constants (all representable in binary16)
+    return (uint32_t)__half_as_ushort(__float2half_rn(v)) * 0x10001u;
+}
+
+__host__ __device__ inline uint32_t bf16x2_bits_of(float lo_hi_same) {
+    // exact conversion for the small constants used by the dequantiser
+    union { float f; uint32_t u; } v;
+    v.f = lo_hi_same;
+    uint32_t b = v.u >> 16;   // all constants used are exact in bf16 (checked on the host)
+    return b | (b << 16);
+}
+
+}  // namespace moe

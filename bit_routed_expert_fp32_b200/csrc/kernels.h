@@ -1,0 +1,46 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kSmallT = 64;        // decode router / decode path threshold
+constexpr int kChunk = 128;        // tokens per chunk of the large-T router
+
+struct RouteArgs {
+    int T, H, E, k, S;
+    const uint16_t* x;
+    const float* Wr;
+    const float* bias;
+    float* logits;      // ws [T][E]
+    int32_t* hist;      // ws [ceil(T/kChunk)][E]
+    int32_t* active;    // ws [E+S]
+    Ctrl* ctrl;
+    moe_routing r;
+};
+
+struct FfnArgs {
+    int T, H, I, E, k, S;
+    const uint8_t* packed;
+    const uint16_t* x;       // bf16 [T][H]
+    const int32_t* perm;
+    const int32_t* inv_perm;
+    const int32_t* counts;
+    const int32_t* offsets;
+    const float* topk_w;
+    const int32_t* active;   // ws
+    Ctrl* ctrl;
+    uint16_t* h;             // ws fp16 [T*(k+S)][I]
+    float* ypart;            // ws f32 [T*(k+S)][H]
+    uint32_t* tile_ctr;      // ws [H/16]
+    uint16_t* y;             // bf16 [T][H]
+    int num_ctas;
+};
+
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_mma(const FfnArgs& a, cudaStream_t s, cudaEvent_t mid_event);
+
+}  // namespace moe

@@ -1,0 +1,181 @@
+// Host-side packer: interchange-form codes and fp16 scales -> packed format v1
+// (layout documented in include/moe.h).  Pure host code, no CUDA calls.
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "moe.h"
+
+namespace {
+
+constexpr uint32_t kMagic = 0x50454F4Du;
+constexpr int kHeader = 256;
+constexpr int kEntry = 64;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int hi_words(int K) { return 4 * ((K + 127) / 128); }
+
+bool shape_ok(const moe_shape* s) {
+    return s && s->hidden > 0 && s->inter > 0 && s->hidden % 64 == 0 && s->inter % 64 == 0 &&
+           s->n_experts >= 1 && s->n_experts <= 256 && s->top_k >= 1 && s->top_k <= 16 &&
+           s->top_k <= s->n_experts && (s->n_shared == 0 || s->n_shared == 1);
+}
+
+struct MatLayout {
+    size_t scales, codes, hi;  // byte offsets (hi = 0 when absent)
+};
+struct ExpertLayout {
+    uint32_t fmt;
+    MatLayout gu, dn;
+};
+
+size_t mat_bytes(int rows, int K, uint32_t fmt, MatLayout* m, size_t off) {
+    off = align256(off);
+    m->scales = off;
+    off = align256(off + (size_t)rows * (K / 64) * 2);
+    m->codes = off;
+    off += (size_t)rows * (K / 16) * 4;
+    if (fmt == MOE_FMT_Q3) {
+        off = align256(off);
+        m->hi = off;
+        off += (size_t)rows * hi_words(K) * 4;
+    } else {
+        m->hi = 0;
+    }
+    return off;
+}
+
+// Computes every expert's offsets; returns the total size.
+size_t layout(const moe_shape* s, const uint8_t* fmt, std::vector<ExpertLayout>* out) {
+    const int H = s->hidden, I = s->inter, n = s->n_experts + s->n_shared;
+    size_t off = align256(kHeader + (size_t)kEntry * n);
+    if (out) out->resize(n);
+    for (int e = 0; e < n; ++e) {
+        ExpertLayout L;
+        L.fmt = fmt[e];
+        off = mat_bytes(2 * I, H, L.fmt, &L.gu, off);
+        off = mat_bytes(H, I, L.fmt, &L.dn, off);
+        if (out) (*out)[e] = L;
+    }
+    return align256(off);
+}
+
+// 16 natural-order 2-bit codes (code i at bits 2i) -> kernel word (even elements in
+// the low half at bits 2p, odd elements in the high half at bits 16 + 2p).
+inline uint32_t squeeze_pairs(uint32_t x) {  // keep fields at bits 4i..4i+1, compact
+    x &= 0x33333333u;
+    x = (x | (x >> 2)) & 0x0F0F0F0Fu;
+    x = (x | (x >> 4)) & 0x00FF00FFu;
+    x = (x | (x >> 8)) & 0x0000FFFFu;
+    return x;
+}
+inline uint32_t code_word(uint32_t nat) { return squeeze_pairs(nat) | (squeeze_pairs(nat >> 2) << 16); }
+
+// 32 natural-order third bits (element i at bit i) -> kernel word (element
+// 16q + 2p + h at bit 16h + 8q + p).
+inline uint32_t squeeze_bits(uint32_t x) {
+    x &= 0x55555555u;
+    x = (x | (x >> 1)) & 0x33333333u;
+    x = (x | (x >> 2)) & 0x0F0F0F0Fu;
+    x = (x | (x >> 4)) & 0x00FF00FFu;
+    x = (x | (x >> 8)) & 0x0000FFFFu;
+    return x;
+}
+inline uint32_t hi_word(uint32_t nat) { return squeeze_bits(nat) | (squeeze_bits(nat >> 1) << 16); }
+
+inline uint32_t load_u32(const uint8_t* p) {
+    return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+inline void store_u32(uint8_t* p, uint32_t v) {
+    p[0] = (uint8_t)v;
+    p[1] = (uint8_t)(v >> 8);
+    p[2] = (uint8_t)(v >> 16);
+    p[3] = (uint8_t)(v >> 24);
+}
+
+// Packs one source row (K elements) into destination row `dr` of a packed matrix.
+bool pack_row(const moe_matrix_src& src, int sr, int K, uint32_t fmt, uint8_t* base, const MatLayout& m, int dr) {
+    const uint8_t* codes = src.codes + (size_t)sr * (K / 4);
+    if (fmt == MOE_FMT_TERNARY) {
+        for (int b = 0; b < K / 4; ++b)
+            if (codes[b] & (codes[b] >> 1) & 0x55) return false;   // a field equal to 3
+    }
+    uint8_t* cdst = base + m.codes + (size_t)dr * (K / 16) * 4;
+    for (int w = 0; w < K / 16; ++w) store_u32(cdst + 4 * w, code_word(load_u32(codes + 4 * w)));
+    uint8_t* sdst = base + m.scales + (size_t)dr * (K / 64) * 2;
+    const uint16_t* ssrc = src.scales + (size_t)sr * (K / 64);
+    for (int g = 0; g < K / 64; ++g) {
+        sdst[2 * g] = (uint8_t)ssrc[g];
+        sdst[2 * g + 1] = (uint8_t)(ssrc[g] >> 8);
+    }
+    if (fmt == MOE_FMT_Q3) {
+        const uint8_t* hi = src.hi + (size_t)sr * (K / 8);
+        const int W1 = hi_words(K);
+        uint8_t* hdst = base + m.hi + (size_t)dr * W1 * 4;
+        for (int w = 0; w < W1; ++w) store_u32(hdst + 4 * w, w < K / 32 ? hi_word(load_u32(hi + 4 * w)) : 0u);
+    }
+    return true;
+}
+
+void write_header(const moe_shape* s, const std::vector<ExpertLayout>& L, size_t total, uint8_t* dst) {
+    memset(dst, 0, kHeader);
+    uint32_t h[8] = {kMagic, 1u, (uint32_t)s->hidden, (uint32_t)s->inter, (uint32_t)s->n_experts,
+                     (uint32_t)s->n_shared, 64u, 8u};
+    for (int i = 0; i < 8; ++i) store_u32(dst + 4 * i, h[i]);
+    store_u32(dst + 32, (uint32_t)total);
+    store_u32(dst + 36, (uint32_t)((uint64_t)total >> 32));
+    for (size_t e = 0; e < L.size(); ++e) {
+        uint8_t* ent = dst + kHeader + e * kEntry;
+        memset(ent, 0, kEntry);
+        uint64_t v[8] = {L[e].fmt, L[e].gu.scales, L[e].gu.codes, L[e].gu.hi,
+                         L[e].dn.scales, L[e].dn.codes, L[e].dn.hi, 0};
+        store_u32(ent, (uint32_t)v[0]);
+        for (int i = 1; i < 8; ++i) {
+            store_u32(ent + 8 * i, (uint32_t)v[i]);
+            store_u32(ent + 8 * i + 4, (uint32_t)(v[i] >> 32));
+        }
+    }
+}
+
+}  // namespace
+
+extern "C" moe_status moe_packed_size(const moe_shape* shape, const uint8_t* h_fmt, size_t* bytes) {
+    if (!shape_ok(shape) || !h_fmt || !bytes) return MOE_ERR_INVALID_ARG;
+    for (int e = 0; e < shape->n_experts + shape->n_shared; ++e)
+        if (h_fmt[e] > MOE_FMT_Q3) return MOE_ERR_INVALID_ARG;
+    *bytes = layout(shape, h_fmt, nullptr);
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_pack_experts(const moe_shape* shape, const uint8_t* h_fmt, int32_t first, int32_t count,
+                                       const moe_matrix_src* h_src, void* h_dst, size_t h_dst_bytes) {
+    if (!shape_ok(shape) || !h_fmt || !h_dst || (count > 0 && !h_src)) return MOE_ERR_INVALID_ARG;
+    const int n = shape->n_experts + shape->n_shared;
+    if (first < 0 || count < 0 || first + count > n) return MOE_ERR_INVALID_ARG;
+    for (int e = 0; e < n; ++e)
+        if (h_fmt[e] > MOE_FMT_Q3) return MOE_ERR_INVALID_ARG;
+    std::vector<ExpertLayout> L;
+    const size_t total = layout(shape, h_fmt, &L);
+    if (h_dst_bytes < total) return MOE_ERR_WORKSPACE;
+    uint8_t* dst = static_cast<uint8_t*>(h_dst);
+    write_header(shape, L, total, dst);
+    const int H = shape->hidden, I = shape->inter;
+    for (int i = 0; i < count; ++i) {
+        const int e = first + i;
+        const uint32_t fmt = h_fmt[e];
+        const moe_matrix_src* m = h_src + 3 * (size_t)i;   // gate, up, down
+        for (int q = 0; q < 3; ++q) {
+            if (!m[q].codes || !m[q].scales || (fmt == MOE_FMT_Q3 && !m[q].hi)) return MOE_ERR_INVALID_ARG;
+        }
+        for (int r = 0; r < 2 * I; ++r) {
+            const int b = r / 16, j = r % 16;
+            const bool gate = j < 8;
+            const int sr = 8 * b + (gate ? j : j - 8);
+            if (!pack_row(gate ? m[0] : m[1], sr, H, fmt, dst, L[e].gu, r)) return MOE_ERR_INVALID_ARG;
+        }
+        for (int r = 0; r < H; ++r)
+            if (!pack_row(m[2], r, I, fmt, dst, L[e].dn, r)) return MOE_ERR_INVALID_ARG;
+    }
+    return MOE_OK;
+}

@@ -1,0 +1,136 @@
+"""Test harness: builds a case (seeded inputs, oracle routing, packed layer) and
+compares the CUDA path with the oracle.  Tests only."""
+from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field
+
+import numpy as np
+
+import oracle
+import synth
+
+GAP = 1e-4          # minimum gap between adjacent top-(k+1) logits (fp64)
+ATOL_RMS = 2e-2     # max |gpu - oracle| <= ATOL_RMS * rms(oracle)
+FROB = 5e-3         # ||gpu - oracle||_F / ||oracle||_F <= FROB
+GATE_RTOL = 1e-5
+
+
+@dataclass
+class Case:
+    cfg: synth.LayerConfig
+    layer: synth.Layer
+    x: np.ndarray                    # uint16 bf16 bits [T][H]
+    L: np.ndarray                    # fp64 logits without bias
+    ids: np.ndarray
+    gates: np.ndarray
+    counts: np.ndarray
+    offsets: np.ndarray
+    perm: np.ndarray
+    inv_perm: np.ndarray
+    redrawn: int = 0
+    extra: dict = field(default_factory=dict)
+
+
+def make_case(cfg, layer_idx=0, step=0, T=None, bias=None, router_w=None, threads=None) -> Case:
+    layer = synth.Layer(cfg, layer_idx)
+    if router_w is not None:
+        layer.router_w = router_w
+    if bias is not None:
+        layer.router_b = bias
+    x = synth.tokens(cfg, layer_idx, step, T)
+    redrawn = 0
+    for rnd in range(20):
+        L = oracle.logits(x, layer.router_w, threads)
+        bad = np.nonzero(oracle.topk_gaps(L, layer.router_b, cfg.k) < GAP)[0]
+        if bad.size == 0:
+            break
+        redrawn += bad.size
+        synth.redraw_tokens(cfg, x, bad, layer_idx, step, rnd)
+    else:
+        raise RuntimeError("could not remove near-ties")
+    ids, gates = oracle.select(L, layer.router_b, cfg.k)
+    counts, offsets, perm, inv = oracle.permute(ids, cfg.E)
+    return Case(cfg, layer, x, L, ids, gates, counts, offsets, perm, inv, redrawn)
+
+
+def pack(case: Case, threads=None) -> np.ndarray:
+    import bit_routed_expert_fp32_b200 as moe
+    cfg, layer = case.cfg, case.layer
+    buf = np.zeros(moe.moe_packed_size(cfg, layer.fmt), dtype=np.uint8)
+
+    def job(e):
+        moe.moe_pack_experts(cfg, layer.fmt, e, [layer.expert(e)], buf)
+
+    with ThreadPoolExecutor(threads or os.cpu_count() or 1) as ex:
+        list(ex.map(job, range(cfg.E + cfg.S)))
+    return buf
+
+
+def run_gpu(case: Case, packed_host=None, path=0, gpu_layer=None):
+    """Route + forward on the GPU; returns (routing dict of numpy arrays, y uint16)."""
+    import torch
+    import bit_routed_expert_fp32_b200 as moe
+    cfg = case.cfg
+    T = case.x.shape[0]
+    if gpu_layer is None:
+        gpu_layer = moe.MoeLayer(cfg, packed_host, case.layer.router_w, case.layer.router_b, T)
+    x = moe.bf16_to_device(case.x)
+    y = torch.full((T, cfg.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gpu_layer.route(x)
+    gpu_layer.forward(x, y, path=path)
+    torch.cuda.synchronize()
+    st, det = moe.moe_get_error(gpu_layer.ws)
+    assert st == 0, f"device error {moe.STATUS[st]} detail {det:#x}"
+    rt = {n: t.cpu().numpy() for n, t in gpu_layer.rt.items()}
+    return rt, moe.bf16_to_host(y)
+
+
+def check_routing(case: Case, rt: dict):
+    cfg = case.cfg
+    T = case.x.shape[0]
+    np.testing.assert_array_equal(rt["topk_ids"][:T], case.ids)
+    np.testing.assert_array_equal(rt["counts"], case.counts)
+    np.testing.assert_array_equal(rt["offsets"], case.offsets)
+    np.testing.assert_array_equal(rt["perm"][:T * cfg.k], case.perm)
+    np.testing.assert_array_equal(rt["inv_perm"][:T * cfg.k], case.inv_perm)
+    np.testing.assert_allclose(rt["topk_w"][:T].astype(np.float64), case.gates, rtol=GATE_RTOL, atol=0)
+
+
+def oracle_outputs(case: Case, tokens, threads=None) -> np.ndarray:
+    return oracle.forward_tokens(case.layer, case.x, case.ids, case.gates, tokens, threads)
+
+
+def check_outputs(y_gpu_bits: np.ndarray, y_ref: np.ndarray):
+    y = synth.bf16_bits_to_f32(y_gpu_bits).astype(np.float64)
+    assert np.all(np.isfinite(y))
+    diff = y - y_ref
+    rms = np.sqrt(np.mean(y_ref ** 2))
+    max_err = np.abs(diff).max()
+    frob = np.linalg.norm(diff) / np.linalg.norm(y_ref)
+    assert max_err <= ATOL_RMS * rms, f"max |err| {max_err:.3e} > {ATOL_RMS} * rms {rms:.3e}"
+    assert frob <= FROB, f"relative Frobenius error {frob:.3e} > {FROB}"
+    return max_err / rms, frob
+
+
+def sample_tokens(case: Case, n_random: int, seed: int = 0) -> list:
+    """Tokens whose outputs the oracle computes at full size: the first and last token
+    of the permuted ranges of 32 experts spread over the ids, tokens at (up to 32)
+    64-row tile boundaries of the hottest expert, and n_random uniform draws."""
+    cfg = case.cfg
+    T = case.x.shape[0]
+    pick = set()
+    for e in range(0, cfg.E, max(1, cfg.E // 32)):           # 32 experts spread over the ids
+        lo, hi = int(case.offsets[e]), int(case.offsets[e + 1])
+        if hi > lo:
+            pick.add(int(case.perm[lo]) // cfg.k)
+            pick.add(int(case.perm[hi - 1]) // cfg.k)
+    hot = int(np.argmax(case.counts))
+    lo, hi = int(case.offsets[hot]), int(case.offsets[hot + 1])
+    step = max(64, ((hi - lo) // 32 + 63) // 64 * 64)         # at most ~32 tile boundaries
+    for r in range(lo, hi, step):
+        pick.add(int(case.perm[r]) // cfg.k)
+    rng = np.random.default_rng(seed)
+    pick.update(int(t) for t in rng.choice(T, size=min(n_random, T), replace=False))
+    return sorted(pick)

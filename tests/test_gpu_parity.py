@@ -1,0 +1,116 @@
+"""Parity of the CUDA path with the CPU oracle (needs a B200).
+
+Routing (ids, counts, offsets, perm, inv_perm) must match bit-exactly and the gates
+to 1e-5 relative; layer outputs must satisfy max |gpu - oracle| <= 2e-2 rms(oracle)
+and relative Frobenius error <= 5e-3.  Inputs are regenerated token by token until
+every adjacent gap among a token's k+1 largest logits is >= 1e-4 (fp64).
+"""
+import numpy as np
+import pytest
+
+import synth
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"decode": 1, "prefill": 2}
+
+
+def _full_check(cfg, path, bias=None, router_w=None, T=None):
+    case = H.make_case(cfg, bias=bias, router_w=router_w, T=T)
+    packed = H.pack(case)
+    rt, y = H.run_gpu(case, packed, path=path)
+    H.check_routing(case, rt)
+    ref = H.oracle_outputs(case, range(case.x.shape[0]))
+    return H.check_outputs(y, ref), case, rt
+
+
+@pytest.mark.parametrize("path", ["decode", "prefill"])
+def test_tiny_layer_both_paths(path):
+    """The 4-token tiny layer (hidden 256, 8 experts, top-2, all 2-bit)."""
+    _full_check(synth.CONFIGS[1], PATHS[path])
+
+
+@pytest.mark.parametrize("T", [1, 7, 63, 64, 65, 130])
+def test_token_counts_around_the_path_switch(T):
+    cfg = synth.micro(T=T, H=128, E=16, k=4, I=64, S=1, formats="mixed", seed=100 + T)
+    _full_check(cfg, 0)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T=9, H=64, E=8, k=2, I=64, S=0, formats="q2"),            # K = 64: one group
+    dict(T=33, H=192, E=32, k=8, I=128, S=1, formats="mixed"),     # odd group counts
+    dict(T=20, H=256, E=256, k=8, I=64, S=1, formats="mixed"),     # full expert count
+    dict(T=5, H=320, E=8, k=1, I=192, S=0, formats="q3"),          # k = 1, 3-bit only
+    dict(T=17, H=128, E=12, k=12, I=64, S=1, formats="ternary"),   # k = E: every expert
+    dict(T=3, H=128, E=40, k=16, I=64, S=0, formats="mixed"),      # k = 16
+])
+def test_micro_shapes(kw):
+    cfg = synth.micro(**kw, seed=sum(kw[k] for k in ("T", "H", "E", "k", "I")))
+    for path in (1, 2):
+        _full_check(cfg, path)
+
+
+def test_one_expert_takes_every_token_and_empty_experts():
+    """A large bias on expert 3 makes every token pick it first; most experts stay
+    empty (k = 2 of 64)."""
+    cfg = synth.micro(T=96, H=128, E=64, k=2, I=64, S=1, formats="mixed", seed=7)
+    bias = np.zeros(cfg.E, np.float32)
+    bias[3] = 30.0
+    bias[40:] = -30.0
+    (_, _), case, rt = _full_check(cfg, 0, bias=bias)
+    assert rt["counts"][3] == cfg.T
+    assert (rt["counts"] == 0).sum() >= 1
+
+
+def test_zero_tokens_is_a_no_op():
+    import torch
+    import bit_routed_expert_fp32_b200 as moe
+    cfg = synth.micro(T=4, H=128, E=8, k=2, I=64, S=1)
+    case = H.make_case(cfg)
+    layer = moe.MoeLayer(cfg, H.pack(case), case.layer.router_w, None, 4)
+    x = moe.bf16_to_device(case.x)
+    y = torch.zeros((4, cfg.H), dtype=torch.bfloat16, device="cuda")
+    layer.route(x, T=0)
+    layer.forward(x, y, T=0)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y.view(torch.int16)) == 0
+
+
+def test_repeated_calls_are_deterministic():
+    """Counters are self-resetting: the same call twice gives identical bits."""
+    import torch
+    import bit_routed_expert_fp32_b200 as moe
+    cfg = synth.micro(T=70, H=256, E=32, k=4, I=128, S=1, formats="mixed", seed=3)
+    case = H.make_case(cfg)
+    layer = moe.MoeLayer(cfg, H.pack(case), case.layer.router_w, None, cfg.T)
+    x = moe.bf16_to_device(case.x)
+    outs = []
+    for path in (1, 1, 2, 2):
+        y = layer(x, path=path)
+        torch.cuda.synchronize()
+        outs.append(moe.bf16_to_host(y))
+    np.testing.assert_array_equal(outs[0], outs[1])
+    np.testing.assert_array_equal(outs[2], outs[3])
+    assert moe.moe_get_error(layer.ws)[0] == 0
+
+
+# ---- full-size workloads (sampled outputs) -------------------------------------
+
+@pytest.mark.parametrize("n", [2, 3, 4, 5])
+def test_full_size_workloads(n):
+    """The four full-size workloads in the launch configuration the benchmark times:
+    routing checked for every token, outputs for a sample the oracle can afford."""
+    import torch
+    cfg = synth.CONFIGS[n]
+    case = H.make_case(cfg)
+    packed = H.pack(case)
+    rt, y = H.run_gpu(case, packed, path=0)
+    H.check_routing(case, rt)
+    toks = list(range(cfg.T)) if cfg.T <= 16 else H.sample_tokens(case, 64, seed=n)
+    ref = H.oracle_outputs(case, toks)
+    H.check_outputs(y[toks], ref)
+    if n == 5:
+        assert case.counts.max() >= 8 * case.counts.mean() and (case.counts == 0).sum() >= 1
+    del packed
+    torch.cuda.empty_cache()

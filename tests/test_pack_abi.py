@@ -1,0 +1,124 @@
+"""Host-side checks of the C ABI library (no GPU): exported symbols, argument
+validation, and the packer checked against the oracle's independent reader of the
+packed format."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import bit_routed_expert_fp32_b200 as moe
+import oracle
+import synth
+from tests.dense_ref import codes_int
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declarations_match_binding():
+    assert declared_functions() == sorted(moe.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in syms, name
+        assert getattr(moe.lib(), name) is not None
+    assert moe.lib().moe_abi_version() == 1
+    assert moe.moe_status_string(0) == "ok"
+
+
+def _shape(H=128, I=64, E=4, k=2, S=1):
+    return moe.Shape(H, I, E, k, S)
+
+
+def test_argument_errors_are_synchronous():
+    L = moe.lib()
+    sz = ctypes.c_size_t(0)
+    fmt = np.ones(5, np.uint8)
+    assert L.moe_packed_size(None, fmt.ctypes.data, ctypes.byref(sz)) == 1
+    bad = _shape(H=100)
+    assert L.moe_packed_size(ctypes.byref(bad), fmt.ctypes.data, ctypes.byref(sz)) == 1
+    assert L.moe_workspace_size(ctypes.byref(_shape(k=5)), 4, ctypes.byref(sz)) == 1       # k > E
+    assert L.moe_workspace_size(ctypes.byref(_shape()), -1, ctypes.byref(sz)) == 1
+    fmt_bad = np.array([1, 1, 3, 1, 1], np.uint8)
+    assert L.moe_packed_size(ctypes.byref(_shape()), fmt_bad.ctypes.data, ctypes.byref(sz)) == 1
+    sh = _shape()
+    fake = ctypes.c_void_p(0x1000)
+    r = moe.Routing(*([0x1000] * 6))
+    assert L.moe_workspace_size(ctypes.byref(sh), 8, ctypes.byref(sz)) == 0
+    need = sz.value
+    # workspace too small, negative T, null x, null routing member: rejected before any launch
+    assert L.moe_route(ctypes.byref(sh), 8, fake, fake, None, ctypes.byref(r), fake, need - 1, None) == 3
+    assert L.moe_route(ctypes.byref(sh), -1, fake, fake, None, ctypes.byref(r), fake, need, None) == 1
+    assert L.moe_route(ctypes.byref(sh), 8, None, fake, None, ctypes.byref(r), fake, need, None) == 1
+    r0 = moe.Routing(0x1000, 0x1000, 0, 0x1000, 0x1000, 0x1000)
+    assert L.moe_route(ctypes.byref(sh), 8, fake, fake, None, ctypes.byref(r0), fake, need, None) == 1
+    assert L.moe_forward(ctypes.byref(sh), 8, fake, fake, ctypes.byref(r), fake, 7, fake, need, None) == 1
+    # T = 0 is a no-op
+    assert L.moe_route(ctypes.byref(sh), 0, fake, fake, None, ctypes.byref(r), fake, need, None) == 0
+    assert L.moe_forward(ctypes.byref(sh), 0, fake, fake, ctypes.byref(r), fake, 0, fake, need, None) == 0
+
+
+@pytest.mark.parametrize("H,I,formats", [(128, 64, "mixed"), (192, 128, "q3"), (256, 64, "ternary"),
+                                         (64, 192, "q2"), (384, 256, "mixed")])
+def test_pack_roundtrip_through_oracle_reader(H, I, formats):
+    cfg = synth.micro(T=1, H=H, E=6, k=2, I=I, S=1, formats=formats, seed=H + I)
+    layer = synth.Layer(cfg)
+    buf = moe.pack_layer(cfg, layer.fmt, layer.expert)
+    assert buf.size == moe.moe_packed_size(cfg, layer.fmt)
+    for e in range(cfg.E + cfg.S):
+        mats = layer.expert(e)
+        for which, name, rows, K in ((0, "gate", I, H), (1, "up", I, H), (2, "down", H, I)):
+            f, codes, scales = oracle.unpack(buf, e, which, rows, K)
+            c, h, s = mats[name]
+            assert f == layer.fmt[e]
+            np.testing.assert_array_equal(codes, codes_int(c, h))
+            np.testing.assert_array_equal(scales, s)
+
+
+def test_pack_edge_codes():
+    """All-minimum and all-maximum codes survive the round trip."""
+    cfg = synth.micro(T=1, H=128, E=2, k=1, I=64, S=0, formats="q3", seed=1)
+    fmt = np.array([2, 2], np.uint8)
+
+    def mats(e):
+        byte = 0x00 if e == 0 else 0xFF
+        out = {}
+        for name, rows, K in (("gate", 64, 128), ("up", 64, 128), ("down", 128, 64)):
+            out[name] = (np.full((rows, K // 4), byte, np.uint8), np.full((rows, K // 8), byte, np.uint8),
+                         np.full((rows, K // 64), 0x3C00, np.uint16))
+        return out
+
+    buf = moe.pack_layer(cfg, fmt, mats)
+    for e, v in ((0, 0), (1, 7)):
+        for which, rows, K in ((0, 64, 128), (1, 64, 128), (2, 128, 64)):
+            f, codes, scales = oracle.unpack(buf, e, which, rows, K)
+            assert np.all(codes == v) and np.all(scales == 0x3C00)
+
+
+def test_pack_rejects_ternary_code_three_and_small_buffer():
+    cfg = synth.micro(T=1, H=64, E=1, k=1, I=64, S=0, formats="ternary", seed=2)
+    layer = synth.Layer(cfg)
+    m = layer.expert(0)
+    size = moe.moe_packed_size(cfg, layer.fmt)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_pack_experts(cfg, layer.fmt, 0, [m], np.zeros(size - 1, np.uint8))
+    assert ei.value.status == 3
+    c, h, s = m["down"]
+    c = c.copy()
+    c[5, 3] |= 0x0C          # one 2-bit field = 3
+    m["down"] = (c, h, s)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_pack_experts(cfg, layer.fmt, 0, [m], np.zeros(size, np.uint8))
+    assert ei.value.status == 1
