@@ -35,8 +35,8 @@ import synth  # noqa: E402
 
 METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B200)"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GATEUP_KERNEL = "ffn_mma_kernel<0>"
-KERNEL_SOURCES = ["bit_routed_expert_fp32_b200/csrc/expert_mma.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]
+GATEUP_KERNEL = "ffn_decode_kernel<0, NT>"
+KERNEL_SOURCES = ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]
 
 
 def peaks():
@@ -73,7 +73,7 @@ def traffic_record(cfg_name: str):
 def gu_bytes(cfg, fmt: int) -> int:
     """Packed bytes of one expert's fused gate/up matrix (codes + scales [+ third bits])."""
     K, rows = cfg.H, 2 * cfg.I
-    b = rows * (K // 4 + K // 32)
+    b = rows * (K // 4 + 16 * ((K // 64 + 7) // 8))
     if fmt == synth.FMT_Q3:
         b += rows * 4 * 4 * ((K + 127) // 128)
     return b
@@ -81,7 +81,7 @@ def gu_bytes(cfg, fmt: int) -> int:
 
 def dn_bytes(cfg, fmt: int) -> int:
     K, rows = cfg.I, cfg.H
-    b = rows * (K // 4 + K // 32)
+    b = rows * (K // 4 + 16 * ((K // 64 + 7) // 8))
     if fmt == synth.FMT_Q3:
         b += rows * 4 * 4 * ((K + 127) // 128)
     return b
@@ -151,13 +151,16 @@ def oracle_tokens_per_s(cfg, layer, xs, budget_s: float, max_tokens: int):
     budget_s has elapsed; returns (tokens/s, tokens, seconds, threads)."""
     import oracle
     threads = os.cpu_count() or 1
-    done, t0 = 0, time.perf_counter()
-    while done < max_tokens and time.perf_counter() - t0 < budget_s:
-        x = xs[done % len(xs)]
+    done, i, t0 = 0, 0, time.perf_counter()
+    while True:                      # at least one batch, then until the budget is used
+        x = xs[i % len(xs)]
         L = oracle.logits(x, layer.router_w, threads)
         ids, gates = oracle.select(L, layer.router_b, cfg.k)
         oracle.forward_tokens(layer, x, ids, gates, range(x.shape[0]), threads)
         done += x.shape[0]
+        i += 1
+        if done >= max_tokens or time.perf_counter() - t0 >= budget_s:
+            break
     dt = time.perf_counter() - t0
     return done / dt, done, dt, min(threads, 9 * max(1, xs[0].shape[0]))
 
@@ -234,6 +237,10 @@ def run_ours(args, cfg):
     ids_log = torch.empty((total, T, cfg.k), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(total)]
+    for row in ev:               # torch creates the CUDA event on first record: do it here so
+        for e in row:            # the handles handed to the library are real events
+            e.record(stream)
+    torch.cuda.synchronize(dev)
 
     def step(s, record=True):
         lay = layers[s % n_layers]

@@ -24,7 +24,7 @@ bool shape_ok(const moe_shape* s) {
 // sit at fixed offsets (independent of T) so that their cleared state survives
 // calls with different token counts; the token-sized arrays follow.
 struct Ws {
-    size_t ctrl, tile_ctr, active, logits, hist, h, ypart, total;
+    size_t ctrl, tile_ctr, active, logits, hist, zx, h, ypart, total;
 };
 
 Ws ws_layout(const moe_shape* s, int64_t T) {
@@ -41,6 +41,8 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     off = align256(off + 4 * (size_t)(T * E));
     w.hist = off;
     off = align256(off + 4 * (size_t)(((T + kChunk - 1) / kChunk) * E));
+    w.zx = off;
+    off = align256(off + 4 * (size_t)(3 * (H / 64) * T));
     w.h = off;
     off = align256(off + 2 * (size_t)(T * (k + S) * I));
     w.ypart = off;
@@ -129,6 +131,7 @@ moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x, con
     a.logits = reinterpret_cast<float*>(ws + w.logits);
     a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
     a.active = reinterpret_cast<int32_t*>(ws + w.active);
+    a.zx = reinterpret_cast<float*>(ws + w.zx);
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.r = *out;
     if (launch_route(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -162,6 +165,7 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.offsets = r->offsets;
     a.topk_w = r->topk_w;
     a.active = reinterpret_cast<const int32_t*>(ws + w.active);
+    a.zx = reinterpret_cast<const float*>(ws + w.zx);
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.h = reinterpret_cast<uint16_t*>(ws + w.h);
     a.ypart = reinterpret_cast<float*>(ws + w.ypart);
@@ -172,9 +176,8 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     if (events)
         for (int i = 0; i < 4; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
     if (ev[0] && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
-    cudaError_t err = launch_ffn_mma(a, s, ev[1]);
+    cudaError_t err = launch_ffn_decode(a, s, ev[1], ev[2]);
     if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
-    if (ev[2] && cudaEventRecord(ev[2], s) != cudaSuccess) return MOE_ERR_CUDA;
     if (ev[3] && cudaEventRecord(ev[3], s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }

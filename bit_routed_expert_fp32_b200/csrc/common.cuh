@@ -9,8 +9,9 @@
 
 namespace moe {
 
-// ---- packed format v1 (see include/moe.h) ----------------------------------
+// ---- packed format (see include/moe.h) ----------------------------------------
 constexpr uint32_t kMagic = 0x50454F4Du;
+constexpr uint32_t kVersion = 2u;
 constexpr int kGroup = 64;
 constexpr int kInterleave = 8;
 constexpr int kHeaderBytes = 256;
@@ -25,7 +26,6 @@ struct __align__(16) PackedEntry {
 };
 static_assert(sizeof(PackedEntry) == kEntryBytes, "entry layout");
 
-__host__ __device__ inline int hi_words(int K) { return 4 * ((K + 127) / 128); }
 
 // ---- workspace control block --------------------------------------------------
 // The first 4 KiB of the workspace; zeroed by moe_workspace_init.

@@ -18,6 +18,7 @@ struct RouteArgs {
     float* logits;      // ws [T][E]
     int32_t* hist;      // ws [ceil(T/kChunk)][E]
     int32_t* active;    // ws [E+S]
+    float* zx;          // ws [3][T][H/64] negated dequantiser offsets (see route.cu)
     Ctrl* ctrl;
     moe_routing r;
 };
@@ -32,6 +33,7 @@ struct FfnArgs {
     const int32_t* offsets;
     const float* topk_w;
     const int32_t* active;   // ws
+    const float* zx;         // ws [3][T][H/64], negated
     Ctrl* ctrl;
     uint16_t* h;             // ws fp16 [T*(k+S)][I]
     float* ypart;            // ws f32 [T*(k+S)][H]
@@ -41,6 +43,8 @@ struct FfnArgs {
 };
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
-cudaError_t launch_ffn_mma(const FfnArgs& a, cudaStream_t s, cudaEvent_t mid_event);
+// decode-path expert kernels + combine; ev_gateup / ev_down (may be null) are recorded
+// after the gate/up and the down kernel
+cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down);
 
 }  // namespace moe

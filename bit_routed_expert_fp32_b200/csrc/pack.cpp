@@ -1,4 +1,4 @@
-// Host-side packer: interchange-form codes and fp16 scales -> packed format v1
+// Host-side packer: interchange-form codes and fp16 scales -> packed format v2
 // (layout documented in include/moe.h).  Pure host code, no CUDA calls.
 #include <stdint.h>
 #include <string.h>
@@ -14,7 +14,8 @@ constexpr int kHeader = 256;
 constexpr int kEntry = 64;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-inline int hi_words(int K) { return 4 * ((K + 127) / 128); }
+// chunks of up to 8 groups of 64 along K
+inline int n_chunks(int K) { return (K / 64 + 7) / 8; }
 
 bool shape_ok(const moe_shape* s) {
     return s && s->hidden > 0 && s->inter > 0 && s->hidden % 64 == 0 && s->inter % 64 == 0 &&
@@ -33,13 +34,13 @@ struct ExpertLayout {
 size_t mat_bytes(int rows, int K, uint32_t fmt, MatLayout* m, size_t off) {
     off = align256(off);
     m->scales = off;
-    off = align256(off + (size_t)rows * (K / 64) * 2);
+    off = align256(off + (size_t)(rows / 16) * 256 * n_chunks(K));
     m->codes = off;
-    off += (size_t)rows * (K / 16) * 4;
+    off += (size_t)rows * (K / 4);
     if (fmt == MOE_FMT_Q3) {
         off = align256(off);
         m->hi = off;
-        off += (size_t)rows * hi_words(K) * 4;
+        off += (size_t)rows * (K / 8);
     } else {
         m->hi = 0;
     }
@@ -94,33 +95,44 @@ inline void store_u32(uint8_t* p, uint32_t v) {
     p[3] = (uint8_t)(v >> 24);
 }
 
-// Packs one source row (K elements) into destination row `dr` of a packed matrix.
+// Packs one source row (K elements) into packed row `dr` (tile dr/16, row dr%16) of a
+// matrix, in the tile/chunk-blocked, swizzled layout documented in moe.h.
 bool pack_row(const moe_matrix_src& src, int sr, int K, uint32_t fmt, uint8_t* base, const MatLayout& m, int dr) {
     const uint8_t* codes = src.codes + (size_t)sr * (K / 4);
     if (fmt == MOE_FMT_TERNARY) {
         for (int b = 0; b < K / 4; ++b)
             if (codes[b] & (codes[b] >> 1) & 0x55) return false;   // a field equal to 3
     }
-    uint8_t* cdst = base + m.codes + (size_t)dr * (K / 16) * 4;
-    for (int w = 0; w < K / 16; ++w) store_u32(cdst + 4 * w, code_word(load_u32(codes + 4 * w)));
-    uint8_t* sdst = base + m.scales + (size_t)dr * (K / 64) * 2;
-    const uint16_t* ssrc = src.scales + (size_t)sr * (K / 64);
-    for (int g = 0; g < K / 64; ++g) {
-        sdst[2 * g] = (uint8_t)ssrc[g];
-        sdst[2 * g + 1] = (uint8_t)(ssrc[g] >> 8);
-    }
-    if (fmt == MOE_FMT_Q3) {
-        const uint8_t* hi = src.hi + (size_t)sr * (K / 8);
-        const int W1 = hi_words(K);
-        uint8_t* hdst = base + m.hi + (size_t)dr * W1 * 4;
-        for (int w = 0; w < W1; ++w) store_u32(hdst + 4 * w, w < K / 32 ? hi_word(load_u32(hi + 4 * w)) : 0u);
+    const int G = K / 64, NC = n_chunks(K), j = dr / 16, r = dr % 16;
+    const uint16_t* ssrc = src.scales + (size_t)sr * G;
+    const uint8_t* hi = fmt == MOE_FMT_Q3 ? src.hi + (size_t)sr * (K / 8) : nullptr;
+    for (int c = 0; c < NC; ++c) {
+        const int ng = G - 8 * c < 8 ? G - 8 * c : 8;
+        uint8_t* cblk = base + m.codes + (size_t)4 * K * j + 2048 * (size_t)c;
+        for (int wl = 0; wl < 4 * ng; ++wl) {
+            const int pos = ng == 8 ? r * 32 + (wl ^ (4 * (r % 8))) : r * 4 * ng + wl;
+            store_u32(cblk + 4 * pos, code_word(load_u32(codes + 4 * (32 * c + wl))));
+        }
+        uint8_t* sblk = base + m.scales + (size_t)256 * NC * j + 256 * (size_t)c + 16 * r;
+        for (int gl = 0; gl < 8; ++gl) {
+            const uint16_t v = 8 * c + gl < G ? ssrc[8 * c + gl] : 0;
+            sblk[2 * gl] = (uint8_t)v;
+            sblk[2 * gl + 1] = (uint8_t)(v >> 8);
+        }
+        if (hi) {
+            uint8_t* hblk = base + m.hi + (size_t)128 * G * j + 1024 * (size_t)c;
+            for (int vl = 0; vl < 2 * ng; ++vl) {
+                const int pos = ng == 8 ? r * 16 + (vl ^ (2 * ((r % 8) / 2))) : r * 2 * ng + vl;
+                store_u32(hblk + 4 * pos, hi_word(load_u32(hi + 4 * (16 * c + vl))));
+            }
+        }
     }
     return true;
 }
 
 void write_header(const moe_shape* s, const std::vector<ExpertLayout>& L, size_t total, uint8_t* dst) {
     memset(dst, 0, kHeader);
-    uint32_t h[8] = {kMagic, 1u, (uint32_t)s->hidden, (uint32_t)s->inter, (uint32_t)s->n_experts,
+    uint32_t h[8] = {kMagic, 2u, (uint32_t)s->hidden, (uint32_t)s->inter, (uint32_t)s->n_experts,
                      (uint32_t)s->n_shared, 64u, 8u};
     for (int i = 0; i < 8; ++i) store_u32(dst + 4 * i, h[i]);
     store_u32(dst + 32, (uint32_t)total);

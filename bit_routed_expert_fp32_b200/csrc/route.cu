@@ -7,9 +7,9 @@
 // L = x Wr^T + b; the k largest logits (ties to the lower id) in descending order;
 // gates = softmax over the k selected logits, which equals p_sel / sum p_sel.
 //
-// Decode (T <= 64): one launch.  64 CTAs stream the 7.3 MB fp32 router (a warp per
-// expert row), and the last CTA to finish (atomic ticket) does top-k, histogram,
-// scan and permutation for all T tokens.
+// Decode (T <= 64): one launch.  E/2 CTAs stream the 7.3 MB fp32 router (four warps
+// per expert row), compute the Z tables of the gate/up dequantiser, and the last
+// CTA to finish (atomic ticket) does top-k, histogram, scan and permutation.
 // Prefill: a tiled fp32 GEMM for the logits, a top-k kernel whose last CTA scans the
 // per-chunk histograms, and a scatter kernel that writes perm/inv_perm per chunk.
 // Ordering inside an expert is token ascending, made deterministic by processing the
@@ -146,37 +146,99 @@ __device__ void warp_active(const int* s_cnt, int E, int S, int32_t* active, Ctr
     }
 }
 
+// ---------------------------------------------------------------- Z tables
+// The gate/up expert kernel feeds the MMA with "base + c" values straight out of the
+// code words (no per-pair subtraction) and starts every 64-wide group's accumulator
+// at -Z.  For token t and group G (elements x_e, e = 0..63 of the group):
+//   Bx = sum_e lo_base(e) x_e,  Hx = sum_e hi_base(e) x_e,  Sx = sum_e x_e,
+// with lo_base / hi_base the magic bases the expert kernel uses for the pair that
+// holds element e (pair p = (e % 16) / 2):  lo 64,32,8,16,4,64,16,4 and
+// hi 512,256,128,64,32,16,8,8.  Then for code offset o:
+//   Z_ternary = Bx + Sx,  Z_q2 = Bx + 1.5 Sx,  Z_q3 = Bx + Hx + 3.5 Sx.
+// Stored negated as zx[format][T][G] (the MMA's accumulator input).
+__device__ void compute_z(const RouteArgs& p, int t, int Gi, int lane) {
+    constexpr float kLo[8] = {64.f, 32.f, 8.f, 16.f, 4.f, 64.f, 16.f, 4.f};
+    constexpr float kHi[8] = {512.f, 256.f, 128.f, 64.f, 32.f, 16.f, 8.f, 8.f};
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * p.H + Gi * 64) + lane);
+    const float x0 = bf16lo(v), x1 = bf16hi(v);
+    const float bl = kLo[lane & 7], bh = kHi[lane & 7];
+    float bx = fmaf(bl, x0, bl * x1), hx = fmaf(bh, x0, bh * x1), sx = x0 + x1;
+    bx = warp_sum(bx);
+    hx = warp_sum(hx);
+    sx = warp_sum(sx);
+    if (lane == 0) {
+        const int G = p.H / 64;
+        const size_t i = (size_t)t * G + Gi, plane = (size_t)p.T * G;
+        p.zx[i] = -(bx + sx);
+        p.zx[plane + i] = -fmaf(1.5f, sx, bx);
+        p.zx[2 * plane + i] = -fmaf(3.5f, sx, bx + hx);
+    }
+}
+
+__global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
+    const int G = p.H / 64;
+    const int warp = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (warp < p.T * G) compute_z(p, warp / G, warp % G, lane);
+}
+
 // ---------------------------------------------------------------- decode router
-__global__ void __launch_bounds__(128) route_small_kernel(RouteArgs p) {
+// 2 experts per CTA, 4 warps per expert row (one K quarter each), 7 float4 loads in
+// flight per lane; then the Z tables; the last CTA does top-k and the permutation.
+__global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
+    constexpr int U = 7;
+    __shared__ float s_part[8][kSmallT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 4 + warp;
+    const int el = warp >> 2, q = warp & 3;
+    const int e = blockIdx.x * 2 + el;
+    const int q4 = p.H / 16;                     // float4 per K quarter
     if (e < p.E) {
-        const float4* w4 = reinterpret_cast<const float4*>(p.Wr + (size_t)e * p.H);
-        const int n4 = p.H / 4;
-        const float b = p.bias ? p.bias[e] : 0.f;
+        const float4* w4 = reinterpret_cast<const float4*>(p.Wr + (size_t)e * p.H) + q * q4;
         for (int tb = 0; tb < p.T; tb += 8) {
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-            for (int i = lane; i < n4; i += 32) {
-                float4 w = __ldg(w4 + i);
+            for (int i0 = lane; i0 < q4; i0 += 32 * U) {
+                float4 w[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = i0 + 32 * u;
+                    w[u] = i < q4 ? __ldg(w4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    if (tb + j < p.T) {
-                        uint2 xv = __ldg(reinterpret_cast<const uint2*>(p.x + (size_t)(tb + j) * p.H) + i);
-                        acc[j] = fmaf(w.x, bf16lo(xv.x), acc[j]);
-                        acc[j] = fmaf(w.y, bf16hi(xv.x), acc[j]);
-                        acc[j] = fmaf(w.z, bf16lo(xv.y), acc[j]);
-                        acc[j] = fmaf(w.w, bf16hi(xv.y), acc[j]);
+                    if (tb + j >= p.T) break;
+                    const uint2* xr = reinterpret_cast<const uint2*>(p.x + (size_t)(tb + j) * p.H) + q * q4;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int i = i0 + 32 * u;
+                        if (i < q4) {
+                            const uint2 xv = __ldg(xr + i);
+                            acc[j] = fmaf(w[u].x, bf16lo(xv.x), acc[j]);
+                            acc[j] = fmaf(w[u].y, bf16hi(xv.x), acc[j]);
+                            acc[j] = fmaf(w[u].z, bf16lo(xv.y), acc[j]);
+                            acc[j] = fmaf(w[u].w, bf16hi(xv.y), acc[j]);
+                        }
                     }
                 }
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                float v = warp_sum(acc[j]);
-                if (lane == 0 && tb + j < p.T) p.logits[(size_t)(tb + j) * p.E + e] = v + b;
+                const float v = warp_sum(acc[j]);
+                if (lane == 0 && tb + j < p.T) s_part[warp][tb + j] = v;
             }
         }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 2 * p.T; i += blockDim.x) {
+        const int l = i / p.T, t = i - l * p.T, ee = blockIdx.x * 2 + l;
+        if (ee < p.E) {
+            const float v = (s_part[4 * l][t] + s_part[4 * l + 1][t]) + (s_part[4 * l + 2][t] + s_part[4 * l + 3][t]);
+            p.logits[(size_t)t * p.E + ee] = v + (p.bias ? p.bias[ee] : 0.f);
+        }
+    }
+    {
+        const int G = p.H / 64;
+        for (int pr = blockIdx.x * 8 + warp; pr < p.T * G; pr += gridDim.x * 8) compute_z(p, pr / G, pr % G, lane);
     }
     __shared__ int s_last;
     __threadfence();
@@ -189,8 +251,8 @@ __global__ void __launch_bounds__(128) route_small_kernel(RouteArgs p) {
     __shared__ int32_t s_ids[kSmallT * 16];
     __shared__ int s_cnt[256];
     __shared__ int s_off[257];
-    // top-k per token: warp w takes tokens w, w+4, ...
-    for (int t = warp; t < p.T; t += 4) {
+    // top-k per token: warp w takes tokens w, w+8, ...
+    for (int t = warp; t < p.T; t += 8) {
         float v[8];
         load_logits_row(p.logits + (size_t)t * p.E, p.E, lane, v);
         warp_topk(v, p.k, lane, p.r.topk_ids + (size_t)t * p.k, p.r.topk_w + (size_t)t * p.k);
@@ -353,9 +415,11 @@ __global__ void __launch_bounds__(32) route_scatter_kernel(RouteArgs p) {
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     if (a.T <= kSmallT) {
-        route_small_kernel<<<(a.E + 3) / 4, 128, 0, s>>>(a);
+        route_small_kernel<<<(a.E + 1) / 2, 256, 0, s>>>(a);
         return cudaGetLastError();
     }
+    const int zwarps = a.T * (a.H / 64);
+    route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
     dim3 g1((a.T + GBM - 1) / GBM, (a.E + GBN - 1) / GBN);
     route_logits_gemm_kernel<<<g1, 256, 0, s>>>(a);
     const int nchunks = (a.T + kChunk - 1) / kChunk;

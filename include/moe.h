@@ -87,12 +87,12 @@ typedef struct {
 } moe_routing;
 
 /* ---------------------------------------------------------------------------
- * Packed expert format, version 1 (defined by this library; the pages name the
+ * Packed expert format, version 2 (defined by this library; the pages name the
  * ternary / 2-bit / 3-bit mix but give no layout).  Little-endian throughout;
  * offsets are from the start of the buffer; every array starts on 256 bytes.
  *
  * Header, 256 bytes:
- *    0 u32 magic 0x50454F4D ('M','O','E','P' in memory)   4 u32 version = 1
+ *    0 u32 magic 0x50454F4D ('M','O','E','P' in memory)   4 u32 version = 2
  *    8 i32 H   12 i32 I   16 i32 E   20 i32 S   24 i32 group = 64
  *   28 i32 interleave R = 8   32 u64 total bytes   40..255 zero
  * Expert table at byte 256: E+S entries (routed experts, then shared) of 64 bytes:
@@ -102,20 +102,35 @@ typedef struct {
  *   56 u64 zero;  *_hi is 0 unless the format is MOE_FMT_Q3
  * Data follows the table, expert by expert, arrays in the order listed.
  *
- * A matrix W[N][K] is stored as
- *   scales fp16 [N][K/64]            s[n][k/64]
- *   codes  u32  [N][K/16]            word w of a row holds elements k = 16w .. 16w+15;
- *                                    element 16w + 2p + h (p = 0..7, h = 0/1) is the
- *                                    2-bit field at bits 16h + 2p .. 16h + 2p + 1
- *   hi     u32  [N][4*ceil(K/128)]   (3-bit only) word w holds the third code bit of
- *                                    elements k = 32w .. 32w+31; element
- *                                    32w + 16q + 2p + h is at bit 16h + 8q + p
- * The value of element (n, k) with code c is
+ * Codes.  Element k of a row has a code c; the 2-bit field lo = c & 3 of elements
+ * 16w .. 16w+15 forms "code word" w of the row (element 16w + 2p + h, p = 0..7,
+ * h = 0/1, at bits 16h + 2p .. 16h + 2p + 1); for 3-bit codes the third bit hi = c >> 2
+ * of elements 32v .. 32v+31 forms "third-bit word" v (element 32v + 16q + 2p + h at
+ * bit 16h + 8q + p).  The value of element (n, k) with code c and scale s is
  *   ternary  (c - 1)   * s,  c in {0,1,2} (c = 3 is rejected by the packer)
  *   q2       (c - 1.5) * s,  c in 0..3
  *   q3       (c - 3.5) * s,  c = lo + 4*hi in 0..7
- * Gate and up are fused into one matrix GU[2I][H]: row r lies in block b = r/16;
- * r%16 < 8 is gate row 8b + r%16, otherwise up row 8b + r%16 - 8.  Down is D[H][I].
+ * with s the fp16 scale of the element's group (64 consecutive k).
+ *
+ * Blocking.  A matrix W[N][K] (N a multiple of 16, K of 64) has G = K/64 groups per
+ * row, cut into NC = ceil(G/8) chunks; chunk c holds groups 8c .. 8c+ng-1 with
+ * ng = min(8, G - 8c).  Rows are cut into tiles of 16 (tile j = rows 16j..16j+15,
+ * r = row within the tile).  Every array stores one contiguous block per
+ * (tile, chunk), blocks in tile-major order:
+ *   codes  block (j,c) at byte 4*K*j + 2048*c, 256*ng bytes: the 4*ng code words
+ *          wl = 4*gl + q (gl = group in chunk, q = 16-element quarter) of each row,
+ *          word (r, wl) at u32 index  r*32 + (wl ^ 4*(r%8))  if ng = 8,
+ *                                     r*4*ng + wl            otherwise;
+ *   hi     (3-bit only) block (j,c) at byte 128*G*j + 1024*c, 128*ng bytes: third-bit
+ *          words vl = 2*gl + half of each row at u32 index
+ *                                     r*16 + (vl ^ 2*((r%8)/2))  if ng = 8,
+ *                                     r*2*ng + vl                 otherwise;
+ *   scales block (j,c) at byte 256*NC*j + 256*c, 256 bytes: fp16 scale of group
+ *          8c + gl of row r at half index r*8 + gl (zero where 8c + gl >= G).
+ * (The XOR swizzles make the fragment reads of a 16-row chunk in shared memory free
+ * of bank conflicts.)  Gate and up are fused into one matrix GU[2I][H]: row r lies in
+ * block b = r/16; r%16 < 8 is gate row 8b + r%16, otherwise up row 8b + r%16 - 8.
+ * Down is D[H][I].
  * ------------------------------------------------------------------------- */
 
 /* One source matrix in the interchange layout the packer reads (host memory):

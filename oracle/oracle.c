@@ -222,16 +222,21 @@ static uint64_t rd64(const uint8_t* p) { return (uint64_t)rd32(p) | ((uint64_t)r
 /* Reads matrix `which` (0 gate [I][H], 1 up [I][H], 2 down [H][I]) of expert table
  * entry `table` from a packed buffer: codes as int8 [rows][K] (full code 0..7) and
  * scales as fp16 bits [rows][K/64].  *fmt receives the format.
- * Layout read here (packed format version 1): header of 256 bytes (magic 'MOEP',
- * version 1, H, I, E, S, group 64, interleave 8); table of 64-byte entries at 256
+ * Layout read here (packed format version 2): header of 256 bytes (magic 'MOEP',
+ * version 2, H, I, E, S, group 64, interleave 8); table of 64-byte entries at 256
  * ({u32 fmt, u32 0, u64 gu_scales, gu_codes, gu_hi, dn_scales, dn_codes, dn_hi});
- * gate/up fused as GU[2I][H] with rows interleaved 8 gate / 8 up; code word w holds
- * element 16w + 2p + h at bit 16h + 2p; third-bit word w (row stride 4*ceil(K/128)
- * words) holds element 32w + 16q + 2p + h at bit 16h + 8q + p.
+ * gate/up fused as GU[2I][H] with rows interleaved 8 gate / 8 up.  Each array holds
+ * one block per (16-row tile j, chunk c of up to 8 groups of 64, ng groups):
+ *   codes  at 4*K*j + 2048*c; word wl = 4*gl + quarter of tile row r at u32 index
+ *          r*32 + (wl ^ 4*(r%8)) when ng == 8, else r*4*ng + wl; element 16w+2p+h of
+ *          a code word at bits 16h+2p..+1;
+ *   hi     at 128*G*j + 1024*c; word vl = 2*gl + half at r*16 + (vl ^ 2*((r%8)/2)) when
+ *          ng == 8, else r*2*ng + vl; element 32v+16q+2p+h at bit 16h+8q+p;
+ *   scales at 256*NC*j + 256*c; scale of group 8c+gl of row r at half r*8 + gl.
  * Returns 0 or a negative error. */
 int oracle_unpack(const uint8_t* buf, size_t bytes, int table, int which, int8_t* codes,
                   uint16_t* scales, int* fmt) {
-    if (bytes < 256 || rd32(buf) != 0x50454F4Du || rd32(buf + 4) != 1u) return -1;
+    if (bytes < 256 || rd32(buf) != 0x50454F4Du || rd32(buf + 4) != 2u) return -1;
     int H = (int)rd32(buf + 8), I = (int)rd32(buf + 12), E = (int)rd32(buf + 16);
     int S = (int)rd32(buf + 20), R = (int)rd32(buf + 28);
     if ((int)rd32(buf + 24) != ORACLE_GROUP || R != 8) return -2;
@@ -241,31 +246,36 @@ int oracle_unpack(const uint8_t* buf, size_t bytes, int table, int which, int8_t
     *fmt = f;
     int rows = which == 2 ? H : I;
     int K = which == 2 ? I : H;
+    int G = K / ORACLE_GROUP;
+    int NC = (G + 7) / 8;
     uint64_t off_s = rd64(ent + (which == 2 ? 32 : 8));
     uint64_t off_c = rd64(ent + (which == 2 ? 40 : 16));
     uint64_t off_h = rd64(ent + (which == 2 ? 48 : 24));
-    int hi_stride = 4 * ((K + 127) / 128);
     for (int n = 0; n < rows; ++n) {
         /* physical row in the packed matrix */
-        int pr;
-        if (which == 2) pr = n;
-        else pr = 16 * (n / 8) + (which == 1 ? 8 : 0) + n % 8;
-        for (int g = 0; g < K / ORACLE_GROUP; ++g) {
-            const uint8_t* sp = buf + off_s + ((size_t)pr * (K / ORACLE_GROUP) + g) * 2;
-            scales[(size_t)n * (K / ORACLE_GROUP) + g] = (uint16_t)(sp[0] | (sp[1] << 8));
+        int pr = which == 2 ? n : 16 * (n / 8) + (which == 1 ? 8 : 0) + n % 8;
+        int j = pr / 16, r = pr % 16;
+        for (int g = 0; g < G; ++g) {
+            int c = g / 8, gl = g % 8;
+            const uint8_t* sp = buf + off_s + (size_t)256 * NC * j + 256 * (size_t)c + 16 * r + 2 * gl;
+            scales[(size_t)n * G + g] = (uint16_t)(sp[0] | (sp[1] << 8));
         }
         for (int k = 0; k < K; ++k) {
-            int w = k / 16, i = k % 16;
-            int p = i / 2, h = i % 2;
-            uint32_t word = rd32(buf + off_c + ((size_t)pr * (K / 16) + w) * 4);
-            int c = (int)((word >> (16 * h + 2 * p)) & 3u);
+            int g = k / 64, c = g / 8, gl = g % 8;
+            int ng = G - 8 * c < 8 ? G - 8 * c : 8;
+            int wl = 4 * gl + (k % 64) / 16;
+            int pos = ng == 8 ? r * 32 + (wl ^ (4 * (r % 8))) : r * 4 * ng + wl;
+            uint32_t word = rd32(buf + off_c + (size_t)4 * K * j + 2048 * (size_t)c + 4 * (size_t)pos);
+            int i = k % 16, p = i / 2, h = i % 2;
+            int code = (int)((word >> (16 * h + 2 * p)) & 3u);
             if (f == 2) {
-                int w1 = k / 32, i1 = k % 32;
-                int q = i1 / 16, p1 = (i1 % 16) / 2, h1 = i1 % 2;
-                uint32_t hw = rd32(buf + off_h + ((size_t)pr * hi_stride + w1) * 4);
-                c += 4 * (int)((hw >> (16 * h1 + 8 * q + p1)) & 1u);
+                int vl = 2 * gl + (k % 64) / 32;
+                int hpos = ng == 8 ? r * 16 + (vl ^ (2 * ((r % 8) / 2))) : r * 2 * ng + vl;
+                uint32_t hw = rd32(buf + off_h + (size_t)128 * G * j + 1024 * (size_t)c + 4 * (size_t)hpos);
+                int e = k % 32, q = e / 16, p1 = (e % 16) / 2, h1 = e % 2;
+                code += 4 * (int)((hw >> (16 * h1 + 8 * q + p1)) & 1u);
             }
-            codes[(size_t)n * K + k] = (int8_t)c;
+            codes[(size_t)n * K + k] = (int8_t)code;
         }
     }
     return 0;

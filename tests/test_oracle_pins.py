@@ -275,40 +275,45 @@ def test_dequant_scale_index_is_per_row_group():
 # ---- the oracle's reader of the packed format -------------------------------
 
 def _hand_packed(fmt, H, I, gu_codes, gu_hi, dn_codes, dn_hi, scale_bits):
-    """Packed buffer for E=1, S=0 built directly from the format's definition:
-    every word is assembled from per-element bit positions (tests only)."""
-    def put_plane(rows, K, code_of):
-        words = np.zeros((rows, K // 16), np.uint32)
-        for r in range(rows):
+    """Packed buffer (format version 2) for E=1, S=0 built directly from the format's
+    definition, element by element (tests only)."""
+    def blocks(rows, K, code_of):
+        G = K // 64
+        NC = (G + 7) // 8
+        codes = np.zeros(rows * K // 16, np.uint32)
+        hi = np.zeros(rows * K // 32, np.uint32)
+        scales = np.zeros((rows // 16) * NC * 128, np.uint16)
+        for pr in range(rows):
+            j, r = divmod(pr, 16)
             for k in range(K):
-                w, i = divmod(k, 16)
-                p, hh = divmod(i, 2)
-                words[r, w] |= np.uint32((code_of(r, k) & 3) << (16 * hh + 2 * p))
-        return words
-
-    def put_hi(rows, K, bit_of):
-        stride = 4 * ((K + 127) // 128)
-        words = np.zeros((rows, stride), np.uint32)
-        for r in range(rows):
-            for k in range(K):
-                w, i = divmod(k, 32)
-                q, rest = divmod(i, 16)
-                p, hh = divmod(rest, 2)
-                words[r, w] |= np.uint32(bit_of(r, k) << (16 * hh + 8 * q + p))
-        return words
+                g, kk = divmod(k, 64)
+                c, gl = divmod(g, 8)
+                ng = min(8, G - 8 * c)
+                wl = 4 * gl + kk // 16
+                pos = r * 32 + (wl ^ (4 * (r % 8))) if ng == 8 else r * 4 * ng + wl
+                idx = (4 * K * j + 2048 * c) // 4 + pos
+                p_, h_ = divmod(k % 16, 2)
+                cv = code_of(pr, k)
+                codes[idx] |= np.uint32((cv & 3) << (16 * h_ + 2 * p_))
+                vl = 2 * gl + kk // 32
+                hpos = r * 16 + (vl ^ (2 * ((r % 8) // 2))) if ng == 8 else r * 2 * ng + vl
+                hidx = (128 * G * j + 1024 * c) // 4 + hpos
+                q_, rest = divmod(k % 32, 16)
+                p1, h1 = divmod(rest, 2)
+                hi[hidx] |= np.uint32(((cv >> 2) & 1) << (16 * h1 + 8 * q_ + p1))
+            for g in range(G):
+                c, gl = divmod(g, 8)
+                scales[(256 * NC * j + 256 * c) // 2 + 8 * r + gl] = scale_bits
+        return scales, codes, hi
 
     def gu_src(r):                   # packed GU row -> (gate?, source row)
-        b, j = divmod(r, 16)
-        return (j < 8), 8 * b + (j % 8)
+        b, jj = divmod(r, 16)
+        return (jj < 8), 8 * b + (jj % 8)
 
     gu_full = lambda r, k: (gu_codes[0] if gu_src(r)[0] else gu_codes[1])[gu_src(r)[1], k]
-    arrays = []
-    arrays.append(np.full((2 * I, H // 64), scale_bits, np.uint16))
-    arrays.append(put_plane(2 * I, H, lambda r, k: gu_full(r, k)))
-    arrays.append(put_hi(2 * I, H, lambda r, k: gu_full(r, k) >> 2) if fmt == FMT_Q3 else None)
-    arrays.append(np.full((H, I // 64), scale_bits, np.uint16))
-    arrays.append(put_plane(H, I, lambda r, k: dn_codes[r, k]))
-    arrays.append(put_hi(H, I, lambda r, k: dn_codes[r, k] >> 2) if fmt == FMT_Q3 else None)
+    gs, gc, gh = blocks(2 * I, H, gu_full)
+    ds, dc, dh = blocks(H, I, lambda r, k: dn_codes[r, k])
+    arrays = [gs, gc, gh if fmt == FMT_Q3 else None, ds, dc, dh if fmt == FMT_Q3 else None]
     off = 256 + 64
     offs = []
     blobs = []
@@ -322,7 +327,7 @@ def _hand_packed(fmt, H, I, gu_codes, gu_hi, dn_codes, dn_hi, scale_bits):
         off += a.nbytes
     total = off
     buf = bytearray(total)
-    hdr = np.array([0x50454F4D, 1, H, I, 1, 0, 64, 8], np.uint32).tobytes()
+    hdr = np.array([0x50454F4D, 2, H, I, 1, 0, 64, 8], np.uint32).tobytes()
     buf[0:32] = hdr
     buf[32:40] = np.uint64(total).tobytes()
     ent = np.zeros(8, np.uint64)
@@ -334,9 +339,10 @@ def _hand_packed(fmt, H, I, gu_codes, gu_hi, dn_codes, dn_hi, scale_bits):
     return np.frombuffer(bytes(buf), np.uint8)
 
 
-@pytest.mark.parametrize("fmt", [FMT_Q2, FMT_Q3])
-def test_oracle_unpack_reads_hand_built_buffer(fmt):
-    H, I = 128, 64
+@pytest.mark.parametrize("fmt,H,I", [(FMT_Q2, 128, 64), (FMT_Q3, 128, 64), (FMT_Q3, 576, 64),
+                                    (FMT_Q2, 64, 1024)])
+def test_oracle_unpack_reads_hand_built_buffer(fmt, H, I):
+    """Covers full 8-group chunks (swizzled) and tail chunks of 1, 2 and 1 groups."""
     rng = np.random.default_rng(10)
     top = 8 if fmt == FMT_Q3 else 4
     g = rng.integers(0, top, size=(I, H))
