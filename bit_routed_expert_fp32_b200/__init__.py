@@ -23,7 +23,9 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 # every symbol include/moe.h declares
 EXPORTS = ["moe_packed_size", "moe_pack_experts", "moe_workspace_size", "moe_workspace_init", "moe_route",
-           "moe_forward", "moe_forward_timed", "moe_get_error", "moe_status_string", "moe_abi_version"]
+           "moe_forward", "moe_forward_timed", "moe_get_error", "moe_decode_static", "moe_status_string",
+           "moe_abi_version"]
+STATIC_WS_BYTES = 8 << 20
 
 
 class MoeError(RuntimeError):
@@ -66,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_timed.argtypes = [sh, i32, vp, vp, ctypes.POINTER(Routing), vp, ctypes.c_int, vp, sz, vp,
                                         ctypes.POINTER(vp), i32]
         L.moe_get_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_decode_static.argtypes = [sh, i32, vp, vp, vp, vp, ctypes.POINTER(Routing), vp, vp]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_abi_version.restype = i32
@@ -172,6 +175,14 @@ def moe_forward(cfg, T, packed, x, rt: dict, y, path=PATH_AUTO, ws=None, stream=
     st = lib().moe_forward_timed(ctypes.byref(_shape(cfg)), T, _ptr(packed), _ptr(x), ctypes.byref(r), _ptr(y),
                                  path, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream), ev, 4)
     _check("moe_forward_timed", st)
+
+
+def moe_decode_static(cfg, T, x, router_w, router_b, packed, rt: dict, y, stream=None) -> None:
+    """Route + decode forward using the library's own scratch array (no workspace)."""
+    r = routing_struct(rt)
+    _check("moe_decode_static", lib().moe_decode_static(ctypes.byref(_shape(cfg)), T, _ptr(x), _ptr(router_w),
+                                                         _ptr(router_b), _ptr(packed), ctypes.byref(r), _ptr(y),
+                                                         _stream(stream)))
 
 
 def moe_get_error(ws, stream=None):

@@ -8,25 +8,15 @@
 #include "kernels.h"
 #include "moe.h"
 
+namespace moe {
+
 namespace {
-
-using namespace moe;
-
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-bool shape_ok(const moe_shape* s) {
-    return s && s->hidden > 0 && s->inter > 0 && s->hidden % 64 == 0 && s->inter % 64 == 0 &&
-           s->n_experts >= 1 && s->n_experts <= 256 && s->top_k >= 1 && s->top_k <= 16 &&
-           s->top_k <= s->n_experts && (s->n_shared == 0 || s->n_shared == 1);
-}
+}  // namespace
 
 // Workspace layout.  The control block, tile counters and the active-expert list
 // sit at fixed offsets (independent of T) so that their cleared state survives
 // calls with different token counts; the token-sized arrays follow.
-struct Ws {
-    size_t ctrl, tile_ctr, active, logits, hist, zx, h, ypart, total;
-};
-
 Ws ws_layout(const moe_shape* s, int64_t T) {
     Ws w;
     const int64_t E = s->n_experts, S = s->n_shared, k = s->top_k, H = s->hidden, I = s->inter;
@@ -49,6 +39,18 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     off = align256(off + 4 * (size_t)(T * (k + S) * H));
     w.total = off;
     return w;
+}
+
+}  // namespace moe
+
+namespace {
+
+using namespace moe;
+
+bool shape_ok(const moe_shape* s) {
+    return s && s->hidden > 0 && s->inter > 0 && s->hidden % 64 == 0 && s->inter % 64 == 0 &&
+           s->n_experts >= 1 && s->n_experts <= 256 && s->top_k >= 1 && s->top_k <= 16 &&
+           s->top_k <= s->n_experts && (s->n_shared == 0 || s->n_shared == 1);
 }
 
 size_t ws_fixed_prefix(const moe_shape* s) { return ws_layout(s, 0).active; }

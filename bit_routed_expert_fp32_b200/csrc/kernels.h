@@ -42,6 +42,13 @@ struct FfnArgs {
     int num_ctas;
 };
 
+// Workspace layout for T tokens (api.cu).  The control block, tile counters and the
+// active-expert list sit at fixed offsets (independent of T).
+struct Ws {
+    size_t ctrl, tile_ctr, active, logits, hist, zx, h, ypart, total;
+};
+Ws ws_layout(const moe_shape* s, int64_t T);
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // decode-path expert kernels + combine; ev_gateup / ev_down (may be null) are recorded
 // after the gate/up and the down kernel

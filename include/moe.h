@@ -206,6 +206,30 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
  * receives a kernel-specific code. For tests and diagnostics; not for hot loops. */
 moe_status moe_get_error(void* d_ws, size_t ws_bytes, void* stream, uint32_t* detail);
 
+/* No-allocation decode entry point.  The source pages have no counterpart to this
+ * call: it exists for callers of this library that cannot allocate device memory,
+ * such as a plugin inside a framework whose pool allocator owns all GPU memory, a
+ * serving loop that cannot afford cudaMalloc / cudaFree (they may synchronise the
+ * device), or code recording a CUDA graph, during which no allocation may happen.
+ * It does what moe_route followed by moe_forward(MOE_PATH_DECODE) do, with the same
+ * arguments and outputs (out: caller-allocated routing arrays; d_y: bf16 [T][H]), but
+ * instead of a caller-given workspace it uses a scratch array that the library holds
+ * in device memory: MOE_STATIC_WS_BYTES (8 MiB), held by every GPU that loads the
+ * library until the process exits.  It allocates nothing itself.
+ *   - If the workspace T tokens need (moe_workspace_size) exceeds MOE_STATIC_WS_BYTES
+ *     it returns MOE_ERR_WORKSPACE and enqueues nothing; with the full-size layer
+ *     (H 7168, I 2048, E 256, k 8, S 1) that allows up to 28 tokens per call.
+ *   - The first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before
+ *     any stream capture.  Later calls only enqueue work.
+ *   - All calls share the one array, and each call first clears its control block.
+ *     Calls that overlap on the GPU (other streams, other host threads, other
+ *     devices' calls do not overlap) race on the array: serialise them. */
+#define MOE_STATIC_WS_BYTES ((size_t)8 << 20)
+moe_status moe_decode_static(const moe_shape* shape, int32_t T, const uint16_t* d_x,
+                             const float* d_router_w, const float* d_router_b, const void* d_packed,
+                             const moe_routing* out, uint16_t* d_y, void* stream);
+
 const char* moe_status_string(moe_status s);
 int32_t moe_abi_version(void);
 
