@@ -35,7 +35,7 @@ import synth  # noqa: E402
 
 METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B200)"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GATEUP_KERNEL = "ffn_decode_kernel<0, NT>"
+GATEUP_KERNEL = "ffn_decode_kernel<0, NT, NW> (gate/up + SwiGLU)"
 KERNEL_SOURCES = ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]
 
 
@@ -146,23 +146,43 @@ def dist_env():
 
 
 # --------------------------------------------------------------------------- oracle
-def oracle_tokens_per_s(cfg, layer, xs, budget_s: float, max_tokens: int):
-    """Times the CPU oracle (routing + experts + combine) on whole tokens until
-    budget_s has elapsed; returns (tokens/s, tokens, seconds, threads)."""
+def _expert_cache(cfg, layer, xs, threads):
+    """Interchange-form weights of every expert the token batches touch (drawn before
+    timing: drawing inputs is not oracle work)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    need = set(range(cfg.E, cfg.E + cfg.S))
+    for x in xs:
+        _, ids, _ = oracle.route(x, layer.router_w, layer.router_b, cfg.k, threads)
+        need.update(int(e) for e in np.unique(ids))
+    with ThreadPoolExecutor(threads) as ex:
+        mats = list(ex.map(layer.expert, sorted(need)))
+    return dict(zip(sorted(need), mats))
+
+
+def oracle_tokens_per_s(cfg, layer, xs, budget_s: float, max_tokens: int, cache=None):
+    """Times the CPU oracle (routing + experts + combine) on whole token batches until
+    budget_s has elapsed (at least one batch); returns (tokens/s, tokens, seconds,
+    threads used).  Each call into the oracle is single-threaded; independent
+    experts run concurrently on the host cores."""
     import oracle
     threads = os.cpu_count() or 1
+    if cache is None:
+        cache = _expert_cache(cfg, layer, xs, threads)
     done, i, t0 = 0, 0, time.perf_counter()
-    while True:                      # at least one batch, then until the budget is used
+    used = 1
+    while True:
         x = xs[i % len(xs)]
         L = oracle.logits(x, layer.router_w, threads)
         ids, gates = oracle.select(L, layer.router_b, cfg.k)
-        oracle.forward_tokens(layer, x, ids, gates, range(x.shape[0]), threads)
+        oracle.forward_tokens(layer, x, ids, gates, range(x.shape[0]), threads, expert_cache=cache)
+        used = max(used, min(threads, len(np.unique(ids)) + cfg.S))
         done += x.shape[0]
         i += 1
         if done >= max_tokens or time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    return done / dt, done, dt, min(threads, 9 * max(1, xs[0].shape[0]))
+    return done / dt, done, dt, used
 
 
 def run_reference(args, cfg):
@@ -172,13 +192,15 @@ def run_reference(args, cfg):
     layer = synth.Layer(cfg, 0)
     per_step = max(1, min(cfg.T, 4))           # bounded sample of tokens per step
     xs = [synth.tokens(cfg, 0, s, per_step) for s in range(args.warmup + args.steps)]
+    cache = _expert_cache(cfg, layer, xs, os.cpu_count() or 1)
     for s in range(args.warmup):
-        oracle_tokens_per_s(cfg, layer, [xs[s]], 0.0, per_step)
+        oracle_tokens_per_s(cfg, layer, [xs[s]], 0.0, per_step, cache)
     t0 = time.perf_counter()
     tok, threads = 0, 1
     for s in range(args.steps):
-        _, n, _, threads = oracle_tokens_per_s(cfg, layer, [xs[args.warmup + s]], 0.0, per_step)
+        _, n, _, used = oracle_tokens_per_s(cfg, layer, [xs[args.warmup + s]], 0.0, per_step, cache)
         tok += n
+        threads = max(threads, used)
     dt = time.perf_counter() - t0
     value = tok / dt
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -187,7 +209,8 @@ def run_reference(args, cfg):
             "data": "synthetic", "config": config_dict(cfg, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": f"{per_step} token(s) of the workload per step, routed and run through "
-                                       f"all selected experts and the shared expert in fp64"},
+                                       f"all selected experts and the shared expert in fp64 (expert weights "
+                                       f"drawn before timing)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -245,20 +268,30 @@ def run_ours(args, cfg):
     def step(s, record=True):
         lay = layers[s % n_layers]
         e = ev[s]
-        e[0].record(stream)
+        if record:
+            e[0].record(stream)
         lay.route(x_dev[s])
         lay.forward(x_dev[s], y, events=e[1:5] if record else None)
-        e[5].record(stream)
-        ids_log[s].copy_(lay.rt["topk_ids"][:T])
+        if record:
+            e[5].record(stream)
+            ids_log[s].copy_(lay.rt["topk_ids"][:T])
 
     for s in range(args.warmup):
         flush.zero_()
         step(s)
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    # clocks are sampled (every 100 ms) over a soak of the same steps that runs right
+    # before the timed region and over the timed region itself
     clocks = Clocks(local)
     clocks.start()
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak_s:
+        for s in range(args.warmup):
+            flush.zero_()
+            step(s, record=False)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
     torch.cuda.synchronize(dev)
     wall0 = time.perf_counter()
     for s in range(args.warmup, total):
@@ -269,9 +302,12 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
     ck = clocks.stop()
+    if ck is not None:
+        ck["sampled_over"] = f"{args.soak_s:.1f} s soak of the same steps + the timed region"
     step_ms = [ev[s][0].elapsed_time(ev[s][5]) for s in range(args.warmup, total)]
     gu_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.warmup, total)]
     dn_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(args.warmup, total)]
+    cb_ms = [ev[s][3].elapsed_time(ev[s][4]) for s in range(args.warmup, total)]
     rt_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.warmup, total)]
     my_ms = float(sum(step_ms))
     t = torch.tensor([my_ms], dtype=torch.float64, device=dev)
@@ -333,7 +369,7 @@ def run_ours(args, cfg):
 
     line = None
     if rank == 0:
-        launches_per_step = (1 if T <= 64 else 3) + 2
+        launches_per_step = (1 if T <= 64 else 4) + 3     # route kernels + gate/up, down, combine
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -341,7 +377,7 @@ def run_ours(args, cfg):
                 "roofline": roofline,
                 "layer_weight_stream_gbs": layer_gbs,
                 "kernel_us": {"route": 1e3 * float(np.mean(rt_ms)), "gate_up": 1e3 * float(np.mean(gu_ms)),
-                              "down_combine": 1e3 * float(np.mean(dn_ms)),
+                              "down": 1e3 * float(np.mean(dn_ms)), "combine": 1e3 * float(np.mean(cb_ms)),
                               "down_gbs": dn_gbs},
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.H * 2,
                         "d2h_bytes_per_step": T * cfg.H * 2},
@@ -350,11 +386,12 @@ def run_ours(args, cfg):
                 "clocks": ck}
         if world == 1 and not args.no_cpu_baseline:
             L0 = synth.Layer(cfg, 0)
-            sample = [xs_host[i][: max(1, min(T, 4))] for i in range(4)]
+            sample = [xs_host[i][: max(1, min(T, 4))] for i in range(min(8, total))]
             v, n, dt, cores = oracle_tokens_per_s(cfg, L0, sample, args.cpu_budget, 64)
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                     "sample": f"{n} token(s) of this workload ({dt:.1f} s), routed and run "
-                                              f"through every selected expert and the shared expert in fp64"}
+                                              f"through every selected expert and the shared expert in fp64 "
+                                              f"(expert weights drawn before timing)"}
         print(json.dumps(line), flush=True)
     for lay in layers:
         del lay
@@ -372,6 +409,7 @@ def main():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--soak-s", type=float, default=1.5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
