@@ -178,7 +178,12 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     if (events)
         for (int i = 0; i < 4; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
     if (ev[0] && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
-    cudaError_t err = launch_ffn_decode(a, s, ev[1], ev[2]);
+    // The prefill kernels tile the gate/up rows and the hidden rows by 128.
+    const bool tc_ok = a.H % 128 == 0 && (2 * a.I) % 128 == 0;
+    if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
+    const bool prefill = path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kSmallT && tc_ok);
+    cudaError_t err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
+                              : launch_ffn_decode(a, s, ev[1], ev[2]);
     if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
     if (ev[3] && cudaEventRecord(ev[3], s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;

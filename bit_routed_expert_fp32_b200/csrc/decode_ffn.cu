@@ -595,8 +595,12 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_g
     err = launch_mode<1>(a, s);
     if (err != cudaSuccess) return err;
     if (ev_down) cudaEventRecord(ev_down, s);
-    const int n = a.T * (a.H / 8);
-    combine_kernel<<<(n + 255) / 256, 256, 0, s>>>(a);
+    return launch_combine(a, s);
+}
+
+cudaError_t launch_combine(const FfnArgs& a, cudaStream_t s) {
+    const long long n = (long long)a.T * (a.H / 8);
+    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -53,5 +53,10 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // decode-path expert kernels + combine; ev_gateup / ev_down (may be null) are recorded
 // after the gate/up and the down kernel
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down);
+// prefill-path expert kernels (tcgen05) + combine; x16: fp16 scratch of T*(k+S)*H
+cudaError_t launch_ffn_prefill(const FfnArgs& a, uint16_t* x16, cudaStream_t s, cudaEvent_t ev_gateup,
+                               cudaEvent_t ev_down);
+// gate-weighted unpermute-combine of the partial rows into y
+cudaError_t launch_combine(const FfnArgs& a, cudaStream_t s);
 
 }  // namespace moe

@@ -1,0 +1,531 @@
+// Prefill path (steps a6, a7, a8): grouped GEMMs over the packed experts on the
+// 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
+//
+// With thousands of tokens each selected expert meets hundreds of tokens, so its
+// FFN is a dense contraction and belongs on the tensor cores.  The engine on the
+// pages sweeps a long prompt in batches of 6-9K tokens (shadowgraph.io README,
+// paragraph under the model table); here one call takes all T tokens.
+//
+// Orientation ("swap-AB"): D[M = 128 weight rows][N <= 256 tokens] = W_tile x X^T.
+// Weights are the A operand, so every tile has a full M of 128 whatever the token
+// count, and a tile's N is the expert's token count rounded up to 16 (experts with
+// more than 256 tokens are split evenly into several N-tiles).
+//
+//  * Dequantisation producers (warps 0-3, one thread per weight row): per 64-wide
+//    K stage, load the row's 16 bytes of codes (plus 8 bytes of third bits and the
+//    fp16 scale) from the packed format, turn them into fp16 (c - o) * s (exact codes,
+//    one rounding) and write the 128-byte row into the stage's A tile in the
+//    canonical K-major SWIZZLE_128B layout, then fence.proxy.async + arrive.
+//  * TMA producer (warp 8): one 2-D tensor-map load per 64 token rows of the stage's B
+//    tile (K-major, SWIZZLE_128B) from the gathered fp16 token rows (gate/up) or from
+//    h (down), completion counted in bytes on the stage's mbarrier.
+//  * MMA issuer (warp 9, one thread): per stage four tcgen05.mma.kind::f16 (K = 16
+//    each), fp32 accumulation in TMEM; tcgen05.commit releases the stage to the
+//    producers and, after the last stage, hands the accumulator to the epilogue.
+//    Two accumulators of 256 TMEM columns alternate between tiles, so the epilogue
+//    of one tile overlaps the main loop of the next.
+//  * Epilogue (warps 4-7, TMEM lanes 32q..32q+31): tcgen05.ld 16 columns at a time.
+//    gate/up: rows 16b..16b+7 are gate rows and 16b+8..16b+15 the matching up rows,
+//    i.e. TMEM lanes l and l+8 of the same warp: h = silu(gate) * up is formed with
+//    one shuffle and stored as fp16.  down: fp32 partial rows per (token, slot) for
+//    the deterministic combine kernel.
+// Every wait is bounded (an error is recorded and the kernel carries on), and TMEM is
+// released on every exit path.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;                       // weight rows per tile (UMMA M)
+constexpr int BN = 256;                       // max tokens per tile (UMMA N)
+constexpr int BK = 64;                        // K per stage (one scale group)
+constexpr int NSTG = 4;                       // pipeline stages
+constexpr int A_BYTES = BM * BK * 2;          // 16 KB
+constexpr int B_BYTES = BN * BK * 2;          // 32 KB
+constexpr int STG_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int BOX_ROWS = 64;                  // token rows per TMA load
+constexpr int kThreads = 320;                 // 10 warps
+constexpr int kDqWarps = 4, kTmaWarp = 8, kMmaWarp = 9;   // warps 4-7: epilogue
+constexpr long long kWaitLimit = 4000000000LL;
+
+constexpr uint32_t kH512 = 0x60006000u, kH256 = 0x5C005C00u, kH64 = 0x54005400u, kH16 = 0x4C004C00u,
+                   kH4 = 0x44004400u, kH4096 = 0x6C006C00u, kH2048 = 0x68006800u, kH1024 = 0x64006400u,
+                   kH128 = 0x58005800u, kH32 = 0x50005000u;
+
+// fp16 pairs (c - o), exact (bases 512, 256, 64, 16, 4 have an ulp <= 1/2).
+__device__ inline void codes_f16(uint32_t w, const uint32_t (&sub)[5], uint32_t (&pr)[8]) {
+    const uint32_t w1 = w << 1, w8 = w >> 8;
+    pr[0] = f16x2_sub(lop3_and_or(w1, 0x00060006u, kH512), sub[0]);
+    pr[1] = f16x2_sub(lop3_and_or(w, 0x000C000Cu, kH256), sub[1]);
+    pr[2] = f16x2_sub(lop3_and_or(w, 0x00300030u, kH64), sub[2]);
+    pr[3] = f16x2_sub(lop3_and_or(w, 0x00C000C0u, kH16), sub[3]);
+    pr[4] = f16x2_sub(lop3_and_or(w, 0x03000300u, kH4), sub[4]);
+    pr[5] = f16x2_sub(lop3_and_or(w8, 0x000C000Cu, kH256), sub[1]);
+    pr[6] = f16x2_sub(lop3_and_or(w8, 0x00300030u, kH64), sub[2]);
+    pr[7] = f16x2_sub(lop3_and_or(w8, 0x00C000C0u, kH16), sub[3]);
+}
+
+// fp16 pairs 4 * (third bit), exact, for bits 0..7 of each half of u.
+__device__ inline void hi_f16(uint32_t u, uint32_t (&pr)[8]) {
+    pr[0] = f16x2_sub(lop3_and_or(u, 0x00010001u, kH4096), kH4096);
+    pr[1] = f16x2_sub(lop3_and_or(u, 0x00020002u, kH2048), kH2048);
+    pr[2] = f16x2_sub(lop3_and_or(u, 0x00040004u, kH1024), kH1024);
+    pr[3] = f16x2_sub(lop3_and_or(u, 0x00080008u, kH512), kH512);
+    pr[4] = f16x2_sub(lop3_and_or(u, 0x00100010u, kH256), kH256);
+    pr[5] = f16x2_sub(lop3_and_or(u, 0x00200020u, kH128), kH128);
+    pr[6] = f16x2_sub(lop3_and_or(u, 0x00400040u, kH64), kH64);
+    pr[7] = f16x2_sub(lop3_and_or(u, 0x00800080u, kH32), kH32);
+}
+
+__device__ inline uint32_t f16x2_add(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ inline uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// ---- tcgen05 / TMA wrappers ---------------------------------------------------------
+__device__ inline void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ inline void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ inline void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ inline void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// SWIZZLE_128B K-major shared-memory matrix descriptor: 8-row groups 1024 bytes apart.
+__device__ inline uint64_t smem_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// kind::f16 instruction descriptor: fp16 A and B (K-major), fp32 D, M = 128, N.
+__device__ inline uint32_t instr_desc(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ inline void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ inline void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ inline void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ inline void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ inline void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ inline const PackedEntry* entry(const uint8_t* packed, int e) {
+    return reinterpret_cast<const PackedEntry*>(packed + kHeaderBytes + (size_t)e * kEntryBytes);
+}
+
+struct TcSched {
+    int ok, n_active, n_tiles, abort_flag;
+    uint32_t tmem;
+    int pad[3];
+    int e[260];
+    int fmt[260];
+    int cnt[260];
+    int nt[260];     // N-tiles per active expert
+    int nb[260];     // tokens per N-tile (multiple of 16, <= 256)
+    int tpre[261];   // tile prefix over active experts
+};
+
+struct TileInfo {
+    int a, e, f, mt, n0, N, row0;   // N: tokens in this tile; row0: first permuted row
+};
+
+__device__ inline int ld_volatile(const int& v) { return *reinterpret_cast<const volatile int*>(&v); }
+__device__ inline void st_volatile(int& v, int x) { *reinterpret_cast<volatile int*>(&v) = x; }
+
+__device__ inline TileInfo tile_info(const TcSched& S, const FfnArgs& p, int tile, int mtiles) {
+    int lo = 0, hi = S.n_active - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (S.tpre[mid] <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    TileInfo ti;
+    ti.a = lo;
+    ti.e = S.e[lo];
+    ti.f = S.fmt[lo];
+    const int r = tile - S.tpre[lo];
+    const int ntile = r / mtiles;
+    ti.mt = r - ntile * mtiles;
+    ti.n0 = ntile * S.nb[lo];
+    ti.N = min(S.nb[lo], S.cnt[lo] - ti.n0);
+    ti.row0 = (ti.e < p.E ? p.offsets[ti.e] : p.T * p.k + (ti.e - p.E) * p.T) + ti.n0;
+    return ti;
+}
+
+__device__ bool wait_or_flag(TcSched& S, uint64_t* bar, uint32_t parity, const FfnArgs& p, uint32_t detail) {
+    if (ld_volatile(S.abort_flag)) return false;
+    if (mbar_wait_bounded(bar, parity, kWaitLimit)) return true;
+    st_volatile(S.abort_flag, 1);
+    report_error(p.ctrl, MOE_ERR_TIMEOUT, detail);
+    return false;
+}
+
+template <int MODE>   // 0: gate/up (B = gathered tokens, K = H); 1: down (B = h, K = I)
+__global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const __grid_constant__ CUtensorMap bmap) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ TcSched S;
+    __shared__ __align__(8) uint64_t full_a[NSTG], full_b[NSTG], empty_[NSTG], acc_full[2], acc_empty[2], mma_done;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int K = MODE == 0 ? p.H : p.I;
+    const int M_total = MODE == 0 ? 2 * p.I : p.H;
+    const int mtiles = M_total / BM;
+    const int KS = K / BK;                 // K stages per tile
+    const int G = K / 64, NC = (G + 7) / 8;
+
+    if (threadIdx.x == 0) {
+        const uint32_t* hd = reinterpret_cast<const uint32_t*>(p.packed);
+        const bool ok = hd[0] == kMagic && hd[1] == kVersion && (int)hd[2] == p.H && (int)hd[3] == p.I &&
+                        (int)hd[4] == p.E && (int)hd[5] == p.S && hd[6] == 64u && hd[7] == (uint32_t)kInterleave;
+        S.ok = ok;
+        S.abort_flag = 0;
+        if (!ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
+        S.n_active = p.ctrl->n_active;
+    }
+    __syncthreads();
+    if (!S.ok) return;
+    const int nA = S.n_active;
+    for (int a = threadIdx.x; a < nA; a += blockDim.x) {
+        const int e = p.active[a];
+        const int c = e < p.E ? p.counts[e] : p.T;
+        const int nt = (c + BN - 1) / BN;
+        int nb = (c + nt - 1) / nt;
+        nb = (nb + 15) & ~15;
+        S.e[a] = e;
+        S.fmt[a] = (int)entry(p.packed, e)->fmt;
+        S.cnt[a] = c;
+        S.nt[a] = nt;
+        S.nb[a] = nb;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int a = 0; a < nA; ++a) {
+            S.tpre[a] = run;
+            run += S.nt[a] * mtiles;
+        }
+        S.tpre[nA] = run;
+        S.n_tiles = run;
+        for (int i = 0; i < NSTG; ++i) {
+            mbar_init(&full_a[i], kDqWarps * 32);
+            mbar_init(&full_b[i], 1);
+            mbar_init(&empty_[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4 * 32);
+        }
+        mbar_init(&mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) tmem_alloc(&S.tmem, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem;
+    const int n_tiles = S.n_tiles;
+
+    if (warp < kDqWarps) {
+        // ======================= dequantisation producers (A) =======================
+        // One thread per weight row; the packed words of the next PF groups are kept in
+        // flight in registers while the current group is converted.
+        constexpr int PF = 4;
+        const int i = threadIdx.x;           // row within the tile
+        const int r16 = i & 15, rs = r16 & 7;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const TileInfo ti = tile_info(S, p, tile, mtiles);
+            const PackedEntry* en = entry(p.packed, ti.e);
+            const int row = ti.mt * BM + i;
+            const int j16 = row >> 4;
+            const uint8_t* cbase = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes) + (size_t)4 * K * j16;
+            const uint8_t* hbase = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi) + (size_t)128 * G * j16;
+            const uint8_t* sbase = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales) + (size_t)256 * NC * j16;
+            const bool q3 = ti.f == MOE_FMT_Q3;
+            const float o = ti.f == MOE_FMT_TERNARY ? 1.f : (ti.f == MOE_FMT_Q2 ? 1.5f : 3.5f);
+            uint32_t sub[5];
+            sub[0] = f16x2_bits_of(512.f + o);
+            sub[1] = f16x2_bits_of(256.f + o);
+            sub[2] = f16x2_bits_of(64.f + o);
+            sub[3] = f16x2_bits_of(16.f + o);
+            sub[4] = f16x2_bits_of(4.f + o);
+            // packed words of group ks of this row (codes contiguous in the swizzled block)
+            auto fetch = [&](int ks, uint4& cw, uint2& hw, uint32_t& sc) {
+                const int c = ks >> 3, gl = ks & 7;
+                const int ng = min(8, G - 8 * c);
+                const int wpos = ng == 8 ? r16 * 32 + 4 * (gl ^ rs) : r16 * 4 * ng + 4 * gl;
+                cw = __ldg(reinterpret_cast<const uint4*>(cbase + 2048 * (size_t)c) + wpos / 4);
+                sc = __ldg(reinterpret_cast<const uint16_t*>(sbase + 256 * (size_t)c) + r16 * 8 + gl);
+                hw = make_uint2(0, 0);
+                if (q3) {
+                    const int hpos = ng == 8 ? r16 * 16 + 2 * (gl ^ (rs >> 1)) : r16 * 2 * ng + 2 * gl;
+                    hw = __ldg(reinterpret_cast<const uint2*>(hbase + 1024 * (size_t)c) + hpos / 2);
+                }
+            };
+            uint4 pc[PF];
+            uint2 ph[PF];
+            uint32_t psc[PF];
+#pragma unroll
+            for (int u = 0; u < PF; ++u)
+                if (u < KS) fetch(u, pc[u], ph[u], psc[u]);
+            for (int ks0 = 0; ks0 < KS; ks0 += PF) {
+#pragma unroll
+                for (int u = 0; u < PF; ++u) {
+                    const int ks = ks0 + u;
+                    if (ks >= KS) break;
+                    const uint4 cw = pc[u];
+                    const uint2 hw = ph[u];
+                    const uint32_t s2 = psc[u] * 0x10001u;
+                    if (ks + PF < KS) fetch(ks + PF, pc[u], ph[u], psc[u]);
+                    const int slot = it & (NSTG - 1);
+                    wait_or_flag(S, &empty_[slot], ((it / NSTG) & 1) ^ 1, p, kDetWaitEmpty | 0x10 | MODE);
+                    uint8_t* arow = smem + (size_t)slot * STG_BYTES + (i >> 3) * 1024 + (i & 7) * 128;
+                    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t pr[8];
+                        codes_f16(words[q], sub, pr);
+                        if (q3) {
+                            uint32_t hp[8];
+                            hi_f16(((q < 2) ? hw.x : hw.y) >> (8 * (q & 1)), hp);
+#pragma unroll
+                            for (int v = 0; v < 8; ++v) pr[v] = f16x2_add(pr[v], hp[v]);
+                        }
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) pr[v] = f16x2_mul(pr[v], s2);
+                        // elements 16q..16q+7 -> 16-byte chunk 2q, 16q+8..16q+15 -> chunk 2q+1
+                        const int c0 = (2 * q) ^ (i & 7), c1 = (2 * q + 1) ^ (i & 7);
+                        *reinterpret_cast<uint4*>(arow + c0 * 16) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+                        *reinterpret_cast<uint4*>(arow + c1 * 16) = make_uint4(pr[4], pr[5], pr[6], pr[7]);
+                    }
+                    fence_proxy_async();
+                    mbar_arrive(&full_a[slot]);
+                    ++it;
+                }
+            }
+        }
+    } else if (warp == kTmaWarp) {
+        // ============================ TMA producer (B) ===============================
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+                const TileInfo ti = tile_info(S, p, tile, mtiles);
+                const int nbox = (ti.N + BOX_ROWS - 1) / BOX_ROWS;
+                for (int ks = 0; ks < KS; ++ks, ++it) {
+                    const int slot = it & (NSTG - 1);
+                    wait_or_flag(S, &empty_[slot], ((it / NSTG) & 1) ^ 1, p, kDetWaitEmpty | 0x20 | MODE);
+                    if (ld_volatile(S.abort_flag)) continue;
+                    uint8_t* bdst = smem + (size_t)slot * STG_BYTES + A_BYTES;
+                    mbar_arrive_expect_tx(&full_b[slot], nbox * BOX_ROWS * BK * 2);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(bdst + b * BOX_ROWS * BK * 2, &bmap, ks * BK, ti.row0 + b * BOX_ROWS, &full_b[slot]);
+                }
+            }
+            // no TMA write may still target shared memory at exit (matters only after an
+            // abort: normally the MMA issuer has consumed every stage)
+            if (ld_volatile(S.abort_flag))
+                for (int d = 0; d < NSTG && d < it; ++d) {
+                    const int q2 = it - 1 - d;
+                    if (!mbar_wait_bounded(&full_b[q2 & (NSTG - 1)], (q2 / NSTG) & 1, kWaitLimit)) {
+                        report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | MODE);
+                        break;
+                    }
+                }
+        }
+    } else if (warp == kMmaWarp) {
+        // ============================== MMA issuer ===================================
+        if (lane == 0) {
+            int it = 0, tc = 0;
+            for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
+                const TileInfo ti = tile_info(S, p, tile, mtiles);
+                const int buf = tc & 1;
+                const int n16 = (ti.N + 15) & ~15;
+                const uint32_t idesc = instr_desc(n16);
+                wait_or_flag(S, &acc_empty[buf], ((tc >> 1) & 1) ^ 1, p, kDetWaitEmpty | 0x30 | MODE);
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * BN;
+                for (int ks = 0; ks < KS; ++ks, ++it) {
+                    const int slot = it & (NSTG - 1);
+                    const uint32_t par = (it / NSTG) & 1;
+                    const bool ok_a = wait_or_flag(S, &full_a[slot], par, p, kDetWaitFull | 0x10 | MODE);
+                    const bool ok_b = wait_or_flag(S, &full_b[slot], par, p, kDetWaitFull | 0x20 | MODE);
+                    tc_fence_after();
+                    if (ok_a && ok_b) {
+                        const uint32_t a0 = smem_u32(smem + (size_t)slot * STG_BYTES);
+                        const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                        for (int k16 = 0; k16 < BK / 16; ++k16)
+                            umma_f16(d_tmem, smem_desc(a0 + 32 * k16), smem_desc(b0 + 32 * k16), idesc,
+                                     (ks > 0 || k16 > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty_[slot]);
+                }
+                umma_commit(&acc_full[buf]);
+            }
+            // every MMA this thread issued has completed once this commit arrives
+            umma_commit(&mma_done);
+            if (!mbar_wait_bounded(&mma_done, 0, kWaitLimit)) report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | 0x40);
+        }
+    } else {
+        // =============================== epilogue ====================================
+        const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
+            const TileInfo ti = tile_info(S, p, tile, mtiles);
+            const int buf = tc & 1;
+            wait_or_flag(S, &acc_full[buf], (tc >> 1) & 1, p, kDetWaitFull | 0x30 | MODE);
+            tc_fence_after();
+            const uint32_t tbase = tmem + buf * BN + ((uint32_t)(32 * q) << 16);
+            const int mrow = ti.mt * BM + 32 * q + lane;    // row of the packed matrix
+            for (int c0 = 0; c0 < ti.N; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tbase + c0, v);
+                if (MODE == 0) {
+                    const bool gate_lane = (lane & 15) < 8;
+                    const int hcol = (mrow >> 4) * 8 + (lane & 7);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const float a = __uint_as_float(v[u]);
+                        const float b = __shfl_down_sync(0xffffffffu, a, 8);
+                        if (gate_lane && c0 + u < ti.N)
+                            p.h[(size_t)(ti.row0 + c0 + u) * p.I + hcol] = f32_to_f16_bits(silu_f(a) * b);
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        if (c0 + u < ti.N) p.ypart[(size_t)(ti.row0 + c0 + u) * p.H + mrow] = __uint_as_float(v[u]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[buf]);
+        }
+    }
+    // all roles are done (waits are bounded): make sure no MMA is still writing, then
+    // release the tensor memory
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// X16[r][:] = fp16(x[token of permuted row r][:]); rows T*k .. are the shared expert's.
+__global__ void __launch_bounds__(256) gather_x16_kernel(FfnArgs p, uint16_t* x16) {
+    const int per_row = p.H / 8;
+    const long long rows = (long long)p.T * (p.k + p.S);
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * per_row) return;
+    const long long r = idx / per_row;
+    const int c8 = (int)(idx - r * per_row) * 8;
+    const int tok = r < (long long)p.T * p.k ? p.perm[r] / p.k : (int)((r - (long long)p.T * p.k) % p.T);
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)tok * p.H + c8));
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const float lo = __uint_as_float(in[u] << 16), hi = __uint_as_float(in[u] & 0xFFFF0000u);
+        out[u] = (uint32_t)f32_to_f16_bits(lo) | ((uint32_t)f32_to_f16_bits(hi) << 16);
+    }
+    *reinterpret_cast<uint4*>(x16 + (size_t)r * p.H + c8) = make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// 2-D fp16 tensor map over rows x K (K-major), 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int K) {
+    auto enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {BK, BOX_ROWS};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kTcSmem = (size_t)NSTG * STG_BYTES + 1024;
+
+template <int MODE>
+cudaError_t launch_tc(const FfnArgs& a, const CUtensorMap& map, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t err =
+            cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+        if (err != cudaSuccess) return err;
+        attr = true;
+    }
+    tc_gemm_kernel<MODE><<<a.num_ctas, kThreads, kTcSmem, s>>>(a, map);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_prefill(const FfnArgs& a, uint16_t* x16, cudaStream_t s, cudaEvent_t ev_gateup,
+                               cudaEvent_t ev_down) {
+    if ((2 * a.I) % BM != 0 || a.H % BM != 0) return cudaErrorInvalidConfiguration;
+    const long long rows = (long long)a.T * (a.k + a.S);
+    const long long n8 = rows * (a.H / 8);
+    gather_x16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a, x16);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    CUtensorMap mx, mh;
+    if (!make_map(&mx, x16, rows, a.H) || !make_map(&mh, a.h, rows, a.I)) return cudaErrorInvalidConfiguration;
+    err = launch_tc<0>(a, mx, s);
+    if (err != cudaSuccess) return err;
+    if (ev_gateup) cudaEventRecord(ev_gateup, s);
+    err = launch_tc<1>(a, mh, s);
+    if (err != cudaSuccess) return err;
+    if (ev_down) cudaEventRecord(ev_down, s);
+    return launch_combine(a, s);
+}
+
+}  // namespace moe
