@@ -410,11 +410,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--soak-s", type=float, default=1.5)
+    ap.add_argument("--tokens", type=int, default=0, help="override the workload's tokens per step (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = synth.CONFIGS[args.config]
+    if args.tokens:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

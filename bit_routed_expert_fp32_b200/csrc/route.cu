@@ -10,8 +10,9 @@
 // Decode (T <= 64): one launch.  E/2 CTAs stream the 7.3 MB fp32 router (four warps
 // per expert row), compute the Z tables of the gate/up dequantiser, and the last
 // CTA to finish (atomic ticket) does top-k, histogram, scan and permutation.
-// Prefill: a tiled fp32 GEMM for the logits, a top-k kernel whose last CTA scans the
-// per-chunk histograms, and a scatter kernel that writes perm/inv_perm per chunk.
+// Prefill: a tensor-core logits GEMM (fp32 router split exactly into three bf16
+// pieces), a top-k kernel whose last CTA scans the per-chunk histograms, and a
+// scatter kernel that writes perm/inv_perm per chunk.
 // Ordering inside an expert is token ascending, made deterministic by processing the
 // flattened (token, slot) pairs in order with warp match/ballot ranks.
 #include "kernels.h"
@@ -280,75 +281,151 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
 }
 
 // ---------------------------------------------------------------- prefill router
-constexpr int GBM = 64, GBN = 64, GBK = 32;
+// Router logits for many tokens on the tensor cores.  x is bf16 (exact); the fp32
+// router weight is split exactly into three bf16 pieces w = w1 + w2 + w3 (each the
+// bf16 rounding of what is left), so x.w1 + x.w2 + x.w3 with fp32 accumulation gives
+// fp32-level logits (the dropped remainder is below 2^-24 |w|).  mma.sync m16n8k16,
+// CTA tile 128 tokens x 64 experts x 32 K, 8 warps of 32 x 32, double-buffered smem.
+constexpr int RBM = 128, RBN = 64, RBK = 32, RPAD = 40;   // smem row: 32 bf16 + 8 pad
 
-__global__ void __launch_bounds__(256) route_logits_gemm_kernel(RouteArgs p) {
-    __shared__ float xs[GBK][GBM + 4];
-    __shared__ float ws[GBK][GBN + 4];
-    const int tid = threadIdx.x;
-    const int t0 = blockIdx.x * GBM, e0 = blockIdx.y * GBN;
-    const int ty = tid >> 4, tx = tid & 15;
-    float acc[4][4] = {};
-    const int lr = tid >> 2, lc = (tid & 3) * 8;
-    for (int h0 = 0; h0 < p.H; h0 += GBK) {
-        {
-            int t = t0 + lr;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (t < p.T) v = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + h0 + lc));
-            xs[lc + 0][lr] = bf16lo(v.x);
-            xs[lc + 1][lr] = bf16hi(v.x);
-            xs[lc + 2][lr] = bf16lo(v.y);
-            xs[lc + 3][lr] = bf16hi(v.y);
-            xs[lc + 4][lr] = bf16lo(v.z);
-            xs[lc + 5][lr] = bf16hi(v.z);
-            xs[lc + 6][lr] = bf16lo(v.w);
-            xs[lc + 7][lr] = bf16hi(v.w);
-            int e = e0 + lr;
-            float4 a = make_float4(0, 0, 0, 0), b = a;
-            if (e < p.E) {
-                const float4* src = reinterpret_cast<const float4*>(p.Wr + (size_t)e * p.H + h0 + lc);
-                a = __ldg(src);
-                b = __ldg(src + 1);
+__device__ inline uint32_t pack_bf16x2(float lo, float hi) {
+    return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+}
+
+__device__ inline void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+constexpr size_t kRouteMmaSmem = (size_t)2 * RBM * RPAD * 2 + (size_t)2 * 3 * RBN * RPAD * 2;   // 51,200 B
+
+__global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
+    extern __shared__ __align__(16) uint8_t rsm[];
+    auto xs = reinterpret_cast<uint16_t(*)[RBM][RPAD]>(rsm);
+    auto ws = reinterpret_cast<uint16_t(*)[3][RBN][RPAD]>(rsm + (size_t)2 * RBM * RPAD * 2);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = blockIdx.x * RBM, e0 = blockIdx.y * RBN;
+    const int wm = warp >> 1, wn = warp & 1;            // warp tile: tokens 32wm.., experts 32wn..
+    float acc[2][4][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = acc[a][b][2] = acc[a][b][3] = 0.f;
+
+    // loaders: x tile 128 x 32 bf16 = 512 x 16 B (2 per thread); w tile 64 x 32 fp32 (8 floats per thread)
+    uint4 xr[2];
+    float4 wr[2];
+    auto load = [&](int h0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int idx = tid + 256 * u, row = idx >> 2, c = (idx & 3) * 8;
+            const int t = t0 + row;
+            xr[u] = t < p.T ? __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + h0 + c))
+                            : make_uint4(0, 0, 0, 0);
+        }
+        const int row = tid >> 2, c = (tid & 3) * 8, e = e0 + row;
+        if (e < p.E) {
+            const float4* src = reinterpret_cast<const float4*>(p.Wr + (size_t)e * p.H + h0 + c);
+            wr[0] = __ldg(src);
+            wr[1] = __ldg(src + 1);
+        } else {
+            wr[0] = wr[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int idx = tid + 256 * u, row = idx >> 2, c = (idx & 3) * 8;
+            *reinterpret_cast<uint4*>(&xs[buf][row][c]) = xr[u];
+        }
+        const int row = tid >> 2, c = (tid & 3) * 8;
+        const float w[8] = {wr[0].x, wr[0].y, wr[0].z, wr[0].w, wr[1].x, wr[1].y, wr[1].z, wr[1].w};
+        float r1[8], r2[8], r3[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            r1[v] = __uint_as_float((uint32_t)f32_to_bf16_bits(w[v]) << 16);
+            const float rem = w[v] - r1[v];
+            r2[v] = __uint_as_float((uint32_t)f32_to_bf16_bits(rem) << 16);
+            r3[v] = rem - r2[v];
+        }
+        *reinterpret_cast<uint4*>(&ws[buf][0][row][c]) =
+            make_uint4(pack_bf16x2(r1[0], r1[1]), pack_bf16x2(r1[2], r1[3]), pack_bf16x2(r1[4], r1[5]),
+                       pack_bf16x2(r1[6], r1[7]));
+        *reinterpret_cast<uint4*>(&ws[buf][1][row][c]) =
+            make_uint4(pack_bf16x2(r2[0], r2[1]), pack_bf16x2(r2[2], r2[3]), pack_bf16x2(r2[4], r2[5]),
+                       pack_bf16x2(r2[6], r2[7]));
+        *reinterpret_cast<uint4*>(&ws[buf][2][row][c]) =
+            make_uint4(pack_bf16x2(r3[0], r3[1]), pack_bf16x2(r3[2], r3[3]), pack_bf16x2(r3[4], r3[5]),
+                       pack_bf16x2(r3[6], r3[7]));
+    };
+
+    const int nk = p.H / RBK;
+    load(0);
+    store(0);
+    __syncthreads();
+    for (int kt = 0; kt < nk; ++kt) {
+        const int buf = kt & 1;
+        if (kt + 1 < nk) load((kt + 1) * RBK);
+        // The MMA rounds its fp32 accumulator towards zero; chaining all of K through it
+        // would let that bias grow with H.  Each 32-wide K tile is therefore summed in a
+        // fresh accumulator and added to the total with round-to-nearest adds.
+        float part[2][4][4];
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) part[a][b][0] = part[a][b][1] = part[a][b][2] = part[a][b][3] = 0.f;
+#pragma unroll
+        for (int k16 = 0; k16 < RBK; k16 += 16) {
+            uint32_t af[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                // A 16x16 (tokens x k): lanes 0-15 rows 0-15 at k, lanes 16-31 rows 0-15 at k+8
+                const int r = 32 * wm + 16 * mt + (lane & 15), cc = k16 + 8 * (lane >> 4);
+                ldsm_x4(smem_u32(&xs[buf][r][cc]), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
             }
-            ws[lc + 0][lr] = a.x;
-            ws[lc + 1][lr] = a.y;
-            ws[lc + 2][lr] = a.z;
-            ws[lc + 3][lr] = a.w;
-            ws[lc + 4][lr] = b.x;
-            ws[lc + 5][lr] = b.y;
-            ws[lc + 6][lr] = b.z;
-            ws[lc + 7][lr] = b.w;
-        }
-        __syncthreads();
-        // two-level sum: each 32-wide K slice is summed on its own, then added to the
-        // running total, so rounding grows with H/32 additions rather than H
-        float part[4][4] = {};
-#pragma unroll 8
-        for (int kk = 0; kk < GBK; ++kk) {
-            float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-            float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-            float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int pl = 0; pl < 3; ++pl) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
+                for (int np = 0; np < 2; ++np) {
+                    // two n8 tiles of B (experts x k): matrices (n 0-7, k), (n 0-7, k+8), (n 8-15, k), (n 8-15, k+8)
+                    const int r = 32 * wn + 16 * np + (lane & 7) + 8 * (lane >> 4), cc = k16 + 8 * ((lane >> 3) & 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(smem_u32(&ws[buf][pl][r][cc]), b0, b1, b2, b3);
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        mma_bf16_16816(part[mt][2 * np][0], part[mt][2 * np][1], part[mt][2 * np][2],
+                                       part[mt][2 * np][3], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b0, b1);
+                        mma_bf16_16816(part[mt][2 * np + 1][0], part[mt][2 * np + 1][1], part[mt][2 * np + 1][2],
+                                       part[mt][2 * np + 1][3], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b2, b3);
+                    }
+                }
+            }
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[a][b][c] += part[a][b][c];
+        if (kt + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
+    const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        int t = t0 + ty * 4 + i;
-        if (t >= p.T) continue;
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int e = e0 + tx * 4 + j;
-            if (e < p.E) p.logits[(size_t)t * p.E + e] = acc[i][j] + (p.bias ? p.bias[e] : 0.f);
-        }
-    }
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int t = t0 + 32 * wm + 16 * mt + g + 8 * h;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int e = e0 + 32 * wn + 8 * nt + 2 * t4 + c;
+                    if (t < p.T && e < p.E)
+                        p.logits[(size_t)t * p.E + e] = acc[mt][nt][2 * h + c] + (p.bias ? p.bias[e] : 0.f);
+                }
+            }
 }
 
 __global__ void __launch_bounds__(256) route_topk_kernel(RouteArgs p) {
@@ -420,8 +497,15 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     }
     const int zwarps = a.T * (a.H / 64);
     route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
-    dim3 g1((a.T + GBM - 1) / GBM, (a.E + GBN - 1) / GBN);
-    route_logits_gemm_kernel<<<g1, 256, 0, s>>>(a);
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t err = cudaFuncSetAttribute(route_logits_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)kRouteMmaSmem);
+        if (err != cudaSuccess) return err;
+        attr = true;
+    }
+    dim3 g1((a.T + RBM - 1) / RBM, (a.E + RBN - 1) / RBN);
+    route_logits_mma_kernel<<<g1, 256, kRouteMmaSmem, s>>>(a);
     const int nchunks = (a.T + kChunk - 1) / kChunk;
     route_topk_kernel<<<nchunks, 256, 0, s>>>(a);
     route_scatter_kernel<<<nchunks, 32, 0, s>>>(a);
