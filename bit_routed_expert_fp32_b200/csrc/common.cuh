@@ -86,12 +86,61 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: gives up after `limit` clock cycles and returns false.
+// Bounded wait: gives up after `limit` clock cycles and returns false.  The clock is
+// read once per 64 polls so that a waiting warp issues few instructions.
 __device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
-    long long t0 = clock64();
+    const long long t0 = clock64();
     while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+
+// One lane of a converged warp (elect.sync): issue single-thread async instructions
+// (bulk copies, tensor-map loads, tcgen05.mma) from warp-uniform code under this
+// predicate, so their operands stay warp-uniform.
+__device__ inline bool elect_one() {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(r));
+    return r != 0;
+}
+
+// Bounded wait with a sleep of about `ns` nanoseconds between polls, for long waits
+// where a little wake-up latency costs nothing.
+__device__ inline bool mbar_wait_bounded_backoff(uint64_t* bar, uint32_t parity, long long limit, uint32_t ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(ns);
         if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+
+// try_wait with a suspend-time hint: a thread whose phase has not completed is
+// suspended (it issues nothing) until the phase completes or about `ns` nanoseconds
+// have passed.
+__device__ inline bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, "
+        "p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait that leaves the issue slots to the working warps while it waits: the
+// thread sleeps in the barrier between checks of the clock.
+__device__ inline bool mbar_wait_bounded_suspend(uint64_t* bar, uint32_t parity, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
         if (clock64() - t0 > limit) return false;
     }
 }
@@ -104,6 +153,11 @@ __device__ inline void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t b
             smem_u32(dst_smem)),
         "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned address and size).
+__device__ inline void bulk_prefetch_l2(const void* src_gmem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes) : "memory");
 }
 
 __device__ inline void bulk_g2s_evict_first(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar,

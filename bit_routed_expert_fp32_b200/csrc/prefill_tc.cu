@@ -11,20 +11,24 @@
 // count, and a tile's N is the expert's token count rounded up to 16 (experts with
 // more than 256 tokens are split evenly into several N-tiles).
 //
-//  * Dequantisation producers (warps 0-3, one thread per weight row): per 64-wide
-//    K stage, load the row's 16 bytes of codes (plus 8 bytes of third bits and the
-//    fp16 scale) from the packed format, turn them into fp16 (c - o) * s (exact codes,
-//    one rounding) and write the 128-byte row into the stage's A tile in the
-//    canonical K-major SWIZZLE_128B layout, then fence.proxy.async + arrive.
-//  * TMA producer (warp 8): one 2-D tensor-map load per 64 token rows of the stage's B
-//    tile (K-major, SWIZZLE_128B) from the gathered fp16 token rows (gate/up) or from
-//    h (down), completion counted in bytes on the stage's mbarrier.
-//  * MMA issuer (warp 9, one thread): per stage four tcgen05.mma.kind::f16 (K = 16
+//  * Dequantisation producers (warps 0-7; warp w owns the tile's 16-row block w, two
+//    lanes per row, 32 of the 64 K of a stage each).  Lane 0 of each warp brings its
+//    block's packed data in by bulk copies, one 512-wide K chunk per slot of a
+//    two-slot ring of its own (eight issuing threads keep enough bytes in flight; one
+//    thread alone issues too few copies per microsecond).  The warp reads the row's
+//    code words (plus third bits and the fp16 scale) from the ring, turns them into
+//    fp16 (c - o) * s (exact codes, one rounding) and writes them into the stage's A
+//    tile in the canonical K-major SWIZZLE_128B layout, then fence.proxy.async + one
+//    arrive per warp.
+//  * TMA producer (warp 12): one 2-D tensor-map load per stage for the B tile (K-major,
+//    SWIZZLE_128B) from the gathered fp16 token rows (gate/up) or from h (down),
+//    completion counted in bytes on the stage's mbarrier.
+//  * MMA issuer (warp 13, one thread): per stage four tcgen05.mma.kind::f16 (K = 16
 //    each), fp32 accumulation in TMEM; tcgen05.commit releases the stage to the
 //    producers and, after the last stage, hands the accumulator to the epilogue.
 //    Two accumulators of 256 TMEM columns alternate between tiles, so the epilogue
 //    of one tile overlaps the main loop of the next.
-//  * Epilogue (warps 4-7, TMEM lanes 32q..32q+31): tcgen05.ld 16 columns at a time.
+//  * Epilogue (warps 8-11, TMEM lanes 32q..32q+31): tcgen05.ld 16 columns at a time.
 //    gate/up: rows 16b..16b+7 are gate rows and 16b+8..16b+15 the matching up rows,
 //    i.e. TMEM lanes l and l+8 of the same warp: h = silu(gate) * up is formed with
 //    one shuffle and stored as fp16.  down: fp32 partial rows per (token, slot) for
@@ -42,13 +46,24 @@ namespace {
 constexpr int BM = 128;                       // weight rows per tile (UMMA M)
 constexpr int BN = 256;                       // max tokens per tile (UMMA N)
 constexpr int BK = 64;                        // K per stage (one scale group)
-constexpr int NSTG = 4;                       // pipeline stages
+constexpr int NSTG = 3;                       // A/B pipeline stages
 constexpr int A_BYTES = BM * BK * 2;          // 16 KB
 constexpr int B_BYTES = BN * BK * 2;          // 32 KB
 constexpr int STG_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int BOX_ROWS = 64;                  // token rows per TMA load
-constexpr int kThreads = 320;                 // 10 warps
-constexpr int kDqWarps = 4, kTmaWarp = 8, kMmaWarp = 9;   // warps 4-7: epilogue
+// Per-warp packed ring: each dequantiser warp streams its own 16-row block, one
+// 8-group chunk (codes, third bits, scales of the packed format) per slot.
+constexpr int NP = 2;
+constexpr int PK_CODES = 0, PK_HI = 2048, PK_SC = 3072, PK_BYTES = 3328;
+constexpr int kThreads = 448;                 // 14 warps
+constexpr int kDqWarps = 8, kEpiWarp0 = 8, kTmaWarp = 12, kMmaWarp = 13;   // warps 8-11: epilogue
+
+// B tiles: one tensor-map load per stage, from the map whose box (64, 128 or 256 token
+// rows) is the smallest that covers the tile's tokens.  A single thread issues bulk
+// loads at a limited rate, so one large box beats several small ones.
+struct BMaps {
+    CUtensorMap m[3];   // box rows 64, 128, 256
+};
+__device__ inline int box_index(int n) { return n <= 64 ? 0 : (n <= 128 ? 1 : 2); }
 constexpr long long kWaitLimit = 4000000000LL;
 
 constexpr uint32_t kH512 = 0x60006000u, kH256 = 0x5C005C00u, kH64 = 0x54005400u, kH16 = 0x4C004C00u,
@@ -79,6 +94,10 @@ __device__ inline void hi_f16(uint32_t u, uint32_t (&pr)[8]) {
     pr[6] = f16x2_sub(lop3_and_or(u, 0x00400040u, kH64), kH64);
     pr[7] = f16x2_sub(lop3_and_or(u, 0x00800080u, kH32), kH32);
 }
+
+// silu(a) = a / (1 + e^-a) with the fast exponential and division (relative error
+// ~1e-6, far below the fp16 rounding of h); for a -> -inf the quotient goes to 0.
+__device__ inline float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
 __device__ inline uint32_t f16x2_add(uint32_t a, uint32_t b) {
     uint32_t r;
@@ -192,17 +211,18 @@ __device__ inline TileInfo tile_info(const TcSched& S, const FfnArgs& p, int til
 
 __device__ bool wait_or_flag(TcSched& S, uint64_t* bar, uint32_t parity, const FfnArgs& p, uint32_t detail) {
     if (ld_volatile(S.abort_flag)) return false;
-    if (mbar_wait_bounded(bar, parity, kWaitLimit)) return true;
+    if (mbar_wait_bounded_suspend(bar, parity, kWaitLimit)) return true;
     st_volatile(S.abort_flag, 1);
     report_error(p.ctrl, MOE_ERR_TIMEOUT, detail);
     return false;
 }
 
 template <int MODE>   // 0: gate/up (B = gathered tokens, K = H); 1: down (B = h, K = I)
-__global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const __grid_constant__ CUtensorMap bmap) {
+__global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const __grid_constant__ BMaps bmaps) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ TcSched S;
-    __shared__ __align__(8) uint64_t full_a[NSTG], full_b[NSTG], empty_[NSTG], acc_full[2], acc_empty[2], mma_done;
+    __shared__ __align__(8) uint64_t full_a[NSTG], full_b[NSTG], empty_[NSTG], acc_full[2], acc_empty[2], mma_done,
+        pk_full[kDqWarps][NP];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = MODE == 0 ? p.H : p.I;
@@ -245,10 +265,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         S.tpre[nA] = run;
         S.n_tiles = run;
         for (int i = 0; i < NSTG; ++i) {
-            mbar_init(&full_a[i], kDqWarps * 32);
+            mbar_init(&full_a[i], kDqWarps);                 // one arrive per dequantiser warp
             mbar_init(&full_b[i], 1);
             mbar_init(&empty_[i], 1);
         }
+        for (int w = 0; w < kDqWarps; ++w)
+            for (int i = 0; i < NP; ++i) mbar_init(&pk_full[w][i], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 4 * 32);
@@ -265,20 +287,62 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
 
     if (warp < kDqWarps) {
         // ======================= dequantisation producers (A) =======================
-        // One thread per weight row; the packed words of the next PF groups are kept in
-        // flight in registers while the current group is converted.
-        constexpr int PF = 4;
-        const int i = threadIdx.x;           // row within the tile
-        const int r16 = i & 15, rs = r16 & 7;
-        int it = 0;
+        const int r16 = lane >> 1, hh = lane & 1, rs = r16 & 7;
+        const int i = 16 * warp + r16;                 // row within the tile
+        uint8_t* const ring = smem + (size_t)NSTG * STG_BYTES + (size_t)warp * NP * PK_BYTES;
+        uint64_t* const pfull = pk_full[warp];
+        // Issue cursor (lane 0): the next (tile, chunk) of this warp's block to bring in.
+        struct Cursor {
+            int tile, c;
+            const uint8_t *cb, *hb, *sb;
+            bool q3;
+        } cur{n_tiles, 0, nullptr, nullptr, nullptr, false};
+        auto load_tile = [&](Cursor& u) {
+            if (u.tile >= n_tiles) return;
+            const TileInfo ti = tile_info(S, p, u.tile, mtiles);
+            const PackedEntry* en = entry(p.packed, ti.e);
+            const int j = ti.mt * (BM / 16) + warp;
+            u.cb = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes) + (size_t)4 * K * j;
+            u.hb = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi) + (size_t)128 * G * j;
+            u.sb = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales) + (size_t)256 * NC * j;
+            u.q3 = ti.f == MOE_FMT_Q3;
+        };
+        int issued = 0, consumed = 0;
+        // (whole warp, converged) bring the cursor's chunk into slot issued % NP and
+        // advance the cursor; one elected lane issues the copies
+        auto issue = [&]() {
+            if (cur.tile >= n_tiles) return;
+            const int ps = issued % NP;
+            const int ng = min(8, G - 8 * cur.c);
+            const uint32_t cbytes = 256 * ng, hbytes = cur.q3 ? 128 * ng : 0;
+            uint8_t* dst = ring + (size_t)ps * PK_BYTES;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&pfull[ps], cbytes + hbytes + 256);
+                bulk_g2s(dst + PK_CODES, cur.cb + 2048 * (size_t)cur.c, cbytes, &pfull[ps]);
+                bulk_g2s(dst + PK_SC, cur.sb + 256 * (size_t)cur.c, 256, &pfull[ps]);
+                if (hbytes) bulk_g2s(dst + PK_HI, cur.hb + 1024 * (size_t)cur.c, hbytes, &pfull[ps]);
+            }
+            __syncwarp();
+            ++issued;
+            if (++cur.c == NC) {
+                cur.c = 0;
+                cur.tile += gridDim.x;
+                load_tile(cur);
+            }
+        };
+        cur.tile = blockIdx.x;
+        cur.c = 0;
+        load_tile(cur);
+        for (int d = 0; d < NP; ++d) issue();
+        // A-tile row of this lane and the 16-byte chunks its two quarters land in
+        // (SWIZZLE_128B: chunk index XOR row % 8)
+        const uint32_t arow_off = (i >> 3) * 1024 + (i & 7) * 128;
+        const uint32_t ch[4] = {(uint32_t)(((4 * hh) ^ (i & 7)) * 16), (uint32_t)(((4 * hh + 1) ^ (i & 7)) * 16),
+                                (uint32_t)(((4 * hh + 2) ^ (i & 7)) * 16), (uint32_t)(((4 * hh + 3) ^ (i & 7)) * 16)};
+        int slot = 0;
+        uint32_t eph = 1;                              // parity of the empty phase awaited
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
-            const PackedEntry* en = entry(p.packed, ti.e);
-            const int row = ti.mt * BM + i;
-            const int j16 = row >> 4;
-            const uint8_t* cbase = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes) + (size_t)4 * K * j16;
-            const uint8_t* hbase = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi) + (size_t)128 * G * j16;
-            const uint8_t* sbase = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales) + (size_t)256 * NC * j16;
             const bool q3 = ti.f == MOE_FMT_Q3;
             const float o = ti.f == MOE_FMT_TERNARY ? 1.f : (ti.f == MOE_FMT_Q2 ? 1.5f : 3.5f);
             uint32_t sub[5];
@@ -287,147 +351,215 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
             sub[2] = f16x2_bits_of(64.f + o);
             sub[3] = f16x2_bits_of(16.f + o);
             sub[4] = f16x2_bits_of(4.f + o);
-            // packed words of group ks of this row (codes contiguous in the swizzled block)
-            auto fetch = [&](int ks, uint4& cw, uint2& hw, uint32_t& sc) {
-                const int c = ks >> 3, gl = ks & 7;
+            for (int c = 0; c < NC; ++c) {
+                const int ps = consumed % NP;
                 const int ng = min(8, G - 8 * c);
-                const int wpos = ng == 8 ? r16 * 32 + 4 * (gl ^ rs) : r16 * 4 * ng + 4 * gl;
-                cw = __ldg(reinterpret_cast<const uint4*>(cbase + 2048 * (size_t)c) + wpos / 4);
-                sc = __ldg(reinterpret_cast<const uint16_t*>(sbase + 256 * (size_t)c) + r16 * 8 + gl);
-                hw = make_uint2(0, 0);
-                if (q3) {
-                    const int hpos = ng == 8 ? r16 * 16 + 2 * (gl ^ (rs >> 1)) : r16 * 2 * ng + 2 * gl;
-                    hw = __ldg(reinterpret_cast<const uint2*>(hbase + 1024 * (size_t)c) + hpos / 2);
-                }
-            };
-            uint4 pc[PF];
-            uint2 ph[PF];
-            uint32_t psc[PF];
+                if (lane == 0 && !mbar_try_wait(&pfull[ps], (consumed / NP) & 1))
+                    wait_or_flag(S, &pfull[ps], (consumed / NP) & 1, p, kDetWaitFull | 0x40 | MODE);
+                __syncwarp();
+                const uint8_t* pk = ring + (size_t)ps * PK_BYTES;
+                // this lane's 2 code words, third-bit word and the row's scales of the chunk
+                const uint8_t* cw_base = pk + PK_CODES + (ng == 8 ? r16 * 128 : r16 * 16 * ng) + 8 * hh;
+                const uint8_t* hw_base = pk + PK_HI + (ng == 8 ? r16 * 64 : r16 * 8 * ng) + 4 * hh;
+                const uint16_t* sc_base = reinterpret_cast<const uint16_t*>(pk + PK_SC + r16 * 16);
+                auto load = [&](int gl, uint2& cw, uint32_t& hw, uint32_t& s2) {
+                    const int cpos = ng == 8 ? gl ^ rs : gl;
+                    const int hpos = ng == 8 ? gl ^ (rs >> 1) : gl;
+                    cw = *reinterpret_cast<const uint2*>(cw_base + 16 * cpos);
+                    hw = q3 ? *reinterpret_cast<const uint32_t*>(hw_base + 8 * hpos) : 0u;
+                    s2 = (uint32_t)sc_base[gl] * 0x10001u;
+                };
+                uint2 cw;
+                uint32_t hw, s2;
+                load(0, cw, hw, s2);
+                for (int gl = 0; gl < ng; ++gl) {
+                    // the next group's words are read while this one is converted
+                    uint2 cw_n = cw;
+                    uint32_t hw_n = hw, s2_n = s2;
+                    if (gl + 1 < ng) load(gl + 1, cw_n, hw_n, s2_n);
+                    uint32_t pr[2][8];
+                    const uint32_t words[2] = {cw.x, cw.y};
 #pragma unroll
-            for (int u = 0; u < PF; ++u)
-                if (u < KS) fetch(u, pc[u], ph[u], psc[u]);
-            for (int ks0 = 0; ks0 < KS; ks0 += PF) {
-#pragma unroll
-                for (int u = 0; u < PF; ++u) {
-                    const int ks = ks0 + u;
-                    if (ks >= KS) break;
-                    const uint4 cw = pc[u];
-                    const uint2 hw = ph[u];
-                    const uint32_t s2 = psc[u] * 0x10001u;
-                    if (ks + PF < KS) fetch(ks + PF, pc[u], ph[u], psc[u]);
-                    const int slot = it & (NSTG - 1);
-                    wait_or_flag(S, &empty_[slot], ((it / NSTG) & 1) ^ 1, p, kDetWaitEmpty | 0x10 | MODE);
-                    uint8_t* arow = smem + (size_t)slot * STG_BYTES + (i >> 3) * 1024 + (i & 7) * 128;
-                    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t pr[8];
-                        codes_f16(words[q], sub, pr);
+                    for (int qq = 0; qq < 2; ++qq) {
+                        codes_f16(words[qq], sub, pr[qq]);
                         if (q3) {
                             uint32_t hp[8];
-                            hi_f16(((q < 2) ? hw.x : hw.y) >> (8 * (q & 1)), hp);
+                            hi_f16(hw >> (8 * qq), hp);
 #pragma unroll
-                            for (int v = 0; v < 8; ++v) pr[v] = f16x2_add(pr[v], hp[v]);
+                            for (int v = 0; v < 8; ++v) pr[qq][v] = f16x2_add(pr[qq][v], hp[v]);
                         }
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) pr[v] = f16x2_mul(pr[v], s2);
-                        // elements 16q..16q+7 -> 16-byte chunk 2q, 16q+8..16q+15 -> chunk 2q+1
-                        const int c0 = (2 * q) ^ (i & 7), c1 = (2 * q + 1) ^ (i & 7);
-                        *reinterpret_cast<uint4*>(arow + c0 * 16) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
-                        *reinterpret_cast<uint4*>(arow + c1 * 16) = make_uint4(pr[4], pr[5], pr[6], pr[7]);
+                        for (int v = 0; v < 8; ++v) pr[qq][v] = f16x2_mul(pr[qq][v], s2);
+                    }
+                    // only now wait for the stage's slot
+                    if (lane == 0 && !mbar_try_wait(&empty_[slot], eph))
+                        wait_or_flag(S, &empty_[slot], eph, p, kDetWaitEmpty | 0x10 | MODE);
+                    __syncwarp();
+                    uint8_t* arow = smem + (size_t)slot * STG_BYTES + arow_off;
+                    // quarter q = 2hh + qq: elements 16q..16q+7 -> chunk 2q, 16q+8.. -> 2q+1
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        *reinterpret_cast<uint4*>(arow + ch[2 * qq]) =
+                            make_uint4(pr[qq][0], pr[qq][1], pr[qq][2], pr[qq][3]);
+                        *reinterpret_cast<uint4*>(arow + ch[2 * qq + 1]) =
+                            make_uint4(pr[qq][4], pr[qq][5], pr[qq][6], pr[qq][7]);
                     }
                     fence_proxy_async();
-                    mbar_arrive(&full_a[slot]);
-                    ++it;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full_a[slot]);
+                    if (++slot == NSTG) {
+                        slot = 0;
+                        eph ^= 1;
+                    }
+                    cw = cw_n;
+                    hw = hw_n;
+                    s2 = s2_n;
                 }
+                // every lane has read the slot: lane 0 refills it with the chunk NP ahead
+                __syncwarp();
+                ++consumed;
+                if (!ld_volatile(S.abort_flag)) issue();
             }
         }
+        // after an abort, no bulk copy may still target shared memory at exit: wait
+        // (bounded) for the most recent phase issued on each slot
+        if (lane == 0 && ld_volatile(S.abort_flag))
+            for (int d = 0; d < NP && d < issued; ++d) {
+                const int q2 = issued - 1 - d;
+                if (!mbar_wait_bounded(&pfull[q2 % NP], (q2 / NP) & 1, kWaitLimit)) {
+                    report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | 0x50 | MODE);
+                    break;
+                }
+            }
     } else if (warp == kTmaWarp) {
         // ============================ TMA producer (B) ===============================
-        if (lane == 0) {
-            int it = 0;
-            for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-                const TileInfo ti = tile_info(S, p, tile, mtiles);
-                const int nbox = (ti.N + BOX_ROWS - 1) / BOX_ROWS;
-                for (int ks = 0; ks < KS; ++ks, ++it) {
-                    const int slot = it & (NSTG - 1);
-                    wait_or_flag(S, &empty_[slot], ((it / NSTG) & 1) ^ 1, p, kDetWaitEmpty | 0x20 | MODE);
-                    if (ld_volatile(S.abort_flag)) continue;
-                    uint8_t* bdst = smem + (size_t)slot * STG_BYTES + A_BYTES;
-                    mbar_arrive_expect_tx(&full_b[slot], nbox * BOX_ROWS * BK * 2);
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(bdst + b * BOX_ROWS * BK * 2, &bmap, ks * BK, ti.row0 + b * BOX_ROWS, &full_b[slot]);
+        // whole warp, converged; one elected lane issues
+        int it = 0, issued = 0, slot = 0;
+        uint32_t eph = 1;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const TileInfo ti = tile_info(S, p, tile, mtiles);
+            const int bx = box_index(ti.N);
+            const uint32_t bbytes = (64u << bx) * BK * 2;
+            for (int ks = 0; ks < KS; ++ks, ++it) {
+                if (!mbar_try_wait(&empty_[slot], eph))
+                    wait_or_flag(S, &empty_[slot], eph, p, kDetWaitEmpty | 0x20 | MODE);
+                __syncwarp();
+                if (!ld_volatile(S.abort_flag)) {
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&full_b[slot], bbytes);
+                        tma_load_2d(smem + (size_t)slot * STG_BYTES + A_BYTES, &bmaps.m[bx], ks * BK, ti.row0,
+                                    &full_b[slot]);
+                    }
+                    __syncwarp();
+                    issued = it + 1;
+                }
+                if (++slot == NSTG) {
+                    slot = 0;
+                    eph ^= 1;
                 }
             }
-            // no TMA write may still target shared memory at exit (matters only after an
-            // abort: normally the MMA issuer has consumed every stage)
-            if (ld_volatile(S.abort_flag))
-                for (int d = 0; d < NSTG && d < it; ++d) {
-                    const int q2 = it - 1 - d;
-                    if (!mbar_wait_bounded(&full_b[q2 & (NSTG - 1)], (q2 / NSTG) & 1, kWaitLimit)) {
-                        report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | MODE);
-                        break;
-                    }
-                }
         }
+        // no TMA write may still target shared memory at exit (matters only after an
+        // abort: normally the MMA issuer has consumed every stage)
+        if (lane == 0 && ld_volatile(S.abort_flag))
+            for (int d = 0; d < NSTG && d < issued; ++d) {
+                const int q2 = issued - 1 - d;
+                if (!mbar_wait_bounded(&full_b[q2 % NSTG], (q2 / NSTG) & 1, kWaitLimit)) {
+                    report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | MODE);
+                    break;
+                }
+            }
     } else if (warp == kMmaWarp) {
         // ============================== MMA issuer ===================================
-        if (lane == 0) {
-            int it = 0, tc = 0;
-            for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
-                const TileInfo ti = tile_info(S, p, tile, mtiles);
-                const int buf = tc & 1;
-                const int n16 = (ti.N + 15) & ~15;
-                const uint32_t idesc = instr_desc(n16);
-                wait_or_flag(S, &acc_empty[buf], ((tc >> 1) & 1) ^ 1, p, kDetWaitEmpty | 0x30 | MODE);
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + buf * BN;
-                for (int ks = 0; ks < KS; ++ks, ++it) {
-                    const int slot = it & (NSTG - 1);
-                    const uint32_t par = (it / NSTG) & 1;
-                    const bool ok_a = wait_or_flag(S, &full_a[slot], par, p, kDetWaitFull | 0x10 | MODE);
-                    const bool ok_b = wait_or_flag(S, &full_b[slot], par, p, kDetWaitFull | 0x20 | MODE);
-                    tc_fence_after();
-                    if (ok_a && ok_b) {
-                        const uint32_t a0 = smem_u32(smem + (size_t)slot * STG_BYTES);
-                        const uint32_t b0 = a0 + A_BYTES;
+        // The whole warp runs the loop (its control flow and the descriptors stay
+        // warp-uniform) and one elected lane issues tcgen05.mma / commit.  The per-stage
+        // path is short, since it bounds the stage rate: slot and phase advance
+        // incrementally, descriptors are precomputed, and the bounded wait is entered
+        // only when the barrier is not already complete.
+        const uint64_t a_desc0 = smem_desc(smem_u32(smem));
+        constexpr uint32_t kSlotStep = STG_BYTES >> 4, kBOff = A_BYTES >> 4;
+        int slot = 0, tc = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
+            const TileInfo ti = tile_info(S, p, tile, mtiles);
+            const int buf = tc & 1;
+            const int n16 = (ti.N + 15) & ~15;
+            const uint32_t idesc = instr_desc(n16);
+            if (!mbar_try_wait(&acc_empty[buf], ((tc >> 1) & 1) ^ 1))
+                ok &= wait_or_flag(S, &acc_empty[buf], ((tc >> 1) & 1) ^ 1, p, kDetWaitEmpty | 0x30 | MODE);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + buf * BN;
+            for (int ks = 0; ks < KS; ++ks) {
+                if (!mbar_try_wait(&full_a[slot], phase))
+                    ok &= wait_or_flag(S, &full_a[slot], phase, p, kDetWaitFull | 0x10 | MODE);
+                if (!mbar_try_wait(&full_b[slot], phase))
+                    ok &= wait_or_flag(S, &full_b[slot], phase, p, kDetWaitFull | 0x20 | MODE);
+                ok = __all_sync(0xffffffffu, ok);
+                const uint64_t ad = a_desc0 + (uint64_t)(slot * kSlotStep), bd = ad + kBOff;
+                if (elect_one()) {
+                    if (ok) {
 #pragma unroll
                         for (int k16 = 0; k16 < BK / 16; ++k16)
-                            umma_f16(d_tmem, smem_desc(a0 + 32 * k16), smem_desc(b0 + 32 * k16), idesc,
-                                     (ks > 0 || k16 > 0) ? 1u : 0u);
+                            umma_f16(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, (ks | k16) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty_[slot]);
                 }
-                umma_commit(&acc_full[buf]);
+                __syncwarp();
+                if (++slot == NSTG) {
+                    slot = 0;
+                    phase ^= 1;
+                }
             }
-            // every MMA this thread issued has completed once this commit arrives
-            umma_commit(&mma_done);
-            if (!mbar_wait_bounded(&mma_done, 0, kWaitLimit)) report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | 0x40);
+            if (elect_one()) umma_commit(&acc_full[buf]);
+            __syncwarp();
         }
-    } else {
+        // every MMA this warp issued has completed once this commit arrives
+        if (elect_one()) umma_commit(&mma_done);
+        __syncwarp();
+        if (lane == 0 && !mbar_wait_bounded(&mma_done, 0, kWaitLimit)) report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | 0x40);
+    } else if (warp >= kEpiWarp0) {
         // =============================== epilogue ====================================
-        const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31
+        const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31 (warps 8-11)
+        uint16_t* const stg = reinterpret_cast<uint16_t*>(smem + (size_t)NSTG * STG_BYTES +
+                                                           (size_t)kDqWarps * NP * PK_BYTES) + q * 256;
         int tc = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
             const int buf = tc & 1;
-            wait_or_flag(S, &acc_full[buf], (tc >> 1) & 1, p, kDetWaitFull | 0x30 | MODE);
+            // a long wait (a whole tile's main loop): poll slowly to leave the issue slots
+            // to the dequantisers on this sub-partition
+            if (!mbar_try_wait(&acc_full[buf], (tc >> 1) & 1) && !ld_volatile(S.abort_flag) &&
+                !mbar_wait_bounded_backoff(&acc_full[buf], (tc >> 1) & 1, kWaitLimit, 256)) {
+                st_volatile(S.abort_flag, 1);
+                report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | 0x30 | MODE);
+            }
             tc_fence_after();
             const uint32_t tbase = tmem + buf * BN + ((uint32_t)(32 * q) << 16);
             const int mrow = ti.mt * BM + 32 * q + lane;    // row of the packed matrix
+            const int hcol0 = (ti.mt * BM + 32 * q) / 2;         // first h column of this warp (gate/up)
             for (int c0 = 0; c0 < ti.N; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld16(tbase + c0, v);
                 if (MODE == 0) {
+                    // lanes l < 8 and 16 <= l < 24 hold gate rows, l + 8 the matching up
+                    // rows: h for 16 tokens x this warp's 16 h columns, transposed through
+                    // shared memory into one 16-byte store per lane
                     const bool gate_lane = (lane & 15) < 8;
-                    const int hcol = (mrow >> 4) * 8 + (lane & 7);
+                    const int lc = ((lane >> 4) << 3) | (lane & 7);    // h column within the warp
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const float a = __uint_as_float(v[u]);
                         const float b = __shfl_down_sync(0xffffffffu, a, 8);
-                        if (gate_lane && c0 + u < ti.N)
-                            p.h[(size_t)(ti.row0 + c0 + u) * p.I + hcol] = f32_to_f16_bits(silu_f(a) * b);
+                        if (gate_lane) stg[u * 16 + lc] = f32_to_f16_bits(silu_fast(a) * b);
                     }
+                    __syncwarp();
+                    const int u = lane >> 1, half = lane & 1;
+                    if (c0 + u < ti.N)
+                        *reinterpret_cast<uint4*>(p.h + (size_t)(ti.row0 + c0 + u) * p.I + hcol0 + 8 * half) =
+                            *reinterpret_cast<const uint4*>(stg + u * 16 + 8 * half);
+                    __syncwarp();
                 } else {
 #pragma unroll
                     for (int u = 0; u < 16; ++u)
@@ -447,23 +579,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
 }
 
 // X16[r][:] = fp16(x[token of permuted row r][:]); rows T*k .. are the shared expert's.
+// One block per row, threads over 8-element column chunks.
 __global__ void __launch_bounds__(256) gather_x16_kernel(FfnArgs p, uint16_t* x16) {
-    const int per_row = p.H / 8;
-    const long long rows = (long long)p.T * (p.k + p.S);
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= rows * per_row) return;
-    const long long r = idx / per_row;
-    const int c8 = (int)(idx - r * per_row) * 8;
-    const int tok = r < (long long)p.T * p.k ? p.perm[r] / p.k : (int)((r - (long long)p.T * p.k) % p.T);
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)tok * p.H + c8));
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[4];
+    const int r = blockIdx.x;
+    const int tk = p.T * p.k;
+    const int tok = r < tk ? __ldg(p.perm + r) / p.k : (r - tk) % p.T;
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)tok * p.H);
+    uint4* dst = reinterpret_cast<uint4*>(x16 + (size_t)r * p.H);
+    for (int c = threadIdx.x; c < p.H / 8; c += blockDim.x) {
+        const uint4 v = __ldg(src + c);
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const float lo = __uint_as_float(in[u] << 16), hi = __uint_as_float(in[u] & 0xFFFF0000u);
-        out[u] = (uint32_t)f32_to_f16_bits(lo) | ((uint32_t)f32_to_f16_bits(hi) << 16);
+        for (int u = 0; u < 4; ++u) {
+            const float lo = __uint_as_float(in[u] << 16), hi = __uint_as_float(in[u] & 0xFFFF0000u);
+            out[u] = (uint32_t)f32_to_f16_bits(lo) | ((uint32_t)f32_to_f16_bits(hi) << 16);
+        }
+        dst[c] = make_uint4(out[0], out[1], out[2], out[3]);
     }
-    *reinterpret_cast<uint4*>(x16 + (size_t)r * p.H + c8) = make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
@@ -479,23 +612,28 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
     return fn;
 }
 
-// 2-D fp16 tensor map over rows x K (K-major), 64 x 64 boxes, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, long long rows, int K) {
+// 2-D fp16 tensor map over rows x K (K-major), boxes of 64 K x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows) {
     auto enc = get_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {BK, BOX_ROWS};
+    cuuint32_t box[2] = {BK, (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kTcSmem = (size_t)NSTG * STG_BYTES + 1024;
+constexpr size_t kTcSmem = (size_t)NSTG * STG_BYTES + (size_t)kDqWarps * NP * PK_BYTES + 4 * 512 + 1024;
+
+bool make_maps(BMaps* b, const void* base, long long rows, int K) {
+    return make_map(&b->m[0], base, rows, K, 64) && make_map(&b->m[1], base, rows, K, 128) &&
+           make_map(&b->m[2], base, rows, K, 256);
+}
 
 template <int MODE>
-cudaError_t launch_tc(const FfnArgs& a, const CUtensorMap& map, cudaStream_t s) {
+cudaError_t launch_tc(const FfnArgs& a, const BMaps& maps, cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
         cudaError_t err =
@@ -503,7 +641,7 @@ cudaError_t launch_tc(const FfnArgs& a, const CUtensorMap& map, cudaStream_t s) 
         if (err != cudaSuccess) return err;
         attr = true;
     }
-    tc_gemm_kernel<MODE><<<a.num_ctas, kThreads, kTcSmem, s>>>(a, map);
+    tc_gemm_kernel<MODE><<<a.num_ctas, kThreads, kTcSmem, s>>>(a, maps);
     return cudaGetLastError();
 }
 
@@ -513,12 +651,12 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, uint16_t* x16, cudaStream_t s, 
                                cudaEvent_t ev_down) {
     if ((2 * a.I) % BM != 0 || a.H % BM != 0) return cudaErrorInvalidConfiguration;
     const long long rows = (long long)a.T * (a.k + a.S);
-    const long long n8 = rows * (a.H / 8);
-    gather_x16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a, x16);
+    if (rows > 2147483647LL) return cudaErrorInvalidConfiguration;
+    gather_x16_kernel<<<(unsigned)rows, 256, 0, s>>>(a, x16);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    CUtensorMap mx, mh;
-    if (!make_map(&mx, x16, rows, a.H) || !make_map(&mh, a.h, rows, a.I)) return cudaErrorInvalidConfiguration;
+    BMaps mx, mh;
+    if (!make_maps(&mx, x16, rows, a.H) || !make_maps(&mh, a.h, rows, a.I)) return cudaErrorInvalidConfiguration;
     err = launch_tc<0>(a, mx, s);
     if (err != cudaSuccess) return err;
     if (ev_gateup) cudaEventRecord(ev_gateup, s);
