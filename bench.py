@@ -11,6 +11,12 @@ reads its experts from HBM.  For N > 1 (torchrun) each rank runs an independent
 replica on its own token stream (the layer is data-parallel: no collective on the
 data path) and the time is the max over ranks.
 
+The roofline object describes the gate/up launch: for the decode path (<= 64 tokens)
+against the measured HBM copy bandwidth (algorithmic bytes = the packed bytes of
+every selected expert and the shared expert, each read once); for the tensor-core
+prefill path against the measured sustained bf16 GEMM rate (algorithmic FLOPs =
+2 x routed rows x 2*ffn x hidden; the fp16 operands run at the bf16 rate).
+
 --impl reference times the CPU oracle (the only reference that exists for this
 layer) on the same workload, a bounded sample per step, on the host cores.
 """
@@ -35,8 +41,42 @@ import synth  # noqa: E402
 
 METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B200)"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GATEUP_KERNEL = "ffn_decode_kernel<0, NT, NW> (gate/up + SwiGLU)"
-KERNEL_SOURCES = ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]
+# gate/up kernel of each path and the sources its ncu traffic record is tied to
+PATHS = {
+    "decode": ("ffn_decode_kernel<0, NT, NW> (gate/up + SwiGLU)",
+               ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
+    "prefill": ("tc_gemm_kernel<0> (gate/up + SwiGLU, tcgen05; interval includes the token gather)",
+                ["bit_routed_expert_fp32_b200/csrc/prefill_tc.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
+}
+
+
+def path_of(cfg) -> str:
+    """The path moe_forward(MOE_PATH_AUTO) takes for this workload."""
+    tc_ok = cfg.H % 128 == 0 and (2 * cfg.I) % 128 == 0
+    return "prefill" if cfg.T > 64 and tc_ok else "decode"
+
+
+def launches_per_step(cfg) -> int:
+    """Kernels one step launches: routing (one fused kernel up to 64 tokens, else four)
+    plus gate/up, down and combine, plus the token gather on the prefill path."""
+    route = 1 if cfg.T <= 64 else 4
+    return route + (4 if path_of(cfg) == "prefill" else 3)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of x over all ranks (x itself for one rank)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's device time."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
 
 
 def peaks():
@@ -48,15 +88,15 @@ def peaks():
     return FALLBACK, "fallback"
 
 
-def kernel_hash() -> str:
+def kernel_hash(path: str) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in PATHS[path][1]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def traffic_record(cfg_name: str):
+def traffic_record(cfg_name: str, path: str):
     """DRAM bytes per launch of the gate/up kernel from the committed ncu summary, if
     it was taken on the current kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -65,7 +105,7 @@ def traffic_record(cfg_name: str):
     with open(p) as f:
         d = json.load(f)
     rec = d.get(cfg_name)
-    if not rec or rec.get("kernel_hash") != kernel_hash():
+    if not rec or rec.get("kernel_hash") != kernel_hash(path):
         return None
     return rec
 
@@ -310,11 +350,8 @@ def run_ours(args, cfg):
     cb_ms = [ev[s][3].elapsed_time(ev[s][4]) for s in range(args.warmup, total)]
     rt_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.warmup, total)]
     my_ms = float(sum(step_ms))
-    t = torch.tensor([my_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    value = world * T * args.steps / (max_ms / 1e3)
+    max_ms = max_over_ranks(my_ms, world, dev)
+    value = throughput(world, T, args.steps, max_ms)
 
     # algorithmic bytes of the gate/up launches from the routing each step produced
     ids_h = ids_log.cpu().numpy()
@@ -332,13 +369,27 @@ def run_ours(args, cfg):
     gu_gbs = (sum(gu_alg) / 1e9) / (sum(gu_ms) / 1e3)
     dn_gbs = (sum(dn_alg) / 1e9) / (sum(dn_ms) / 1e3)
     layer_gbs = ((sum(gu_alg) + sum(dn_alg)) / 1e9) / (my_ms / 1e3)
-    tr = traffic_record(cfg.name)
-    roofline = {"bound": "hbm", "kernel": GATEUP_KERNEL, "achieved": gu_gbs, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": gu_gbs / pk["hbm_gbs"],
-                "traffic": None if tr is None else tr["dram_bytes_per_launch"],
-                "algorithmic_bytes_per_launch": float(np.mean(gu_alg)),
-                "peak_source": f"{pk_kind} (MEASURED_PEAKS.json hbm_gbs)" if pk_kind == "measured" else "fallback",
-                "avg_launch_us": 1e3 * float(np.mean(gu_ms))}
+    path = path_of(cfg)
+    tr = traffic_record(cfg.name, path)
+    traffic = None if tr is None else tr["dram_bytes_per_launch"]
+    if path == "decode":
+        roofline = {"bound": "hbm", "kernel": PATHS[path][0], "achieved": gu_gbs, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": gu_gbs / pk["hbm_gbs"], "traffic": traffic,
+                    "algorithmic_bytes_per_launch": float(np.mean(gu_alg)),
+                    "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)",
+                    "avg_launch_us": 1e3 * float(np.mean(gu_ms))}
+    else:
+        rows = T * (cfg.k + cfg.S)
+        flops = 2.0 * rows * (2 * cfg.I) * cfg.H
+        tflops = flops / (float(np.mean(gu_ms)) / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        roofline = {"bound": "tensor", "kernel": PATHS[path][0], "achieved": tflops, "peak": peak,
+                    "unit": "TFLOP/s", "frac": tflops / peak, "traffic": traffic,
+                    "algorithmic_flops_per_launch": flops,
+                    "peak_source": f"{pk_kind} bf16_tflops_sustained (cuBLAS bf16 GEMM looped under the power cap; "
+                                   f"the launch runs inside a multi-millisecond step)",
+                    "avg_launch_us": 1e3 * float(np.mean(gu_ms)),
+                    "weight_stream_gbs": gu_gbs}
 
     # end to end through the public API with host buffers (pinned), copies timed
     x_pin = torch.from_numpy(xs_host.view(np.int16)).pin_memory()
@@ -359,17 +410,13 @@ def run_ours(args, cfg):
             e2e_ms.append((a, b))
     torch.cuda.synchronize(dev)
     e2e_total = sum(a.elapsed_time(b) for a, b in e2e_ms)
-    t2 = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_value = world * T * args.steps / (float(t2.item()) / 1e3)
+    e2e_value = throughput(world, T, args.steps, max_over_ranks(e2e_total, world, dev))
     st, det = moe.moe_get_error(layers[0].ws)
     if st != 0:
         raise RuntimeError(f"device error {moe.STATUS[st]} {det:#x}")
 
     line = None
     if rank == 0:
-        launches_per_step = (1 if T <= 64 else 4) + 3     # route kernels + gate/up, down, combine
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -381,7 +428,8 @@ def run_ours(args, cfg):
                               "down_gbs": dn_gbs},
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.H * 2,
                         "d2h_bytes_per_step": T * cfg.H * 2},
-                "gpu_launches": launches_per_step * args.steps,
+                "gpu_launches": launches_per_step(cfg) * args.steps,
+                "path": path,
                 "wall_s_timed_region": wall,
                 "clocks": ck}
         if world == 1 and not args.no_cpu_baseline:

@@ -277,7 +277,7 @@ struct RingProducer {
         if (item != cur_item) load_item(p, S, tiles);
         const int st = issued & (NS - 1);
         const int ng = min(CG, G - c * CG);
-        if (lane == 0) {
+        if (elect_one()) {                      // warp-uniform issue, one elected lane
             uint8_t* dst = ring + (size_t)st * STAGE;
             const uint32_t cb = 256 * ng, hb = q3 ? 128 * ng : 0;
             mbar_arrive_expect_tx(&bar[st], cb + hb + 256);
