@@ -256,10 +256,13 @@ def run_reference(args, cfg):
     return 0
 
 
-def config_dict(cfg, world):
-    return {"workload": cfg.name, "tokens_per_step": cfg.T, "hidden": cfg.H, "experts": cfg.E, "top_k": cfg.k,
-            "ffn": cfg.I, "shared": cfg.S, "formats": cfg.formats, "layers": cfg.layers,
-            "l2": "flushed between timed steps (512 MiB write)", "parallelism": f"replicas x{world}"}
+def config_dict(cfg, world, launch=None):
+    d = {"workload": cfg.name, "tokens_per_step": cfg.T, "hidden": cfg.H, "experts": cfg.E, "top_k": cfg.k,
+         "ffn": cfg.I, "shared": cfg.S, "formats": cfg.formats, "layers": cfg.layers,
+         "l2": "flushed between timed steps (512 MiB write)", "parallelism": f"replicas x{world}"}
+    if launch:
+        d["launch"] = launch
+    return d
 
 
 # --------------------------------------------------------------------------- ours
@@ -299,26 +302,58 @@ def run_ours(args, cfg):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     ids_log = torch.empty((total, T, cfg.k), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(total)]
-    for row in ev:               # torch creates the CUDA event on first record: do it here so
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(total)]      # step pass
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(total)]     # kernel pass
+    for row in ev + evk:         # torch creates the CUDA event on first record: do it here so
         for e in row:            # the handles handed to the library are real events
             e.record(stream)
     torch.cuda.synchronize(dev)
 
-    def step(s, record=True):
+    def step(s, record=None, per_kernel=False):
+        """One layer step; record = the step's 6 events (0 and 5 bracket the step; 1-4
+        go between the kernels when per_kernel, which serialises the launches)."""
+        st = torch.cuda.current_stream(dev)          # the capture stream while capturing
         lay = layers[s % n_layers]
-        e = ev[s]
-        if record:
-            e[0].record(stream)
-        lay.route(x_dev[s])
-        lay.forward(x_dev[s], y, events=e[1:5] if record else None)
-        if record:
-            e[5].record(stream)
+        if record is not None:
+            moe.moe_event_record(record[0], st)
+        lay.route(x_dev[s], stream=st)
+        lay.forward(x_dev[s], y, events=record[1:5] if (record is not None and per_kernel) else None, stream=st)
+        if record is not None:
+            moe.moe_event_record(record[5], st)
             ids_log[s].copy_(lay.rt["topk_ids"][:T])
+
+    # Each step (route + forward) is captured as one CUDA graph and replayed.  The
+    # kernels are launched with programmatic dependent launch, so a kernel's launch
+    # overlaps its predecessor's tail; the timed pass records events only around the
+    # whole step.  A second pass over the same steps (same flushes) puts an event
+    # between the kernels, which serialises them, to give the per-kernel times and the
+    # gate/up launch duration for the roofline.  --no-graph launches eagerly instead.
+    graphs = gk = None
+    if not args.no_graph:
+        for s in range(min(2, total)):              # first-call set-up happens outside capture
+            step(s)
+        torch.cuda.synchronize(dev)
+        graphs, gk = [], []
+        for s in range(total):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(s, ev[s])
+            graphs.append(g)
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                step(s, evk[s], per_kernel=True)
+            gk.append(g2)
+        torch.cuda.synchronize(dev)
+
+    def run(s, per_kernel=False):
+        if graphs is not None:
+            (gk if per_kernel else graphs)[s].replay()
+        else:
+            step(s, evk[s] if per_kernel else ev[s], per_kernel)
 
     for s in range(args.warmup):
         flush.zero_()
-        step(s)
+        run(s)
     torch.cuda.synchronize(dev)
     # clocks are sampled (every 100 ms) over a soak of the same steps that runs right
     # before the timed region and over the timed region itself
@@ -328,7 +363,7 @@ def run_ours(args, cfg):
     while time.perf_counter() - t_soak < args.soak_s:
         for s in range(args.warmup):
             flush.zero_()
-            step(s, record=False)
+            run(s)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -336,19 +371,25 @@ def run_ours(args, cfg):
     wall0 = time.perf_counter()
     for s in range(args.warmup, total):
         flush.zero_()
-        step(s)
+        run(s)
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
+    # per-kernel pass (not part of the headline number)
+    for s in range(args.warmup, total):
+        flush.zero_()
+        run(s, per_kernel=True)
+    torch.cuda.synchronize(dev)
     ck = clocks.stop()
     if ck is not None:
         ck["sampled_over"] = f"{args.soak_s:.1f} s soak of the same steps + the timed region"
     step_ms = [ev[s][0].elapsed_time(ev[s][5]) for s in range(args.warmup, total)]
-    gu_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.warmup, total)]
-    dn_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(args.warmup, total)]
-    cb_ms = [ev[s][3].elapsed_time(ev[s][4]) for s in range(args.warmup, total)]
-    rt_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.warmup, total)]
+    gu_ms = [evk[s][1].elapsed_time(evk[s][2]) for s in range(args.warmup, total)]
+    dn_ms = [evk[s][2].elapsed_time(evk[s][3]) for s in range(args.warmup, total)]
+    cb_ms = [evk[s][3].elapsed_time(evk[s][4]) for s in range(args.warmup, total)]
+    rt_ms = [evk[s][0].elapsed_time(evk[s][1]) for s in range(args.warmup, total)]
+    step_serial_ms = [evk[s][0].elapsed_time(evk[s][5]) for s in range(args.warmup, total)]
     my_ms = float(sum(step_ms))
     max_ms = max_over_ranks(my_ms, world, dev)
     value = throughput(world, T, args.steps, max_ms)
@@ -420,12 +461,14 @@ def run_ours(args, cfg):
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": config_dict(cfg, world),
+                "config": config_dict(cfg, world, "eager launches" if graphs is None else
+                                      "one CUDA graph per step (route + forward), replayed"),
                 "roofline": roofline,
                 "layer_weight_stream_gbs": layer_gbs,
                 "kernel_us": {"route": 1e3 * float(np.mean(rt_ms)), "gate_up": 1e3 * float(np.mean(gu_ms)),
                               "down": 1e3 * float(np.mean(dn_ms)), "combine": 1e3 * float(np.mean(cb_ms)),
-                              "down_gbs": dn_gbs},
+                              "down_gbs": dn_gbs, "step_with_events_between_kernels": 1e3 * float(np.mean(step_serial_ms)),
+                              "measured": "second pass over the same steps with an event between kernels"},
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.H * 2,
                         "d2h_bytes_per_step": T * cfg.H * 2},
                 "gpu_launches": launches_per_step(cfg) * args.steps,
@@ -460,6 +503,7 @@ def main():
     ap.add_argument("--soak-s", type=float, default=1.5)
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's tokens per step (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every call eagerly instead of replaying graphs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

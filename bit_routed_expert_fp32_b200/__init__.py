@@ -23,8 +23,8 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 # every symbol include/moe.h declares
 EXPORTS = ["moe_packed_size", "moe_pack_experts", "moe_workspace_size", "moe_workspace_init", "moe_route",
-           "moe_forward", "moe_forward_timed", "moe_get_error", "moe_decode_static", "moe_status_string",
-           "moe_abi_version"]
+           "moe_forward", "moe_forward_timed", "moe_get_error", "moe_decode_static", "moe_event_record",
+           "moe_status_string", "moe_abi_version"]
 STATIC_WS_BYTES = 8 << 20
 
 
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(vp), i32]
         L.moe_get_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_decode_static.argtypes = [sh, i32, vp, vp, vp, vp, ctypes.POINTER(Routing), vp, vp]
+        L.moe_event_record.argtypes = [vp, vp]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_abi_version.restype = i32
@@ -175,6 +176,12 @@ def moe_forward(cfg, T, packed, x, rt: dict, y, path=PATH_AUTO, ws=None, stream=
     st = lib().moe_forward_timed(ctypes.byref(_shape(cfg)), T, _ptr(packed), _ptr(x), ctypes.byref(r), _ptr(y),
                                  path, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream), ev, 4)
     _check("moe_forward_timed", st)
+
+
+def moe_event_record(event, stream=None) -> None:
+    """Records a torch.cuda.Event on the stream; inside graph capture the record becomes a
+    graph node that every replay executes."""
+    _check("moe_event_record", lib().moe_event_record(ctypes.c_void_p(event.cuda_event), _stream(stream)))
 
 
 def moe_decode_static(cfg, T, x, router_w, router_b, packed, rt: dict, y, stream=None) -> None:

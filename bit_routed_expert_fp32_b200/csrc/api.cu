@@ -85,6 +85,13 @@ extern "C" {
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+moe_status moe_event_record(void* event, void* stream) {
+    if (!event) return MOE_ERR_INVALID_ARG;
+    return moe::record_event(static_cast<cudaEvent_t>(event), static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 const char* moe_status_string(moe_status s) {
     switch (s) {
         case MOE_OK: return "ok";
@@ -177,7 +184,7 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
     if (events)
         for (int i = 0; i < 4; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
-    if (ev[0] && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (ev[0] && record_event(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
     // The prefill kernels tile the gate/up rows and the hidden rows by 128.
     const bool tc_ok = a.H % 128 == 0 && (2 * a.I) % 128 == 0;
     if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
@@ -185,7 +192,7 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     cudaError_t err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
                               : launch_ffn_decode(a, s, ev[1], ev[2]);
     if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
-    if (ev[3] && cudaEventRecord(ev[3], s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (ev[3] && record_event(ev[3], s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 

@@ -155,6 +155,19 @@ __device__ inline void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t b
         : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start before its predecessor in the stream has finished: it must
+// call griddep_wait() before it reads anything the predecessor writes (or overwrites
+// anything the predecessor reads).  griddep_launch_dependents() lets the next kernel's
+// launch begin; kernels call it only when all of their CTAs are resident at once, so
+// the successor's CTAs never take an SM that one of their own still needs.  Both are
+// no-ops for kernels launched without the attribute.
+__device__ inline void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// Prefetch the line holding p into L1 (no register result, never blocks).
+__device__ inline void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
+
 // Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned address and size).
 __device__ inline void bulk_prefetch_l2(const void* src_gmem, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes) : "memory");

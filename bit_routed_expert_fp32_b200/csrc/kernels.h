@@ -1,5 +1,6 @@
 // Internal launcher interface between the C ABI (api.cu) and the kernels.
 #pragma once
+#include <utility>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -58,5 +59,35 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, uint16_t* x16, cudaStream_t s, 
                                cudaEvent_t ev_down);
 // gate-weighted unpermute-combine of the partial rows into y
 cudaError_t launch_combine(const FfnArgs& a, cudaStream_t s);
+
+// Launches kern<<<grid, block, smem, s>>>(args...) with programmatic stream
+// serialization: the kernel may begin while its predecessor in s is still running and
+// synchronises with it through griddep_wait().
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Records event e on stream s.  While s is being captured into a CUDA graph the record
+// becomes an event node of the graph (cudaEventRecordExternal), so that every replay
+// records the event as an eager launch would; otherwise a plain record.
+inline cudaError_t record_event(cudaEvent_t e, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const cudaError_t err = cudaStreamIsCapturing(s, &cs);
+    if (err != cudaSuccess) return err;
+    return cudaEventRecordWithFlags(e, s, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                              : cudaEventRecordDefault);
+}
 
 }  // namespace moe

@@ -231,6 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
     const int KS = K / BK;                 // K stages per tile
     const int G = K / 64, NC = (G + 7) / 8;
 
+    // launched with programmatic serialization: the launch overlaps the predecessor's
+    // tail; nothing is read before the predecessor has finished
+    griddep_launch_dependents();        // one CTA per SM: every CTA of this grid is resident
+    griddep_wait();
     if (threadIdx.x == 0) {
         const uint32_t* hd = reinterpret_cast<const uint32_t*>(p.packed);
         const bool ok = hd[0] == kMagic && hd[1] == kVersion && (int)hd[2] == p.H && (int)hd[3] == p.I &&
@@ -581,6 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
 // X16[r][:] = fp16(x[token of permuted row r][:]); rows T*k .. are the shared expert's.
 // One block per row, threads over 8-element column chunks.
 __global__ void __launch_bounds__(256) gather_x16_kernel(FfnArgs p, uint16_t* x16) {
+    griddep_wait();                     // perm comes from the router
     const int r = blockIdx.x;
     const int tk = p.T * p.k;
     const int tok = r < tk ? __ldg(p.perm + r) / p.k : (r - tk) % p.T;
@@ -641,8 +646,7 @@ cudaError_t launch_tc(const FfnArgs& a, const BMaps& maps, cudaStream_t s) {
         if (err != cudaSuccess) return err;
         attr = true;
     }
-    tc_gemm_kernel<MODE><<<a.num_ctas, kThreads, kTcSmem, s>>>(a, maps);
-    return cudaGetLastError();
+    return launch_pdl(tc_gemm_kernel<MODE>, dim3(a.num_ctas), dim3(kThreads), kTcSmem, s, a, maps);
 }
 
 }  // namespace
@@ -652,17 +656,16 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, uint16_t* x16, cudaStream_t s, 
     if ((2 * a.I) % BM != 0 || a.H % BM != 0) return cudaErrorInvalidConfiguration;
     const long long rows = (long long)a.T * (a.k + a.S);
     if (rows > 2147483647LL) return cudaErrorInvalidConfiguration;
-    gather_x16_kernel<<<(unsigned)rows, 256, 0, s>>>(a, x16);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(gather_x16_kernel, dim3((unsigned)rows), dim3(256), 0, s, a, x16);
     if (err != cudaSuccess) return err;
     BMaps mx, mh;
     if (!make_maps(&mx, x16, rows, a.H) || !make_maps(&mh, a.h, rows, a.I)) return cudaErrorInvalidConfiguration;
     err = launch_tc<0>(a, mx, s);
     if (err != cudaSuccess) return err;
-    if (ev_gateup) cudaEventRecord(ev_gateup, s);
+    if (ev_gateup && (err = record_event(ev_gateup, s)) != cudaSuccess) return err;
     err = launch_tc<1>(a, mh, s);
     if (err != cudaSuccess) return err;
-    if (ev_down) cudaEventRecord(ev_down, s);
+    if (ev_down && (err = record_event(ev_down, s)) != cudaSuccess) return err;
     return launch_combine(a, s);
 }
 

@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
 // 2 experts per CTA, 4 warps per expert row (one K quarter each), 7 float4 loads in
 // flight per lane; then the Z tables; the last CTA does top-k and the permutation.
 __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
+    griddep_launch_dependents();        // one wave of CTAs: the expert pass may start launching
     constexpr int U = 7;
     __shared__ float s_part[8][kSmallT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -480,6 +481,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(RouteArgs p) {
 }
 
 __global__ void __launch_bounds__(32) route_scatter_kernel(RouteArgs p) {
+    griddep_launch_dependents();        // one wave of CTAs: the expert pass may start launching
     __shared__ int s_run[256];
     const int c = blockIdx.x, lane = threadIdx.x;
     for (int e = lane; e < p.E; e += 32) s_run[e] = p.hist[(size_t)c * p.E + e];

@@ -230,6 +230,15 @@ moe_status moe_decode_static(const moe_shape* shape, int32_t T, const uint16_t* 
                              const float* d_router_w, const float* d_router_b, const void* d_packed,
                              const moe_routing* out, uint16_t* d_y, void* stream);
 
+/* Records a caller-created CUDA event (cudaEvent_t, passed as void*) on a stream.
+ * While the stream is being captured into a CUDA graph the record is captured as an
+ * event node of the graph (cudaEventRecordExternal), so every replay of the graph
+ * records the event; otherwise it is a plain cudaEventRecord.  moe_forward_timed
+ * records its events the same way.  The pages have no counterpart: this exists so
+ * that callers can time graph-replayed layer steps.
+ * Errors: MOE_ERR_INVALID_ARG for a null event, MOE_ERR_CUDA if the record fails. */
+moe_status moe_event_record(void* event, void* stream);
+
 const char* moe_status_string(moe_status s);
 int32_t moe_abi_version(void);
 

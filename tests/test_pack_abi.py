@@ -47,6 +47,7 @@ def test_argument_errors_are_synchronous():
     sz = ctypes.c_size_t(0)
     fmt = np.ones(5, np.uint8)
     assert L.moe_packed_size(None, fmt.ctypes.data, ctypes.byref(sz)) == 1
+    assert L.moe_event_record(None, None) == 1          # null event: rejected before any CUDA call
     bad = _shape(H=100)
     assert L.moe_packed_size(ctypes.byref(bad), fmt.ctypes.data, ctypes.byref(sz)) == 1
     assert L.moe_workspace_size(ctypes.byref(_shape(k=5)), 4, ctypes.byref(sz)) == 1       # k > E
