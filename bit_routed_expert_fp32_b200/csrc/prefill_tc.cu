@@ -6,28 +6,32 @@
 // pages sweeps a long prompt in batches of 6-9K tokens (shadowgraph.io README,
 // paragraph under the model table); here one call takes all T tokens.
 //
-// Orientation ("swap-AB"): D[M = 128 weight rows][N <= 256 tokens] = W_tile x X^T.
+// Orientation ("swap-AB"): D[M = 128 weight rows][N <= 192 tokens] = W_tile x X^T.
 // Weights are the A operand, so every tile has a full M of 128 whatever the token
 // count, and a tile's N is the expert's token count rounded up to 16 (experts with
-// more than 256 tokens are split evenly into several N-tiles).
+// more than 192 tokens are split evenly into several N-tiles).
 //
-//  * Dequantisation producers (warps 0-7; warp w owns the tile's 16-row block w, two
-//    lanes per row, 32 of the 64 K of a stage each).  Lane 0 of each warp brings its
-//    block's packed data in by bulk copies, one 512-wide K chunk per slot of a
-//    two-slot ring of its own (eight issuing threads keep enough bytes in flight; one
-//    thread alone issues too few copies per microsecond).  The warp reads the row's
-//    code words (plus third bits and the fp16 scale) from the ring, turns them into
-//    fp16 (c - o) * s (exact codes, one rounding) and writes them into the stage's A
-//    tile in the canonical K-major SWIZZLE_128B layout, then fence.proxy.async + one
-//    arrive per warp.
+// The dequantised A tile lives in tensor memory, not shared memory: shared memory then
+// carries only the B tiles and the packed weights, which halves its traffic per stage
+// (with A in shared memory the tile was written and read back every stage).
+//
+//  * Dequantisation producers (warps 0-7; warp w owns TMEM lane quarter w % 4, i.e.
+//    tile rows 32q .. 32q+31 one per lane, and K half w / 4 of every 64-wide stage).
+//    Lane 0 of each warp brings its two 16-row packed blocks in by bulk copies, one
+//    512-wide K chunk per slot of a two-slot ring of its own (eight issuing threads
+//    keep enough bytes in flight).  A lane reads its row's code words (plus third bits
+//    and the fp16 scale) from the ring, turns them into fp16 (c - o) * s (exact codes,
+//    one rounding) and stores the 16 pairs with one tcgen05.st into the stage's A
+//    columns; tcgen05.wait::st + fence, one arrive per warp.
 //  * TMA producer (warp 12): one 2-D tensor-map load per stage for the B tile (K-major,
 //    SWIZZLE_128B) from the gathered fp16 token rows (gate/up) or from h (down),
 //    completion counted in bytes on the stage's mbarrier.
-//  * MMA issuer (warp 13, one thread): per stage four tcgen05.mma.kind::f16 (K = 16
-//    each), fp32 accumulation in TMEM; tcgen05.commit releases the stage to the
-//    producers and, after the last stage, hands the accumulator to the epilogue.
-//    Two accumulators of 256 TMEM columns alternate between tiles, so the epilogue
-//    of one tile overlaps the main loop of the next.
+//  * MMA issuer (warp 13, one elected lane): per stage four tcgen05.mma.kind::f16
+//    (K = 16 each) with A from tensor memory and B from shared memory, fp32
+//    accumulation in TMEM; tcgen05.commit releases the stage to the producers and,
+//    after the last stage, hands the accumulator to the epilogue.  Two accumulators of
+//    192 columns alternate between tiles, so the epilogue of one tile overlaps the main
+//    loop of the next.
 //  * Epilogue (warps 8-11, TMEM lanes 32q..32q+31): tcgen05.ld 16 columns at a time.
 //    gate/up: rows 16b..16b+7 are gate rows and 16b+8..16b+15 the matching up rows,
 //    i.e. TMEM lanes l and l+8 of the same warp: h = silu(gate) * up is formed with
@@ -44,16 +48,20 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128;                       // weight rows per tile (UMMA M)
-constexpr int BN = 256;                       // max tokens per tile (UMMA N)
+constexpr int BN = 192;                       // max tokens per tile (UMMA N)
 constexpr int BK = 64;                        // K per stage (one scale group)
-constexpr int NSTG = 3;                       // A/B pipeline stages
-constexpr int A_BYTES = BM * BK * 2;          // 16 KB
-constexpr int B_BYTES = BN * BK * 2;          // 32 KB
-constexpr int STG_BYTES = A_BYTES + B_BYTES;  // 48 KB
-// Per-warp packed ring: each dequantiser warp streams its own 16-row block, one
-// 8-group chunk (codes, third bits, scales of the packed format) per slot.
+constexpr int NSTG = 4;                       // pipeline stages
+constexpr int B_BYTES = BN * BK * 2;          // 24 KB: a stage's shared memory is its B tile
+constexpr int STG_BYTES = B_BYTES;
+// Tensor memory (512 columns x 128 lanes x 32 bit): two fp32 accumulators of BN
+// columns, then NSTG A stages of 32 columns (128 rows x 64 fp16, two per column).
+constexpr uint32_t kACol0 = 2 * BN;
+static_assert(kACol0 + 32 * NSTG <= 512, "TMEM columns");
+// Per-warp packed ring: each dequantiser warp streams the two 16-row blocks of its TMEM
+// lane quarter, one 8-group chunk (codes, third bits, scales of the packed format) of
+// both per slot.
 constexpr int NP = 2;
-constexpr int PK_CODES = 0, PK_HI = 2048, PK_SC = 3072, PK_BYTES = 3328;
+constexpr int PK_CODES = 0, PK_HI = 2048, PK_SC = 3072, PK_BYTES = 3328, PKW_BYTES = 2 * PK_BYTES;
 constexpr int kThreads = 448;                 // 14 warps
 constexpr int kDqWarps = 8, kEpiWarp0 = 8, kTmaWarp = 12, kMmaWarp = 13;   // warps 8-11: epilogue
 
@@ -61,9 +69,10 @@ constexpr int kDqWarps = 8, kEpiWarp0 = 8, kTmaWarp = 12, kMmaWarp = 13;   // wa
 // rows) is the smallest that covers the tile's tokens.  A single thread issues bulk
 // loads at a limited rate, so one large box beats several small ones.
 struct BMaps {
-    CUtensorMap m[3];   // box rows 64, 128, 256
+    CUtensorMap m[3];   // box rows 64, 128, BN
 };
 __device__ inline int box_index(int n) { return n <= 64 ? 0 : (n <= 128 ? 1 : 2); }
+__host__ __device__ constexpr int box_rows(int i) { return i == 0 ? 64 : (i == 1 ? 128 : BN); }
 constexpr long long kWaitLimit = 4000000000LL;
 
 constexpr uint32_t kH512 = 0x60006000u, kH256 = 0x5C005C00u, kH64 = 0x54005400u, kH16 = 0x4C004C00u,
@@ -134,13 +143,26 @@ __device__ inline uint32_t instr_desc(int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-__device__ inline void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+// D[M = 128][N] (+)= A[M][K = 16] B[N][K]^T with A read from tensor memory (128 lanes =
+// rows, 8 columns = 16 fp16 along K) and B from shared memory (descriptor).
+__device__ inline void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
         : "memory");
 }
+
+// Each thread writes 16 consecutive 32-bit columns of its own TMEM lane.
+__device__ inline void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ inline void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ inline void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -164,7 +186,6 @@ __device__ inline void tma_load_2d(void* dst, const CUtensorMap* map, int x, int
         : "memory");
 }
 
-__device__ inline void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ inline const PackedEntry* entry(const uint8_t* packed, int e) {
     return reinterpret_cast<const PackedEntry*>(packed + kHeaderBytes + (size_t)e * kEntryBytes);
@@ -291,11 +312,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
 
     if (warp < kDqWarps) {
         // ======================= dequantisation producers (A) =======================
-        const int r16 = lane >> 1, hh = lane & 1, rs = r16 & 7;
-        const int i = 16 * warp + r16;                 // row within the tile
-        uint8_t* const ring = smem + (size_t)NSTG * STG_BYTES + (size_t)warp * NP * PK_BYTES;
+        // Warp w writes TMEM lane quarter q = w % 4 (tile rows 32q .. 32q+31, one per
+        // lane) and K half kh = w / 4 of every stage (columns 16 kh .. 16 kh + 15 of the
+        // stage's 32); a lane's row is row r16 of packed block 2q + blk.
+        const int q = warp & 3, kh = warp >> 2;
+        const int blk = lane >> 4, r16 = lane & 15, rs = r16 & 7;
+        uint8_t* const ring = smem + (size_t)NSTG * STG_BYTES + (size_t)warp * NP * PKW_BYTES;
         uint64_t* const pfull = pk_full[warp];
-        // Issue cursor (lane 0): the next (tile, chunk) of this warp's block to bring in.
+        const uint32_t a_lane = tmem + ((uint32_t)(32 * q) << 16) + kACol0 + 16 * kh;
+        // Issue cursor: the next (tile, chunk) of this warp's two blocks to bring in.
         struct Cursor {
             int tile, c;
             const uint8_t *cb, *hb, *sb;
@@ -305,26 +330,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
             if (u.tile >= n_tiles) return;
             const TileInfo ti = tile_info(S, p, u.tile, mtiles);
             const PackedEntry* en = entry(p.packed, ti.e);
-            const int j = ti.mt * (BM / 16) + warp;
+            const int j = ti.mt * (BM / 16) + 2 * q;
             u.cb = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes) + (size_t)4 * K * j;
             u.hb = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi) + (size_t)128 * G * j;
             u.sb = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales) + (size_t)256 * NC * j;
             u.q3 = ti.f == MOE_FMT_Q3;
         };
         int issued = 0, consumed = 0;
-        // (whole warp, converged) bring the cursor's chunk into slot issued % NP and
-        // advance the cursor; one elected lane issues the copies
+        // (whole warp, converged) bring the cursor's chunk of both blocks into slot
+        // issued % NP and advance the cursor; one elected lane issues the copies
         auto issue = [&]() {
             if (cur.tile >= n_tiles) return;
             const int ps = issued % NP;
             const int ng = min(8, G - 8 * cur.c);
             const uint32_t cbytes = 256 * ng, hbytes = cur.q3 ? 128 * ng : 0;
-            uint8_t* dst = ring + (size_t)ps * PK_BYTES;
+            uint8_t* dst = ring + (size_t)ps * PKW_BYTES;
             if (elect_one()) {
-                mbar_arrive_expect_tx(&pfull[ps], cbytes + hbytes + 256);
-                bulk_g2s(dst + PK_CODES, cur.cb + 2048 * (size_t)cur.c, cbytes, &pfull[ps]);
-                bulk_g2s(dst + PK_SC, cur.sb + 256 * (size_t)cur.c, 256, &pfull[ps]);
-                if (hbytes) bulk_g2s(dst + PK_HI, cur.hb + 1024 * (size_t)cur.c, hbytes, &pfull[ps]);
+                mbar_arrive_expect_tx(&pfull[ps], 2 * (cbytes + hbytes + 256));
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    uint8_t* d = dst + b * PK_BYTES;
+                    bulk_g2s(d + PK_CODES, cur.cb + (size_t)4 * K * b + 2048 * (size_t)cur.c, cbytes, &pfull[ps]);
+                    bulk_g2s(d + PK_SC, cur.sb + (size_t)256 * NC * b + 256 * (size_t)cur.c, 256, &pfull[ps]);
+                    if (hbytes)
+                        bulk_g2s(d + PK_HI, cur.hb + (size_t)128 * G * b + 1024 * (size_t)cur.c, hbytes, &pfull[ps]);
+                }
             }
             __syncwarp();
             ++issued;
@@ -338,11 +368,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         cur.c = 0;
         load_tile(cur);
         for (int d = 0; d < NP; ++d) issue();
-        // A-tile row of this lane and the 16-byte chunks its two quarters land in
-        // (SWIZZLE_128B: chunk index XOR row % 8)
-        const uint32_t arow_off = (i >> 3) * 1024 + (i & 7) * 128;
-        const uint32_t ch[4] = {(uint32_t)(((4 * hh) ^ (i & 7)) * 16), (uint32_t)(((4 * hh + 1) ^ (i & 7)) * 16),
-                                (uint32_t)(((4 * hh + 2) ^ (i & 7)) * 16), (uint32_t)(((4 * hh + 3) ^ (i & 7)) * 16)};
         int slot = 0;
         uint32_t eph = 1;                              // parity of the empty phase awaited
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -361,10 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
                 if (lane == 0 && !mbar_try_wait(&pfull[ps], (consumed / NP) & 1))
                     wait_or_flag(S, &pfull[ps], (consumed / NP) & 1, p, kDetWaitFull | 0x40 | MODE);
                 __syncwarp();
-                const uint8_t* pk = ring + (size_t)ps * PK_BYTES;
+                const uint8_t* pk = ring + (size_t)ps * PKW_BYTES + blk * PK_BYTES;
                 // this lane's 2 code words, third-bit word and the row's scales of the chunk
-                const uint8_t* cw_base = pk + PK_CODES + (ng == 8 ? r16 * 128 : r16 * 16 * ng) + 8 * hh;
-                const uint8_t* hw_base = pk + PK_HI + (ng == 8 ? r16 * 64 : r16 * 8 * ng) + 4 * hh;
+                const uint8_t* cw_base = pk + PK_CODES + (ng == 8 ? r16 * 128 : r16 * 16 * ng) + 8 * kh;
+                const uint8_t* hw_base = pk + PK_HI + (ng == 8 ? r16 * 64 : r16 * 8 * ng) + 4 * kh;
                 const uint16_t* sc_base = reinterpret_cast<const uint16_t*>(pk + PK_SC + r16 * 16);
                 auto load = [&](int gl, uint2& cw, uint32_t& hw, uint32_t& s2) {
                     const int cpos = ng == 8 ? gl ^ rs : gl;
@@ -381,34 +406,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
                     uint2 cw_n = cw;
                     uint32_t hw_n = hw, s2_n = s2;
                     if (gl + 1 < ng) load(gl + 1, cw_n, hw_n, s2_n);
-                    uint32_t pr[2][8];
+                    // fp16 (c - o) * s of K elements 32 kh .. 32 kh + 31 of this group, as
+                    // 16 pairs in K order (quarter qq of the half -> columns 8 qq .. 8 qq + 7)
+                    uint32_t r[16];
                     const uint32_t words[2] = {cw.x, cw.y};
 #pragma unroll
                     for (int qq = 0; qq < 2; ++qq) {
-                        codes_f16(words[qq], sub, pr[qq]);
+                        uint32_t pr[8];
+                        codes_f16(words[qq], sub, pr);
                         if (q3) {
                             uint32_t hp[8];
                             hi_f16(hw >> (8 * qq), hp);
 #pragma unroll
-                            for (int v = 0; v < 8; ++v) pr[qq][v] = f16x2_add(pr[qq][v], hp[v]);
+                            for (int v = 0; v < 8; ++v) pr[v] = f16x2_add(pr[v], hp[v]);
                         }
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) pr[qq][v] = f16x2_mul(pr[qq][v], s2);
+                        for (int v = 0; v < 8; ++v) r[8 * qq + v] = f16x2_mul(pr[v], s2);
                     }
                     // only now wait for the stage's slot
                     if (lane == 0 && !mbar_try_wait(&empty_[slot], eph))
                         wait_or_flag(S, &empty_[slot], eph, p, kDetWaitEmpty | 0x10 | MODE);
                     __syncwarp();
-                    uint8_t* arow = smem + (size_t)slot * STG_BYTES + arow_off;
-                    // quarter q = 2hh + qq: elements 16q..16q+7 -> chunk 2q, 16q+8.. -> 2q+1
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        *reinterpret_cast<uint4*>(arow + ch[2 * qq]) =
-                            make_uint4(pr[qq][0], pr[qq][1], pr[qq][2], pr[qq][3]);
-                        *reinterpret_cast<uint4*>(arow + ch[2 * qq + 1]) =
-                            make_uint4(pr[qq][4], pr[qq][5], pr[qq][6], pr[qq][7]);
-                    }
-                    fence_proxy_async();
+                    tmem_st16(a_lane + 32 * slot, r);
+                    tmem_wait_st();
+                    tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&full_a[slot]);
                     if (++slot == NSTG) {
@@ -419,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
                     hw = hw_n;
                     s2 = s2_n;
                 }
-                // every lane has read the slot: lane 0 refills it with the chunk NP ahead
+                // every lane has read the slot: refill it with the chunk NP ahead
                 __syncwarp();
                 ++consumed;
                 if (!ld_volatile(S.abort_flag)) issue();
@@ -443,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
             const int bx = box_index(ti.N);
-            const uint32_t bbytes = (64u << bx) * BK * 2;
+            const uint32_t bbytes = (uint32_t)box_rows(bx) * BK * 2;
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 if (!mbar_try_wait(&empty_[slot], eph))
                     wait_or_flag(S, &empty_[slot], eph, p, kDetWaitEmpty | 0x20 | MODE);
@@ -451,8 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
                 if (!ld_volatile(S.abort_flag)) {
                     if (elect_one()) {
                         mbar_arrive_expect_tx(&full_b[slot], bbytes);
-                        tma_load_2d(smem + (size_t)slot * STG_BYTES + A_BYTES, &bmaps.m[bx], ks * BK, ti.row0,
-                                    &full_b[slot]);
+                        tma_load_2d(smem + (size_t)slot * STG_BYTES, &bmaps.m[bx], ks * BK, ti.row0, &full_b[slot]);
                     }
                     __syncwarp();
                     issued = it + 1;
@@ -480,8 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         // path is short, since it bounds the stage rate: slot and phase advance
         // incrementally, descriptors are precomputed, and the bounded wait is entered
         // only when the barrier is not already complete.
-        const uint64_t a_desc0 = smem_desc(smem_u32(smem));
-        constexpr uint32_t kSlotStep = STG_BYTES >> 4, kBOff = A_BYTES >> 4;
+        const uint64_t b_desc0 = smem_desc(smem_u32(smem));
+        constexpr uint32_t kSlotStep = STG_BYTES >> 4;
         int slot = 0, tc = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -501,12 +521,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
                 if (!mbar_try_wait(&full_b[slot], phase))
                     ok &= wait_or_flag(S, &full_b[slot], phase, p, kDetWaitFull | 0x20 | MODE);
                 ok = __all_sync(0xffffffffu, ok);
-                const uint64_t ad = a_desc0 + (uint64_t)(slot * kSlotStep), bd = ad + kBOff;
+                tc_fence_after();                       // A was written by tcgen05.st of other warps
+                const uint32_t a_tm = tmem + kACol0 + 32 * slot;
+                const uint64_t bd = b_desc0 + (uint64_t)(slot * kSlotStep);
                 if (elect_one()) {
                     if (ok) {
 #pragma unroll
                         for (int k16 = 0; k16 < BK / 16; ++k16)
-                            umma_f16(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, (ks | k16) != 0 ? 1u : 0u);
+                            umma_f16_ts(d_tmem, a_tm + 8 * k16, bd + 2 * k16, idesc, (ks | k16) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty_[slot]);
                 }
@@ -527,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         // =============================== epilogue ====================================
         const int q = warp & 3;                       // TMEM lanes 32q .. 32q+31 (warps 8-11)
         uint16_t* const stg = reinterpret_cast<uint16_t*>(smem + (size_t)NSTG * STG_BYTES +
-                                                           (size_t)kDqWarps * NP * PK_BYTES) + q * 256;
+                                                           (size_t)kDqWarps * NP * PKW_BYTES) + q * 256;
         int tc = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
@@ -630,11 +652,11 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_r
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kTcSmem = (size_t)NSTG * STG_BYTES + (size_t)kDqWarps * NP * PK_BYTES + 4 * 512 + 1024;
+constexpr size_t kTcSmem = (size_t)NSTG * STG_BYTES + (size_t)kDqWarps * NP * PKW_BYTES + 4 * 512 + 1024;
 
 bool make_maps(BMaps* b, const void* base, long long rows, int K) {
-    return make_map(&b->m[0], base, rows, K, 64) && make_map(&b->m[1], base, rows, K, 128) &&
-           make_map(&b->m[2], base, rows, K, 256);
+    return make_map(&b->m[0], base, rows, K, box_rows(0)) && make_map(&b->m[1], base, rows, K, box_rows(1)) &&
+           make_map(&b->m[2], base, rows, K, box_rows(2));
 }
 
 template <int MODE>
