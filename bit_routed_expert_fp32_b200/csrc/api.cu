@@ -35,8 +35,20 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     off = align256(off + 4 * (size_t)(3 * (H / 64) * T));
     w.h = off;
     off = align256(off + 2 * (size_t)(T * (k + S) * I));
+    // ypart, and the decode gate/up partial sums that alias it: the largest need of any
+    // token count up to T (the split into K parts shrinks as T grows), so a workspace
+    // sized for T tokens serves every smaller T.
+    size_t yfl = (size_t)(T * (k + S) * H);
+    for (int64_t t = 1; t <= T && t <= kSmallT; ++t) {
+        int ngu = 1, ndn = 1;
+        decode_kparts(s, t, &ngu, &ndn);
+        const size_t rows = (size_t)(t * (k + S));
+        const size_t need_dn = (size_t)ndn * rows * H, need_gu = ngu > 1 ? (size_t)ngu * rows * 2 * I : 0;
+        yfl = yfl > need_dn ? yfl : need_dn;
+        yfl = yfl > need_gu ? yfl : need_gu;
+    }
     w.ypart = off;
-    off = align256(off + 4 * (size_t)(T * (k + S) * H));
+    off = align256(off + 4 * yfl);
     w.total = off;
     return w;
 }
@@ -178,6 +190,8 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.h = reinterpret_cast<uint16_t*>(ws + w.h);
     a.ypart = reinterpret_cast<float*>(ws + w.ypart);
+    a.gpart = a.ypart;
+    a.nkp_gu = a.nkp_dn = 1;
     a.tile_ctr = reinterpret_cast<uint32_t*>(ws + w.tile_ctr);
     a.y = d_y;
     a.num_ctas = sm_count();
@@ -189,6 +203,7 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     const bool tc_ok = a.H % 128 == 0 && (2 * a.I) % 128 == 0;
     if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
     const bool prefill = path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kSmallT && tc_ok);
+    if (!prefill) decode_kparts(shape, T, &a.nkp_gu, &a.nkp_dn);
     cudaError_t err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
                               : launch_ffn_decode(a, s, ev[1], ev[2]);
     if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;

@@ -8,33 +8,41 @@
 // expert once for its 4-8 tokens).  So every selected expert's packed bytes are
 // streamed exactly once and applied to all of its tokens:
 //
-//  * Work item = (active expert, 16-row tile of the packed matrix, token pass of up
-//    to 8*NT tokens).  Every warp owns whole items (items w, w + P, w + 2P, ... for P
-//    warps in the grid) and walks the full K of each; no two warps share an item, so
-//    there is no cross-warp reduction and no CTA-wide barrier in the main loop.
-//  * Each warp streams its items through its own ring of NS shared-memory stages with
+//  * Work unit = (active expert, 32-row block = two 16-row tiles of the packed
+//    matrix, K part, token pass of up to 8 tokens).  With one or two tokens there are
+//    fewer 32-row blocks than warps on the GPU, so K is cut into parts (whole 8-group
+//    chunks) and every part writes its own fp32 partial sums; the parts are added in
+//    a fixed order afterwards (finalize_gateup_kernel, combine_kernel), so the result
+//    does not depend on which warp ran what.  Units are dealt round-robin to the
+//    warps of a persistent grid (one CTA of 16 warps per SM), CTAs first.  An expert
+//    with more than 8 tokens has one unit per pass; the passes of a block are
+//    consecutive units, which start together on neighbouring SMs, so the block's
+//    bytes come from HBM once and from L2 for the other passes.
+//  * Each warp streams its units through its own ring of NS shared-memory stages with
 //    1-D bulk copies (cp.async.bulk on the TMA engine, completion on a per-stage
-//    mbarrier); a stage holds one 8-group (512-wide) chunk of K for the 16 rows:
-//    codes, third bits and fp16 scales, each a contiguous block of the packed format
-//    (three copies per chunk).  The format's XOR swizzle keeps the fragment reads
-//    free of bank conflicts.  The ring runs NS-1 chunks ahead, across items.
-//  * A 32-bit code word (16 codes of one row) becomes eight bf16 / fp16 pairs with
-//    shifts and lop3 (magic-number exponent trick: the code lands in the mantissa of
-//    a power-of-two base, exactly), the A operand of mma.sync m16n8k16; the tokens
-//    are N (8 per n-tile) and the B fragments come straight from the token rows.
-//      gate/up: pairs stay "base + c"; each 64-wide group's accumulator starts at
+//    mbarrier); a stage holds one 8-group (512-wide) chunk of K for both tiles:
+//    codes, third bits and fp16 scales, each a contiguous block of the packed format.
+//    The format's XOR swizzle keeps the fragment reads free of bank conflicts.  The
+//    ring runs ahead across units; there is no CTA-wide barrier in the main loop.
+//  * A full chunk is processed fully unrolled: per 64-wide group and tile, two code
+//    words become sixteen bf16 / fp16 pairs with shifts and lop3 (magic-number
+//    exponent trick: the code lands in the mantissa of a power-of-two base, exactly),
+//    the A operand of mma.sync m16n8k16; the tokens are N (8 per n-tile) and the B
+//    fragments come straight from the token rows (L1-resident).
+//      gate/up: pairs stay "base + c"; each group's accumulator starts at
 //        -Z[token, group] (Z = sum base(k) x_k + o sum x_k, plus the third-bit bases
 //        for 3-bit experts; computed by the router), so the MMA yields
 //        sum (c_k - o) x_k.  bf16 MMAs: the tokens are bf16.
 //      down: pairs are (c - o) exactly (one fp16x2 subtract); fp16 MMAs, h is fp16.
 //    Each group result is scaled by its fp16 scale into an fp32 accumulator.
-//    3-bit experts add an MMA for 4 * (third bit).
+//    3-bit experts add an MMA per k-step for 4 * (third bit).
 //  * gate/up: the 16 rows of a tile are 8 gate rows and the matching 8 up rows, which
-//    the MMA places in the same thread (rows g and g + 8), so h = silu(gate) * up is
-//    formed in registers and stored as fp16.
-//  * down: partial rows (fp32) per (token, slot); the combine kernel then sums each
-//    token's k slots in slot order with the gates, adds the shared expert and writes
-//    y in bf16: deterministic, no floating-point atomics.
+//    the MMA places in the same thread (rows g and g + 8), so with a single K part
+//    h = silu(gate) * up is formed in registers and stored as fp16; with several K
+//    parts the raw sums go to gpart and finalize_gateup_kernel forms h.
+//  * down: partial rows (fp32) per (K part, token, slot); the combine kernel then
+//    sums the parts, each token's k slots in slot order with the gates, adds the
+//    shared expert and writes y in bf16: deterministic, no floating-point atomics.
 // Every wait is bounded; a wait that runs out records an error in the workspace and
 // the warp carries on without waiting, so the kernel always terminates.
 #include "kernels.h"
@@ -45,13 +53,17 @@ namespace {
 constexpr int CG = 8;                                  // 64-wide groups per chunk
 constexpr int OFF_HI = 2048;                           // codes block: 16 rows x 32 words
 constexpr int OFF_SC = OFF_HI + 1024;                  // third-bit block: 16 rows x 16 words
-constexpr int STAGE = OFF_SC + 256;                    // scales block: 16 rows x 8 halves
-constexpr int NS = 4;                                  // stages per warp (power of two)
+constexpr int TSTAGE = OFF_SC + 256;                   // scales block: 16 rows x 8 halves
+constexpr int NTL = 2;                                 // 16-row tiles per block
+constexpr int STAGE = NTL * TSTAGE;                    // one chunk of both tiles of a block
+constexpr int NW = 16;                                 // warps per CTA
+constexpr int NS = 2;                                  // stages per warp
+constexpr int TP = 8;                                  // tokens per pass (one n-tile)
 constexpr long long kWaitLimit = 4000000000LL;         // clock cycles (~2 s)
 
 // bf16 magic bases (exponent-only bit patterns) of the gate/up dequantiser
-constexpr uint32_t kMag64 = 0x42804280u, kMag32 = 0x42004200u, kMag16 = 0x41804180u, kMag8 = 0x41004100u,
-                   kMag4 = 0x40804080u, kMag512 = 0x44004400u, kMag256 = 0x43804380u, kMag128 = 0x43004300u;
+constexpr uint32_t kMag128 = 0x43004300u, kMag32 = 0x42004200u, kMag8 = 0x41004100u, kMag64 = 0x42804280u,
+                   kMag16 = 0x41804180u, kMag512 = 0x44004400u, kMag256 = 0x43804380u;
 // fp16 magic bases of the down dequantiser
 constexpr uint32_t kH512 = 0x60006000u, kH256 = 0x5C005C00u, kH64 = 0x54005400u, kH16 = 0x4C004C00u,
                    kH4 = 0x44004400u, kH4096 = 0x6C006C00u, kH2048 = 0x68006800u, kH1024 = 0x64006400u,
@@ -59,22 +71,23 @@ constexpr uint32_t kH512 = 0x60006000u, kH256 = 0x5C005C00u, kH64 = 0x54005400u,
 
 // ---- dequantisers (code word: element 2p + h of its 16 at bits 16h + 2p .. +1) ----
 
-// bf16 pairs "base_p + c"; base per pair p: 64, 32, 8, 16, 4, 64, 16, 4.
-__device__ inline void raw_codes_bf16(uint32_t w, uint32_t (&pr)[8]) {
-    const uint32_t w1 = w << 1, w3 = w >> 3, w9 = w >> 9;
-    pr[0] = lop3_and_or(w1, 0x00060006u, kMag64);   // bits 0-1 -> 1-2
-    pr[1] = lop3_and_or(w, 0x000C000Cu, kMag32);    // bits 2-3
-    pr[2] = lop3_and_or(w, 0x00300030u, kMag8);     // bits 4-5
-    pr[3] = lop3_and_or(w3, 0x00180018u, kMag16);   // bits 6-7 -> 3-4
-    pr[4] = lop3_and_or(w3, 0x00600060u, kMag4);    // bits 8-9 -> 5-6
-    pr[5] = lop3_and_or(w9, 0x00060006u, kMag64);   // bits 10-11 -> 1-2
-    pr[6] = lop3_and_or(w9, 0x00180018u, kMag16);   // bits 12-13 -> 3-4
-    pr[7] = lop3_and_or(w9, 0x00600060u, kMag4);    // bits 14-15 -> 5-6
+// bf16 pairs "base_p + c"; base per pair p: 128, 32, 8, 128, 32, 8, 128, 32 (a code
+// at mantissa bits 0-1 / 2-3 / 4-5 of 128 / 32 / 8 has weight exactly 1).
+__device__ __forceinline__ void raw_codes_bf16(uint32_t w, uint32_t (&pr)[8]) {
+    const uint32_t w6 = w >> 6, w12 = w >> 12;
+    pr[0] = lop3_and_or(w, 0x00030003u, kMag128);     // bits 0-1
+    pr[1] = lop3_and_or(w, 0x000C000Cu, kMag32);      // bits 2-3
+    pr[2] = lop3_and_or(w, 0x00300030u, kMag8);       // bits 4-5
+    pr[3] = lop3_and_or(w6, 0x00030003u, kMag128);    // bits 6-7 -> 0-1
+    pr[4] = lop3_and_or(w6, 0x000C000Cu, kMag32);     // bits 8-9 -> 2-3
+    pr[5] = lop3_and_or(w6, 0x00300030u, kMag8);      // bits 10-11 -> 4-5
+    pr[6] = lop3_and_or(w12, 0x00030003u, kMag128);   // bits 12-13 -> 0-1
+    pr[7] = lop3_and_or(w12, 0x000C000Cu, kMag32);    // bits 14-15 -> 2-3
 }
 
 // bf16 pairs "base_p + 4 * bit" of the third code bit (bits 0..7 of each half of u);
 // base per pair p: 512, 256, 128, 64, 32, 16, 8, 8.
-__device__ inline void raw_hi_bf16(uint32_t u, uint32_t (&pr)[8]) {
+__device__ __forceinline__ void raw_hi_bf16(uint32_t u, uint32_t (&pr)[8]) {
     pr[0] = lop3_and_or(u, 0x00010001u, kMag512);
     pr[1] = lop3_and_or(u, 0x00020002u, kMag256);
     pr[2] = lop3_and_or(u, 0x00040004u, kMag128);
@@ -86,7 +99,7 @@ __device__ inline void raw_hi_bf16(uint32_t u, uint32_t (&pr)[8]) {
 }
 
 // fp16 pairs (c - o), exact: the bases 512, 256, 64, 16, 4 have an ulp <= 1/2.
-__device__ inline void exact_codes_f16(uint32_t w, const uint32_t (&sub)[5], uint32_t (&pr)[8]) {
+__device__ __forceinline__ void exact_codes_f16(uint32_t w, const uint32_t (&sub)[5], uint32_t (&pr)[8]) {
     const uint32_t w1 = w << 1, w8 = w >> 8;
     pr[0] = f16x2_sub(lop3_and_or(w1, 0x00060006u, kH512), sub[0]);    // bits 0-1 -> 1-2
     pr[1] = f16x2_sub(lop3_and_or(w, 0x000C000Cu, kH256), sub[1]);     // bits 2-3
@@ -99,7 +112,7 @@ __device__ inline void exact_codes_f16(uint32_t w, const uint32_t (&sub)[5], uin
 }
 
 // fp16 pairs 4 * (third bit), exact.
-__device__ inline void exact_hi_f16(uint32_t u, uint32_t (&pr)[8]) {
+__device__ __forceinline__ void exact_hi_f16(uint32_t u, uint32_t (&pr)[8]) {
     pr[0] = f16x2_sub(lop3_and_or(u, 0x00010001u, kH4096), kH4096);
     pr[1] = f16x2_sub(lop3_and_or(u, 0x00020002u, kH2048), kH2048);
     pr[2] = f16x2_sub(lop3_and_or(u, 0x00040004u, kH1024), kH1024);
@@ -110,21 +123,402 @@ __device__ inline void exact_hi_f16(uint32_t u, uint32_t (&pr)[8]) {
     pr[7] = f16x2_sub(lop3_and_or(u, 0x00800080u, kH32), kH32);
 }
 
-// L1 prefetch of chunk c's token lines and Z values for this lane's columns: lane t of a
-// row takes the 128-byte lines of groups t and t + 4 (the row's B operand for the
-// chunk is 8 lines), so the loads of the chunk hit L1 instead of waiting on L2.
-// Only groups inside the row are touched (a partial last chunk has fewer).
-template <int MODE, int NT, typename View>
-__device__ inline void prefetch_chunk(const View& v, int c, int t, int G) {
-    const int ng = min(CG, G - c * CG);
+// Rows g (wa) and g + 8 (wb) straight into MMA A-fragment order: k-step s uses
+// {pair 2s of wa, pair 2s of wb, pair 2s+1 of wa, pair 2s+1 of wb}.
+template <int MODE>
+__device__ __forceinline__ void dequant_rows(uint32_t wa, uint32_t wb, const uint32_t (&sub)[5], uint32_t (&pa)[8],
+                                             uint32_t (&pb)[8]) {
+    if (MODE == 0) {
+        raw_codes_bf16(wa, pa);
+        raw_codes_bf16(wb, pb);
+    } else {
+        exact_codes_f16(wa, sub, pa);
+        exact_codes_f16(wb, sub, pb);
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ void dequant_hi_rows(uint32_t ua, uint32_t ub, uint32_t (&pa)[8], uint32_t (&pb)[8]) {
+    if (MODE == 0) {
+        raw_hi_bf16(ua, pa);
+        raw_hi_bf16(ub, pb);
+    } else {
+        exact_hi_f16(ua, pa);
+        exact_hi_f16(ub, pb);
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ void mma_acc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+    if (MODE == 0)
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The four k-steps of one 64-wide group of one tile against one n-tile (xb: the B
+// fragments of the group, pairs 0..7 of this lane's 16 elements).
+template <int MODE>
+__device__ __forceinline__ void mma_group(float (&d)[4], const uint32_t (&pa)[8], const uint32_t (&pb)[8],
+                                          const uint4& x0, const uint4& x1) {
+    mma_acc<MODE>(d, pa[0], pb[0], pa[1], pb[1], x0.x, x0.y);
+    mma_acc<MODE>(d, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
+    mma_acc<MODE>(d, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
+    mma_acc<MODE>(d, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
+}
+
+__device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xFFFFu))); }
+__device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w >> 16))); }
+__device__ __forceinline__ const PackedEntry* entry(const uint8_t* packed, int e) {
+    return reinterpret_cast<const PackedEntry*>(packed + kHeaderBytes + (size_t)e * kEntryBytes);
+}
+
+// ---- the CTA's copy of the schedule -------------------------------------------------
+constexpr int kMaxActive = 260;
+constexpr int kPermSmem = 1024;                        // routed pairs staged in shared memory
+
+struct CtaSched {
+    int ok;
+    int n_active;
+    int n_units;
+    int perm_in_smem;
+    int e[kMaxActive];
+    int fmt[kMaxActive];
+    int cnt[kMaxActive];       // tokens of the expert
+    int off[kMaxActive];       // first permuted row (routed experts)
+    int upre[kMaxActive + 1];  // unit prefix over active experts
+    int tok[kPermSmem];        // source token of permuted row r (perm[r] / k)
+};
+
+struct UnitPos {
+    int a, pass, jb, kp;
+};
+
+// Units are ordered (active expert, 32-row block, K part, token pass), pass fastest.
+__device__ __forceinline__ UnitPos unit_pos(const CtaSched& S, int u, int blocks, int nkp) {
+    int lo = 0, hi = S.n_active - 1;                   // largest a with upre[a] <= u
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (S.upre[mid] <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    UnitPos q;
+    q.a = lo;
+    int r = u - S.upre[lo];
+    const int np = (S.cnt[lo] + TP - 1) / TP;
+    q.pass = r % np;
+    r /= np;
+    q.kp = r % nkp;
+    q.jb = r / nkp;
+    return q;
+}
+
+// Walks consecutive units (pass fastest, then K part, block, expert) without
+// divisions; seek() places it on any unit.
+struct UnitIt {
+    int u, a, jb, kp, pass, np;
+    __device__ __forceinline__ void seek(const CtaSched& S, int u0, int blocks, int nkp) {
+        u = u0;
+        if (u0 >= S.n_units) return;
+        const UnitPos q = unit_pos(S, u0, blocks, nkp);
+        a = q.a;
+        jb = q.jb;
+        kp = q.kp;
+        pass = q.pass;
+        np = (S.cnt[a] + TP - 1) / TP;
+    }
+    __device__ __forceinline__ void next(const CtaSched& S, int blocks, int nkp) {
+        ++u;
+        if (++pass < np) return;
+        pass = 0;
+        if (++kp < nkp) return;
+        kp = 0;
+        if (++jb < blocks) return;
+        jb = 0;
+        if (++a < S.n_active) np = (S.cnt[a] + TP - 1) / TP;
+    }
+};
+
+__device__ __forceinline__ int src_token(const FfnArgs& p, const CtaSched& S, int row) {
+    return S.perm_in_smem ? S.tok[row] : __ldg(p.perm + row) / p.k;
+}
+
+// Per-lane view of one unit: B row, -Z rows and output rows of this lane's columns.
+struct UnitView {
+    const uint16_t* b;         // B-operand row of token column g (+16t elements)
+    const float* z0;           // -Z rows of output columns 2t, 2t+1 (gate/up only)
+    const float* z1;
+    int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token)
+};
+
+// Columns without a token read a valid row (the pass's first token); their MMA
+// outputs are never stored.
+template <int MODE>
+__device__ __forceinline__ void make_view(const FfnArgs& p, const CtaSched& S, int a, int pass, int g, int t,
+                                          UnitView& v) {
+    const int e = S.e[a], f = S.fmt[a], cnt = S.cnt[a];
+    const int tb = pass * TP, nb = min(TP, cnt - tb);
+    const bool routed = e < p.E;
+    const int G = p.H / 64;
+    const int srow0 = p.T * p.k + (e - p.E) * p.T;     // first row of a shared expert
+    const int i = tb + (g < nb ? g : 0);
+    int brow;
+    if (routed) {
+        const int hr = S.off[a] + i;
+        brow = MODE == 0 ? src_token(p, S, hr) : hr;
+    } else {
+        brow = MODE == 0 ? i : srow0 + i;
+    }
+    v.b = (MODE == 0 ? p.x : p.h) + (size_t)brow * (MODE == 0 ? p.H : p.I) + 16 * t;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        const uint16_t* line0 = v.b[n] - 16 * t + c * CG * 64;
-        if (t < ng) prefetch_l1(line0 + 64 * t);
-        if (t + 4 < ng) prefetch_l1(line0 + 64 * (t + 4));
-        if (MODE == 0) {
-            prefetch_l1(v.z[n][0] + c * CG);
-            prefetch_l1(v.z[n][1] + c * CG);
+    for (int cc = 0; cc < 2; ++cc) {
+        const int col = 2 * t + cc;
+        const int ii = tb + (col < nb ? col : 0);
+        const int orow = routed ? S.off[a] + ii : srow0 + ii;
+        v.orow[cc] = col < nb ? orow : -1;
+        const float* zr = nullptr;
+        if (MODE == 0) zr = p.zx + ((size_t)f * p.T + (routed ? src_token(p, S, orow) : ii)) * G;
+        if (cc == 0) v.z0 = zr;
+        else v.z1 = zr;
+    }
+}
+
+// Lane constants for reading a stage: cw_lane = 32g + t and g4 = 4g locate the code
+// words (row g; row g + 8 is 256 words on), hw_lane = 16g + t/2 and g2 = 2(g/2) the
+// third-bit words (row g + 8: 128 words on), sh the third-bit half of this lane.
+struct LaneGeo {
+    int g, t, cw_lane, g4, hw_lane, g2, sh;
+};
+
+// Group gl of a full chunk, every tile of the block: code words from the swizzled
+// stage, the B fragments of the group, the MMAs and the scaled fold into acc.  s2:
+// per tile, the scale words of rows g and g + 8 that hold groups gl & ~1 and gl | 1;
+// HI selects the half of group gl.
+template <int MODE, bool Q3, int HI>
+__device__ __forceinline__ void group_full(const uint8_t* stg, int gl, const uint16_t* bx, const float* zc0,
+                                           const float* zc1, const LaneGeo& L, const uint32_t (&s2)[NTL][2],
+                                           const uint32_t (&sub)[5], float (&acc)[NTL][4]) {
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(stg);
+    const int cpos = L.cw_lane + ((4 * gl) ^ L.g4);
+    uint32_t w[NTL][2], u[NTL][2];
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        w[tl][0] = cw[cpos + tl * (TSTAGE / 4)];
+        w[tl][1] = cw[cpos + tl * (TSTAGE / 4) + 256];
+        u[tl][0] = u[tl][1] = 0;
+    }
+    if (Q3) {
+        const uint32_t* hw = reinterpret_cast<const uint32_t*>(stg + OFF_HI);
+        const int hpos = L.hw_lane + ((2 * gl) ^ L.g2);
+#pragma unroll
+        for (int tl = 0; tl < NTL; ++tl) {
+            u[tl][0] = hw[hpos + tl * (TSTAGE / 4)] >> L.sh;
+            u[tl][1] = hw[hpos + tl * (TSTAGE / 4) + 128] >> L.sh;
+        }
+    }
+    const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(bx + 64 * gl));
+    const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(bx + 64 * gl) + 1);
+    const float z0 = MODE == 0 ? __ldg(zc0 + gl) : 0.f;
+    const float z1 = MODE == 0 ? __ldg(zc1 + gl) : 0.f;
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        uint32_t pa[8], pb[8];
+        dequant_rows<MODE>(w[tl][0], w[tl][1], sub, pa, pb);
+        float d[4] = {z0, z1, z0, z1};
+        mma_group<MODE>(d, pa, pb, x0, x1);
+        if (Q3) {
+            dequant_hi_rows<MODE>(u[tl][0], u[tl][1], pa, pb);
+            mma_group<MODE>(d, pa, pb, x0, x1);
+        }
+        const float s0 = HI ? half_hi(s2[tl][0]) : half_lo(s2[tl][0]);
+        const float s1 = HI ? half_hi(s2[tl][1]) : half_lo(s2[tl][1]);
+        acc[tl][0] = fmaf(s0, d[0], acc[tl][0]);
+        acc[tl][1] = fmaf(s0, d[1], acc[tl][1]);
+        acc[tl][2] = fmaf(s1, d[2], acc[tl][2]);
+        acc[tl][3] = fmaf(s1, d[3], acc[tl][3]);
+    }
+}
+
+// One full 8-group chunk of every tile of a block against this lane's token column,
+// as four steps of two groups (a rolled loop keeps the code inside the instruction
+// cache).  stg: the stage; c: chunk index (selects the B columns and the Z entries).
+template <int MODE, bool Q3>
+__device__ __forceinline__ void chunk_full(const uint8_t* stg, int c, const UnitView& v, const LaneGeo& L,
+                                           const uint32_t (&sub)[5], float (&acc)[NTL][4]) {
+    const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + OFF_SC);   // row r: words 4r .. 4r+3
+    const uint16_t* bx = v.b + c * (CG * 64);
+    const float* zc0 = MODE == 0 ? v.z0 + c * CG : nullptr;
+    const float* zc1 = MODE == 0 ? v.z1 + c * CG : nullptr;
+#pragma unroll 1
+    for (int gp = 0; gp < CG / 2; ++gp) {
+        uint32_t s2[NTL][2];
+#pragma unroll
+        for (int tl = 0; tl < NTL; ++tl) {
+            s2[tl][0] = scw[tl * (TSTAGE / 4) + 4 * L.g + gp];
+            s2[tl][1] = scw[tl * (TSTAGE / 4) + 4 * (L.g + 8) + gp];
+        }
+        group_full<MODE, Q3, 0>(stg, 2 * gp, bx, zc0, zc1, L, s2, sub, acc);
+        group_full<MODE, Q3, 1>(stg, 2 * gp + 1, bx, zc0, zc1, L, s2, sub, acc);
+    }
+}
+
+// A chunk with ng < 8 groups (the last one when K / 64 is not a multiple of 8):
+// unswizzled rows of 4 ng code words and 2 ng third-bit words.
+template <int MODE, bool Q3>
+__device__ __forceinline__ void chunk_partial(const uint8_t* stg, int c, int ng, const UnitView& v,
+                                              const LaneGeo& L, const uint32_t (&sub)[5], float (&acc)[NTL][4]) {
+    const int g = L.g, t = L.t;
+    for (int gl = 0; gl < ng; ++gl) {
+        const uint16_t* bp = v.b + c * (CG * 64) + 64 * gl;
+        const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(bp));
+        const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(bp) + 1);
+        const float z0 = MODE == 0 ? __ldg(v.z0 + c * CG + gl) : 0.f;
+        const float z1 = MODE == 0 ? __ldg(v.z1 + c * CG + gl) : 0.f;
+#pragma unroll
+        for (int tl = 0; tl < NTL; ++tl) {
+            const uint8_t* tb = stg + tl * TSTAGE;
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(tb);
+            const uint32_t* hw = reinterpret_cast<const uint32_t*>(tb + OFF_HI);
+            const uint16_t* scs = reinterpret_cast<const uint16_t*>(tb + OFF_SC);
+            uint32_t pa[8], pb[8];
+            dequant_rows<MODE>(cw[g * 4 * ng + 4 * gl + t], cw[(g + 8) * 4 * ng + 4 * gl + t], sub, pa, pb);
+            float d[4] = {z0, z1, z0, z1};
+            mma_group<MODE>(d, pa, pb, x0, x1);
+            if (Q3) {
+                dequant_hi_rows<MODE>(hw[g * 2 * ng + 2 * gl + (t >> 1)] >> L.sh,
+                                      hw[(g + 8) * 2 * ng + 2 * gl + (t >> 1)] >> L.sh, pa, pb);
+                mma_group<MODE>(d, pa, pb, x0, x1);
+            }
+            const float s0 = __half2float(__ushort_as_half(scs[g * 8 + gl]));
+            const float s1 = __half2float(__ushort_as_half(scs[(g + 8) * 8 + gl]));
+            acc[tl][0] = fmaf(s0, d[0], acc[tl][0]);
+            acc[tl][1] = fmaf(s0, d[1], acc[tl][1]);
+            acc[tl][2] = fmaf(s1, d[2], acc[tl][2]);
+            acc[tl][3] = fmaf(s1, d[3], acc[tl][3]);
+        }
+    }
+}
+
+// Per-launch geometry of one expert pass (gate/up: K = H, rows 2I; down: K = I, rows H).
+struct Geo {
+    int K, G, NC, blocks, nkp, cpk;
+};
+
+// Producer side of a warp's ring: issues the bulk copies of the next chunk of the
+// unit it is on (both tiles of the block: up to six copies), from one elected lane of
+// the converged warp, then moves to the next chunk / unit.
+template <int MODE>
+struct Producer {
+    const uint8_t* codes;
+    const uint8_t* hi;
+    const uint8_t* sc;
+    UnitIt it;
+    int u_end, c, c_end, q3, issued, cur_a;
+    __device__ void begin(const FfnArgs& p, const CtaSched& S, const Geo& geo) {
+        if (it.u >= u_end) return;
+        c = it.kp * geo.cpk;
+        c_end = min(geo.NC, c + geo.cpk);
+        if (it.a != cur_a) {
+            cur_a = it.a;
+            const PackedEntry* en = entry(p.packed, S.e[it.a]);
+            codes = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes);
+            hi = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi);
+            sc = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales);
+            q3 = S.fmt[it.a] == MOE_FMT_Q3;
+        }
+    }
+    __device__ void issue(const FfnArgs& p, const CtaSched& S, const Geo& geo, uint8_t* ring, uint64_t* bar,
+                          uint64_t pol) {
+        if (it.u >= u_end) return;
+        const int st = issued % NS;
+        const int ng = min(CG, geo.G - c * CG);
+        if (elect_one()) {
+            uint8_t* dst = ring + (size_t)st * STAGE;
+            const uint32_t cb = 256 * ng, hb = q3 ? 128 * ng : 0;
+            mbar_arrive_expect_tx(&bar[st], NTL * (cb + hb + 256));
+#pragma unroll
+            for (int tl = 0; tl < NTL; ++tl) {
+                const int j = NTL * it.jb + tl;
+                uint8_t* d = dst + tl * TSTAGE;
+                bulk_g2s_evict_first(d, codes + (size_t)4 * geo.K * j + 2048 * (size_t)c, cb, &bar[st], pol);
+                bulk_g2s_evict_first(d + OFF_SC, sc + (size_t)256 * geo.NC * j + 256 * (size_t)c, 256, &bar[st],
+                                     pol);
+                if (hb)
+                    bulk_g2s_evict_first(d + OFF_HI, hi + (size_t)128 * geo.G * j + 1024 * (size_t)c, hb, &bar[st],
+                                         pol);
+            }
+        }
+        __syncwarp();
+        ++issued;
+        if (++c == c_end) {
+            it.next(S, geo.blocks, geo.nkp);
+            begin(p, S, geo);
+        }
+    }
+};
+
+// One unit: its chunks through the ring, then the epilogue.
+template <int MODE, bool Q3>
+__device__ __forceinline__ void run_unit(const FfnArgs& p, const CtaSched& S, const Geo& geo, const UnitPos& q,
+                                         Producer<MODE>& prod, int& consumed, bool& aborted, uint8_t* ring,
+                                         uint64_t* bar, uint64_t pol, const LaneGeo& L) {
+    UnitView v;
+    make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
+    uint32_t sub[5] = {0, 0, 0, 0, 0};
+    if (MODE == 1) {
+        const int f = S.fmt[q.a];
+        const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
+        sub[0] = f16x2_bits_of(512.f + o);
+        sub[1] = f16x2_bits_of(256.f + o);
+        sub[2] = f16x2_bits_of(64.f + o);
+        sub[3] = f16x2_bits_of(16.f + o);
+        sub[4] = f16x2_bits_of(4.f + o);
+    }
+    float acc[NTL][4];
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) acc[tl][0] = acc[tl][1] = acc[tl][2] = acc[tl][3] = 0.f;
+    const int c0 = q.kp * geo.cpk, c1 = min(geo.NC, c0 + geo.cpk);
+    for (int c = c0; c < c1; ++c) {
+        prod.issue(p, S, geo, ring, bar, pol);
+        const int st = consumed % NS;
+        if (!aborted && !mbar_wait_bounded(&bar[st], (uint32_t)(consumed / NS) & 1, kWaitLimit)) {
+            aborted = true;
+            report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | MODE);
+        }
+        const uint8_t* stg = ring + (size_t)st * STAGE;
+        const int ng = min(CG, geo.G - c * CG);
+        if (ng == CG) chunk_full<MODE, Q3>(stg, c, v, L, sub, acc);
+        else chunk_partial<MODE, Q3>(stg, c, ng, v, L, sub, acc);
+        __syncwarp();          // every lane is done with this stage before it is refilled
+        ++consumed;
+    }
+    // epilogue: tile j = NTL jb + tl, rows g (gate / first half) and g + 8 (up / second half)
+    const size_t R = (size_t)p.T * (p.k + p.S);
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        const int j = NTL * q.jb + tl;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int orow = v.orow[cc];
+            if (orow < 0) continue;
+            if (MODE == 0 && geo.nkp == 1) {
+                p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(silu_f(acc[tl][cc]) * acc[tl][2 + cc]);
+            } else if (MODE == 0) {
+                float* dst = p.gpart + ((size_t)q.kp * R + orow) * (2 * p.I) + j * 16 + L.g;
+                dst[0] = acc[tl][cc];
+                dst[8] = acc[tl][2 + cc];
+            } else {
+                float* dst = p.ypart + ((size_t)q.kp * R + orow) * p.H + j * 16 + L.g;
+                dst[0] = acc[tl][cc];
+                dst[8] = acc[tl][2 + cc];
+            }
         }
     }
 }
@@ -150,287 +544,21 @@ __device__ inline void warm_z(const FfnArgs& p) {
         prefetch_l1(reinterpret_cast<const uint8_t*>(p.zx) + i * 128);
 }
 
-__device__ inline float half_bits_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
-
 template <int MODE>
-__device__ inline void mma4(float& d0, float& d1, float& d2, float& d3, const uint32_t (&pa)[8],
-                            const uint32_t (&pb)[8], const uint32_t (&xb)[8]) {
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        if (MODE == 0)
-            mma_bf16_16816(d0, d1, d2, d3, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], xb[2 * s],
-                           xb[2 * s + 1]);
-        else
-            mma_f16_16816(d0, d1, d2, d3, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], xb[2 * s],
-                          xb[2 * s + 1]);
-    }
-}
-
-__device__ inline const PackedEntry* entry(const uint8_t* packed, int e) {
-    return reinterpret_cast<const PackedEntry*>(packed + kHeaderBytes + (size_t)e * kEntryBytes);
-}
-
-struct CtaSched {
-    int ok;
-    int n_active;
-    int n_items;
-    int e[260];
-    int fmt[260];
-    int cnt[260];
-    int ipre[261];   // item prefix over active experts
-};
-
-__device__ inline int find_active(const CtaSched& S, int item) {
-    int lo = 0, hi = S.n_active - 1;     // largest a with ipre[a] <= item
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (S.ipre[mid] <= item) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
-template <int MODE>
-__device__ inline void mma_acc(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1, uint32_t a2,
-                               uint32_t a3, uint32_t b0, uint32_t b1) {
-    if (MODE == 0)
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    else
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Per-lane view of one work item (16-row tile x token pass).
-template <int NT>
-struct ItemView {
-    const uint16_t* b[NT];     // B-operand row of token column g of n-tile n (+16t elements)
-    const float* z[NT][2];     // -Z rows of output columns 2t, 2t+1 (gate/up only)
-    int orow[NT][2];           // output rows of columns 2t, 2t+1 (-1: no token)
-};
-
-// Dequantise the code words of rows g (wa) and g + 8 (wb) straight into MMA
-// A-fragment order: quad s = {pair 2s of wa, pair 2s of wb, pair 2s+1 of wa, pair 2s+1 of wb}.
-template <int MODE>
-__device__ __forceinline__ void dequant_quads(uint32_t wa, uint32_t wb, const uint32_t (&sub)[5], uint32_t (&q)[16]) {
-    uint32_t pa[8], pb[8];
-    if (MODE == 0) {
-        raw_codes_bf16(wa, pa);
-        raw_codes_bf16(wb, pb);
-    } else {
-        exact_codes_f16(wa, sub, pa);
-        exact_codes_f16(wb, sub, pb);
-    }
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        q[4 * s + 0] = pa[2 * s];
-        q[4 * s + 1] = pb[2 * s];
-        q[4 * s + 2] = pa[2 * s + 1];
-        q[4 * s + 3] = pb[2 * s + 1];
-    }
-}
-
-template <int MODE>
-__device__ __forceinline__ void dequant_hi_quads(uint32_t ua, uint32_t ub, uint32_t (&q)[16]) {
-    uint32_t pa[8], pb[8];
-    if (MODE == 0) {
-        raw_hi_bf16(ua, pa);
-        raw_hi_bf16(ub, pb);
-    } else {
-        exact_hi_f16(ua, pa);
-        exact_hi_f16(ub, pb);
-    }
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        q[4 * s + 0] = pa[2 * s];
-        q[4 * s + 1] = pb[2 * s];
-        q[4 * s + 2] = pa[2 * s + 1];
-        q[4 * s + 3] = pb[2 * s + 1];
-    }
-}
-
-// One 64-wide group: dequantise rows g and g+8, MMA against every n-tile, fold the
-// scaled group result into acc.  wa/wb: code words, ua/ub: third-bit words (already
-// shifted), s0/s1: scales, bx[n]: B row pointers of this group, zc[n]: -Z rows at
-// this group (gate/up).
-template <int MODE, int NT, bool Q3>
-__device__ __forceinline__ void group_step(uint32_t wa, uint32_t wb, uint32_t ua, uint32_t ub, float s0, float s1,
-                                           const uint16_t* const (&bx)[NT], const float* const (&zc)[NT][2],
-                                           const uint32_t (&sub)[5], float (&acc)[NT][4]) {
-    uint32_t q[16], hq[16];
-    dequant_quads<MODE>(wa, wb, sub, q);
-    if (Q3) dequant_hi_quads<MODE>(ua, ub, hq);
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(bx[n]));
-        const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(bx[n]) + 1);
-        float d0, d1, d2, d3;
-        if (MODE == 0) {
-            d0 = __ldg(zc[n][0]);
-            d1 = __ldg(zc[n][1]);
-            d2 = d0;
-            d3 = d1;
-        } else {
-            d0 = d1 = d2 = d3 = 0.f;
-        }
-        mma_acc<MODE>(d0, d1, d2, d3, q[0], q[1], q[2], q[3], b0.x, b0.y);
-        mma_acc<MODE>(d0, d1, d2, d3, q[4], q[5], q[6], q[7], b0.z, b0.w);
-        mma_acc<MODE>(d0, d1, d2, d3, q[8], q[9], q[10], q[11], b1.x, b1.y);
-        mma_acc<MODE>(d0, d1, d2, d3, q[12], q[13], q[14], q[15], b1.z, b1.w);
-        if (Q3) {
-            mma_acc<MODE>(d0, d1, d2, d3, hq[0], hq[1], hq[2], hq[3], b0.x, b0.y);
-            mma_acc<MODE>(d0, d1, d2, d3, hq[4], hq[5], hq[6], hq[7], b0.z, b0.w);
-            mma_acc<MODE>(d0, d1, d2, d3, hq[8], hq[9], hq[10], hq[11], b1.x, b1.y);
-            mma_acc<MODE>(d0, d1, d2, d3, hq[12], hq[13], hq[14], hq[15], b1.z, b1.w);
-        }
-        acc[n][0] = fmaf(s0, d0, acc[n][0]);
-        acc[n][1] = fmaf(s0, d1, acc[n][1]);
-        acc[n][2] = fmaf(s1, d2, acc[n][2]);
-        acc[n][3] = fmaf(s1, d3, acc[n][3]);
-    }
-}
-
-// Producer side of a warp's ring: issues the three bulk copies of the next chunk.
-template <int MODE>
-struct RingProducer {
-    const uint8_t* codes;
-    const uint8_t* hi;
-    const uint8_t* sc;
-    int item, c, issued, j, q3, cur_item;
-    __device__ void load_item(const FfnArgs& p, const CtaSched& S, int tiles) {
-        const int a = find_active(S, item);
-        j = (item - S.ipre[a]) % tiles;
-        const PackedEntry* en = entry(p.packed, S.e[a]);
-        codes = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes);
-        hi = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi);
-        sc = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales);
-        q3 = S.fmt[a] == MOE_FMT_Q3;
-        cur_item = item;
-    }
-    __device__ void issue(const FfnArgs& p, const CtaSched& S, int n_items, int P, int tiles, int K, int G, int NC,
-                          uint8_t* ring, uint64_t* bar, uint64_t pol, int lane) {
-        if (item >= n_items) return;
-        if (item != cur_item) load_item(p, S, tiles);
-        const int st = issued & (NS - 1);
-        const int ng = min(CG, G - c * CG);
-        if (elect_one()) {                      // warp-uniform issue, one elected lane
-            uint8_t* dst = ring + (size_t)st * STAGE;
-            const uint32_t cb = 256 * ng, hb = q3 ? 128 * ng : 0;
-            mbar_arrive_expect_tx(&bar[st], cb + hb + 256);
-            bulk_g2s_evict_first(dst, codes + (size_t)4 * K * j + 2048 * (size_t)c, cb, &bar[st], pol);
-            bulk_g2s_evict_first(dst + OFF_SC, sc + (size_t)256 * NC * j + 256 * (size_t)c, 256, &bar[st], pol);
-            if (hb) bulk_g2s_evict_first(dst + OFF_HI, hi + (size_t)128 * G * j + 1024 * (size_t)c, hb, &bar[st], pol);
-        }
-        ++issued;
-        if (++c == NC) {
-            c = 0;
-            item += P;
-        }
-    }
-};
-
-template <int MODE, int NT, bool Q3>
-__device__ __forceinline__ void run_item(const FfnArgs& p, const CtaSched& S, RingProducer<MODE>& prod,
-                                         int& consumed, bool& aborted, const ItemView<NT>& v, const uint32_t (&sub)[5],
-                                         float (&acc)[NT][4], int n_items, int P, int tiles, int K, int G, int NC,
-                                         uint8_t* ring, uint64_t* bar, uint64_t pol, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    const int sh = 8 * (t & 1);
-    // swizzle offsets of group gl inside a full chunk: codes 4*(gl^g), third bits 2*(gl^(g/2))
-    int sw4[CG], sw2[CG];
-#pragma unroll
-    for (int gl = 0; gl < CG; ++gl) {
-        sw4[gl] = 4 * (gl ^ g);
-        sw2[gl] = 2 * (gl ^ (g >> 1));
-    }
-    prefetch_chunk<MODE, NT>(v, 0, t, G);
-    for (int c = 0; c < NC; ++c) {
-        prod.issue(p, S, n_items, P, tiles, K, G, NC, ring, bar, pol, lane);
-        if (c + 1 < NC) prefetch_chunk<MODE, NT>(v, c + 1, t, G);
-        const int st = consumed & (NS - 1);
-        if (!aborted && !mbar_wait_bounded(&bar[st], (uint32_t)(consumed / NS) & 1, kWaitLimit)) {
-            aborted = true;
-            report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | MODE);
-        }
-        const uint8_t* stg = ring + (size_t)st * STAGE;
-        const uint32_t* cw = reinterpret_cast<const uint32_t*>(stg);
-        const uint32_t* hw = reinterpret_cast<const uint32_t*>(stg + OFF_HI);
-        const uint16_t* scs = reinterpret_cast<const uint16_t*>(stg + OFF_SC) + g * 8;
-        // this chunk's B rows and -Z rows (constant offsets per group below)
-        const uint16_t* bc[NT];
-        const float* zcb[NT][2];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            bc[n] = v.b[n] + c * CG * 64;
-            zcb[n][0] = MODE == 0 ? v.z[n][0] + c * CG : nullptr;
-            zcb[n][1] = MODE == 0 ? v.z[n][1] + c * CG : nullptr;
-        }
-        const int ng = min(CG, G - c * CG);
-        if (ng == CG) {
-            const uint32_t* cwa = cw + g * 32 + t;          // row g; row g + 8 is 256 words on
-            const uint32_t* hwa = hw + g * 16 + (t >> 1);   // row g; row g + 8 is 128 words on
-#pragma unroll
-            for (int gl = 0; gl < CG; ++gl) {
-                const uint32_t wa = cwa[sw4[gl]], wb = cwa[sw4[gl] + 256];
-                uint32_t ua = 0, ub = 0;
-                if (Q3) {
-                    ua = hwa[sw2[gl]] >> sh;
-                    ub = hwa[sw2[gl] + 128] >> sh;
-                }
-                const uint16_t* bx[NT];
-                const float* zc[NT][2];
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    bx[n] = bc[n] + gl * 64;
-                    zc[n][0] = zcb[n][0] + gl;
-                    zc[n][1] = zcb[n][1] + gl;
-                }
-                group_step<MODE, NT, Q3>(wa, wb, ua, ub, half_bits_to_f32(scs[gl]), half_bits_to_f32(scs[64 + gl]),
-                                         bx, zc, sub, acc);
-            }
-        } else {
-            for (int gl = 0; gl < ng; ++gl) {
-                const uint32_t wa = cw[g * 4 * ng + 4 * gl + t], wb = cw[(g + 8) * 4 * ng + 4 * gl + t];
-                uint32_t ua = 0, ub = 0;
-                if (Q3) {
-                    ua = hw[g * 2 * ng + 2 * gl + (t >> 1)] >> sh;
-                    ub = hw[(g + 8) * 2 * ng + 2 * gl + (t >> 1)] >> sh;
-                }
-                const uint16_t* bx[NT];
-                const float* zc[NT][2];
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    bx[n] = bc[n] + gl * 64;
-                    zc[n][0] = zcb[n][0] + gl;
-                    zc[n][1] = zcb[n][1] + gl;
-                }
-                group_step<MODE, NT, Q3>(wa, wb, ua, ub, half_bits_to_f32(scs[gl]), half_bits_to_f32(scs[64 + gl]),
-                                         bx, zc, sub, acc);
-            }
-        }
-        __syncwarp();          // every lane is done with this stage before it is refilled
-        ++consumed;
-    }
-}
-
-template <int MODE, int NT, int NW>
 __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
-    constexpr int TB = 8 * NT;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ CtaSched S;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int K = MODE == 0 ? p.H : p.I;
-    const int tiles = MODE == 0 ? (2 * p.I) / 16 : p.H / 16;
-    const int G = K / 64, NC = (G + CG - 1) / CG;
+    Geo geo;
+    geo.K = MODE == 0 ? p.H : p.I;
+    geo.G = geo.K / 64;
+    geo.NC = (geo.G + CG - 1) / CG;
+    geo.blocks = MODE == 0 ? (2 * p.I) / (16 * NTL) : p.H / (16 * NTL);
+    geo.nkp = MODE == 0 ? p.nkp_gu : p.nkp_dn;
+    geo.cpk = (geo.NC + geo.nkp - 1) / geo.nkp;
     uint8_t* ring = smem + (size_t)warp * NS * STAGE;
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)NW * NS * STAGE) + warp * NS;
 
-    // ---- header check and the CTA's copy of the expert schedule --------------------
     // Work that does not depend on the router's (or the previous pass's) outputs runs
     // before griddep_wait() and overlaps the predecessor's tail: the header check and
     // the token rows; the schedule and everything after read the predecessor's data.
@@ -445,6 +573,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     if (threadIdx.x == 0) {
         if (!S.ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
         S.n_active = p.ctrl->n_active;
+        S.perm_in_smem = p.T * p.k <= kPermSmem;
     }
     __syncthreads();
     if (!S.ok) return;
@@ -454,552 +583,211 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         S.e[a] = e;
         S.fmt[a] = (int)entry(p.packed, e)->fmt;
         S.cnt[a] = e < p.E ? p.counts[e] : p.T;
+        S.off[a] = e < p.E ? p.offsets[e] : 0;
     }
+    if (S.perm_in_smem)
+        for (int r = threadIdx.x; r < p.T * p.k; r += blockDim.x) S.tok[r] = p.perm[r] / p.k;
     __syncthreads();
     if (threadIdx.x == 0) {
         int run = 0;
         for (int a = 0; a < nA; ++a) {
-            S.ipre[a] = run;
-            run += tiles * ((S.cnt[a] + TB - 1) / TB);
+            S.upre[a] = run;
+            run += ((S.cnt[a] + TP - 1) / TP) * geo.blocks * geo.nkp;
         }
-        S.ipre[nA] = run;
-        S.n_items = run;
+        S.upre[nA] = run;
+        S.n_units = run;
     }
     if (MODE == 0) warm_z(p);
     if (lane == 0)
         for (int s = 0; s < NS; ++s) mbar_init(&bar[s], 1);
     fence_mbar_init();
     __syncthreads();
-    const int n_items = S.n_items;
+    const int n_units = S.n_units;
+    // Every warp takes a contiguous range of units.  Range r goes to CTA r % grid and
+    // warp slot r / grid, with warp = 5 * slot mod 16: consecutive ranges (one
+    // expert's units) spread over all SMs, and the slots of one SM over its four
+    // schedulers.
     const int P = gridDim.x * NW;
-    // items dealt round-robin over the CTAs first (spreads each expert over many SMs)
-    const int gw = warp * gridDim.x + blockIdx.x;
+    const int slot = (warp * 13) & (NW - 1);           // the inverse of 5 mod 16
+    const int r = slot * gridDim.x + blockIdx.x;
+    const int u0 = (int)(((long long)n_units * r) / P), u1 = (int)(((long long)n_units * (r + 1)) / P);
     const uint64_t pol = l2_policy_evict_first();
 
-    RingProducer<MODE> prod;
-    prod.item = gw;
-    prod.c = 0;
+    Producer<MODE> prod;
+    prod.u_end = u1;
     prod.issued = 0;
-    prod.cur_item = -1;
-    for (int i = 0; i < NS - 1; ++i) prod.issue(p, S, n_items, P, tiles, K, G, NC, ring, bar, pol, lane);
+    prod.cur_a = -1;
+    prod.it.seek(S, u0, geo.blocks, geo.nkp);
+    prod.begin(p, S, geo);
+    for (int i = 0; i < NS - 1; ++i) prod.issue(p, S, geo, ring, bar, pol);
 
+    LaneGeo L;
+    L.g = lane >> 2;
+    L.t = lane & 3;
+    L.cw_lane = 32 * L.g + L.t;
+    L.g4 = 4 * L.g;
+    L.hw_lane = 16 * L.g + (L.t >> 1);
+    L.g2 = 2 * (L.g >> 1);
+    L.sh = 8 * (L.t & 1);
     bool aborted = false;
     int consumed = 0;
-    for (int item = gw; item < n_items; item += P) {
-        const int a = find_active(S, item);
-        const int r = item - S.ipre[a];
-        const int pass = r / tiles, j = r - pass * tiles;
-        const int e = S.e[a], f = S.fmt[a], cnt = S.cnt[a];
-        const int tb = pass * TB, nb = min(TB, cnt - tb);
-        // Token columns of this pass.  Columns without a token read a valid row (the
-        // pass's first token): their MMA outputs are never stored.
-        ItemView<NT> v;
-        const uint16_t* bsrc = MODE == 0 ? p.x : p.h;
-        const int bld = MODE == 0 ? p.H : p.I;
-        const float* zf = MODE == 0 ? p.zx + (size_t)f * p.T * G : nullptr;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int cb = n * 8 + g;
-            const int i = tb + (cb < nb ? cb : 0);
-            int brow;
-            if (e < p.E) {
-                const int hr = p.offsets[e] + i;
-                brow = MODE == 0 ? p.perm[hr] / p.k : hr;
-            } else {
-                brow = MODE == 0 ? i : p.T * p.k + (e - p.E) * p.T + i;
-            }
-            v.b[n] = bsrc + (size_t)brow * bld + 16 * t;
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int col = n * 8 + 2 * t + cc;
-                const int ii = tb + (col < nb ? col : 0);
-                int orow, ztok;
-                if (e < p.E) {
-                    orow = p.offsets[e] + ii;
-                    ztok = p.perm[orow] / p.k;
-                } else {
-                    orow = p.T * p.k + (e - p.E) * p.T + ii;
-                    ztok = ii;
-                }
-                v.orow[n][cc] = col < nb ? orow : -1;
-                v.z[n][cc] = MODE == 0 ? zf + (size_t)ztok * G : nullptr;
-            }
-        }
-        uint32_t sub[5] = {0, 0, 0, 0, 0};
-        if (MODE == 1) {
-            const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
-            sub[0] = f16x2_bits_of(512.f + o);
-            sub[1] = f16x2_bits_of(256.f + o);
-            sub[2] = f16x2_bits_of(64.f + o);
-            sub[3] = f16x2_bits_of(16.f + o);
-            sub[4] = f16x2_bits_of(4.f + o);
-        }
-        float acc[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-        if (f == MOE_FMT_Q3)
-            run_item<MODE, NT, true>(p, S, prod, consumed, aborted, v, sub, acc, n_items, P, tiles, K, G, NC, ring, bar,
-                                     pol, lane);
+    UnitIt it;
+    it.seek(S, u0, geo.blocks, geo.nkp);
+    for (; it.u < u1; it.next(S, geo.blocks, geo.nkp)) {
+        UnitPos q;
+        q.a = it.a;
+        q.jb = it.jb;
+        q.kp = it.kp;
+        q.pass = it.pass;
+        if (S.fmt[q.a] == MOE_FMT_Q3)
+            run_unit<MODE, true>(p, S, geo, q, prod, consumed, aborted, ring, bar, pol, L);
         else
-            run_item<MODE, NT, false>(p, S, prod, consumed, aborted, v, sub, acc, n_items, P, tiles, K, G, NC, ring,
-                                      bar, pol, lane);
-        // epilogue
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                if (v.orow[n][cc] < 0) continue;
-                if (MODE == 0) {
-                    p.h[(size_t)v.orow[n][cc] * p.I + j * 8 + g] =
-                        f32_to_f16_bits(silu_f(acc[n][cc]) * acc[n][2 + cc]);
-                } else {
-                    p.ypart[(size_t)v.orow[n][cc] * p.H + j * 16 + g] = acc[n][cc];
-                    p.ypart[(size_t)v.orow[n][cc] * p.H + j * 16 + g + 8] = acc[n][2 + cc];
-                }
-            }
-        }
+            run_unit<MODE, false>(p, S, geo, q, prod, consumed, aborted, ring, bar, pol, L);
     }
     // after a timeout the ring may still hold copies in flight: wait for them (bounded)
     if (aborted) {
-        for (int q = consumed; q < prod.issued; ++q)
-            if (!mbar_wait_bounded(&bar[q & (NS - 1)], (uint32_t)(q / NS) & 1, kWaitLimit)) {
+        for (int qd = consumed; qd < prod.issued; ++qd)
+            if (!mbar_wait_bounded(&bar[qd % NS], (uint32_t)(qd / NS) & 1, kWaitLimit)) {
                 report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | MODE);
                 break;
             }
     }
+}
+
+// h[row][i] = silu(sum_kp gate) * (sum_kp up) for every (token, slot) row, the K parts
+// added in order.  One thread per 4 consecutive h columns (4 gate and 4 up sums per
+// part); every part's loads are issued before the first add, so the kernel costs one
+// L2 round trip.
+constexpr int kMaxParts = 16;                           // K parts: at most ceil(K / 512)
+
+__global__ void __launch_bounds__(128) finalize_gateup_kernel(FfnArgs p) {
+    griddep_launch_dependents();                        // a single small wave
+    griddep_wait();                                     // gpart comes from the gate/up pass
+    const int per_row = p.I / 4;
+    const size_t R = (size_t)p.T * (p.k + p.S);
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= R * per_row) return;
+    const size_t row = idx / per_row;
+    const int q = (int)(idx - row * per_row);           // columns 4q .. 4q+3
+    const int j = q >> 1, half = q & 1;                 // tile j: gate sums at 16j + 4half, up at +8
+    const float* base = p.gpart + row * (2 * p.I) + j * 16 + 4 * half;
+    const size_t pstride = R * (2 * p.I);
+    float4 gv[kMaxParts], uv[kMaxParts];
+#pragma unroll
+    for (int kp = 0; kp < kMaxParts; ++kp) {
+        if (kp < p.nkp_gu) {
+            gv[kp] = __ldcg(reinterpret_cast<const float4*>(base + kp * pstride));
+            uv[kp] = __ldcg(reinterpret_cast<const float4*>(base + kp * pstride + 8));
+        }
+    }
+    float4 gs = make_float4(0.f, 0.f, 0.f, 0.f), us = gs;
+#pragma unroll
+    for (int kp = 0; kp < kMaxParts; ++kp) {
+        if (kp < p.nkp_gu) {
+            gs.x += gv[kp].x; gs.y += gv[kp].y; gs.z += gv[kp].z; gs.w += gv[kp].w;
+            us.x += uv[kp].x; us.y += uv[kp].y; us.z += uv[kp].z; us.w += uv[kp].w;
+        }
+    }
+    uint2 o;
+    o.x = (uint32_t)f32_to_f16_bits(silu_f(gs.x) * us.x) | ((uint32_t)f32_to_f16_bits(silu_f(gs.y) * us.y) << 16);
+    o.y = (uint32_t)f32_to_f16_bits(silu_f(gs.z) * us.z) | ((uint32_t)f32_to_f16_bits(silu_f(gs.w) * us.w) << 16);
+    *reinterpret_cast<uint2*>(p.h + row * p.I + 4 * q) = o;
 }
 
 // y[t] = sum_j g[t,j] * ypart[inv_perm[t*k + j]] + sum_s ypart[T*k + s*T + t], in slot
-// order, fp32, stored as bf16.  One thread per 8 consecutive outputs.
-__global__ void __launch_bounds__(256) combine_kernel(FfnArgs p) {
+// order, each row first summed over its K parts in order; fp32, stored as bf16.  One
+// thread per 4 consecutive outputs.  For few tokens the slot rows and gates are loaded
+// first, then every partial row, so the pass costs two L2 round trips.
+constexpr int kMaxRows = 12;                            // k + S rows per token ...
+constexpr int kMaxKp = 4;                               // ... and K parts held in registers
+
+__device__ __forceinline__ void add4(float4& a, const float4& b) {
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+}
+
+template <bool SMALL>
+__global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
     griddep_wait();                                     // ypart comes from the down pass
-    const int per_tok = p.H / 8;
-    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= p.T * per_tok) return;
-    const int tok = idx / per_tok, c8 = (idx - tok * per_tok) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int sl = 0; sl < p.k; ++sl) {
-        const int row = p.inv_perm[(size_t)tok * p.k + sl];
-        const float gw = p.topk_w[(size_t)tok * p.k + sl];
-        const float4* src = reinterpret_cast<const float4*>(p.ypart + (size_t)row * p.H + c8);
-        const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
-        acc[0] = fmaf(gw, v0.x, acc[0]);
-        acc[1] = fmaf(gw, v0.y, acc[1]);
-        acc[2] = fmaf(gw, v0.z, acc[2]);
-        acc[3] = fmaf(gw, v0.w, acc[3]);
-        acc[4] = fmaf(gw, v1.x, acc[4]);
-        acc[5] = fmaf(gw, v1.y, acc[5]);
-        acc[6] = fmaf(gw, v1.z, acc[6]);
-        acc[7] = fmaf(gw, v1.w, acc[7]);
-    }
-    for (int s = 0; s < p.S; ++s) {
-        const float4* src =
-            reinterpret_cast<const float4*>(p.ypart + ((size_t)p.T * p.k + (size_t)s * p.T + tok) * p.H + c8);
-        const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
-        acc[0] += v0.x;
-        acc[1] += v0.y;
-        acc[2] += v0.z;
-        acc[3] += v0.w;
-        acc[4] += v1.x;
-        acc[5] += v1.y;
-        acc[6] += v1.z;
-        acc[7] += v1.w;
-    }
-    uint4 o;
-    o.x = (uint32_t)f32_to_bf16_bits(acc[0]) | ((uint32_t)f32_to_bf16_bits(acc[1]) << 16);
-    o.y = (uint32_t)f32_to_bf16_bits(acc[2]) | ((uint32_t)f32_to_bf16_bits(acc[3]) << 16);
-    o.z = (uint32_t)f32_to_bf16_bits(acc[4]) | ((uint32_t)f32_to_bf16_bits(acc[5]) << 16);
-    o.w = (uint32_t)f32_to_bf16_bits(acc[6]) | ((uint32_t)f32_to_bf16_bits(acc[7]) << 16);
-    *reinterpret_cast<uint4*>(p.y + (size_t)tok * p.H + c8) = o;
-}
-
-// ---- warp-pair kernel for up to 16 tokens -------------------------------------------
-// A work item is (active expert, 32-row block = two 16-row tiles, token pass).  The two
-// warps of a pair (w and w + NW/2 of a CTA) stream the first and the second half of the
-// item's K chunks; the second adds its accumulators into the first's through shared
-// memory, and the first runs the epilogue.  Against one tile per warp this shares the
-// token fragments, the Z values, the loop and the address arithmetic between two tiles
-// and gives each warp two independent MMA chains, while the K split keeps as many
-// warps busy as there were items before.
-constexpr int NS2 = 2;                                  // stages per warp
-constexpr int STAGE2 = 2 * STAGE;                       // one stage: both tiles' blocks
-
-template <int MODE, int NT, bool Q3>
-__device__ __forceinline__ void group_step2(const uint32_t (&w)[2][2], const uint32_t (&u)[2][2],
-                                            const float (&sc)[2][2], const uint16_t* const (&bx)[NT],
-                                            const float* const (&zc)[NT][2], const uint32_t (&sub)[5],
-                                            float (&acc)[2][NT][4]) {
-    uint4 b0[NT], b1[NT];
-    float z0[NT], z1[NT];
+    const int per_tok = p.H / 4;
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (size_t)p.T * per_tok) return;
+    const int tok = (int)(idx / per_tok), c4 = (int)(idx - (size_t)tok * per_tok) * 4;
+    const size_t R = (size_t)p.T * (p.k + p.S);
+    const size_t pstride = R * p.H;
+    const int nrows = p.k + p.S;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (SMALL && nrows <= kMaxRows && p.nkp_dn <= kMaxKp) {
+        int rows[kMaxRows];
+        float gw[kMaxRows];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        b0[n] = __ldg(reinterpret_cast<const uint4*>(bx[n]));
-        b1[n] = __ldg(reinterpret_cast<const uint4*>(bx[n]) + 1);
-        z0[n] = MODE == 0 ? __ldg(zc[n][0]) : 0.f;
-        z1[n] = MODE == 0 ? __ldg(zc[n][1]) : 0.f;
-    }
-#pragma unroll
-    for (int tl = 0; tl < 2; ++tl) {
-        uint32_t q[16], hq[16];
-        dequant_quads<MODE>(w[tl][0], w[tl][1], sub, q);
-        if (Q3) dequant_hi_quads<MODE>(u[tl][0], u[tl][1], hq);
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            float d0 = z0[n], d1 = z1[n], d2 = z0[n], d3 = z1[n];
-            mma_acc<MODE>(d0, d1, d2, d3, q[0], q[1], q[2], q[3], b0[n].x, b0[n].y);
-            mma_acc<MODE>(d0, d1, d2, d3, q[4], q[5], q[6], q[7], b0[n].z, b0[n].w);
-            mma_acc<MODE>(d0, d1, d2, d3, q[8], q[9], q[10], q[11], b1[n].x, b1[n].y);
-            mma_acc<MODE>(d0, d1, d2, d3, q[12], q[13], q[14], q[15], b1[n].z, b1[n].w);
-            if (Q3) {
-                mma_acc<MODE>(d0, d1, d2, d3, hq[0], hq[1], hq[2], hq[3], b0[n].x, b0[n].y);
-                mma_acc<MODE>(d0, d1, d2, d3, hq[4], hq[5], hq[6], hq[7], b0[n].z, b0[n].w);
-                mma_acc<MODE>(d0, d1, d2, d3, hq[8], hq[9], hq[10], hq[11], b1[n].x, b1[n].y);
-                mma_acc<MODE>(d0, d1, d2, d3, hq[12], hq[13], hq[14], hq[15], b1[n].z, b1[n].w);
-            }
-            acc[tl][n][0] = fmaf(sc[tl][0], d0, acc[tl][n][0]);
-            acc[tl][n][1] = fmaf(sc[tl][0], d1, acc[tl][n][1]);
-            acc[tl][n][2] = fmaf(sc[tl][1], d2, acc[tl][n][2]);
-            acc[tl][n][3] = fmaf(sc[tl][1], d3, acc[tl][n][3]);
-        }
-    }
-}
-
-// Producer side of a pair warp's ring: the next chunk of both tiles (six bulk copies at
-// most), issued by one elected lane of the converged warp.
-template <int MODE>
-struct PairProducer {
-    const uint8_t* codes;
-    const uint8_t* hi;
-    const uint8_t* sc;
-    int item, c, issued, jb, q3, cur_item;
-    __device__ void load_item(const FfnArgs& p, const CtaSched& S, int blocks) {
-        const int a = find_active(S, item);
-        jb = (item - S.ipre[a]) % blocks;
-        const PackedEntry* en = entry(p.packed, S.e[a]);
-        codes = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes);
-        hi = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi);
-        sc = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales);
-        q3 = S.fmt[a] == MOE_FMT_Q3;
-        cur_item = item;
-    }
-    __device__ void issue(const FfnArgs& p, const CtaSched& S, int n_items, int P, int blocks, int K, int G, int NC,
-                          int c_lo, int c_hi, uint8_t* ring, uint64_t* bar, uint64_t pol) {
-        if (item >= n_items || c_lo >= c_hi) return;
-        if (item != cur_item) load_item(p, S, blocks);
-        const int st = issued % NS2;
-        const int ng = min(CG, G - c * CG);
-        if (elect_one()) {
-            uint8_t* dst = ring + (size_t)st * STAGE2;
-            const uint32_t cb = 256 * ng, hb = q3 ? 128 * ng : 0;
-            mbar_arrive_expect_tx(&bar[st], 2 * (cb + hb + 256));
-#pragma unroll
-            for (int tl = 0; tl < 2; ++tl) {
-                const int j = 2 * jb + tl;
-                uint8_t* d = dst + tl * STAGE;
-                bulk_g2s_evict_first(d, codes + (size_t)4 * K * j + 2048 * (size_t)c, cb, &bar[st], pol);
-                bulk_g2s_evict_first(d + OFF_SC, sc + (size_t)256 * NC * j + 256 * (size_t)c, 256, &bar[st], pol);
-                if (hb) bulk_g2s_evict_first(d + OFF_HI, hi + (size_t)128 * G * j + 1024 * (size_t)c, hb, &bar[st], pol);
+        for (int r = 0; r < kMaxRows; ++r) {
+            if (r < p.k) {
+                rows[r] = __ldg(p.inv_perm + (size_t)tok * p.k + r);
+                gw[r] = __ldg(p.topk_w + (size_t)tok * p.k + r);
+            } else if (r < nrows) {
+                rows[r] = p.T * p.k + (r - p.k) * p.T + tok;
+                gw[r] = 1.f;
             }
         }
-        __syncwarp();
-        ++issued;
-        if (++c == c_hi) {
-            c = c_lo;
-            item += P;
-        }
-    }
-};
-
-template <int MODE, int NT, bool Q3>
-__device__ __forceinline__ void run_item2(const FfnArgs& p, const CtaSched& S, PairProducer<MODE>& prod,
-                                          int& consumed, bool& aborted, const ItemView<NT>& v,
-                                          const uint32_t (&sub)[5], float (&acc)[2][NT][4], int n_items, int P,
-                                          int blocks, int K, int G, int NC, int c_lo, int c_hi, uint8_t* ring,
-                                          uint64_t* bar, uint64_t pol, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    const int sh = 8 * (t & 1);
-    if (c_lo < c_hi) prefetch_chunk<MODE, NT>(v, c_lo, t, G);
-    for (int c = c_lo; c < c_hi; ++c) {
-        prod.issue(p, S, n_items, P, blocks, K, G, NC, c_lo, c_hi, ring, bar, pol);
-        if (c + 1 < c_hi) prefetch_chunk<MODE, NT>(v, c + 1, t, G);
-        const int st = consumed % NS2;
-        if (!aborted && !mbar_wait_bounded(&bar[st], (uint32_t)(consumed / NS2) & 1, kWaitLimit)) {
-            aborted = true;
-            report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | MODE);
-        }
-        const uint8_t* stg = ring + (size_t)st * STAGE2;
-        const uint16_t* bc[NT];
-        const float* zcb[NT][2];
+        float4 v[kMaxKp][kMaxRows];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            bc[n] = v.b[n] + c * CG * 64;
-            zcb[n][0] = MODE == 0 ? v.z[n][0] + c * CG : nullptr;
-            zcb[n][1] = MODE == 0 ? v.z[n][1] + c * CG : nullptr;
-        }
-        const int ng = min(CG, G - c * CG);
-        // word offsets of rows g (and g + 8: +256 codes words, +128 third-bit words)
-        const int cw_row = ng == CG ? g * 32 + t : g * 4 * ng + t;
-        const int cw_row8 = ng == CG ? 256 : 8 * 4 * ng;
-        const int hw_row = ng == CG ? g * 16 + (t >> 1) : g * 2 * ng + (t >> 1);
-        const int hw_row8 = ng == CG ? 128 : 8 * 2 * ng;
-        for (int gl = 0; gl < ng; ++gl) {
-            const int cpos = cw_row + (ng == CG ? 4 * (gl ^ g) : 4 * gl);
-            const int hpos = hw_row + (ng == CG ? 2 * (gl ^ (g >> 1)) : 2 * gl);
-            uint32_t w[2][2], u[2][2] = {{0, 0}, {0, 0}};
-            float scv[2][2];
+        for (int kp = 0; kp < kMaxKp; ++kp)
 #pragma unroll
-            for (int tl = 0; tl < 2; ++tl) {
-                const uint8_t* tb = stg + tl * STAGE;
-                const uint32_t* cw = reinterpret_cast<const uint32_t*>(tb);
-                w[tl][0] = cw[cpos];
-                w[tl][1] = cw[cpos + cw_row8];
-                if (Q3) {
-                    const uint32_t* hw = reinterpret_cast<const uint32_t*>(tb + OFF_HI);
-                    u[tl][0] = hw[hpos] >> sh;
-                    u[tl][1] = hw[hpos + hw_row8] >> sh;
-                }
-                const uint16_t* scs = reinterpret_cast<const uint16_t*>(tb + OFF_SC) + g * 8;
-                scv[tl][0] = half_bits_to_f32(scs[gl]);
-                scv[tl][1] = half_bits_to_f32(scs[64 + gl]);
-            }
-            const uint16_t* bx[NT];
-            const float* zc[NT][2];
+            for (int r = 0; r < kMaxRows; ++r)
+                if (r < nrows && kp < p.nkp_dn)
+                    v[kp][r] = __ldcg(reinterpret_cast<const float4*>(p.ypart + kp * pstride + (size_t)rows[r] * p.H + c4));
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                bx[n] = bc[n] + gl * 64;
-                zc[n][0] = zcb[n][0] + gl;
-                zc[n][1] = zcb[n][1] + gl;
-            }
-            group_step2<MODE, NT, Q3>(w, u, scv, bx, zc, sub, acc);
-        }
-        __syncwarp();          // every lane is done with this stage before it is refilled
-        ++consumed;
-    }
-}
-
-template <int MODE, int NT, int NW>
-__global__ void __launch_bounds__(NW * 32, 1) ffn_decode_pair_kernel(FfnArgs p) {
-    constexpr int TB = 8 * NT, NPAIR = NW / 2;
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ CtaSched S;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int pair = warp % NPAIR, kh = warp / NPAIR;
-    const int g = lane >> 2, t = lane & 3;
-    const int K = MODE == 0 ? p.H : p.I;
-    const int blocks = MODE == 0 ? (2 * p.I) / 32 : p.H / 32;
-    const int G = K / 64, NC = (G + CG - 1) / CG;
-    const int c_mid = (NC + 1) / 2;
-    const int c_lo = kh == 0 ? 0 : c_mid, c_hi = kh == 0 ? c_mid : NC;
-    uint8_t* ring = smem + (size_t)warp * NS2 * STAGE2;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)NW * NS2 * STAGE2) + warp * NS2;
-    float* red = reinterpret_cast<float*>(smem + (size_t)NW * NS2 * STAGE2 + (size_t)NW * NS2 * 8) +
-                 (size_t)pair * (2 * NT * 4 * 32);
-
-    // Work that does not depend on the router's (or the previous pass's) outputs runs
-    // before griddep_wait() and overlaps the predecessor's tail: the header check and
-    // the token rows; the schedule and everything after read the predecessor's data.
-    griddep_launch_dependents();                        // all CTAs of this grid are resident
-    if (threadIdx.x == 0) {
-        const uint32_t* hd = reinterpret_cast<const uint32_t*>(p.packed);
-        S.ok = hd[0] == kMagic && hd[1] == kVersion && (int)hd[2] == p.H && (int)hd[3] == p.I &&
-               (int)hd[4] == p.E && (int)hd[5] == p.S && hd[6] == 64u && hd[7] == (uint32_t)kInterleave;
-    }
-    if (MODE == 0) warm_rows(p);
-    griddep_wait();
-    if (threadIdx.x == 0) {
-        if (!S.ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
-        S.n_active = p.ctrl->n_active;
-    }
-    __syncthreads();
-    if (!S.ok) return;
-    const int nA = S.n_active;
-    for (int a = threadIdx.x; a < nA; a += blockDim.x) {
-        const int e = p.active[a];
-        S.e[a] = e;
-        S.fmt[a] = (int)entry(p.packed, e)->fmt;
-        S.cnt[a] = e < p.E ? p.counts[e] : p.T;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int a = 0; a < nA; ++a) {
-            S.ipre[a] = run;
-            run += blocks * ((S.cnt[a] + TB - 1) / TB);
-        }
-        S.ipre[nA] = run;
-        S.n_items = run;
-    }
-    if (MODE == 0) warm_z(p);
-    if (lane == 0)
-        for (int s = 0; s < NS2; ++s) mbar_init(&bar[s], 1);
-    fence_mbar_init();
-    __syncthreads();
-    const int n_items = S.n_items;
-    const int P = gridDim.x * NPAIR;
-    // items are dealt round-robin over the CTAs first, so that one expert's items (the
-    // heavier 3-bit ones in particular) spread over many SMs instead of filling a few
-    const int gp = pair * gridDim.x + blockIdx.x;
-    const uint64_t pol = l2_policy_evict_first();
-
-    PairProducer<MODE> prod;
-    prod.item = gp;
-    prod.c = c_lo;
-    prod.issued = 0;
-    prod.cur_item = -1;
-    for (int i = 0; i < NS2 - 1; ++i) prod.issue(p, S, n_items, P, blocks, K, G, NC, c_lo, c_hi, ring, bar, pol);
-
-    bool aborted = false;
-    int consumed = 0;
-    for (int item = gp; item < n_items; item += P) {
-        const int a = find_active(S, item);
-        const int r = item - S.ipre[a];
-        const int pass = r / blocks, jb = r - pass * blocks;
-        const int e = S.e[a], f = S.fmt[a], cnt = S.cnt[a];
-        const int tb = pass * TB, nb = min(TB, cnt - tb);
-        // Token columns of this pass.  Columns without a token read a valid row (the
-        // pass's first token): their MMA outputs are never stored.
-        ItemView<NT> v;
-        const uint16_t* bsrc = MODE == 0 ? p.x : p.h;
-        const int bld = MODE == 0 ? p.H : p.I;
-        const float* zf = MODE == 0 ? p.zx + (size_t)f * p.T * G : nullptr;
+        for (int r = 0; r < kMaxRows; ++r) {
+            if (r >= nrows) continue;
+            float4 s = v[0][r];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int cb = n * 8 + g;
-            const int i = tb + (cb < nb ? cb : 0);
-            int brow;
-            if (e < p.E) {
-                const int hr = p.offsets[e] + i;
-                brow = MODE == 0 ? p.perm[hr] / p.k : hr;
+            for (int kp = 1; kp < kMaxKp; ++kp)
+                if (kp < p.nkp_dn) add4(s, v[kp][r]);
+            if (r < p.k) {
+                acc.x = fmaf(gw[r], s.x, acc.x);
+                acc.y = fmaf(gw[r], s.y, acc.y);
+                acc.z = fmaf(gw[r], s.z, acc.z);
+                acc.w = fmaf(gw[r], s.w, acc.w);
             } else {
-                brow = MODE == 0 ? i : p.T * p.k + (e - p.E) * p.T + i;
-            }
-            v.b[n] = bsrc + (size_t)brow * bld + 16 * t;
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int col = n * 8 + 2 * t + cc;
-                const int ii = tb + (col < nb ? col : 0);
-                int orow, ztok;
-                if (e < p.E) {
-                    orow = p.offsets[e] + ii;
-                    ztok = p.perm[orow] / p.k;
-                } else {
-                    orow = p.T * p.k + (e - p.E) * p.T + ii;
-                    ztok = ii;
-                }
-                v.orow[n][cc] = col < nb ? orow : -1;
-                v.z[n][cc] = MODE == 0 ? zf + (size_t)ztok * G : nullptr;
+                add4(acc, s);
             }
         }
-        uint32_t sub[5] = {0, 0, 0, 0, 0};
-        if (MODE == 1) {
-            const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
-            sub[0] = f16x2_bits_of(512.f + o);
-            sub[1] = f16x2_bits_of(256.f + o);
-            sub[2] = f16x2_bits_of(64.f + o);
-            sub[3] = f16x2_bits_of(16.f + o);
-            sub[4] = f16x2_bits_of(4.f + o);
-        }
-        float acc[2][NT][4];
-#pragma unroll
-        for (int tl = 0; tl < 2; ++tl)
-#pragma unroll
-            for (int n = 0; n < NT; ++n) acc[tl][n][0] = acc[tl][n][1] = acc[tl][n][2] = acc[tl][n][3] = 0.f;
-        if (f == MOE_FMT_Q3)
-            run_item2<MODE, NT, true>(p, S, prod, consumed, aborted, v, sub, acc, n_items, P, blocks, K, G, NC, c_lo,
-                                      c_hi, ring, bar, pol, lane);
-        else
-            run_item2<MODE, NT, false>(p, S, prod, consumed, aborted, v, sub, acc, n_items, P, blocks, K, G, NC, c_lo,
-                                       c_hi, ring, bar, pol, lane);
-        // the second K half hands its sums to the first through shared memory
-        if (kh == 1) {
-#pragma unroll
-            for (int tl = 0; tl < 2; ++tl)
-#pragma unroll
-                for (int n = 0; n < NT; ++n)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) red[((tl * NT + n) * 4 + i) * 32 + lane] = acc[tl][n][i];
-        }
-        named_bar_sync(1 + pair, 64);
-        if (kh == 0) {
-#pragma unroll
-            for (int tl = 0; tl < 2; ++tl)
-#pragma unroll
-                for (int n = 0; n < NT; ++n)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[tl][n][i] += red[((tl * NT + n) * 4 + i) * 32 + lane];
-            // epilogue: tile j = 2 jb + tl
-#pragma unroll
-            for (int tl = 0; tl < 2; ++tl) {
-                const int j = 2 * jb + tl;
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        if (v.orow[n][cc] < 0) continue;
-                        if (MODE == 0) {
-                            p.h[(size_t)v.orow[n][cc] * p.I + j * 8 + g] =
-                                f32_to_f16_bits(silu_f(acc[tl][n][cc]) * acc[tl][n][2 + cc]);
-                        } else {
-                            p.ypart[(size_t)v.orow[n][cc] * p.H + j * 16 + g] = acc[tl][n][cc];
-                            p.ypart[(size_t)v.orow[n][cc] * p.H + j * 16 + g + 8] = acc[tl][n][2 + cc];
-                        }
-                    }
-                }
+    } else {
+        // many parts: the same sums, one row at a time
+        for (int r = 0; r < nrows; ++r) {
+            const int row = r < p.k ? p.inv_perm[(size_t)tok * p.k + r] : p.T * p.k + (r - p.k) * p.T + tok;
+            const float* src = p.ypart + (size_t)row * p.H + c4;
+            float4 s = __ldcg(reinterpret_cast<const float4*>(src));
+            for (int kp = 1; kp < p.nkp_dn; ++kp) add4(s, __ldcg(reinterpret_cast<const float4*>(src + kp * pstride)));
+            if (r < p.k) {
+                const float g = p.topk_w[(size_t)tok * p.k + r];
+                acc.x = fmaf(g, s.x, acc.x);
+                acc.y = fmaf(g, s.y, acc.y);
+                acc.z = fmaf(g, s.z, acc.z);
+                acc.w = fmaf(g, s.w, acc.w);
+            } else {
+                add4(acc, s);
             }
         }
-        named_bar_sync(1 + pair, 64);          // the first half has read the shared sums
     }
-    // after a timeout the ring may still hold copies in flight: wait for them (bounded)
-    if (aborted && lane == 0) {
-        for (int q = consumed; q < prod.issued; ++q)
-            if (!mbar_wait_bounded(&bar[q % NS2], (uint32_t)(q / NS2) & 1, kWaitLimit)) {
-                report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetDrain | MODE);
-                break;
-            }
-    }
+    uint2 o;
+    o.x = (uint32_t)f32_to_bf16_bits(acc.x) | ((uint32_t)f32_to_bf16_bits(acc.y) << 16);
+    o.y = (uint32_t)f32_to_bf16_bits(acc.z) | ((uint32_t)f32_to_bf16_bits(acc.w) << 16);
+    *reinterpret_cast<uint2*>(p.y + (size_t)tok * p.H + c4) = o;
 }
 
-template <int NT, int NW>
-constexpr size_t dyn_smem_pair() {
-    return (size_t)NW * NS2 * STAGE2 + (size_t)NW * NS2 * 8 + (size_t)(NW / 2) * 2 * NT * 4 * 32 * 4;
-}
+constexpr size_t kDynSmem = (size_t)NW * NS * STAGE + (size_t)NW * NS * 8;
 
-template <int MODE, int NT, int NW>
-cudaError_t launch_pair(const FfnArgs& a, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_decode_pair_kernel<MODE, NT, NW>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)dyn_smem_pair<NT, NW>());
-        if (err != cudaSuccess) return err;
-        attr = true;
-    }
-    return launch_pdl(ffn_decode_pair_kernel<MODE, NT, NW>, dim3(a.num_ctas), dim3(NW * 32), dyn_smem_pair<NT, NW>(),
-                      s, a);
-}
-
-template <int NW>
-constexpr size_t dyn_smem() { return (size_t)NW * NS * STAGE + (size_t)NW * NS * 8; }
-
-template <int MODE, int NT, int NW>
-cudaError_t launch_one(const FfnArgs& a, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_decode_kernel<MODE, NT, NW>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem<NW>());
-        if (err != cudaSuccess) return err;
-        attr = true;
-    }
-    return launch_pdl(ffn_decode_kernel<MODE, NT, NW>, dim3(a.num_ctas), dim3(NW * 32), dyn_smem<NW>(), s, a);
-}
-
-// warps per CTA shrink as the token tile grows, to leave room for the accumulators
 template <int MODE>
 cudaError_t launch_mode(const FfnArgs& a, cudaStream_t s) {
-    if (a.T <= 8) return launch_pair<MODE, 1, 16>(a, s);
-    if (a.T <= 16) return launch_pair<MODE, 2, 12>(a, s);
-    if (a.T <= 32) return launch_one<MODE, 4, 8>(a, s);
-    return launch_one<MODE, 8, 8>(a, s);
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t err = cudaFuncSetAttribute(ffn_decode_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)kDynSmem);
+        if (err != cudaSuccess) return err;
+        attr = true;
+    }
+    return launch_pdl(ffn_decode_kernel<MODE>, dim3(a.num_ctas), dim3(NW * 32), kDynSmem, s, a);
 }
 
 }  // namespace
@@ -1007,6 +795,11 @@ cudaError_t launch_mode(const FfnArgs& a, cudaStream_t s) {
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down) {
     cudaError_t err = launch_mode<0>(a, s);
     if (err != cudaSuccess) return err;
+    if (a.nkp_gu > 1) {
+        const long long n = (long long)a.T * (a.k + a.S) * (a.I / 4);
+        err = launch_pdl(finalize_gateup_kernel, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, s, a);
+        if (err != cudaSuccess) return err;
+    }
     if (ev_gateup && (err = record_event(ev_gateup, s)) != cudaSuccess) return err;
     err = launch_mode<1>(a, s);
     if (err != cudaSuccess) return err;
@@ -1015,8 +808,11 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_g
 }
 
 cudaError_t launch_combine(const FfnArgs& a, cudaStream_t s) {
-    const long long n = (long long)a.T * (a.H / 8);
-    return launch_pdl(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, a);
+    const long long n = (long long)a.T * (a.H / 4);
+    const dim3 grid((unsigned)((n + 127) / 128));
+    // few tokens: a latency-bound pass, every load issued up front; many tokens: plain
+    return a.T <= kSmallT ? launch_pdl(combine_kernel<true>, grid, dim3(128), 0, s, a)
+                          : launch_pdl(combine_kernel<false>, grid, dim3(128), 0, s, a);
 }
 
 }  // namespace moe

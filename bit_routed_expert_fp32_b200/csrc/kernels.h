@@ -37,7 +37,9 @@ struct FfnArgs {
     const float* zx;         // ws [3][T][H/64], negated
     Ctrl* ctrl;
     uint16_t* h;             // ws fp16 [T*(k+S)][I]
-    float* ypart;            // ws f32 [T*(k+S)][H]
+    float* ypart;            // ws f32 [nkp_dn][T*(k+S)][H]
+    float* gpart;            // ws f32 [nkp_gu][T*(k+S)][2I] (aliases ypart; decode, nkp_gu > 1)
+    int nkp_gu, nkp_dn;      // K parts of the decode gate/up and down passes (1 on the prefill path)
     uint32_t* tile_ctr;      // ws [H/16]
     uint16_t* y;             // bf16 [T][H]
     int num_ctas;
@@ -49,6 +51,28 @@ struct Ws {
     size_t ctrl, tile_ctr, active, logits, hist, zx, h, ypart, total;
 };
 Ws ws_layout(const moe_shape* s, int64_t T);
+
+// K parts of the decode-path expert passes for T tokens.  With few tokens only a few
+// experts are active and their 32-row blocks are fewer than the warps of the GPU, so
+// K is split (into whole 8-group chunks) until there are about three units per warp
+// of a reference 148-SM part.  Only for T <= kSmallT; 1 otherwise.
+inline void decode_kparts(const moe_shape* s, int64_t T, int* nkp_gu, int* nkp_dn) {
+    *nkp_gu = *nkp_dn = 1;
+    if (T < 1 || T > kSmallT) return;
+    const int64_t active = (T * s->top_k < s->n_experts ? T * s->top_k : s->n_experts) + s->n_shared;
+    const int64_t target = 3 * 148 * 16;
+    auto pick = [&](int K, int rows) {
+        const int nc = (K / 64 + 7) / 8;
+        const int64_t base = active * (rows / 32);
+        for (int n = 1; n <= nc; ++n) {
+            const int cpk = (nc + n - 1) / n, eff = (nc + cpk - 1) / cpk;
+            if (base * eff >= target || n == nc) return eff;
+        }
+        return 1;
+    };
+    *nkp_gu = pick(s->hidden, 2 * s->inter);
+    *nkp_dn = pick(s->inter, s->hidden);
+}
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // decode-path expert kernels + combine; ev_gateup / ev_down (may be null) are recorded

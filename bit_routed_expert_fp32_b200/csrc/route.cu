@@ -153,12 +153,12 @@ __device__ void warp_active(const int* s_cnt, int E, int S, int32_t* active, Ctr
 // at -Z.  For token t and group G (elements x_e, e = 0..63 of the group):
 //   Bx = sum_e lo_base(e) x_e,  Hx = sum_e hi_base(e) x_e,  Sx = sum_e x_e,
 // with lo_base / hi_base the magic bases the expert kernel uses for the pair that
-// holds element e (pair p = (e % 16) / 2):  lo 64,32,8,16,4,64,16,4 and
+// holds element e (pair p = (e % 16) / 2):  lo 128,32,8,128,32,8,128,32 and
 // hi 512,256,128,64,32,16,8,8.  Then for code offset o:
 //   Z_ternary = Bx + Sx,  Z_q2 = Bx + 1.5 Sx,  Z_q3 = Bx + Hx + 3.5 Sx.
 // Stored negated as zx[format][T][G] (the MMA's accumulator input).
 __device__ void compute_z(const RouteArgs& p, int t, int Gi, int lane) {
-    constexpr float kLo[8] = {64.f, 32.f, 8.f, 16.f, 4.f, 64.f, 16.f, 4.f};
+    constexpr float kLo[8] = {128.f, 32.f, 8.f, 128.f, 32.f, 8.f, 128.f, 32.f};
     constexpr float kHi[8] = {512.f, 256.f, 128.f, 64.f, 32.f, 16.f, 8.f, 8.f};
     const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * p.H + Gi * 64) + lane);
     const float x0 = bf16lo(v), x1 = bf16hi(v);
@@ -183,60 +183,113 @@ __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
 }
 
 // ---------------------------------------------------------------- decode router
-// 2 experts per CTA, 4 warps per expert row (one K quarter each), 7 float4 loads in
-// flight per lane; then the Z tables; the last CTA does top-k and the permutation.
+// Top-k of one token by one warp with 32-bit reductions: lane l holds the logits of
+// experts 8l .. 8l+7 (v[j], -inf padding) as order-preserving keys; each round takes
+// the largest key over the warp (redux.sync), the lowest lane holding it and, inside
+// that lane, the lowest j, so equal logits go to the lower expert id.  Writes ids and
+// renormalised gates for slots < k to ids_out / gates_out and to s_ids (shared).
+__device__ inline uint32_t order_key(float f) {
+    const uint32_t b = f == 0.f ? 0u : __float_as_uint(f);          // -0 and +0 are equal
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ void warp_topk_redux(const float (&v)[8], int k, int lane, int32_t* ids_out, float* gates_out,
+                                int32_t* s_ids) {
+    uint32_t key[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) key[j] = v[j] == -INFINITY ? 0u : order_key(v[j]);
+    float my_sel = 0.f, top = 0.f;
+    int my_id = 0;
+    for (int r = 0; r < k; ++r) {
+        uint32_t bk = key[0];
+        int bj = 0;
+#pragma unroll
+        for (int j = 1; j < 8; ++j)
+            if (key[j] > bk) {              // strict: an equal key keeps the lower j
+                bk = key[j];
+                bj = j;
+            }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+        const int wl = __ffs(__ballot_sync(0xffffffffu, bk == m)) - 1;
+        const int wj = __shfl_sync(0xffffffffu, bj, wl);
+        float val = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j == bj) val = v[j];
+        val = __shfl_sync(0xffffffffu, val, wl);
+        if (r == 0) top = val;
+        if (lane == r) {
+            my_sel = val;
+            my_id = 8 * wl + wj;
+        }
+        if (lane == wl) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j == wj) key[j] = 0u;
+        }
+    }
+    const float ex = lane < k ? expf(my_sel - top) : 0.f;
+    const float sum = warp_sum(ex);
+    if (lane < k) {
+        ids_out[lane] = my_id;
+        gates_out[lane] = ex / sum;
+        s_ids[lane] = my_id;
+    }
+}
+
+// One CTA per expert row: 8 warps hold the whole fp32 row in registers (one load
+// each, all in flight at once) and form its logit for every token; then the Z
+// tables; the last CTA to finish (atomic ticket) does top-k, histogram, scan and the
+// permutation.
+constexpr int kRouteVec = 7;                           // float4 of the row per thread (H <= 7168)
+
 __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
     griddep_launch_dependents();        // one wave of CTAs: the expert pass may start launching
-    constexpr int U = 7;
     __shared__ float s_part[8][kSmallT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int el = warp >> 2, q = warp & 3;
-    const int e = blockIdx.x * 2 + el;
-    const int q4 = p.H / 16;                     // float4 per K quarter
-    if (e < p.E) {
-        const float4* w4 = reinterpret_cast<const float4*>(p.Wr + (size_t)e * p.H) + q * q4;
+    const int e = blockIdx.x;
+    const int n4 = p.H / 4;                                        // float4 per row
+    const float4* w4 = reinterpret_cast<const float4*>(p.Wr + (size_t)e * p.H);
+    for (int i0 = 0; i0 < n4; i0 += 256 * kRouteVec) {
+        float4 w[kRouteVec];
+#pragma unroll
+        for (int u = 0; u < kRouteVec; ++u) {
+            const int i = i0 + threadIdx.x + 256 * u;
+            w[u] = i < n4 ? __ldg(w4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         for (int tb = 0; tb < p.T; tb += 8) {
             float acc[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-            for (int i0 = lane; i0 < q4; i0 += 32 * U) {
-                float4 w[U];
+            for (int j = 0; j < 8; ++j) {
+                acc[j] = 0.f;
+                if (tb + j >= p.T) continue;
+                const uint2* xr = reinterpret_cast<const uint2*>(p.x + (size_t)(tb + j) * p.H);
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int i = i0 + 32 * u;
-                    w[u] = i < q4 ? __ldg(w4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (tb + j >= p.T) break;
-                    const uint2* xr = reinterpret_cast<const uint2*>(p.x + (size_t)(tb + j) * p.H) + q * q4;
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const int i = i0 + 32 * u;
-                        if (i < q4) {
-                            const uint2 xv = __ldg(xr + i);
-                            acc[j] = fmaf(w[u].x, bf16lo(xv.x), acc[j]);
-                            acc[j] = fmaf(w[u].y, bf16hi(xv.x), acc[j]);
-                            acc[j] = fmaf(w[u].z, bf16lo(xv.y), acc[j]);
-                            acc[j] = fmaf(w[u].w, bf16hi(xv.y), acc[j]);
-                        }
+                for (int u = 0; u < kRouteVec; ++u) {
+                    const int i = i0 + threadIdx.x + 256 * u;
+                    if (i < n4) {
+                        const uint2 xv = __ldg(xr + i);
+                        acc[j] = fmaf(w[u].x, bf16lo(xv.x), acc[j]);
+                        acc[j] = fmaf(w[u].y, bf16hi(xv.x), acc[j]);
+                        acc[j] = fmaf(w[u].z, bf16lo(xv.y), acc[j]);
+                        acc[j] = fmaf(w[u].w, bf16hi(xv.y), acc[j]);
                     }
                 }
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
+                if (tb + j >= p.T) break;
                 const float v = warp_sum(acc[j]);
-                if (lane == 0 && tb + j < p.T) s_part[warp][tb + j] = v;
+                if (lane == 0) s_part[warp][tb + j] = (i0 == 0 ? 0.f : s_part[warp][tb + j]) + v;
             }
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < 2 * p.T; i += blockDim.x) {
-        const int l = i / p.T, t = i - l * p.T, ee = blockIdx.x * 2 + l;
-        if (ee < p.E) {
-            const float v = (s_part[4 * l][t] + s_part[4 * l + 1][t]) + (s_part[4 * l + 2][t] + s_part[4 * l + 3][t]);
-            p.logits[(size_t)t * p.E + ee] = v + (p.bias ? p.bias[ee] : 0.f);
-        }
+    for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += s_part[w][t];
+        p.logits[(size_t)t * p.E + e] = v + (p.bias ? p.bias[e] : 0.f);
     }
     {
         const int G = p.H / 64;
@@ -253,15 +306,18 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
     __shared__ int32_t s_ids[kSmallT * 16];
     __shared__ int s_cnt[256];
     __shared__ int s_off[257];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_cnt[i] = 0;
     // top-k per token: warp w takes tokens w, w+8, ...
     for (int t = warp; t < p.T; t += 8) {
         float v[8];
-        load_logits_row(p.logits + (size_t)t * p.E, p.E, lane, v);
-        warp_topk(v, p.k, lane, p.r.topk_ids + (size_t)t * p.k, p.r.topk_w + (size_t)t * p.k);
-        __syncwarp();
-        if (lane < p.k) s_ids[t * p.k + lane] = p.r.topk_ids[(size_t)t * p.k + lane];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int ee = 8 * lane + j;
+            v[j] = ee < p.E ? ldcg_f32(p.logits + (size_t)t * p.E + ee) : -INFINITY;
+        }
+        warp_topk_redux(v, p.k, lane, p.r.topk_ids + (size_t)t * p.k, p.r.topk_w + (size_t)t * p.k,
+                        s_ids + t * p.k);
     }
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_cnt[i] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < p.T * p.k; i += blockDim.x) atomicAdd(&s_cnt[s_ids[i]], 1);
     __syncthreads();
@@ -276,8 +332,9 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
         __syncwarp();
         // s_off doubles as the running position per expert
         warp_scatter(s_ids, 0, p.T * p.k, s_off, p.r.perm, p.r.inv_perm, lane);
-        warp_active(s_cnt, p.E, p.S, p.active, p.ctrl, p.T, lane);
         if (lane == 0) p.ctrl->route_ticket = 0;
+    } else if (warp == 1) {
+        warp_active(s_cnt, p.E, p.S, p.active, p.ctrl, p.T, lane);
     }
 }
 
@@ -494,7 +551,7 @@ __global__ void __launch_bounds__(32) route_scatter_kernel(RouteArgs p) {
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     if (a.T <= kSmallT) {
-        route_small_kernel<<<(a.E + 1) / 2, 256, 0, s>>>(a);
+        route_small_kernel<<<a.E, 256, 0, s>>>(a);
         return cudaGetLastError();
     }
     const int zwarps = a.T * (a.H / 64);
