@@ -43,7 +43,7 @@ METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B2
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # gate/up kernel of each path and the sources its ncu traffic record is tied to
 PATHS = {
-    "decode": ("ffn_decode_kernel<0, NT, NW> (gate/up + SwiGLU)",
+    "decode": ("ffn_decode_kernel<0> (gate/up + SwiGLU; interval includes the K-part reduction when K is split)",
                ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "prefill": ("tc_gemm_kernel<0> (gate/up + SwiGLU, tcgen05; interval includes the token gather)",
                 ["bit_routed_expert_fp32_b200/csrc/prefill_tc.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
@@ -56,11 +56,35 @@ def path_of(cfg) -> str:
     return "prefill" if cfg.T > 64 and tc_ok else "decode"
 
 
+def decode_kparts(cfg):
+    """K parts of the decode gate/up and down passes: the library's split rule (kernels.h,
+    decode_kparts) restated, so that the launch count below is exact."""
+    if cfg.T < 1 or cfg.T > 64:
+        return 1, 1
+    active = min(cfg.T * cfg.k, cfg.E) + cfg.S
+    target = 3 * 148 * 16 // 2
+
+    def pick(K, rows):
+        nc = (K // 64 + 7) // 8
+        base = active * (rows // 32)
+        for n in range(1, nc + 1):
+            cpk = (nc + n - 1) // n
+            eff = (nc + cpk - 1) // cpk
+            if base * eff >= target or n == nc:
+                return eff
+        return 1
+
+    return pick(cfg.H, 2 * cfg.I), pick(cfg.I, cfg.H)
+
+
 def launches_per_step(cfg) -> int:
     """Kernels one step launches: routing (one fused kernel up to 64 tokens, else four)
-    plus gate/up, down and combine, plus the token gather on the prefill path."""
+    plus gate/up, down and combine, plus the token gather on the prefill path and the
+    K-part reduction of gate/up on the decode path when K is split."""
     route = 1 if cfg.T <= 64 else 4
-    return route + (4 if path_of(cfg) == "prefill" else 3)
+    if path_of(cfg) == "prefill":
+        return route + 4
+    return route + 3 + (1 if decode_kparts(cfg)[0] > 1 else 0)
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
