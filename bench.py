@@ -62,7 +62,7 @@ def decode_kparts(cfg):
     if cfg.T < 1 or cfg.T > 64:
         return 1, 1
     active = min(cfg.T * cfg.k, cfg.E) + cfg.S
-    target = 3 * 148 * 16 // 2
+    target = 3 * 148 * 16
 
     def pick(K, rows):
         nc = (K // 64 + 7) // 8

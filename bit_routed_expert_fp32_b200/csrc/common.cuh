@@ -36,7 +36,8 @@ struct Ctrl {
     uint32_t topk_ticket;
     int32_t n_active;       // experts with tokens + shared experts, written by moe_route
     int32_t routed_T;       // T of the last moe_route
-    uint32_t pad[58];
+    uint32_t work[2];       // decode work counters (gate/up, down); zeroed by the router and the combine
+    uint32_t pad[56];
 };
 
 // error detail codes

@@ -193,7 +193,9 @@ struct CtaSched {
     int fmt[kMaxActive];
     int cnt[kMaxActive];       // tokens of the expert
     int off[kMaxActive];       // first permuted row (routed experts)
-    int upre[kMaxActive + 1];  // unit prefix over active experts
+    int upre[kMaxActive + 1];  // expert-pass prefix over active experts
+    int one_pass;              // every active expert has at most 8 tokens
+    int n_ep;                  // expert passes
     int tok[kPermSmem];        // source token of permuted row r (perm[r] / k)
 };
 
@@ -201,50 +203,47 @@ struct UnitPos {
     int a, pass, jb, kp;
 };
 
-// Units are ordered (active expert, 32-row block, K part, token pass), pass fastest.
-__device__ __forceinline__ UnitPos unit_pos(const CtaSched& S, int u, int blocks, int nkp) {
-    int lo = 0, hi = S.n_active - 1;                   // largest a with upre[a] <= u
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (S.upre[mid] <= u) lo = mid;
-        else hi = mid - 1;
+// Division by a divisor fixed for the launch, through a float reciprocal and one
+// correction step (exact for dividends below 2^22).
+struct FastDiv {
+    int d;
+    float inv;
+    __device__ __forceinline__ void init(int dd) {
+        d = dd;
+        inv = 1.0f / (float)dd;
     }
-    UnitPos q;
-    q.a = lo;
-    int r = u - S.upre[lo];
-    const int np = (S.cnt[lo] + TP - 1) / TP;
-    q.pass = r % np;
-    r /= np;
-    q.kp = r % nkp;
-    q.jb = r / nkp;
-    return q;
-}
-
-// Walks consecutive units (pass fastest, then K part, block, expert) without
-// divisions; seek() places it on any unit.
-struct UnitIt {
-    int u, a, jb, kp, pass, np;
-    __device__ __forceinline__ void seek(const CtaSched& S, int u0, int blocks, int nkp) {
-        u = u0;
-        if (u0 >= S.n_units) return;
-        const UnitPos q = unit_pos(S, u0, blocks, nkp);
-        a = q.a;
-        jb = q.jb;
-        kp = q.kp;
-        pass = q.pass;
-        np = (S.cnt[a] + TP - 1) / TP;
-    }
-    __device__ __forceinline__ void next(const CtaSched& S, int blocks, int nkp) {
-        ++u;
-        if (++pass < np) return;
-        pass = 0;
-        if (++kp < nkp) return;
-        kp = 0;
-        if (++jb < blocks) return;
-        jb = 0;
-        if (++a < S.n_active) np = (S.cnt[a] + TP - 1) / TP;
+    __device__ __forceinline__ int div(int n) const {
+        int q = (int)((float)n * inv);
+        if ((q + 1) * d <= n) ++q;
+        else if (q * d > n) --q;
+        return q;
     }
 };
+
+// Units are ordered (active expert, token pass, 32-row block, K part), K part fastest;
+// unit u -> expert pass ep = u / (blocks * nkp), then block and K part.  ep is the
+// active expert itself when every active expert has one pass (at most 8 tokens).
+__device__ __forceinline__ UnitPos unit_pos(const CtaSched& S, int u, const FastDiv& per_ep, const FastDiv& nkp) {
+    UnitPos q;
+    const int ep = per_ep.div(u);
+    const int r = u - ep * per_ep.d;
+    q.jb = nkp.div(r);
+    q.kp = r - q.jb * nkp.d;
+    if (S.one_pass) {
+        q.a = ep;
+        q.pass = 0;
+    } else {
+        int lo = 0, hi = S.n_active - 1;               // largest a with upre[a] <= ep
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (S.upre[mid] <= ep) lo = mid;
+            else hi = mid - 1;
+        }
+        q.a = lo;
+        q.pass = ep - S.upre[lo];
+    }
+    return q;
+}
 
 __device__ __forceinline__ int src_token(const FfnArgs& p, const CtaSched& S, int row) {
     return S.perm_in_smem ? S.tok[row] : __ldg(p.perm + row) / p.k;
@@ -411,32 +410,57 @@ struct Geo {
     int K, G, NC, blocks, nkp, cpk;
 };
 
-// Producer side of a warp's ring: issues the bulk copies of the next chunk of the
-// unit it is on (both tiles of the block: up to six copies), from one elected lane of
-// the converged warp, then moves to the next chunk / unit.
+// Producer side of a warp's ring.  Units are handed out at run time: the elected lane
+// takes the next unit index from the launch's work counter one unit ahead of need, so
+// the atomic's latency hides behind a chunk of work and every warp keeps busy until
+// the counter runs out.  The producer issues the bulk copies of one chunk (both tiles
+// of the block) per call and remembers which unit and chunk each of the last NS
+// issues carried, which is what the consumer reads back NS - 1 calls later.
 template <int MODE>
 struct Producer {
     const uint8_t* codes;
     const uint8_t* hi;
     const uint8_t* sc;
-    UnitIt it;
-    int u_end, c, c_end, q3, issued, cur_a;
-    __device__ void begin(const FfnArgs& p, const CtaSched& S, const Geo& geo) {
-        if (it.u >= u_end) return;
-        c = it.kp * geo.cpk;
+    int cur, jb, c, c_end, q3, cur_a, issued;
+    int pend;                                         // lane 0: the unit grabbed for after cur
+    int hu[NS], hc[NS];                               // unit / chunk of the last NS issues (0 = latest)
+    __device__ __forceinline__ int grab(uint32_t* ctr, int lane) {
+        int g = 0;
+        if (lane == 0) g = (int)atomicAdd(ctr, 1u);
+        return g;
+    }
+    __device__ void start(const FfnArgs& p, const CtaSched& S, const Geo& geo, const FastDiv& per_ep,
+                          const FastDiv& nkp, uint32_t* ctr, int lane, int unit) {
+        cur = unit;
+        if (cur >= S.n_units) {
+            cur = -1;
+            return;
+        }
+        const UnitPos q = unit_pos(S, cur, per_ep, nkp);
+        jb = q.jb;
+        c = q.kp * geo.cpk;
         c_end = min(geo.NC, c + geo.cpk);
-        if (it.a != cur_a) {
-            cur_a = it.a;
-            const PackedEntry* en = entry(p.packed, S.e[it.a]);
+        if (q.a != cur_a) {
+            cur_a = q.a;
+            const PackedEntry* en = entry(p.packed, S.e[q.a]);
             codes = p.packed + (MODE == 0 ? en->gu_codes : en->dn_codes);
             hi = p.packed + (MODE == 0 ? en->gu_hi : en->dn_hi);
             sc = p.packed + (MODE == 0 ? en->gu_scales : en->dn_scales);
-            q3 = S.fmt[it.a] == MOE_FMT_Q3;
+            q3 = S.fmt[q.a] == MOE_FMT_Q3;
         }
+        pend = grab(ctr, lane);                       // the unit after this one
     }
-    __device__ void issue(const FfnArgs& p, const CtaSched& S, const Geo& geo, uint8_t* ring, uint64_t* bar,
+    __device__ void issue(const FfnArgs& p, const CtaSched& S, const Geo& geo, const FastDiv& per_ep,
+                          const FastDiv& nkp, uint32_t* ctr, int lane, uint8_t* ring, uint64_t* bar,
                           uint64_t pol) {
-        if (it.u >= u_end) return;
+#pragma unroll
+        for (int i = NS - 1; i > 0; --i) {
+            hu[i] = hu[i - 1];
+            hc[i] = hc[i - 1];
+        }
+        hu[0] = cur;
+        hc[0] = c;
+        if (cur < 0) return;
         const int st = issued % NS;
         const int ng = min(CG, geo.G - c * CG);
         if (elect_one()) {
@@ -445,7 +469,7 @@ struct Producer {
             mbar_arrive_expect_tx(&bar[st], NTL * (cb + hb + 256));
 #pragma unroll
             for (int tl = 0; tl < NTL; ++tl) {
-                const int j = NTL * it.jb + tl;
+                const int j = NTL * jb + tl;
                 uint8_t* d = dst + tl * TSTAGE;
                 bulk_g2s_evict_first(d, codes + (size_t)4 * geo.K * j + 2048 * (size_t)c, cb, &bar[st], pol);
                 bulk_g2s_evict_first(d + OFF_SC, sc + (size_t)256 * geo.NC * j + 256 * (size_t)c, 256, &bar[st],
@@ -457,49 +481,15 @@ struct Producer {
         }
         __syncwarp();
         ++issued;
-        if (++c == c_end) {
-            it.next(S, geo.blocks, geo.nkp);
-            begin(p, S, geo);
-        }
+        if (++c == c_end) start(p, S, geo, per_ep, nkp, ctr, lane, __shfl_sync(0xffffffffu, pend, 0));
     }
 };
 
-// One unit: its chunks through the ring, then the epilogue.
-template <int MODE, bool Q3>
-__device__ __forceinline__ void run_unit(const FfnArgs& p, const CtaSched& S, const Geo& geo, const UnitPos& q,
-                                         Producer<MODE>& prod, int& consumed, bool& aborted, uint8_t* ring,
-                                         uint64_t* bar, uint64_t pol, const LaneGeo& L) {
-    UnitView v;
-    make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
-    uint32_t sub[5] = {0, 0, 0, 0, 0};
-    if (MODE == 1) {
-        const int f = S.fmt[q.a];
-        const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
-        sub[0] = f16x2_bits_of(512.f + o);
-        sub[1] = f16x2_bits_of(256.f + o);
-        sub[2] = f16x2_bits_of(64.f + o);
-        sub[3] = f16x2_bits_of(16.f + o);
-        sub[4] = f16x2_bits_of(4.f + o);
-    }
-    float acc[NTL][4];
-#pragma unroll
-    for (int tl = 0; tl < NTL; ++tl) acc[tl][0] = acc[tl][1] = acc[tl][2] = acc[tl][3] = 0.f;
-    const int c0 = q.kp * geo.cpk, c1 = min(geo.NC, c0 + geo.cpk);
-    for (int c = c0; c < c1; ++c) {
-        prod.issue(p, S, geo, ring, bar, pol);
-        const int st = consumed % NS;
-        if (!aborted && !mbar_wait_bounded(&bar[st], (uint32_t)(consumed / NS) & 1, kWaitLimit)) {
-            aborted = true;
-            report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | MODE);
-        }
-        const uint8_t* stg = ring + (size_t)st * STAGE;
-        const int ng = min(CG, geo.G - c * CG);
-        if (ng == CG) chunk_full<MODE, Q3>(stg, c, v, L, sub, acc);
-        else chunk_partial<MODE, Q3>(stg, c, ng, v, L, sub, acc);
-        __syncwarp();          // every lane is done with this stage before it is refilled
-        ++consumed;
-    }
-    // epilogue: tile j = NTL jb + tl, rows g (gate / first half) and g + 8 (up / second half)
+// The output of one finished unit: tile j = NTL jb + tl, rows g (gate / first half) and
+// g + 8 (up / second half) of this lane's token columns.
+template <int MODE>
+__device__ __forceinline__ void unit_epilogue(const FfnArgs& p, const Geo& geo, const UnitPos& q, const UnitView& v,
+                                              const LaneGeo& L, const float (&acc)[NTL][4]) {
     const size_t R = (size_t)p.T * (p.k + p.S);
 #pragma unroll
     for (int tl = 0; tl < NTL; ++tl) {
@@ -589,37 +579,39 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         for (int r = threadIdx.x; r < p.T * p.k; r += blockDim.x) S.tok[r] = p.perm[r] / p.k;
     __syncthreads();
     if (threadIdx.x == 0) {
-        int run = 0;
+        int run = 0, one = 1;
         for (int a = 0; a < nA; ++a) {
             S.upre[a] = run;
-            run += ((S.cnt[a] + TP - 1) / TP) * geo.blocks * geo.nkp;
+            const int np = (S.cnt[a] + TP - 1) / TP;
+            run += np;
+            one &= np == 1;
         }
         S.upre[nA] = run;
-        S.n_units = run;
+        S.n_ep = run;
+        S.one_pass = one;
+        S.n_units = run * geo.blocks * geo.nkp;
     }
     if (MODE == 0) warm_z(p);
     if (lane == 0)
         for (int s = 0; s < NS; ++s) mbar_init(&bar[s], 1);
     fence_mbar_init();
     __syncthreads();
-    const int n_units = S.n_units;
-    // Every warp takes a contiguous range of units.  Range r goes to CTA r % grid and
-    // warp slot r / grid, with warp = 5 * slot mod 16: consecutive ranges (one
-    // expert's units) spread over all SMs, and the slots of one SM over its four
-    // schedulers.
-    const int P = gridDim.x * NW;
-    const int slot = (warp * 13) & (NW - 1);           // the inverse of 5 mod 16
-    const int r = slot * gridDim.x + blockIdx.x;
-    const int u0 = (int)(((long long)n_units * r) / P), u1 = (int)(((long long)n_units * (r + 1)) / P);
+    // Units come from the launch's work counter (zeroed by the router and by the
+    // combine, so every forward starts from 0); a warp grabs its first unit here and
+    // each following one a unit ahead of need (Producer).
+    uint32_t* ctr = &p.ctrl->work[MODE];
+    FastDiv per_ep, fkp;
+    per_ep.init(geo.blocks * geo.nkp);
+    fkp.init(geo.nkp);
     const uint64_t pol = l2_policy_evict_first();
 
     Producer<MODE> prod;
-    prod.u_end = u1;
     prod.issued = 0;
     prod.cur_a = -1;
-    prod.it.seek(S, u0, geo.blocks, geo.nkp);
-    prod.begin(p, S, geo);
-    for (int i = 0; i < NS - 1; ++i) prod.issue(p, S, geo, ring, bar, pol);
+#pragma unroll
+    for (int i = 0; i < NS; ++i) prod.hu[i] = -1;
+    prod.start(p, S, geo, per_ep, fkp, ctr, lane, __shfl_sync(0xffffffffu, prod.grab(ctr, lane), 0));
+    for (int i = 0; i < NS - 1; ++i) prod.issue(p, S, geo, per_ep, fkp, ctr, lane, ring, bar, pol);
 
     LaneGeo L;
     L.g = lane >> 2;
@@ -631,18 +623,60 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     L.sh = 8 * (L.t & 1);
     bool aborted = false;
     int consumed = 0;
-    UnitIt it;
-    it.seek(S, u0, geo.blocks, geo.nkp);
-    for (; it.u < u1; it.next(S, geo.blocks, geo.nkp)) {
-        UnitPos q;
-        q.a = it.a;
-        q.jb = it.jb;
-        q.kp = it.kp;
-        q.pass = it.pass;
-        if (S.fmt[q.a] == MOE_FMT_Q3)
-            run_unit<MODE, true>(p, S, geo, q, prod, consumed, aborted, ring, bar, pol, L);
-        else
-            run_unit<MODE, false>(p, S, geo, q, prod, consumed, aborted, ring, bar, pol, L);
+    // The chunk to consume is the one issued NS - 1 issues ago (hu / hc[NS - 1] after
+    // the next issue).  A unit ends when the next chunk belongs to another unit.
+    int unit = -1, view_a = -1, view_pass = -1;
+    bool q3 = false;
+    UnitPos q;
+    q.a = q.pass = q.jb = q.kp = 0;
+    UnitView v;
+    uint32_t sub[5] = {0, 0, 0, 0, 0};
+    float acc[NTL][4];
+    while (true) {
+        prod.issue(p, S, geo, per_ep, fkp, ctr, lane, ring, bar, pol);
+        const int hu = prod.hu[NS - 1], c = prod.hc[NS - 1];
+        if (hu < 0) {                                   // nothing left (or nothing at all)
+            if (unit >= 0) unit_epilogue<MODE>(p, geo, q, v, L, acc);
+            break;
+        }
+        if (hu != unit) {
+            if (unit >= 0) unit_epilogue<MODE>(p, geo, q, v, L, acc);
+            unit = hu;
+            q = unit_pos(S, unit, per_ep, fkp);
+            if (q.a != view_a || q.pass != view_pass) {
+                view_a = q.a;
+                view_pass = q.pass;
+                make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
+                q3 = S.fmt[q.a] == MOE_FMT_Q3;
+                if (MODE == 1) {
+                    const int f = S.fmt[q.a];
+                    const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
+                    sub[0] = f16x2_bits_of(512.f + o);
+                    sub[1] = f16x2_bits_of(256.f + o);
+                    sub[2] = f16x2_bits_of(64.f + o);
+                    sub[3] = f16x2_bits_of(16.f + o);
+                    sub[4] = f16x2_bits_of(4.f + o);
+                }
+            }
+#pragma unroll
+            for (int tl = 0; tl < NTL; ++tl) acc[tl][0] = acc[tl][1] = acc[tl][2] = acc[tl][3] = 0.f;
+        }
+        const int st = consumed % NS;
+        if (!aborted && !mbar_wait_bounded(&bar[st], (uint32_t)(consumed / NS) & 1, kWaitLimit)) {
+            aborted = true;
+            report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | MODE);
+        }
+        const uint8_t* stg = ring + (size_t)st * STAGE;
+        const int ng = min(CG, geo.G - c * CG);
+        if (ng == CG) {
+            if (q3) chunk_full<MODE, true>(stg, c, v, L, sub, acc);
+            else chunk_full<MODE, false>(stg, c, v, L, sub, acc);
+        } else {
+            if (q3) chunk_partial<MODE, true>(stg, c, ng, v, L, sub, acc);
+            else chunk_partial<MODE, false>(stg, c, ng, v, L, sub, acc);
+        }
+        __syncwarp();          // every lane is done with this stage before it is refilled
+        ++consumed;
     }
     // after a timeout the ring may still hold copies in flight: wait for them (bounded)
     if (aborted) {
@@ -708,6 +742,10 @@ __device__ __forceinline__ void add4(float4& a, const float4& b) {
 template <bool SMALL>
 __global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
     griddep_wait();                                     // ypart comes from the down pass
+    if (blockIdx.x == 0 && threadIdx.x == 0) {          // both expert passes are complete
+        p.ctrl->work[0] = 0;
+        p.ctrl->work[1] = 0;
+    }
     const int per_tok = p.H / 4;
     const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (size_t)p.T * per_tok) return;

@@ -54,14 +54,14 @@ Ws ws_layout(const moe_shape* s, int64_t T);
 
 // K parts of the decode-path expert passes for T tokens.  With few tokens only a few
 // experts are active and their 32-row blocks are fewer than the warps of the GPU, so
-// K is split (into whole 8-group chunks) until there are about one and a half units
-// per warp of a reference 148-SM part (finer splits measured no faster: more partial
-// traffic and per-unit work).  Only for T <= kSmallT; 1 otherwise.
+// K is split (into whole 8-group chunks) until there are about three units per warp
+// of a reference 148-SM part; the warps take units at run time, which balances the
+// SMs (finer splits measured no faster).  Only for T <= kSmallT; 1 otherwise.
 inline void decode_kparts(const moe_shape* s, int64_t T, int* nkp_gu, int* nkp_dn) {
     *nkp_gu = *nkp_dn = 1;
     if (T < 1 || T > kSmallT) return;
     const int64_t active = (T * s->top_k < s->n_experts ? T * s->top_k : s->n_experts) + s->n_shared;
-    const int64_t target = 3 * 148 * 16 / 2;
+    const int64_t target = 3 * 148 * 16;
     auto pick = [&](int K, int rows) {
         const int nc = (K / 64 + 7) / 8;
         const int64_t base = active * (rows / 32);

@@ -177,6 +177,10 @@ __device__ void compute_z(const RouteArgs& p, int t, int Gi, int lane) {
 }
 
 __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {          // no expert pass of this workspace runs now
+        p.ctrl->work[0] = 0;
+        p.ctrl->work[1] = 0;
+    }
     const int G = p.H / 64;
     const int warp = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (warp < p.T * G) compute_z(p, warp / G, warp % G, lane);
@@ -245,6 +249,10 @@ constexpr int kRouteVec = 7;                           // float4 of the row per 
 
 __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
     griddep_launch_dependents();        // one wave of CTAs: the expert pass may start launching
+    if (blockIdx.x == 0 && threadIdx.x == 0) {          // no expert pass of this workspace runs now
+        p.ctrl->work[0] = 0;
+        p.ctrl->work[1] = 0;
+    }
     __shared__ float s_part[8][kSmallT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x;

@@ -58,6 +58,6 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
 def test_paths_and_launch_counts():
     c2, c4 = synth.CONFIGS[2], synth.CONFIGS[4]
     # one token: 9 active experts, so gate/up K is split into parts and reduced by one more kernel
-    assert bench.decode_kparts(c2) == (4, 2)
+    assert bench.decode_kparts(c2) == (7, 4)
     assert bench.path_of(c2) == "decode" and bench.launches_per_step(c2) == 1 + 4
     assert bench.path_of(c4) == "prefill" and bench.launches_per_step(c4) == 4 + 4
