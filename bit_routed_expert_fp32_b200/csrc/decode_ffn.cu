@@ -729,9 +729,9 @@ __global__ void __launch_bounds__(128) finalize_gateup_kernel(FfnArgs p) {
 }
 
 // y[t] = sum_j g[t,j] * ypart[inv_perm[t*k + j]] + sum_s ypart[T*k + s*T + t], in slot
-// order, each row first summed over its K parts in order; fp32, stored as bf16.  One
-// thread per 4 consecutive outputs.  For few tokens the slot rows and gates are loaded
-// first, then every partial row, so the pass costs two L2 round trips.
+// order, each row first summed over its K parts in order; fp32, stored as bf16.  For few
+// tokens: one thread per 4 consecutive outputs, the slot rows and gates loaded first,
+// then every partial row, so the pass costs two L2 round trips.
 constexpr int kMaxRows = 12;                            // k + S rows per token ...
 constexpr int kMaxKp = 4;                               // ... and K parts held in registers
 
@@ -739,7 +739,6 @@ __device__ __forceinline__ void add4(float4& a, const float4& b) {
     a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
 }
 
-template <bool SMALL>
 __global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
     griddep_wait();                                     // ypart comes from the down pass
     if (blockIdx.x == 0 && threadIdx.x == 0) {          // both expert passes are complete
@@ -754,7 +753,7 @@ __global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
     const size_t pstride = R * p.H;
     const int nrows = p.k + p.S;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (SMALL && nrows <= kMaxRows && p.nkp_dn <= kMaxKp) {
+    if (nrows <= kMaxRows && p.nkp_dn <= kMaxKp) {
         int rows[kMaxRows];
         float gw[kMaxRows];
 #pragma unroll
@@ -814,6 +813,51 @@ __global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
     *reinterpret_cast<uint2*>(p.y + (size_t)tok * p.H + c4) = o;
 }
 
+// The same combine for many tokens: one thread per 8 consecutive outputs of a token
+// (two 16-byte loads per row and part), rows one after another.
+__global__ void __launch_bounds__(256) combine_rows_kernel(FfnArgs p) {
+    griddep_wait();                                     // ypart comes from the down pass
+    if (blockIdx.x == 0 && threadIdx.x == 0) {          // both expert passes are complete
+        p.ctrl->work[0] = 0;
+        p.ctrl->work[1] = 0;
+    }
+    const int per_tok = p.H / 8;
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (size_t)p.T * per_tok) return;
+    const int tok = (int)(idx / per_tok), c8 = (int)(idx - (size_t)tok * per_tok) * 8;
+    const size_t pstride = (size_t)p.T * (p.k + p.S) * p.H;
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    for (int r = 0; r < p.k + p.S; ++r) {
+        const int row = r < p.k ? p.inv_perm[(size_t)tok * p.k + r] : p.T * p.k + (r - p.k) * p.T + tok;
+        const float4* src = reinterpret_cast<const float4*>(p.ypart + (size_t)row * p.H + c8);
+        float4 s0 = __ldcg(src), s1 = __ldcg(src + 1);
+        for (int kp = 1; kp < p.nkp_dn; ++kp) {
+            add4(s0, __ldcg(src + kp * (pstride / 4)));
+            add4(s1, __ldcg(src + kp * (pstride / 4) + 1));
+        }
+        if (r < p.k) {
+            const float g = p.topk_w[(size_t)tok * p.k + r];
+            a0.x = fmaf(g, s0.x, a0.x);
+            a0.y = fmaf(g, s0.y, a0.y);
+            a0.z = fmaf(g, s0.z, a0.z);
+            a0.w = fmaf(g, s0.w, a0.w);
+            a1.x = fmaf(g, s1.x, a1.x);
+            a1.y = fmaf(g, s1.y, a1.y);
+            a1.z = fmaf(g, s1.z, a1.z);
+            a1.w = fmaf(g, s1.w, a1.w);
+        } else {
+            add4(a0, s0);
+            add4(a1, s1);
+        }
+    }
+    uint4 o;
+    o.x = (uint32_t)f32_to_bf16_bits(a0.x) | ((uint32_t)f32_to_bf16_bits(a0.y) << 16);
+    o.y = (uint32_t)f32_to_bf16_bits(a0.z) | ((uint32_t)f32_to_bf16_bits(a0.w) << 16);
+    o.z = (uint32_t)f32_to_bf16_bits(a1.x) | ((uint32_t)f32_to_bf16_bits(a1.y) << 16);
+    o.w = (uint32_t)f32_to_bf16_bits(a1.z) | ((uint32_t)f32_to_bf16_bits(a1.w) << 16);
+    *reinterpret_cast<uint4*>(p.y + (size_t)tok * p.H + c8) = o;
+}
+
 constexpr size_t kDynSmem = (size_t)NW * NS * STAGE + (size_t)NW * NS * 8;
 
 template <int MODE>
@@ -846,11 +890,13 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_g
 }
 
 cudaError_t launch_combine(const FfnArgs& a, cudaStream_t s) {
-    const long long n = (long long)a.T * (a.H / 4);
-    const dim3 grid((unsigned)((n + 127) / 128));
-    // few tokens: a latency-bound pass, every load issued up front; many tokens: plain
-    return a.T <= kSmallT ? launch_pdl(combine_kernel<true>, grid, dim3(128), 0, s, a)
-                          : launch_pdl(combine_kernel<false>, grid, dim3(128), 0, s, a);
+    // few tokens: a latency-bound pass, every load issued up front; many tokens: rows
+    if (a.T <= kSmallT) {
+        const long long n = (long long)a.T * (a.H / 4);
+        return launch_pdl(combine_kernel, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, s, a);
+    }
+    const long long n = (long long)a.T * (a.H / 8);
+    return launch_pdl(combine_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, a);
 }
 
 }  // namespace moe
