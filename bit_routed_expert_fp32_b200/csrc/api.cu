@@ -32,7 +32,7 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     w.hist = off;
     off = align256(off + 4 * (size_t)(((T + kChunk - 1) / kChunk) * E));
     w.zx = off;
-    off = align256(off + 4 * (size_t)(3 * (H / 64) * T));
+    off = align256(off + 4 * (size_t)(3 * (8 * ((H / 64 + 7) / 8)) * T));   // two fp16 planes
     w.h = off;
     off = align256(off + 2 * (size_t)(T * (k + S) * I));
     // ypart, and the decode gate/up partial sums that alias it: the largest need of any

@@ -29,10 +29,11 @@
 //    exponent trick: the code lands in the mantissa of a power-of-two base, exactly),
 //    the A operand of mma.sync m16n8k16; the tokens are N (8 per n-tile) and the B
 //    fragments come straight from the token rows (L1-resident).
-//      gate/up: pairs stay "base + c"; each group's accumulator starts at
-//        -Z[token, group] (Z = sum base(k) x_k + o sum x_k, plus the third-bit bases
-//        for 3-bit experts; computed by the router), so the MMA yields
-//        sum (c_k - o) x_k.  bf16 MMAs: the tokens are bf16.
+//      gate/up: pairs stay "base + c", so a group's MMAs yield sum (base_k + c_k) x_k;
+//        once per chunk a small fp16 MMA of the scales against the router's table of
+//        -Z (Z = sum base(k) x_k + o sum x_k, plus the third-bit bases for 3-bit
+//        experts) removes the offsets, leaving sum (c_k - o) x_k.  bf16 MMAs: the
+//        tokens are bf16.
 //      down: pairs are (c - o) exactly (one fp16x2 subtract); fp16 MMAs, h is fp16.
 //    Each group result is scaled by its fp16 scale into an fp32 accumulator.
 //    3-bit experts add an MMA per k-step for 4 * (third bit).
@@ -174,6 +175,34 @@ __device__ __forceinline__ void mma_group(float (&d)[4], const uint32_t (&pa)[8]
     mma_acc<MODE>(d, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
 }
 
+// The same four k-steps with a zero accumulator input (the group's sum starts at 0).
+template <int MODE>
+__device__ __forceinline__ void mma_group_first(float (&d)[4], const uint32_t (&pa)[8], const uint32_t (&pb)[8],
+                                                const uint4& x0, const uint4& x1) {
+    const float zero = 0.f;
+    if (MODE == 0)
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(pa[0]), "r"(pb[0]), "r"(pa[1]), "r"(pb[1]), "r"(x0.x), "r"(x0.y), "f"(zero));
+    else
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(pa[0]), "r"(pb[0]), "r"(pa[1]), "r"(pb[1]), "r"(x0.x), "r"(x0.y), "f"(zero));
+    mma_acc<MODE>(d, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
+    mma_acc<MODE>(d, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
+    mma_acc<MODE>(d, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
+}
+
+// acc += A B with A 16 x 8 fp16 (row-major fragment: rows g and g + 8, k = 2t, 2t+1)
+// and B 8 x 8 fp16 (k = 2t, 2t+1 of column g); fp32 accumulation.
+__device__ __forceinline__ void mma_f16_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(b0));
+}
+
 __device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xFFFFu))); }
 __device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w >> 16))); }
 __device__ __forceinline__ const PackedEntry* entry(const uint8_t* packed, int e) {
@@ -252,8 +281,7 @@ __device__ __forceinline__ int src_token(const FfnArgs& p, const CtaSched& S, in
 // Per-lane view of one unit: B row, -Z rows and output rows of this lane's columns.
 struct UnitView {
     const uint16_t* b;         // B-operand row of token column g (+16t elements)
-    const float* z0;           // -Z rows of output columns 2t, 2t+1 (gate/up only)
-    const float* z1;
+    const uint16_t* z;         // gate/up: -Z/16 (hi plane) of token column g, groups 2t, 2t+1
     int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token)
 };
 
@@ -276,16 +304,14 @@ __device__ __forceinline__ void make_view(const FfnArgs& p, const CtaSched& S, i
         brow = MODE == 0 ? i : srow0 + i;
     }
     v.b = (MODE == 0 ? p.x : p.h) + (size_t)brow * (MODE == 0 ? p.H : p.I) + 16 * t;
+    const int G8 = 8 * ((G + 7) / 8);
+    v.z = MODE == 0 ? reinterpret_cast<const uint16_t*>(p.zx) + ((size_t)f * p.T + brow) * G8 + 2 * t : nullptr;
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
         const int col = 2 * t + cc;
         const int ii = tb + (col < nb ? col : 0);
         const int orow = routed ? S.off[a] + ii : srow0 + ii;
         v.orow[cc] = col < nb ? orow : -1;
-        const float* zr = nullptr;
-        if (MODE == 0) zr = p.zx + ((size_t)f * p.T + (routed ? src_token(p, S, orow) : ii)) * G;
-        if (cc == 0) v.z0 = zr;
-        else v.z1 = zr;
     }
 }
 
@@ -294,16 +320,44 @@ __device__ __forceinline__ void make_view(const FfnArgs& p, const CtaSched& S, i
 // third-bit words (row g + 8: 128 words on), sh the third-bit half of this lane.
 struct LaneGeo {
     int g, t, cw_lane, g4, hw_lane, g2, sh;
+    int zplane;                // elements from the hi to the lo plane of the Z table
 };
+
+__device__ __forceinline__ uint32_t f16x2_mul16(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Gate/up: the group MMAs sum (base + c) x from zero; this subtracts the offsets of a
+// whole 8-group chunk at once, acc[row][col] += sum_gl 16 s[row][gl] * (-Z[col][gl] / 16),
+// as two m16n8k8 fp16 MMAs per tile (the hi and lo halves of -Z / 16).  A: this lane's
+// scale words of rows g and g + 8 (groups 2t, 2t+1), times 16 (exact); B: the two
+// fp16 halves of -Z / 16 for token column g at groups 2t, 2t+1.  Groups past K in a
+// partial chunk have zero scales and zero Z.
+__device__ __forceinline__ void z_correction(const uint8_t* stg, int c, const UnitView& v, const LaneGeo& L,
+                                             float (&acc)[NTL][4]) {
+    constexpr uint32_t kSixteen = 0x4C004C00u;         // fp16 16.0 in both halves
+    const uint32_t bhi = __ldg(reinterpret_cast<const uint32_t*>(v.z + 8 * c));
+    const uint32_t blo = __ldg(reinterpret_cast<const uint32_t*>(v.z + L.zplane + 8 * c));
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + tl * TSTAGE + OFF_SC);
+        const uint32_t a0 = f16x2_mul16(scw[4 * L.g + L.t], kSixteen);
+        const uint32_t a1 = f16x2_mul16(scw[4 * (L.g + 8) + L.t], kSixteen);
+        mma_f16_1688(acc[tl], a0, a1, bhi);
+        mma_f16_1688(acc[tl], a0, a1, blo);
+    }
+}
 
 // Group gl of a full chunk, every tile of the block: code words from the swizzled
 // stage, the B fragments of the group, the MMAs and the scaled fold into acc.  s2:
 // per tile, the scale words of rows g and g + 8 that hold groups gl & ~1 and gl | 1;
 // HI selects the half of group gl.
 template <int MODE, bool Q3, int HI>
-__device__ __forceinline__ void group_full(const uint8_t* stg, int gl, const uint16_t* bx, const float* zc0,
-                                           const float* zc1, const LaneGeo& L, const uint32_t (&s2)[NTL][2],
-                                           const uint32_t (&sub)[5], float (&acc)[NTL][4]) {
+__device__ __forceinline__ void group_full(const uint8_t* stg, int gl, const uint16_t* bx, const LaneGeo& L,
+                                           const uint32_t (&s2)[NTL][2], const uint32_t (&sub)[5],
+                                           float (&acc)[NTL][4]) {
     const uint32_t* cw = reinterpret_cast<const uint32_t*>(stg);
     const int cpos = L.cw_lane + ((4 * gl) ^ L.g4);
     uint32_t w[NTL][2], u[NTL][2];
@@ -324,14 +378,12 @@ __device__ __forceinline__ void group_full(const uint8_t* stg, int gl, const uin
     }
     const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(bx + 64 * gl));
     const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(bx + 64 * gl) + 1);
-    const float z0 = MODE == 0 ? __ldg(zc0 + gl) : 0.f;
-    const float z1 = MODE == 0 ? __ldg(zc1 + gl) : 0.f;
 #pragma unroll
     for (int tl = 0; tl < NTL; ++tl) {
         uint32_t pa[8], pb[8];
         dequant_rows<MODE>(w[tl][0], w[tl][1], sub, pa, pb);
-        float d[4] = {z0, z1, z0, z1};
-        mma_group<MODE>(d, pa, pb, x0, x1);
+        float d[4];
+        mma_group_first<MODE>(d, pa, pb, x0, x1);
         if (Q3) {
             dequant_hi_rows<MODE>(u[tl][0], u[tl][1], pa, pb);
             mma_group<MODE>(d, pa, pb, x0, x1);
@@ -353,8 +405,7 @@ __device__ __forceinline__ void chunk_full(const uint8_t* stg, int c, const Unit
                                            const uint32_t (&sub)[5], float (&acc)[NTL][4]) {
     const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + OFF_SC);   // row r: words 4r .. 4r+3
     const uint16_t* bx = v.b + c * (CG * 64);
-    const float* zc0 = MODE == 0 ? v.z0 + c * CG : nullptr;
-    const float* zc1 = MODE == 0 ? v.z1 + c * CG : nullptr;
+    if (MODE == 0) z_correction(stg, c, v, L, acc);
 #pragma unroll 1
     for (int gp = 0; gp < CG / 2; ++gp) {
         uint32_t s2[NTL][2];
@@ -363,8 +414,8 @@ __device__ __forceinline__ void chunk_full(const uint8_t* stg, int c, const Unit
             s2[tl][0] = scw[tl * (TSTAGE / 4) + 4 * L.g + gp];
             s2[tl][1] = scw[tl * (TSTAGE / 4) + 4 * (L.g + 8) + gp];
         }
-        group_full<MODE, Q3, 0>(stg, 2 * gp, bx, zc0, zc1, L, s2, sub, acc);
-        group_full<MODE, Q3, 1>(stg, 2 * gp + 1, bx, zc0, zc1, L, s2, sub, acc);
+        group_full<MODE, Q3, 0>(stg, 2 * gp, bx, L, s2, sub, acc);
+        group_full<MODE, Q3, 1>(stg, 2 * gp + 1, bx, L, s2, sub, acc);
     }
 }
 
@@ -374,12 +425,11 @@ template <int MODE, bool Q3>
 __device__ __forceinline__ void chunk_partial(const uint8_t* stg, int c, int ng, const UnitView& v,
                                               const LaneGeo& L, const uint32_t (&sub)[5], float (&acc)[NTL][4]) {
     const int g = L.g, t = L.t;
+    if (MODE == 0) z_correction(stg, c, v, L, acc);
     for (int gl = 0; gl < ng; ++gl) {
         const uint16_t* bp = v.b + c * (CG * 64) + 64 * gl;
         const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(bp));
         const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(bp) + 1);
-        const float z0 = MODE == 0 ? __ldg(v.z0 + c * CG + gl) : 0.f;
-        const float z1 = MODE == 0 ? __ldg(v.z1 + c * CG + gl) : 0.f;
 #pragma unroll
         for (int tl = 0; tl < NTL; ++tl) {
             const uint8_t* tb = stg + tl * TSTAGE;
@@ -388,8 +438,8 @@ __device__ __forceinline__ void chunk_partial(const uint8_t* stg, int c, int ng,
             const uint16_t* scs = reinterpret_cast<const uint16_t*>(tb + OFF_SC);
             uint32_t pa[8], pb[8];
             dequant_rows<MODE>(cw[g * 4 * ng + 4 * gl + t], cw[(g + 8) * 4 * ng + 4 * gl + t], sub, pa, pb);
-            float d[4] = {z0, z1, z0, z1};
-            mma_group<MODE>(d, pa, pb, x0, x1);
+            float d[4];
+            mma_group_first<MODE>(d, pa, pb, x0, x1);
             if (Q3) {
                 dequant_hi_rows<MODE>(hw[g * 2 * ng + 2 * gl + (t >> 1)] >> L.sh,
                                       hw[(g + 8) * 2 * ng + 2 * gl + (t >> 1)] >> L.sh, pa, pb);
@@ -518,9 +568,8 @@ __device__ __forceinline__ void unit_epilogue(const FfnArgs& p, const Geo& geo, 
 // the router ran); the Z values are the router's output and are prefetched only after
 // griddep_wait(), so no stale line can enter L1.  The zx region is padded to 256 bytes,
 // so whole lines stay inside it.
-__device__ inline bool warm_fits(const FfnArgs& p) {
-    return (size_t)p.T * p.H * 2 + (size_t)3 * p.T * (p.H / 64) * 4 <= 48 * 1024;
-}
+__device__ inline size_t z_bytes(const FfnArgs& p) { return (size_t)3 * p.T * (8 * ((p.H / 64 + 7) / 8)) * 4; }
+__device__ inline bool warm_fits(const FfnArgs& p) { return (size_t)p.T * p.H * 2 + z_bytes(p) <= 48 * 1024; }
 __device__ inline void warm_rows(const FfnArgs& p) {
     if (!warm_fits(p)) return;
     const size_t xb = (size_t)p.T * p.H * 2;
@@ -529,7 +578,7 @@ __device__ inline void warm_rows(const FfnArgs& p) {
 }
 __device__ inline void warm_z(const FfnArgs& p) {
     if (!warm_fits(p)) return;
-    const size_t zb = (size_t)3 * p.T * (p.H / 64) * 4;
+    const size_t zb = z_bytes(p);
     for (size_t i = threadIdx.x; i < (zb + 127) / 128; i += blockDim.x)
         prefetch_l1(reinterpret_cast<const uint8_t*>(p.zx) + i * 128);
 }
@@ -621,6 +670,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     L.hw_lane = 16 * L.g + (L.t >> 1);
     L.g2 = 2 * (L.g >> 1);
     L.sh = 8 * (L.t & 1);
+    L.zplane = 3 * p.T * (8 * ((p.H / 64 + 7) / 8));
     bool aborted = false;
     int consumed = 0;
     // The chunk to consume is the one issued NS - 1 issues ago (hu / hc[NS - 1] after

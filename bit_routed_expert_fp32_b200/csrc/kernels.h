@@ -19,7 +19,7 @@ struct RouteArgs {
     float* logits;      // ws [T][E]
     int32_t* hist;      // ws [ceil(T/kChunk)][E]
     int32_t* active;    // ws [E+S]
-    float* zx;          // ws [3][T][H/64] negated dequantiser offsets (see route.cu)
+    float* zx;          // ws fp16 planes [2][3][T][G8] of -Z/16, hi and lo (see route.cu)
     Ctrl* ctrl;
     moe_routing r;
 };
@@ -34,7 +34,7 @@ struct FfnArgs {
     const int32_t* offsets;
     const float* topk_w;
     const int32_t* active;   // ws
-    const float* zx;         // ws [3][T][H/64], negated
+    const float* zx;         // ws fp16 planes [2][3][T][G8] of -Z/16, hi and lo
     Ctrl* ctrl;
     uint16_t* h;             // ws fp16 [T*(k+S)][I]
     float* ypart;            // ws f32 [nkp_dn][T*(k+S)][H]

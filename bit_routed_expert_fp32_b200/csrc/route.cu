@@ -149,30 +149,44 @@ __device__ void warp_active(const int* s_cnt, int E, int S, int32_t* active, Ctr
 
 // ---------------------------------------------------------------- Z tables
 // The gate/up expert kernel feeds the MMA with "base + c" values straight out of the
-// code words (no per-pair subtraction) and starts every 64-wide group's accumulator
-// at -Z.  For token t and group G (elements x_e, e = 0..63 of the group):
+// code words (no per-pair subtraction), so each 64-wide group's MMA yields
+// sum (base + c) x, and the kernel subtracts Z once per 8-group chunk with a small MMA
+// of the scales against Z.  For token t and group G (elements x_e, e = 0..63):
 //   Bx = sum_e lo_base(e) x_e,  Hx = sum_e hi_base(e) x_e,  Sx = sum_e x_e,
 // with lo_base / hi_base the magic bases the expert kernel uses for the pair that
 // holds element e (pair p = (e % 16) / 2):  lo 128,32,8,128,32,8,128,32 and
 // hi 512,256,128,64,32,16,8,8.  Then for code offset o:
 //   Z_ternary = Bx + Sx,  Z_q2 = Bx + 1.5 Sx,  Z_q3 = Bx + Hx + 3.5 Sx.
-// Stored negated as zx[format][T][G] (the MMA's accumulator input).
+// Stored as -Z / 16 split exactly into two fp16 halves (hi = the rounding, lo = the
+// rounding of what is left), in planes z16[hl][format][T][G8] with the group count
+// padded to whole chunks (G8 = 8 ceil(G / 8); the padding is zero): the B fragments of
+// the correction MMA.  The 1/16 keeps Z inside the fp16 range; the kernel scales the
+// A side (the fp16 scales) by 16, exactly.
 __device__ void compute_z(const RouteArgs& p, int t, int Gi, int lane) {
     constexpr float kLo[8] = {128.f, 32.f, 8.f, 128.f, 32.f, 8.f, 128.f, 32.f};
     constexpr float kHi[8] = {512.f, 256.f, 128.f, 64.f, 32.f, 16.f, 8.f, 8.f};
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * p.H + Gi * 64) + lane);
-    const float x0 = bf16lo(v), x1 = bf16hi(v);
-    const float bl = kLo[lane & 7], bh = kHi[lane & 7];
-    float bx = fmaf(bl, x0, bl * x1), hx = fmaf(bh, x0, bh * x1), sx = x0 + x1;
-    bx = warp_sum(bx);
-    hx = warp_sum(hx);
-    sx = warp_sum(sx);
-    if (lane == 0) {
-        const int G = p.H / 64;
-        const size_t i = (size_t)t * G + Gi, plane = (size_t)p.T * G;
-        p.zx[i] = -(bx + sx);
-        p.zx[plane + i] = -fmaf(1.5f, sx, bx);
-        p.zx[2 * plane + i] = -fmaf(3.5f, sx, bx + hx);
+    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
+    float z[3] = {0.f, 0.f, 0.f};
+    if (Gi < G) {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * p.H + Gi * 64) + lane);
+        const float x0 = bf16lo(v), x1 = bf16hi(v);
+        const float bl = kLo[lane & 7], bh = kHi[lane & 7];
+        float bx = fmaf(bl, x0, bl * x1), hx = fmaf(bh, x0, bh * x1), sx = x0 + x1;
+        bx = warp_sum(bx);
+        hx = warp_sum(hx);
+        sx = warp_sum(sx);
+        z[0] = bx + sx;
+        z[1] = fmaf(1.5f, sx, bx);
+        z[2] = fmaf(3.5f, sx, bx + hx);
+    }
+    if (lane < 3) {
+        const float zs = -0.0625f * (lane == 0 ? z[0] : (lane == 1 ? z[1] : z[2]));
+        const __half hi = __float2half_rn(zs);
+        const __half lo = __float2half_rn(zs - __half2float(hi));
+        uint16_t* z16 = reinterpret_cast<uint16_t*>(p.zx);
+        const size_t i = ((size_t)lane * p.T + t) * G8 + Gi, plane = (size_t)3 * p.T * G8;
+        z16[i] = __half_as_ushort(hi);
+        z16[plane + i] = __half_as_ushort(lo);
     }
 }
 
@@ -181,9 +195,9 @@ __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
         p.ctrl->work[0] = 0;
         p.ctrl->work[1] = 0;
     }
-    const int G = p.H / 64;
+    const int G8 = 8 * ((p.H / 64 + 7) / 8);
     const int warp = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (warp < p.T * G) compute_z(p, warp / G, warp % G, lane);
+    if (warp < p.T * G8) compute_z(p, warp / G8, warp % G8, lane);
 }
 
 // ---------------------------------------------------------------- decode router
@@ -300,8 +314,8 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
         p.logits[(size_t)t * p.E + e] = v + (p.bias ? p.bias[e] : 0.f);
     }
     {
-        const int G = p.H / 64;
-        for (int pr = blockIdx.x * 8 + warp; pr < p.T * G; pr += gridDim.x * 8) compute_z(p, pr / G, pr % G, lane);
+        const int G8 = 8 * ((p.H / 64 + 7) / 8);
+        for (int pr = blockIdx.x * 8 + warp; pr < p.T * G8; pr += gridDim.x * 8) compute_z(p, pr / G8, pr % G8, lane);
     }
     __shared__ int s_last;
     __threadfence();
@@ -562,7 +576,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
         route_small_kernel<<<a.E, 256, 0, s>>>(a);
         return cudaGetLastError();
     }
-    const int zwarps = a.T * (a.H / 64);
+    const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);
     route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
     static bool attr = false;
     if (!attr) {
