@@ -33,6 +33,8 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     off = align256(off + 4 * (size_t)(((T + kChunk - 1) / kChunk) * E));
     w.zx = off;
     off = align256(off + 4 * (size_t)(3 * (8 * ((H / 64 + 7) / 8)) * T));   // two fp16 planes
+    w.iq = off;
+    off = align256(off + iq_bytes(T, H));
     w.h = off;
     off = align256(off + 2 * (size_t)(T * (k + S) * I));
     // ypart, and the decode gate/up partial sums that alias it: the largest need of any
@@ -153,6 +155,7 @@ moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x, con
     a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
     a.active = reinterpret_cast<int32_t*>(ws + w.active);
     a.zx = reinterpret_cast<float*>(ws + w.zx);
+    a.iq = T <= kIqMaxT ? ws + w.iq : nullptr;
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.r = *out;
     if (launch_route(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -187,6 +190,8 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.topk_w = r->topk_w;
     a.active = reinterpret_cast<const int32_t*>(ws + w.active);
     a.zx = reinterpret_cast<const float*>(ws + w.zx);
+    a.iq = T <= kIqMaxT ? ws + w.iq : nullptr;
+    a.iq_on = 0;
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.h = reinterpret_cast<uint16_t*>(ws + w.h);
     a.ypart = reinterpret_cast<float*>(ws + w.ypart);
@@ -203,7 +208,10 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     const bool tc_ok = a.H % 128 == 0 && (2 * a.I) % 128 == 0;
     if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
     const bool prefill = path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kSmallT && tc_ok);
-    if (!prefill) decode_kparts(shape, T, &a.nkp_gu, &a.nkp_dn);
+    if (!prefill) {
+        decode_kparts(shape, T, &a.nkp_gu, &a.nkp_dn);
+        a.iq_on = T <= kIqMaxT;
+    }
     cudaError_t err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
                               : launch_ffn_decode(a, s, ev[1], ev[2]);
     if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;

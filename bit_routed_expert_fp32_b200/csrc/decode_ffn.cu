@@ -282,7 +282,9 @@ __device__ __forceinline__ int src_token(const FfnArgs& p, const CtaSched& S, in
 struct UnitView {
     const uint16_t* b;         // B-operand row of token column g (+16t elements)
     const uint16_t* z;         // gate/up: -Z/16 (hi plane) of token column g, groups 2t, 2t+1
-    int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token)
+    const uint4* bq;           // integer path: digit record of column g, lane t, group 0
+    const float* pq;           // integer path: factors p of token t, group 0
+    int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token); integer path: token t
 };
 
 // Columns without a token read a valid row (the pass's first token); their MMA
@@ -321,6 +323,7 @@ __device__ __forceinline__ void make_view(const FfnArgs& p, const CtaSched& S, i
 struct LaneGeo {
     int g, t, cw_lane, g4, hw_lane, g2, sh;
     int zplane;                // elements from the hi to the lo plane of the Z table
+    int zplane_iq;             // the same for the integer path's offset planes
 };
 
 __device__ __forceinline__ uint32_t f16x2_mul16(uint32_t a, uint32_t b) {
@@ -455,6 +458,147 @@ __device__ __forceinline__ void chunk_partial(const uint8_t* stg, int c, int ng,
     }
 }
 
+// ---- few-token gate/up on the integer tensor path (ternary and 2-bit experts) ----
+// With at most kIqMaxT tokens a pass uses one n8 tile as two signed-byte digit
+// columns per token (column 2j + d: digit d of token j; route.cu writes the digit
+// records).  A code word w of row g gives four u8 A registers without any add:
+// w & 0x03030303 (the codes themselves), w & 0x0C0C0C0C (4 x the codes) and the same
+// of w >> 4; B carries 4q or q to match, so each group is two m16n8k32 u8 x s8 MMAs
+// with exact int32 sums.  The accumulator starts at the bit pattern of 1.5 * 2^23, so
+// the int32 result read as fp32 is 1.5 * 2^23 + D exactly (|D| < 2^17) and one
+// subtract recovers D.  Per group, acc += s p (D) with p = 2^-e / 4 of this lane's
+// token; the chunk's offsets are removed by the fp16 Z MMAs as on the bf16 path, with
+// the Z columns of the high digits zero.  Lane (g, t) ends with rows g, g + 8 of
+// token t: acc[.][0] + 256 acc[.][1] and acc[.][2] + 256 acc[.][3].
+constexpr uint32_t kIqMagic = 0x4B400000u;             // 1.5 * 2^23
+constexpr float kIqMagicF = 12582912.0f;
+
+__device__ __forceinline__ void imma_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(kIqMagic));
+}
+__device__ __forceinline__ void imma_acc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 64-group of one tile: wa, wb the code words of rows g and g + 8, b the lane's
+// digit record (MMA 0: b.x, b.y; MMA 1: b.z, b.w), s0, s1 the two rows' scales times p.
+__device__ __forceinline__ void group_iq_tile(uint32_t wa, uint32_t wb, const uint4& b, float s0, float s1,
+                                              float (&acc)[4]) {
+    const uint32_t wa4 = wa >> 4, wb4 = wb >> 4;
+    int d[4];
+    imma_first(d, wa & 0x03030303u, wb & 0x03030303u, wa & 0x0C0C0C0Cu, wb & 0x0C0C0C0Cu, b.x, b.y);
+    imma_acc(d, wa4 & 0x03030303u, wb4 & 0x03030303u, wa4 & 0x0C0C0C0Cu, wb4 & 0x0C0C0C0Cu, b.z, b.w);
+    acc[0] = fmaf(s0, __int_as_float(d[0]) - kIqMagicF, acc[0]);
+    acc[1] = fmaf(s0, __int_as_float(d[1]) - kIqMagicF, acc[1]);
+    acc[2] = fmaf(s1, __int_as_float(d[2]) - kIqMagicF, acc[2]);
+    acc[3] = fmaf(s1, __int_as_float(d[3]) - kIqMagicF, acc[3]);
+}
+
+// The chunk's offset correction on the integer path: the bf16 path's z_correction
+// with this lane's Z column (zero for the high-digit columns: v.z == nullptr).
+__device__ __forceinline__ void z_correction_iq(const uint8_t* stg, int c, const UnitView& v, const LaneGeo& L,
+                                                float (&acc)[NTL][4]) {
+    constexpr uint32_t kSixteen = 0x4C004C00u;
+    const uint32_t bhi = v.z ? __ldg(reinterpret_cast<const uint32_t*>(v.z + 8 * c)) : 0u;
+    const uint32_t blo = v.z ? __ldg(reinterpret_cast<const uint32_t*>(v.z + L.zplane_iq + 8 * c)) : 0u;
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + tl * TSTAGE + OFF_SC);
+        const uint32_t a0 = f16x2_mul16(scw[4 * L.g + L.t], kSixteen);
+        const uint32_t a1 = f16x2_mul16(scw[4 * (L.g + 8) + L.t], kSixteen);
+        mma_f16_1688(acc[tl], a0, a1, bhi);
+        mma_f16_1688(acc[tl], a0, a1, blo);
+    }
+}
+
+template <int HI>
+__device__ __forceinline__ void group_iq(const uint8_t* stg, int gl, const uint4* bq, float pf, const LaneGeo& L,
+                                         const uint32_t (&s2)[NTL][2], float (&acc)[NTL][4]) {
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(stg);
+    const int cpos = L.cw_lane + ((4 * gl) ^ L.g4);
+    uint32_t w[NTL][2];
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        w[tl][0] = cw[cpos + tl * (TSTAGE / 4)];
+        w[tl][1] = cw[cpos + tl * (TSTAGE / 4) + 256];
+    }
+    const uint4 b = __ldg(bq + 8 * gl);
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        const float s0 = (HI ? half_hi(s2[tl][0]) : half_lo(s2[tl][0])) * pf;
+        const float s1 = (HI ? half_hi(s2[tl][1]) : half_lo(s2[tl][1])) * pf;
+        group_iq_tile(w[tl][0], w[tl][1], b, s0, s1, acc[tl]);
+    }
+}
+
+__device__ __forceinline__ void chunk_full_iq(const uint8_t* stg, int c, const UnitView& v, const LaneGeo& L,
+                                              float (&acc)[NTL][4]) {
+    const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + OFF_SC);
+    const uint4* bq = v.bq + c * (CG * 8);
+    const float2* pq = reinterpret_cast<const float2*>(v.pq + c * CG);
+    z_correction_iq(stg, c, v, L, acc);
+#pragma unroll 1
+    for (int gp = 0; gp < CG / 2; ++gp) {
+        uint32_t s2[NTL][2];
+#pragma unroll
+        for (int tl = 0; tl < NTL; ++tl) {
+            s2[tl][0] = scw[tl * (TSTAGE / 4) + 4 * L.g + gp];
+            s2[tl][1] = scw[tl * (TSTAGE / 4) + 4 * (L.g + 8) + gp];
+        }
+        const float2 pf = __ldg(pq + gp);
+        group_iq<0>(stg, 2 * gp, bq, pf.x, L, s2, acc);
+        group_iq<1>(stg, 2 * gp + 1, bq, pf.y, L, s2, acc);
+    }
+}
+
+__device__ __forceinline__ void chunk_partial_iq(const uint8_t* stg, int c, int ng, const UnitView& v,
+                                                 const LaneGeo& L, float (&acc)[NTL][4]) {
+    const int g = L.g, t = L.t;
+    z_correction_iq(stg, c, v, L, acc);
+    for (int gl = 0; gl < ng; ++gl) {
+        const uint4 b = __ldg(v.bq + c * (CG * 8) + 8 * gl);
+        const float pf = __ldg(v.pq + c * CG + gl);
+#pragma unroll
+        for (int tl = 0; tl < NTL; ++tl) {
+            const uint8_t* tb = stg + tl * TSTAGE;
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(tb);
+            const uint16_t* scs = reinterpret_cast<const uint16_t*>(tb + OFF_SC);
+            const float s0 = __half2float(__ushort_as_half(scs[g * 8 + gl])) * pf;
+            const float s1 = __half2float(__ushort_as_half(scs[(g + 8) * 8 + gl])) * pf;
+            group_iq_tile(cw[g * 4 * ng + 4 * gl + t], cw[(g + 8) * 4 * ng + 4 * gl + t], b, s0, s1, acc[tl]);
+        }
+    }
+}
+
+// View of an integer-path unit (one pass: cnt <= kIqMaxT).  B column g is digit g & 1
+// of the pass's token g >> 1; the outputs of this lane are token t's.  Columns and
+// outputs without a token read the pass's first token and are never stored.
+__device__ __forceinline__ void make_view_iq(const FfnArgs& p, const CtaSched& S, int a, int g, int t,
+                                             UnitView& v) {
+    const int e = S.e[a], f = S.fmt[a], nb = min(kIqMaxT, S.cnt[a]);
+    const bool routed = e < p.E;
+    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
+    const int ib = (g >> 1) < nb ? (g >> 1) : 0, it = t < nb ? t : 0;
+    const int tb = routed ? src_token(p, S, S.off[a] + ib) : ib;
+    const int tt = routed ? src_token(p, S, S.off[a] + it) : it;
+    v.bq = reinterpret_cast<const uint4*>(p.iq) + ((size_t)tb * G * 2 + (g & 1)) * 4 + t;
+    v.pq = reinterpret_cast<const float*>(p.iq + iq_pq_off(p.T, p.H)) + (size_t)tt * G8;
+    v.z = (g & 1) ? nullptr
+                  : reinterpret_cast<const uint16_t*>(p.iq + iq_zq_off(p.T, p.H)) + ((size_t)f * p.T + tb) * G8 + 2 * t;
+    v.orow[0] = t < nb ? (routed ? S.off[a] + t : p.T * p.k + (e - p.E) * p.T + t) : -1;
+    v.orow[1] = -1;
+}
+
 // Per-launch geometry of one expert pass (gate/up: K = H, rows 2I; down: K = I, rows H).
 struct Geo {
     int K, G, NC, blocks, nkp, cpk;
@@ -563,6 +707,28 @@ __device__ __forceinline__ void unit_epilogue(const FfnArgs& p, const Geo& geo, 
     }
 }
 
+// Integer-path unit end: combine the digit columns of token t and store as the bf16
+// path does (h directly, or this K part's gate and up sums).
+__device__ __forceinline__ void unit_epilogue_iq(const FfnArgs& p, const Geo& geo, const UnitPos& q,
+                                                 const UnitView& v, const LaneGeo& L, const float (&acc)[NTL][4]) {
+    const int orow = v.orow[0];
+    if (orow < 0) return;
+    const size_t R = (size_t)p.T * (p.k + p.S);
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        const int j = NTL * q.jb + tl;
+        const float gs = fmaf(256.f, acc[tl][1], acc[tl][0]);
+        const float us = fmaf(256.f, acc[tl][3], acc[tl][2]);
+        if (geo.nkp == 1) {
+            p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(silu_f(gs) * us);
+        } else {
+            float* dst = p.gpart + ((size_t)q.kp * R + orow) * (2 * p.I) + j * 16 + L.g;
+            dst[0] = gs;
+            dst[8] = us;
+        }
+    }
+}
+
 // Gate/up with few tokens: every SM reads the same token rows and Z values, so each CTA
 // pulls them into L1 at the start.  The token rows are the caller's input (ready before
 // the router ran); the Z values are the router's output and are prefetched only after
@@ -583,7 +749,8 @@ __device__ inline void warm_z(const FfnArgs& p) {
         prefetch_l1(reinterpret_cast<const uint8_t*>(p.zx) + i * 128);
 }
 
-template <int MODE>
+// IQ (gate/up only): ternary and 2-bit experts take the integer path (T <= kIqMaxT).
+template <int MODE, bool IQ>
 __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ CtaSched S;
@@ -671,12 +838,13 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     L.g2 = 2 * (L.g >> 1);
     L.sh = 8 * (L.t & 1);
     L.zplane = 3 * p.T * (8 * ((p.H / 64 + 7) / 8));
+    L.zplane_iq = 2 * p.T * (8 * ((p.H / 64 + 7) / 8));
     bool aborted = false;
     int consumed = 0;
     // The chunk to consume is the one issued NS - 1 issues ago (hu / hc[NS - 1] after
     // the next issue).  A unit ends when the next chunk belongs to another unit.
     int unit = -1, view_a = -1, view_pass = -1;
-    bool q3 = false;
+    bool q3 = false, iqu = false;                      // iqu: the current unit is on the integer path
     UnitPos q;
     q.a = q.pass = q.jb = q.kp = 0;
     UnitView v;
@@ -686,18 +854,26 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         prod.issue(p, S, geo, per_ep, fkp, ctr, lane, ring, bar, pol);
         const int hu = prod.hu[NS - 1], c = prod.hc[NS - 1];
         if (hu < 0) {                                   // nothing left (or nothing at all)
-            if (unit >= 0) unit_epilogue<MODE>(p, geo, q, v, L, acc);
+            if (unit >= 0) {
+                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, acc);
+                else unit_epilogue<MODE>(p, geo, q, v, L, acc);
+            }
             break;
         }
         if (hu != unit) {
-            if (unit >= 0) unit_epilogue<MODE>(p, geo, q, v, L, acc);
+            if (unit >= 0) {
+                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, acc);
+                else unit_epilogue<MODE>(p, geo, q, v, L, acc);
+            }
             unit = hu;
             q = unit_pos(S, unit, per_ep, fkp);
             if (q.a != view_a || q.pass != view_pass) {
                 view_a = q.a;
                 view_pass = q.pass;
-                make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
                 q3 = S.fmt[q.a] == MOE_FMT_Q3;
+                iqu = IQ && !q3;
+                if (IQ && iqu) make_view_iq(p, S, q.a, L.g, L.t, v);
+                else make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
                 if (MODE == 1) {
                     const int f = S.fmt[q.a];
                     const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
@@ -718,7 +894,10 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         }
         const uint8_t* stg = ring + (size_t)st * STAGE;
         const int ng = min(CG, geo.G - c * CG);
-        if (ng == CG) {
+        if (IQ && iqu) {
+            if (ng == CG) chunk_full_iq(stg, c, v, L, acc);
+            else chunk_partial_iq(stg, c, ng, v, L, acc);
+        } else if (ng == CG) {
             if (q3) chunk_full<MODE, true>(stg, c, v, L, sub, acc);
             else chunk_full<MODE, false>(stg, c, v, L, sub, acc);
         } else {
@@ -910,22 +1089,22 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(FfnArgs p) {
 
 constexpr size_t kDynSmem = (size_t)NW * NS * STAGE + (size_t)NW * NS * 8;
 
-template <int MODE>
+template <int MODE, bool IQ>
 cudaError_t launch_mode(const FfnArgs& a, cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_decode_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kDynSmem);
+        cudaError_t err = cudaFuncSetAttribute(ffn_decode_kernel<MODE, IQ>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDynSmem);
         if (err != cudaSuccess) return err;
         attr = true;
     }
-    return launch_pdl(ffn_decode_kernel<MODE>, dim3(a.num_ctas), dim3(NW * 32), kDynSmem, s, a);
+    return launch_pdl(ffn_decode_kernel<MODE, IQ>, dim3(a.num_ctas), dim3(NW * 32), kDynSmem, s, a);
 }
 
 }  // namespace
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down) {
-    cudaError_t err = launch_mode<0>(a, s);
+    cudaError_t err = a.iq_on && a.iq ? launch_mode<0, true>(a, s) : launch_mode<0, false>(a, s);
     if (err != cudaSuccess) return err;
     if (a.nkp_gu > 1) {
         const long long n = (long long)a.T * (a.k + a.S) * (a.I / 4);
@@ -933,7 +1112,7 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_g
         if (err != cudaSuccess) return err;
     }
     if (ev_gateup && (err = record_event(ev_gateup, s)) != cudaSuccess) return err;
-    err = launch_mode<1>(a, s);
+    err = launch_mode<1, false>(a, s);
     if (err != cudaSuccess) return err;
     if (ev_down && (err = record_event(ev_down, s)) != cudaSuccess) return err;
     return launch_combine(a, s);

@@ -20,6 +20,7 @@ struct RouteArgs {
     int32_t* hist;      // ws [ceil(T/kChunk)][E]
     int32_t* active;    // ws [E+S]
     float* zx;          // ws fp16 planes [2][3][T][G8] of -Z/16, hi and lo (see route.cu)
+    uint8_t* iq;        // ws integer gate/up operands for T <= kIqMaxT (see route.cu), else null
     Ctrl* ctrl;
     moe_routing r;
 };
@@ -35,6 +36,8 @@ struct FfnArgs {
     const float* topk_w;
     const int32_t* active;   // ws
     const float* zx;         // ws fp16 planes [2][3][T][G8] of -Z/16, hi and lo
+    const uint8_t* iq;       // ws integer gate/up operands (T <= kIqMaxT), else null
+    int iq_on;               // gate/up of ternary / 2-bit experts on the integer path
     Ctrl* ctrl;
     uint16_t* h;             // ws fp16 [T*(k+S)][I]
     float* ypart;            // ws f32 [nkp_dn][T*(k+S)][H]
@@ -48,8 +51,26 @@ struct FfnArgs {
 // Workspace layout for T tokens (api.cu).  The control block, tile counters and the
 // active-expert list sit at fixed offsets (independent of T).
 struct Ws {
-    size_t ctrl, tile_ctr, active, logits, hist, zx, h, ypart, total;
+    size_t ctrl, tile_ctr, active, logits, hist, zx, iq, h, ypart, total;
 };
+
+// Few-token gate/up on the integer tensor path (decode_ffn.cu, route.cu): up to
+// kIqMaxT tokens, each as two signed-byte digit columns of one n8 MMA tile.  The
+// region holds, per token t and 64-group g (G groups, G8 = G padded to whole chunks):
+//   digit records  [T][G][2 digits][4 lanes] x 16 bytes          (offset 0)
+//   factors p      fp32 [T][G8]                                   (iq_pq_off)
+//   offset planes  fp16 [2 hi/lo][2 formats][T][G8] of -o sum x / 16  (iq_zq_off)
+constexpr int kIqMaxT = 4;
+__host__ __device__ inline size_t iq_pq_off(int64_t T, int64_t H) { return (size_t)T * (H / 64) * 128; }
+__host__ __device__ inline size_t iq_zq_off(int64_t T, int64_t H) {
+    return iq_pq_off(T, H) + (size_t)4 * T * (8 * ((H / 64 + 7) / 8));
+}
+// Reserved for min(T, kIqMaxT) tokens at every T >= 1, so that the workspace size
+// never shrinks as T grows; used only when T <= kIqMaxT.
+inline size_t iq_bytes(int64_t T, int64_t H) {
+    const int64_t t = T < kIqMaxT ? T : kIqMaxT;
+    return t >= 1 ? iq_zq_off(t, H) + (size_t)2 * 2 * 2 * t * (8 * ((H / 64 + 7) / 8)) : 0;
+}
 Ws ws_layout(const moe_shape* s, int64_t T);
 
 // K parts of the decode-path expert passes for T tokens.  With few tokens only a few

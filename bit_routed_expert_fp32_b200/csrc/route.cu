@@ -190,6 +190,57 @@ __device__ void compute_z(const RouteArgs& p, int t, int Gi, int lane) {
     }
 }
 
+// Integer operands of the few-token gate/up pass (T <= kIqMaxT; ternary and 2-bit
+// experts, decode_ffn.cu).  Per token t and 64-group Gi: e = 11 - floor(log2 max |x|)
+// puts the group on a 12-bit grid, q = rint(x 2^e) (exact for every x above 2^-4 of
+// the group maximum).  The kernel masks each code word into four byte classes c (two
+// per MMA): classes 0 and 2 hold the code, 1 and 3 four times the code, so B = 4q for
+// even c and q for odd c makes every product 4 c q.  Element k of the group sits in
+// lane k / 16 of the record, class c = (k mod 8) / 2, byte 2 (k mod 2) + (k mod 16) / 8
+// (the inverse of the code word's element order); B is split into signed bytes
+// lo + 256 hi, one record per digit.  p = 2^-e / 4 turns the integer sums into x
+// units; the offset planes hold -o sum(q 2^-e) / 16 as fp16 hi + lo for o = 1 and 1.5.
+__device__ void compute_iq(const RouteArgs& p, int t, int Gi, int lane) {
+    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
+    float* pq = reinterpret_cast<float*>(p.iq + iq_pq_off(p.T, p.H));
+    uint16_t* zq = reinterpret_cast<uint16_t*>(p.iq + iq_zq_off(p.T, p.H));
+    const size_t zplane = (size_t)2 * p.T * G8;
+    if (Gi >= G) {                                      // padding of the last chunk
+        if (lane == 0) pq[(size_t)t * G8 + Gi] = 0.f;
+        if (lane < 4) zq[(lane >> 1) * zplane + ((size_t)(lane & 1) * p.T + t) * G8 + Gi] = 0;
+        return;
+    }
+    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * p.H + Gi * 64) + lane);
+    const float x[2] = {bf16lo(v), bf16hi(v)};
+    const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(x[0]), fabsf(x[1])))));
+    const int e = m > 0.f ? 11 - ilogbf(m) : 0;
+    uint8_t* rec = p.iq + ((size_t)t * G + Gi) * 128;
+    int qsum = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int q = (int)rintf(ldexpf(x[h], e));
+        qsum += q;
+        const int k = 2 * lane + h, lt = k >> 4, off = k & 15;
+        const int c = (off & 7) >> 1, b = 2 * (off & 1) + (off >> 3);
+        const int bv = (c & 1) ? q : 4 * q;
+        const int lo = (int)(int8_t)(uint8_t)(bv & 0xFF), hi = (bv - lo) >> 8;
+        const int pos = 16 * lt + 4 * c + b;
+        rec[pos] = (uint8_t)lo;
+        rec[64 + pos] = (uint8_t)hi;
+    }
+    qsum = (int)__reduce_add_sync(0xffffffffu, (uint32_t)qsum);
+    if (lane == 0) pq[(size_t)t * G8 + Gi] = ldexpf(0.25f, -e);
+    if (lane < 2) {
+        const float sx = ldexpf((float)qsum, -e);
+        const float zs = -0.0625f * (lane == 0 ? sx : 1.5f * sx);
+        const __half hi = __float2half_rn(zs);
+        const __half lo = __float2half_rn(zs - __half2float(hi));
+        const size_t i = ((size_t)lane * p.T + t) * G8 + Gi;
+        zq[i] = __half_as_ushort(hi);
+        zq[zplane + i] = __half_as_ushort(lo);
+    }
+}
+
 __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {          // no expert pass of this workspace runs now
         p.ctrl->work[0] = 0;
@@ -197,7 +248,10 @@ __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
     }
     const int G8 = 8 * ((p.H / 64 + 7) / 8);
     const int warp = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (warp < p.T * G8) compute_z(p, warp / G8, warp % G8, lane);
+    if (warp < p.T * G8) {
+        compute_z(p, warp / G8, warp % G8, lane);
+        if (p.iq) compute_iq(p, warp / G8, warp % G8, lane);
+    }
 }
 
 // ---------------------------------------------------------------- decode router
@@ -315,7 +369,10 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
     }
     {
         const int G8 = 8 * ((p.H / 64 + 7) / 8);
-        for (int pr = blockIdx.x * 8 + warp; pr < p.T * G8; pr += gridDim.x * 8) compute_z(p, pr / G8, pr % G8, lane);
+        for (int pr = blockIdx.x * 8 + warp; pr < p.T * G8; pr += gridDim.x * 8) {
+            compute_z(p, pr / G8, pr % G8, lane);
+            if (p.iq) compute_iq(p, pr / G8, pr % G8, lane);
+        }
     }
     __shared__ int s_last;
     __threadfence();
