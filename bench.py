@@ -43,7 +43,8 @@ METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B2
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # gate/up kernel of each path and the sources its ncu traffic record is tied to
 PATHS = {
-    "decode": ("ffn_decode_kernel<0> (gate/up + SwiGLU; interval includes the K-part reduction when K is split)",
+    "decode": ("ffn_decode_kernel<0, *> (gate/up + SwiGLU; integer MMAs for ternary / 2-bit experts at <= 4 "
+               "tokens; interval includes the K-part reduction when K is split)",
                ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "prefill": ("tc_gemm_kernel<0> (gate/up + SwiGLU, tcgen05; interval includes the token gather)",
                 ["bit_routed_expert_fp32_b200/csrc/prefill_tc.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),

@@ -218,7 +218,7 @@ moe_status moe_get_error(void* d_ws, size_t ws_bytes, void* stream, uint32_t* de
  * library until the process exits.  It allocates nothing itself.
  *   - If the workspace T tokens need (moe_workspace_size) exceeds MOE_STATIC_WS_BYTES
  *     it returns MOE_ERR_WORKSPACE and enqueues nothing; with the full-size layer
- *     (H 7168, I 2048, E 256, k 8, S 1) that allows up to 28 tokens per call.
+ *     (H 7168, I 2048, E 256, k 8, S 1) that allows up to 27 tokens per call.
  *   - The first call on each device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before
  *     any stream capture.  Later calls only enqueue work.

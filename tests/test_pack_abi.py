@@ -71,6 +71,18 @@ def test_argument_errors_are_synchronous():
     assert L.moe_forward(ctypes.byref(sh), 0, fake, fake, ctypes.byref(r), fake, 0, fake, need, None) == 0
 
 
+def test_workspace_size_never_shrinks_as_tokens_grow():
+    # A workspace sized for max_tokens must serve every smaller T: the K-part split
+    # of the decode passes and the few-token integer operands must not make a smaller
+    # T need more bytes than a larger one.
+    for cfg in (synth.CONFIGS[2], synth.micro(T=8, H=256, E=8, k=2, I=128, S=0)):
+        sizes = [moe.moe_workspace_size(cfg, T) for T in range(0, 97)]
+        assert all(b >= a for a, b in zip(sizes, sizes[1:]))
+    # the full-size layer: the library's static scratch holds 27 tokens, not 28
+    cfg = synth.CONFIGS[2]
+    assert moe.moe_workspace_size(cfg, 27) <= moe.STATIC_WS_BYTES < moe.moe_workspace_size(cfg, 28)
+
+
 @pytest.mark.parametrize("H,I,formats", [(128, 64, "mixed"), (192, 128, "q3"), (256, 64, "ternary"),
                                          (64, 192, "q2"), (384, 256, "mixed")])
 def test_pack_roundtrip_through_oracle_reader(H, I, formats):
