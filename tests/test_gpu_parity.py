@@ -149,3 +149,16 @@ def test_full_size_decode_split_k_and_determinism():
     assert {(7, 4), (4, 2), (3, 2), (2, 1)} <= seen
     del layer, packed
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("T,shared_format", [(1, synth.FMT_TERNARY), (2, synth.FMT_Q2), (4, synth.FMT_TERNARY)])
+def test_few_token_integer_gate_up_full_chunks(T, shared_format):
+    """Gate/up with at most 4 tokens runs ternary and 2-bit experts on integer MMAs:
+    hidden 1024 gives whole 8-group chunks (the micro shapes above only reach the
+    partial-chunk code), all routed experts ternary exercises the o = 1 offset plane,
+    and a ternary or 2-bit shared expert takes the integer path's shared-expert rows
+    (every other workload's shared expert is 3-bit, which stays on the bf16 path)."""
+    import dataclasses
+    cfg = synth.micro(T=T, H=1024, E=16, k=8, I=128, S=1, formats="ternary", seed=40 + T)
+    cfg = dataclasses.replace(cfg, shared_format=shared_format)
+    _full_check(cfg, PATHS["decode"])
