@@ -13,18 +13,20 @@
 //    fewer 32-row blocks than warps on the GPU, so K is cut into parts (whole 8-group
 //    chunks) and every part writes its own fp32 partial sums; the parts are added in
 //    a fixed order afterwards (finalize_gateup_kernel, combine_kernel), so the result
-//    does not depend on which warp ran what.  Units are dealt round-robin to the
-//    warps of a persistent grid (one CTA of 16 warps per SM), CTAs first.  An expert
-//    with more than 8 tokens has one unit per pass; the passes of a block are
-//    consecutive units, which start together on neighbouring SMs, so the block's
-//    bytes come from HBM once and from L2 for the other passes.
+//    does not depend on which warp ran what.  The warps of a persistent grid (one CTA
+//    of 16 warps per SM) take units at run time from a per-launch counter, one unit
+//    ahead of need, which balances SMs and SM sub-partitions whatever the expert mix.
+//    An expert with more than 8 tokens has one unit per pass; the passes of a block
+//    are consecutive units, taken at about the same time, so the block's bytes come
+//    from HBM once and from L2 for the other passes.
 //  * Each warp streams its units through its own ring of NS shared-memory stages with
 //    1-D bulk copies (cp.async.bulk on the TMA engine, completion on a per-stage
 //    mbarrier); a stage holds one 8-group (512-wide) chunk of K for both tiles:
 //    codes, third bits and fp16 scales, each a contiguous block of the packed format.
 //    The format's XOR swizzle keeps the fragment reads free of bank conflicts.  The
 //    ring runs ahead across units; there is no CTA-wide barrier in the main loop.
-//  * A full chunk is processed fully unrolled: per 64-wide group and tile, two code
+//  * A full chunk is processed in four steps of two groups (a rolled loop keeps the
+//    code inside the instruction cache): per 64-wide group and tile, two code
 //    words become sixteen bf16 / fp16 pairs with shifts and lop3 (magic-number
 //    exponent trick: the code lands in the mantissa of a power-of-two base, exactly),
 //    the A operand of mma.sync m16n8k16; the tokens are N (8 per n-tile) and the B
@@ -37,6 +39,10 @@
 //      down: pairs are (c - o) exactly (one fp16x2 subtract); fp16 MMAs, h is fp16.
 //    Each group result is scaled by its fp16 scale into an fp32 accumulator.
 //    3-bit experts add an MMA per k-step for 4 * (third bit).
+//  * gate/up with at most 4 tokens, ternary and 2-bit experts: integer MMAs instead
+//    (u8 codes masked out of the code words against signed-byte digits of the tokens
+//    on a 12-bit grid per group; see "few-token gate/up on the integer tensor path"
+//    below), which halves the dequantiser's ALU work and the MMA chain per group.
 //  * gate/up: the 16 rows of a tile are 8 gate rows and the matching 8 up rows, which
 //    the MMA places in the same thread (rows g and g + 8), so with a single K part
 //    h = silu(gate) * up is formed in registers and stored as fp16; with several K
