@@ -1,6 +1,6 @@
-// Expert FFN kernels of the decode path (steps a4, a5, a8) and the gate-weighted
-// unpermute-combine (a9): grouped skinny GEMMs over the packed ternary / 2-bit /
-// 3-bit experts, for few tokens per expert.
+// Expert FFN kernels of the decode path (gate/up + SwiGLU and down, routed and
+// shared experts) and the gate-weighted unpermute-combine: grouped skinny GEMMs over
+// the packed ternary / 2-bit / 3-bit experts, for few tokens per expert.
 //
 // Decode speed is set by the expert bytes moved per token (ossradar.top, Xolotl
 // README, "Fast mode (DeepSeek-V4.1)"), and each selected expert is read once for

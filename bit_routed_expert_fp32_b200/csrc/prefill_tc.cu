@@ -1,4 +1,4 @@
-// Prefill path (steps a6, a7, a8): grouped GEMMs over the packed experts on the
+// Prefill path (routed and shared experts): grouped GEMMs over the packed experts on the
 // 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
 //
 // With thousands of tokens each selected expert meets hundreds of tokens, so its

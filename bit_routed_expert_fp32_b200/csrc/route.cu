@@ -1,5 +1,5 @@
-// Router: fp32 logits (a1), softmax + top-k + renormalised gates (a2), and the
-// per-expert histogram / exclusive scan / permutation (a3).
+// Router: fp32 logits, softmax + top-k + renormalised gates, and the per-expert
+// histogram / exclusive scan / permutation.
 //
 // The pages only say that each token's router picks a few experts and that only
 // those experts are read (ossradar.top, Xolotl README, "How it works, in one

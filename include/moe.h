@@ -169,8 +169,8 @@ moe_status moe_workspace_size(const moe_shape* shape, int32_t max_tokens, size_t
  * Every later call leaves the counters cleared again. */
 moe_status moe_workspace_init(void* d_ws, size_t ws_bytes, void* stream);
 
-/* Route T tokens: fp32 router logits (step a1), softmax + top-k + renormalised gates
- * (a2), per-expert histogram, prefix sum and permutation (a3).
+/* Route T tokens: fp32 router logits, softmax + top-k + renormalised gates,
+ * per-expert histogram, prefix sum and permutation.
  *   d_x        bf16 bit patterns [T][H], row-major
  *   d_router_w fp32 [E][H], row-major
  *   d_router_b fp32 [E] added to the logits before the softmax, or NULL
@@ -181,8 +181,8 @@ moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x,
                      const float* d_router_w, const float* d_router_b, const moe_routing* out,
                      void* d_ws, size_t ws_bytes, void* stream);
 
-/* Expert FFNs of the routed and shared experts and the gate-weighted combine
- * (steps a4-a9), using the routing of the preceding moe_route on the same d_ws.
+/* Expert FFNs of the routed and shared experts and the gate-weighted combine,
+ * using the routing of the preceding moe_route on the same d_ws.
  *   d_packed  packed experts (format above), device memory
  *   d_x       bf16 [T][H] (the same tokens as routed)
  *   r         the routing moe_route wrote

@@ -72,7 +72,7 @@ def _threads(n: int | None) -> int:
     return max(1, n if n else (os.cpu_count() or 1))
 
 
-# ---- a1 / a2 ---------------------------------------------------------------
+# ---- router logits, top-k, gates ------------------------------------------
 
 def logits(x: np.ndarray, Wr: np.ndarray, threads: int | None = None) -> np.ndarray:
     """fp64 [T][E] router logits (no bias)."""
@@ -130,7 +130,7 @@ def topk_gaps(L: np.ndarray, bias, k: int) -> np.ndarray:
     return np.min(top[:, :-1] - top[:, 1:], axis=1)
 
 
-# ---- a3 --------------------------------------------------------------------
+# ---- histogram, scan, permutation -----------------------------------------
 
 def permute(ids: np.ndarray, E: int):
     ids = np.ascontiguousarray(ids, dtype=np.int32)
@@ -143,7 +143,7 @@ def permute(ids: np.ndarray, E: int):
     return counts, offsets, perm, inv
 
 
-# ---- a4-a9 -----------------------------------------------------------------
+# ---- expert FFNs and the combine ------------------------------------------
 
 def _ptr(a):
     return None if a is None else a.ctypes.data

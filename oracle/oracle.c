@@ -83,7 +83,7 @@ static int dequant_row(const uint8_t* codes, const uint8_t* hi, const uint16_t* 
     return 0;
 }
 
-/* ---- a1: router logits --------------------------------------------------- */
+/* ---- router logits ------------------------------------------------------- */
 
 /* L[t][e] = sum_h x[t][h] * Wr[e][h], in fp64 (x bf16, Wr fp32, both exact in fp64). */
 void oracle_logits(int T, int H, int E, const uint16_t* x, const float* Wr, double* L) {
@@ -97,7 +97,7 @@ void oracle_logits(int T, int H, int E, const uint16_t* x, const float* Wr, doub
     }
 }
 
-/* ---- a2: softmax, top-k, renormalised gates ------------------------------ */
+/* ---- softmax, top-k, renormalised gates ---------------------------------- */
 
 /* For each token: z = L + b (b may be NULL), p = softmax(z) (max subtracted),
  * ids = k largest p in descending order (equal p: lower id first),
@@ -139,7 +139,7 @@ void oracle_select(int T, int E, int k, const double* L, const float* bias, int3
     }
 }
 
-/* ---- a3: histogram, exclusive scan, permutation --------------------------- */
+/* ---- histogram, exclusive scan, permutation ------------------------------- */
 
 /* counts[e] = #{(t,j): ids[t][j] == e}; offsets = exclusive prefix sum (E+1 entries);
  * perm lists pairs t*k + j expert by expert (ascending), token ascending within an
@@ -158,7 +158,7 @@ void oracle_permute(int T, int E, int k, const int32_t* ids, int32_t* counts, in
     for (int i = 0; i < T * k; ++i) inv_perm[perm[i]] = i;
 }
 
-/* ---- a4-a8: one expert FFN on a list of tokens ----------------------------- */
+/* ---- one expert FFN (routed or shared) on a list of tokens ----------------- */
 
 /* y[i][:] = Wd (silu(Wg x_i) * (Wu x_i)) for n_tok tokens x_i (bf16 rows of H).
  * Gate/up are [I][H], down is [H][I], each as (codes, hi, scales) in the
@@ -199,7 +199,7 @@ int oracle_expert_ffn(int H, int I, int fmt,
     return 0;
 }
 
-/* ---- a9: gate-weighted combine ---------------------------------------------- */
+/* ---- gate-weighted combine -------------------------------------------------- */
 
 /* y[h] = sum_j gates[j] * y_routed[j][h] + sum_s y_shared[s][h], slot order j = 0..k-1. */
 void oracle_combine(int H, int k, int S, const double* gates, const double* y_routed,

@@ -36,7 +36,7 @@ def test_bf16_decode(bits, val):
     assert oracle.lib().oracle_bf16_to_f64(bits) == val
 
 
-# ---- a1/a2: routing ---------------------------------------------------------
+# ---- routing: logits, top-k, gates -------------------------------------------
 
 def test_route_closed_form():
     """x = e_0 makes the logits the first column of Wr; gates by hand."""
@@ -107,7 +107,7 @@ def test_logits_match_exact_dot():
     np.testing.assert_allclose(L, ref, rtol=1e-12, atol=1e-13)
 
 
-# ---- a3: histogram / scan / permutation -------------------------------------
+# ---- histogram / scan / permutation -----------------------------------------
 
 @pytest.mark.parametrize("T,E,k,seed", [(1, 8, 2, 0), (37, 16, 4, 1), (200, 256, 8, 2)])
 def test_permute_invariants(T, E, k, seed):
@@ -130,7 +130,7 @@ def test_permute_invariants(T, E, k, seed):
     np.testing.assert_array_equal(xp[inv], x)
 
 
-# ---- a4-a9: expert math -----------------------------------------------------
+# ---- expert math and combine ------------------------------------------------
 
 def _layer(cfg):
     return synth.Layer(cfg)
