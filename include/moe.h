@@ -176,7 +176,10 @@ moe_status moe_workspace_init(void* d_ws, size_t ws_bytes, void* stream);
  *   d_router_b fp32 [E] added to the logits before the softmax, or NULL
  *   out        caller-allocated device arrays (see moe_routing)
  * Also leaves in d_ws the expert schedule that moe_forward reads, so moe_forward
- * must be given the same d_ws and T.  T = 0 is a no-op returning MOE_OK. */
+ * must be given the same d_ws and T.  T = 0 is a no-op returning MOE_OK.
+ * Tokens, router weights and bias must be finite: a NaN or infinity gives
+ * unspecified routing and outputs (the few-token integer path does not carry a NaN
+ * token through to y); nothing checks this on the device. */
 moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x,
                      const float* d_router_w, const float* d_router_b, const moe_routing* out,
                      void* d_ws, size_t ws_bytes, void* stream);
