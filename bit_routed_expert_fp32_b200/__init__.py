@@ -22,7 +22,8 @@ FMT_TERNARY, FMT_Q2, FMT_Q3 = 0, 1, 2
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 # every symbol include/moe.h declares
-EXPORTS = ["moe_packed_size", "moe_pack_experts", "moe_workspace_size", "moe_workspace_init", "moe_route",
+EXPORTS = ["moe_packed_size", "moe_pack_experts", "moe_requantize_q3_to_q2", "moe_workspace_size",
+           "moe_workspace_init", "moe_route",
            "moe_forward", "moe_forward_timed", "moe_get_error", "moe_decode_static", "moe_event_record",
            "moe_status_string", "moe_abi_version"]
 STATIC_WS_BYTES = 8 << 20
@@ -61,6 +62,7 @@ def lib() -> ctypes.CDLL:
         sh = ctypes.POINTER(Shape)
         L.moe_packed_size.argtypes = [sh, vp, ctypes.POINTER(sz)]
         L.moe_pack_experts.argtypes = [sh, vp, i32, i32, ctypes.POINTER(MatrixSrc), vp, sz]
+        L.moe_requantize_q3_to_q2.argtypes = [i32, i32, ctypes.POINTER(MatrixSrc), vp, vp]
         L.moe_workspace_size.argtypes = [sh, i32, ctypes.POINTER(sz)]
         L.moe_workspace_init.argtypes = [vp, sz, vp]
         L.moe_route.argtypes = [sh, i32, vp, vp, vp, ctypes.POINTER(Routing), vp, sz, vp]
@@ -132,6 +134,41 @@ def pack_layer(cfg, fmt: np.ndarray, expert_fn) -> np.ndarray:
     for e in range(cfg.E + cfg.S):
         moe_pack_experts(cfg, fmt, e, [expert_fn(e)], buf)
     return buf
+
+
+def moe_requantize_q3_to_q2(codes: np.ndarray, hi: np.ndarray, scales: np.ndarray):
+    """2-bit copy of one 3-bit matrix (interchange form): codes [rows][K/4], hi
+    [rows][K/8], fp16 scales [rows][K/64] -> (codes, None, scales) of c >> 1, 2 s."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    h = np.ascontiguousarray(hi, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.uint16)
+    rows, K = c.shape[0], 4 * c.shape[1]
+    if h.shape != (rows, K // 8) or s.shape != (rows, K // 64):
+        raise ValueError("moe_requantize_q3_to_q2: codes, hi and scales disagree on the matrix shape")
+    oc = np.empty_like(c)
+    osc = np.empty_like(s)
+    src = MatrixSrc(c.ctypes.data, h.ctypes.data, s.ctypes.data)
+    _check("moe_requantize_q3_to_q2",
+           lib().moe_requantize_q3_to_q2(rows, K, ctypes.byref(src), oc.ctypes.data, osc.ctypes.data))
+    return oc, None, osc
+
+
+def fast_copy(fmt: np.ndarray, expert_fn):
+    """Formats and expert source of the fast-mode copy of a layer: every 3-bit expert
+    (routed or shared) becomes its 2-bit copy (moe_requantize_q3_to_q2), the others
+    are unchanged.  Pack the result with pack_layer / moe_pack_experts into a second
+    buffer and pass that buffer, instead of the layer's own, to the calls that should
+    read the 2-bit copy."""
+    fmt = np.ascontiguousarray(fmt, dtype=np.uint8)
+    fast = np.where(fmt == FMT_Q3, FMT_Q2, fmt).astype(np.uint8)
+
+    def fn(e):
+        m = expert_fn(e)
+        if fmt[e] != FMT_Q3:
+            return m
+        return {name: moe_requantize_q3_to_q2(*m[name]) for name in ("gate", "up", "down")}
+
+    return fast, fn
 
 
 # ---- device calls -----------------------------------------------------------------

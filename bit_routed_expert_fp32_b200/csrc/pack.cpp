@@ -191,3 +191,38 @@ extern "C" moe_status moe_pack_experts(const moe_shape* shape, const uint8_t* h_
     }
     return MOE_OK;
 }
+
+extern "C" moe_status moe_requantize_q3_to_q2(int32_t rows, int32_t K, const moe_matrix_src* src,
+                                              uint8_t* h_codes, uint16_t* h_scales) {
+    if (rows < 1 || K < 64 || K % 64 != 0 || !src || !src->codes || !src->hi || !src->scales || !h_codes ||
+        !h_scales)
+        return MOE_ERR_INVALID_ARG;
+    const size_t G = (size_t)K / 64, nsc = (size_t)rows * G;
+    // fp16 doubling: one more in the exponent field, or a left shift of a subnormal's
+    // mantissa (which carries into the exponent field exactly when the result is
+    // normal); an exponent field of 30 or 31 (largest binade, inf, nan) is refused
+    for (size_t i = 0; i < nsc; ++i)
+        if (((src->scales[i] >> 10) & 0x1F) >= 30) return MOE_ERR_INVALID_ARG;
+    for (size_t i = 0; i < nsc; ++i) {
+        const uint16_t b = src->scales[i], sign = b & 0x8000, mag = b & 0x7FFF;
+        h_scales[i] = (uint16_t)(sign | ((mag >> 10) ? mag + 0x0400 : mag << 1));
+    }
+    // element k: 2-bit field at bits 2(k%4) of byte k/4, third bit at bit k%8 of byte k/8;
+    // c >> 1 has the field's high bit as its low bit and the third bit as its high bit
+    const size_t cb = (size_t)K / 4, hb = (size_t)K / 8;
+    for (int r = 0; r < rows; ++r) {
+        const uint8_t* c = src->codes + r * cb;
+        const uint8_t* h = src->hi + r * hb;
+        uint8_t* o = h_codes + r * cb;
+        for (size_t j = 0; j < cb; ++j) {
+            uint8_t v = 0;
+            for (int i = 0; i < 4; ++i) {
+                const size_t k = 4 * j + i;
+                const unsigned lo = (c[j] >> (2 * i)) & 3u, third = (h[k / 8] >> (k % 8)) & 1u;
+                v |= (uint8_t)(((lo >> 1) | (third << 1)) << (2 * i));
+            }
+            o[j] = v;
+        }
+    }
+    return MOE_OK;
+}

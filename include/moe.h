@@ -161,6 +161,25 @@ moe_status moe_pack_experts(const moe_shape* shape, const uint8_t* h_fmt, int32_
                             int32_t count, const moe_matrix_src* h_src, void* h_dst,
                             size_t h_dst_bytes);
 
+/* The 2-bit copy of one 3-bit matrix, for the fast mode: a second packed buffer in
+ * which the 3-bit experts are 2-bit, read instead of the model's own buffer on the
+ * calls that ask for it (Indras-Mirror/Xolotl README, "Fast mode (DeepSeek-V4.1)":
+ * decode speed follows the expert bytes read per token, so a lossy 2-bit copy of the
+ * biggest expert format is kept beside the model and read instead; the model buffer
+ * itself is unchanged).  The pages give no requantisation rule; this one keeps the
+ * 64-weight groups and their layout: the code c = field + 4 hi (0..7) becomes
+ * c' = c >> 1 (0..3) and the group scale s becomes s' = 2 s (exact in fp16), so each
+ * weight (c' - 1.5) s' differs from (c - 3.5) s by exactly s / 2, the nearest of the
+ * four 2-bit levels to each of the eight 3-bit ones.  Pack the result with
+ * MOE_FMT_Q2 for that expert.  Host memory only, no CUDA calls.
+ *   src       the 3-bit matrix in the interchange form (hi required), [rows][K]
+ *   h_codes   out [rows][K/4]: 2-bit fields in the interchange form
+ *   h_scales  out [rows][K/64]: fp16 bit patterns of 2 s
+ * MOE_ERR_INVALID_ARG (nothing written): a null pointer, rows < 1, K < 64 or not a
+ * multiple of 64, a scale that is not finite or whose double is not finite in fp16. */
+moe_status moe_requantize_q3_to_q2(int32_t rows, int32_t K, const moe_matrix_src* src,
+                                   uint8_t* h_codes, uint16_t* h_scales);
+
 /* Device workspace needed for up to max_tokens tokens per call (both paths). */
 moe_status moe_workspace_size(const moe_shape* shape, int32_t max_tokens, size_t* bytes);
 

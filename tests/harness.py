@@ -55,6 +55,35 @@ def make_case(cfg, layer_idx=0, step=0, T=None, bias=None, router_w=None, thread
     return Case(cfg, layer, x, L, ids, gates, counts, offsets, perm, inv, redrawn)
 
 
+class FastLayer:
+    """The fast-mode copy of a synthetic layer for the oracle, requantised here in
+    numpy (not by the library): every 3-bit expert's code c becomes c >> 1 (2-bit
+    field = the old field's high bit, then the third bit) and its fp16 scales double;
+    other experts are unchanged.  Same interface as synth.Layer for the oracle."""
+
+    def __init__(self, layer):
+        self.base = layer
+        self.cfg = layer.cfg
+        self.router_w, self.router_b = layer.router_w, layer.router_b
+        self.fmt = np.where(layer.fmt == synth.FMT_Q3, synth.FMT_Q2, layer.fmt).astype(np.uint8)
+
+    def expert(self, e):
+        m = self.base.expert(e)
+        if self.base.fmt[e] != synth.FMT_Q3:
+            return m
+        out = {}
+        for name, (c, h, s) in m.items():
+            bits = np.unpackbits(h, axis=1, bitorder="little")           # third bit of element k
+            f = np.zeros_like(c)
+            for i in range(4):
+                lo = (c >> (2 * i)) & 3
+                third = bits[:, i::4]
+                f |= (((lo >> 1) | (third << 1)) << (2 * i)).astype(np.uint8)
+            s2 = (s.view(np.float16).astype(np.float32) * 2).astype(np.float16).view(np.uint16)
+            out[name] = (f, None, s2)
+        return out
+
+
 def pack(case: Case, threads=None) -> np.ndarray:
     import bit_routed_expert_fp32_b200 as moe
     cfg, layer = case.cfg, case.layer

@@ -162,3 +162,20 @@ def test_few_token_integer_gate_up_full_chunks(T, shared_format):
     cfg = synth.micro(T=T, H=1024, E=16, k=8, I=128, S=1, formats="ternary", seed=40 + T)
     cfg = dataclasses.replace(cfg, shared_format=shared_format)
     _full_check(cfg, PATHS["decode"])
+
+
+@pytest.mark.parametrize("formats,T,path", [("q2", 1, "decode"), ("mixed", 12, "decode"), ("mixed", 96, "prefill")])
+def test_fast_mode_copy(formats, T, path):
+    """The fast mode's second buffer (every 3-bit expert replaced by its 2-bit copy)
+    through both paths: the GPU reads the library's requantised and packed copy, the
+    oracle the test harness's own numpy requantisation of the same layer."""
+    import oracle
+    import bit_routed_expert_fp32_b200 as moe
+    cfg = synth.micro(T=T, H=256, E=16, k=4, I=128, S=1, formats=formats, seed=60 + T)
+    case = H.make_case(cfg)
+    fmt2, fn2 = moe.fast_copy(case.layer.fmt, case.layer.expert)
+    packed = moe.pack_layer(cfg, fmt2, fn2)
+    rt, y = H.run_gpu(case, packed, path=PATHS[path])
+    H.check_routing(case, rt)
+    ref = oracle.forward_tokens(H.FastLayer(case.layer), case.x, case.ids, case.gates, range(T))
+    H.check_outputs(y, ref)
