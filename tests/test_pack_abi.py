@@ -135,3 +135,44 @@ def test_pack_rejects_ternary_code_three_and_small_buffer():
     with pytest.raises(moe.MoeError) as ei:
         moe.moe_pack_experts(cfg, layer.fmt, 0, [m], np.zeros(size, np.uint8))
     assert ei.value.status == 1
+
+
+def test_pack_roundtrip_random_shapes_and_formats():
+    """Property check of the packer against the oracle's independent reader: random
+    shapes (H, I multiples of 64, partial chunks included), expert counts and a random
+    format per expert, shared expert in any format."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=25, deadline=None, derandomize=True)
+    @given(st.integers(1, 9), st.integers(1, 6), st.integers(1, 6), st.integers(0, 1), st.data())
+    def check(hg, ig, E, S, data):
+        H, I = 64 * hg, 64 * ig
+        fmts = np.array(data.draw(st.lists(st.integers(0, 2), min_size=E + S, max_size=E + S)), np.uint8)
+        cfg = synth.micro(T=1, H=H, E=E, k=1, I=I, S=S, formats="mixed", seed=hg * 100 + ig * 10 + E)
+        rng = np.random.default_rng(int(fmts.sum()) + H + I)
+
+        def mats(e):
+            out = {}
+            for name, rows, K in (("gate", I, H), ("up", I, H), ("down", H, I)):
+                codes = rng.integers(0, 256, (rows, K // 4), dtype=np.uint8)
+                if fmts[e] == synth.FMT_TERNARY:          # fields 0..2 only
+                    f = np.stack([(codes >> (2 * i)) & 3 for i in range(4)])
+                    f = np.where(f == 3, 2, f)
+                    codes = (f[0] | (f[1] << 2) | (f[2] << 4) | (f[3] << 6)).astype(np.uint8)
+                hi = rng.integers(0, 256, (rows, K // 8), dtype=np.uint8) if fmts[e] == synth.FMT_Q3 else None
+                sc = np.float16(rng.uniform(-0.05, 0.05, (rows, K // 64))).view(np.uint16)
+                out[name] = (codes, hi, sc)
+            return out
+
+        cache = {e: mats(e) for e in range(E + S)}
+        buf = moe.pack_layer(cfg, fmts, lambda e: cache[e])
+        assert buf.size == moe.moe_packed_size(cfg, fmts)
+        for e in range(E + S):
+            for which, name, rows, K in ((0, "gate", I, H), (1, "up", I, H), (2, "down", H, I)):
+                f, codes, scales = oracle.unpack(buf, e, which, rows, K)
+                c, h, s = cache[e][name]
+                assert f == fmts[e]
+                np.testing.assert_array_equal(codes, codes_int(c, h))
+                np.testing.assert_array_equal(scales, s)
+
+    check()
