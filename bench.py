@@ -11,11 +11,13 @@ reads its experts from HBM.  For N > 1 (torchrun) each rank runs an independent
 replica on its own token stream (the layer is data-parallel: no collective on the
 data path) and the time is the max over ranks.
 
-The roofline object describes the gate/up launch: for the decode path (<= 64 tokens)
-against the measured HBM copy bandwidth (algorithmic bytes = the packed bytes of
-every selected expert and the shared expert, each read once); for the tensor-core
-prefill path against the measured sustained bf16 GEMM rate (algorithmic FLOPs =
-2 x routed rows x 2*ffn x hidden; the fp16 operands run at the bf16 rate).
+The roofline object describes the dominant launch.  Up to 16 tokens the whole decode
+forward is one kernel (ffn_fused_kernel): against the measured HBM copy bandwidth, with
+algorithmic bytes = the packed gate/up and down bytes of every selected expert and the
+shared expert, each read once.  From 17 to 64 tokens, the decode gate/up launch against
+the same peak (its packed gate/up bytes).  For the tensor-core prefill path, the gate/up
+launch against the measured sustained bf16 GEMM rate (algorithmic FLOPs = 2 x routed rows
+x 2*ffn x hidden; the fp16 operands run at the bf16 rate).
 
 --impl reference times the CPU oracle (the only reference that exists for this
 layer) on the same workload, a bounded sample per step, on the host cores.
@@ -43,6 +45,10 @@ METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B2
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # gate/up kernel of each path and the sources its ncu traffic record is tied to
 PATHS = {
+    "fused": ("ffn_fused_kernel (the whole decode forward: token operands, gate/up + SwiGLU, down and the "
+              "combine, one persistent launch; integer MMAs for ternary / 2-bit gate/up)",
+              ["bit_routed_expert_fp32_b200/csrc/decode_fused.cu", "bit_routed_expert_fp32_b200/csrc/dequant.cuh",
+               "bit_routed_expert_fp32_b200/csrc/operands.cuh", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "decode": ("ffn_decode_kernel<0, *> (gate/up + SwiGLU; integer MMAs for ternary / 2-bit experts at <= 4 "
                "tokens; interval includes the K-part reduction when K is split)",
                ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
@@ -51,10 +57,15 @@ PATHS = {
 }
 
 
+FUSED_MAX_T = 16       # the library's fused decode kernel serves up to this many tokens
+
+
 def path_of(cfg) -> str:
     """The path moe_forward(MOE_PATH_AUTO) takes for this workload."""
     tc_ok = cfg.H % 128 == 0 and (2 * cfg.I) % 128 == 0
-    return "prefill" if cfg.T > 64 and tc_ok else "decode"
+    if cfg.T > 64 and tc_ok:
+        return "prefill"
+    return "fused" if 1 <= cfg.T <= FUSED_MAX_T and cfg.E + cfg.S <= 272 else "decode"
 
 
 def decode_kparts(cfg):
@@ -85,6 +96,8 @@ def launches_per_step(cfg) -> int:
     route = 1 if cfg.T <= 64 else 4
     if path_of(cfg) == "prefill":
         return route + 4
+    if path_of(cfg) == "fused":
+        return route + 1
     return route + 3 + (1 if decode_kparts(cfg)[0] > 1 else 0)
 
 
@@ -438,7 +451,15 @@ def run_ours(args, cfg):
     path = path_of(cfg)
     tr = traffic_record(cfg.name, path)
     traffic = None if tr is None else tr["dram_bytes_per_launch"]
-    if path == "decode":
+    if path == "fused":
+        fused_alg = [a + b for a, b in zip(gu_alg, dn_alg)]
+        fused_gbs = (sum(fused_alg) / 1e9) / (sum(gu_ms) / 1e3)
+        roofline = {"bound": "hbm", "kernel": PATHS[path][0], "achieved": fused_gbs, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": fused_gbs / pk["hbm_gbs"], "traffic": traffic,
+                    "algorithmic_bytes_per_launch": float(np.mean(fused_alg)),
+                    "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)",
+                    "avg_launch_us": 1e3 * float(np.mean(gu_ms))}
+    elif path == "decode":
         roofline = {"bound": "hbm", "kernel": PATHS[path][0], "achieved": gu_gbs, "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": gu_gbs / pk["hbm_gbs"], "traffic": traffic,
                     "algorithmic_bytes_per_launch": float(np.mean(gu_alg)),
@@ -490,10 +511,16 @@ def run_ours(args, cfg):
                                       "one CUDA graph per step (route + forward), replayed"),
                 "roofline": roofline,
                 "layer_weight_stream_gbs": layer_gbs,
-                "kernel_us": {"route": 1e3 * float(np.mean(rt_ms)), "gate_up": 1e3 * float(np.mean(gu_ms)),
-                              "down": 1e3 * float(np.mean(dn_ms)), "combine": 1e3 * float(np.mean(cb_ms)),
-                              "down_gbs": dn_gbs, "step_with_events_between_kernels": 1e3 * float(np.mean(step_serial_ms)),
-                              "measured": "second pass over the same steps with an event between kernels"},
+                "kernel_us": ({"route": 1e3 * float(np.mean(rt_ms)), "forward_fused": 1e3 * float(np.mean(gu_ms)),
+                               "step_with_events_between_kernels": 1e3 * float(np.mean(step_serial_ms)),
+                               "measured": "second pass over the same steps with an event between the router "
+                                           "and the forward kernel (which also stops their overlap)"}
+                              if path == "fused" else
+                              {"route": 1e3 * float(np.mean(rt_ms)), "gate_up": 1e3 * float(np.mean(gu_ms)),
+                               "down": 1e3 * float(np.mean(dn_ms)), "combine": 1e3 * float(np.mean(cb_ms)),
+                               "down_gbs": dn_gbs,
+                               "step_with_events_between_kernels": 1e3 * float(np.mean(step_serial_ms)),
+                               "measured": "second pass over the same steps with an event between kernels"}),
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.H * 2,
                         "d2h_bytes_per_step": T * cfg.H * 2},
                 "gpu_launches": launches_per_step(cfg) * args.steps,
@@ -527,6 +554,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--soak-s", type=float, default=1.5)
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's tokens per step (profiling)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the routed expert count (profiling: the same per-step work on a smaller layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every call eagerly instead of replaying graphs")
     args = ap.parse_args()
@@ -536,6 +565,9 @@ def main():
     if args.tokens:
         import dataclasses
         cfg = dataclasses.replace(cfg, T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
+    if args.experts:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, E=args.experts, name=f"{cfg.name}_E{args.experts}")
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

@@ -20,12 +20,18 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_DEVICE_CHECK"}
 FMT_TERNARY, FMT_Q2, FMT_Q3 = 0, 1, 2
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+OUT_F32 = 0x10          # OR into a path: moe_forward writes fp32 y
 
 # every symbol include/moe.h declares
 EXPORTS = ["moe_packed_size", "moe_pack_experts", "moe_requantize_q3_to_q2", "moe_workspace_size",
            "moe_workspace_init", "moe_route",
-           "moe_forward", "moe_forward_timed", "moe_get_error", "moe_decode_static", "moe_event_record",
-           "moe_status_string", "moe_abi_version"]
+           "moe_forward", "moe_forward_timed", "moe_get_error", "moe_decode_static", "moe_decode_static_get_error",
+           "moe_workspace_set_test_stall", "moe_event_record", "moe_status_string", "moe_abi_version",
+           "moe_route_fixed", "moe_gather_rows", "moe_combine_pairs", "moe_cache_size", "moe_cache_init",
+           "moe_cache_load"]
+# detail codes beside MOE_ERR_TIMEOUT / MOE_ERR_DEVICE_CHECK (high bits: what; low byte: where)
+DETAIL = {"WAIT_FULL": 0x100, "WAIT_EMPTY": 0x200, "DRAIN": 0x300, "HEADER": 0x400, "ROUTED_T": 0x500,
+          "RANGE": 0x600, "TEST_STALL": 0x700, "LOOP_CAP": 0x800}
 STATIC_WS_BYTES = 8 << 20
 
 
@@ -71,6 +77,14 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(vp), i32]
         L.moe_get_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_decode_static.argtypes = [sh, i32, vp, vp, vp, vp, ctypes.POINTER(Routing), vp, vp]
+        L.moe_decode_static_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_workspace_set_test_stall.argtypes = [vp, sz, ctypes.c_uint32, vp]
+        L.moe_route_fixed.argtypes = [sh, i32, vp, vp, vp, ctypes.POINTER(Routing), vp, sz, vp]
+        L.moe_gather_rows.argtypes = [i32, i32, vp, i32, vp, i32, vp, vp, sz, vp]
+        L.moe_combine_pairs.argtypes = [i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_cache_size.argtypes = [sh, vp, i32, ctypes.POINTER(sz)]
+        L.moe_cache_init.argtypes = [sh, vp, i32, vp, sz, vp]
+        L.moe_cache_load.argtypes = [sh, vp, i32, vp, sz, vp, vp, i32, vp]
         L.moe_event_record.argtypes = [vp, vp]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -227,6 +241,44 @@ def moe_decode_static(cfg, T, x, router_w, router_b, packed, rt: dict, y, stream
     _check("moe_decode_static", lib().moe_decode_static(ctypes.byref(_shape(cfg)), T, _ptr(x), _ptr(router_w),
                                                          _ptr(router_b), _ptr(packed), ctypes.byref(r), _ptr(y),
                                                          _stream(stream)))
+
+
+def moe_decode_static_get_error(stream=None):
+    """(status, detail) recorded on the device by moe_decode_static calls since the last
+    read; synchronises the stream and clears the record."""
+    d = ctypes.c_uint32(0)
+    st = lib().moe_decode_static_get_error(_stream(stream), ctypes.byref(d))
+    return st, d.value
+
+
+def moe_workspace_set_test_stall(ws, cycles: int, stream=None) -> None:
+    """Failure-path tests only: the expert kernels of the next moe_forward calls on ws
+    first wait up to `cycles` SM cycles on a barrier nothing completes (0 = off)."""
+    _check("moe_workspace_set_test_stall",
+           lib().moe_workspace_set_test_stall(_ptr(ws), ws.numel() * ws.element_size(), cycles, _stream(stream)))
+
+
+def moe_route_fixed(cfg, T, x, ids, gates, rt: dict, ws, stream=None) -> None:
+    """Routing of caller-given expert ids / gates (device int32 / float32 [T][k])."""
+    r = routing_struct(rt)
+    _check("moe_route_fixed", lib().moe_route_fixed(ctypes.byref(_shape(cfg)), T, _ptr(x), _ptr(ids), _ptr(gates),
+                                                     ctypes.byref(r), _ptr(ws), ws.numel() * ws.element_size(),
+                                                     _stream(stream)))
+
+
+def moe_gather_rows(src, index, divisor, dst, ws, n=None, stream=None) -> None:
+    """dst[i] = src[index[i] // divisor] for the first n rows (bf16 [rows][H] tensors)."""
+    n = index.numel() if n is None else n
+    _check("moe_gather_rows", lib().moe_gather_rows(n, src.shape[1], _ptr(src), src.shape[0], _ptr(index), divisor,
+                                                     _ptr(dst), _ptr(ws), ws.numel() * ws.element_size(),
+                                                     _stream(stream)))
+
+
+def moe_combine_pairs(T, k, rows, inv_perm, gates, shared, y, ws, stream=None) -> None:
+    """y[t] = sum_j gates[t][j] rows[inv_perm[t k + j]] + shared[t] (bf16 rows)."""
+    _check("moe_combine_pairs", lib().moe_combine_pairs(T, k, y.shape[1], _ptr(rows), rows.shape[0], _ptr(inv_perm),
+                                                         _ptr(gates), _ptr(shared), _ptr(y), _ptr(ws),
+                                                         ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_get_error(ws, stream=None):

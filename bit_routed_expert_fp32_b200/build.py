@@ -21,9 +21,9 @@ NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", 
               "-Xcompiler", "-fPIC", "-Xptxas", "-v", "-I", INCLUDE, "-I", CSRC]
 CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-I", INCLUDE]
 
-CU = ["route.cu", "decode_ffn.cu", "prefill_tc.cu", "api.cu", "static_ws.cu"]
+CU = ["route.cu", "decode_ffn.cu", "decode_fused.cu", "prefill_tc.cu", "ep.cu", "cache.cu", "api.cu", "static_ws.cu"]
 CPP = ["pack.cpp"]
-HEADERS = ["common.cuh", "kernels.h"]
+HEADERS = ["common.cuh", "kernels.h", "dequant.cuh", "operands.cuh"]
 
 
 def _newer(src_list, target):

@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "kernels.h"
 #include "moe.h"
 
@@ -35,6 +37,12 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     off = align256(off + 4 * (size_t)(3 * (8 * ((H / 64 + 7) / 8)) * T));   // two fp16 planes
     w.iq = off;
     off = align256(off + iq_bytes(T, H));
+    // the fused decode kernel's fp32 h and its integer operands, for min(T, kFusedMaxT) tokens
+    const int64_t r16 = (T < kFusedMaxT ? T : kFusedMaxT) * (k + S);
+    w.hf = off;
+    off = align256(off + 4 * (size_t)(r16 * I));
+    w.hq = off;
+    off = align256(off + (r16 > 0 ? iq_size(r16, I) : 0));
     w.h = off;
     off = align256(off + 2 * (size_t)(T * (k + S) * I));
     // ypart, and the decode gate/up partial sums that alias it: the largest need of any
@@ -57,9 +65,7 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
 
 }  // namespace moe
 
-namespace {
-
-using namespace moe;
+namespace moe {
 
 bool shape_ok(const moe_shape* s) {
     return s && s->hidden > 0 && s->inter > 0 && s->hidden % 64 == 0 && s->inter % 64 == 0 &&
@@ -67,18 +73,20 @@ bool shape_ok(const moe_shape* s) {
            s->top_k <= s->n_experts && (s->n_shared == 0 || s->n_shared == 1);
 }
 
+namespace {
+
 size_t ws_fixed_prefix(const moe_shape* s) { return ws_layout(s, 0).active; }
 
 int sm_count() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = n > 0 ? n : 148;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 bool routing_ok(const moe_routing* r) {
@@ -93,6 +101,35 @@ moe_status check_common(const moe_shape* shape, int32_t T, const void* d_ws, siz
     return MOE_OK;
 }
 
+}  // namespace
+
+moe_status check_route_args(const moe_shape* shape, int32_t T, const uint16_t* d_x, const float* d_router_w,
+                            const moe_routing* out, const void* d_ws, size_t ws_bytes) {
+    const moe_status st = check_common(shape, T, d_ws, ws_bytes);
+    if (st != MOE_OK) return st;
+    if (!d_x || !d_router_w || !routing_ok(out)) return MOE_ERR_INVALID_ARG;
+    if (ws_fixed_prefix(shape) > 4096 + 65536) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status check_forward_args(const moe_shape* shape, int32_t T, const void* d_packed, const uint16_t* d_x,
+                              const moe_routing* r, const uint16_t* d_y, moe_path path, const void* d_ws,
+                              size_t ws_bytes) {
+    const moe_status st = check_common(shape, T, d_ws, ws_bytes);
+    if (st != MOE_OK) return st;
+    if (!d_packed || !d_x || !d_y || !routing_ok(r)) return MOE_ERR_INVALID_ARG;
+    const int base = (int)path & ~MOE_OUT_F32;
+    if (base != MOE_PATH_AUTO && base != MOE_PATH_DECODE && base != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Writes the test-stall word of a workspace's control block (one thread).
+__global__ void set_test_stall_kernel(Ctrl* c, uint32_t cycles) { c->test_stall = cycles; }
+
+}  // namespace moe
+
+namespace {
+using namespace moe;
 }  // namespace
 
 extern "C" {
@@ -133,16 +170,20 @@ moe_status moe_workspace_init(void* d_ws, size_t ws_bytes, void* stream) {
     return MOE_OK;
 }
 
+moe_status moe_workspace_set_test_stall(void* d_ws, size_t ws_bytes, uint32_t cycles, void* stream) {
+    if (!d_ws || ws_bytes < 4096) return MOE_ERR_INVALID_ARG;
+    set_test_stall_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<Ctrl*>(d_ws), cycles);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x, const float* d_router_w,
                      const float* d_router_b, const moe_routing* out, void* d_ws, size_t ws_bytes, void* stream) {
-    moe_status st = check_common(shape, T, d_ws, ws_bytes);
+    const moe_status st = check_route_args(shape, T, d_x, d_router_w, out, d_ws, ws_bytes);
     if (st != MOE_OK) return st;
-    if (!d_x || !d_router_w || !routing_ok(out)) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (ws_fixed_prefix(shape) > 4096 + 65536) return MOE_ERR_UNSUPPORTED;
     const Ws w = ws_layout(shape, T);
     uint8_t* ws = static_cast<uint8_t*>(d_ws);
-    RouteArgs a;
+    RouteArgs a = {};     // every field not set below is zero (no fixed routing)
     a.T = T;
     a.H = shape->hidden;
     a.E = shape->n_experts;
@@ -155,26 +196,79 @@ moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x, con
     a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
     a.active = reinterpret_cast<int32_t*>(ws + w.active);
     a.zx = reinterpret_cast<float*>(ws + w.zx);
-    a.iq = T <= kIqMaxT ? ws + w.iq : nullptr;
+    // The decode operands are formed by the router only for the decode kernels that do
+    // not form them themselves (more than kFusedMaxT tokens).
+    a.ops = T > kFusedMaxT;
+    a.iq = nullptr;
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.r = *out;
     if (launch_route(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 
+moe_status moe_route_fixed(const moe_shape* shape, int32_t T, const uint16_t* d_x, const int32_t* d_ids,
+                           const float* d_gates, const moe_routing* out, void* d_ws, size_t ws_bytes, void* stream) {
+    // the same checks as moe_route, with the caller's ids and gates in place of the router
+    const float* present = reinterpret_cast<const float*>(d_ids);
+    const moe_status st = check_route_args(shape, T, d_x, present, out, d_ws, ws_bytes);
+    if (st != MOE_OK) return st;
+    if (!d_ids || !d_gates) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    const Ws w = ws_layout(shape, T);
+    uint8_t* ws = static_cast<uint8_t*>(d_ws);
+    RouteArgs a = {};
+    a.T = T;
+    a.H = shape->hidden;
+    a.E = shape->n_experts;
+    a.k = shape->top_k;
+    a.S = shape->n_shared;
+    a.x = d_x;
+    a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
+    a.active = reinterpret_cast<int32_t*>(ws + w.active);
+    a.zx = reinterpret_cast<float*>(ws + w.zx);
+    a.ops = T > kFusedMaxT;
+    a.iq = nullptr;
+    a.fixed_ids = d_ids;
+    a.fixed_w = d_gates;
+    a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
+    a.r = *out;
+    return launch_route_fixed(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_gather_rows(int32_t n, int32_t hidden, const uint16_t* d_src, int32_t n_src, const int32_t* d_index,
+                           int32_t divisor, uint16_t* d_dst, void* d_ws, size_t ws_bytes, void* stream) {
+    if (n < 0 || hidden <= 0 || hidden % 64 != 0 || n_src < 0 || divisor < 1) return MOE_ERR_INVALID_ARG;
+    if (n == 0) return MOE_OK;
+    if (!d_src || !d_index || !d_dst || !d_ws || ws_bytes < 4096) return MOE_ERR_INVALID_ARG;
+    return launch_gather_rows(n, hidden, d_src, d_index, divisor, n_src, d_dst, static_cast<Ctrl*>(d_ws),
+                              static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+moe_status moe_combine_pairs(int32_t T, int32_t top_k, int32_t hidden, const float* d_rows, int32_t n_rows,
+                             const int32_t* d_inv_perm, const float* d_gates, const float* d_shared, uint16_t* d_y,
+                             void* d_ws, size_t ws_bytes, void* stream) {
+    if (T < 0 || top_k < 1 || top_k > 16 || hidden <= 0 || hidden % 64 != 0 || n_rows < 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!d_rows || !d_inv_perm || !d_gates || !d_y || !d_ws || ws_bytes < 4096) return MOE_ERR_INVALID_ARG;
+    return launch_combine_pairs(T, top_k, hidden, n_rows, d_rows, d_inv_perm, d_gates, d_shared, d_y,
+                                static_cast<Ctrl*>(d_ws), static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_packed, const uint16_t* d_x,
                              const moe_routing* r, uint16_t* d_y, moe_path path, void* d_ws, size_t ws_bytes,
                              void* stream, void* const* events, int32_t n_events) {
-    moe_status st = check_common(shape, T, d_ws, ws_bytes);
+    const moe_status st = check_forward_args(shape, T, d_packed, d_x, r, d_y, path, d_ws, ws_bytes);
     if (st != MOE_OK) return st;
-    if (!d_packed || !d_x || !d_y || !routing_ok(r)) return MOE_ERR_INVALID_ARG;
-    if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
     if (events && n_events < 4) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const Ws w = ws_layout(shape, T);
     uint8_t* ws = static_cast<uint8_t*>(d_ws);
-    FfnArgs a;
+    FfnArgs a = {};
     a.T = T;
     a.H = shape->hidden;
     a.I = shape->inter;
@@ -190,8 +284,13 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.topk_w = r->topk_w;
     a.active = reinterpret_cast<const int32_t*>(ws + w.active);
     a.zx = reinterpret_cast<const float*>(ws + w.zx);
-    a.iq = T <= kIqMaxT ? ws + w.iq : nullptr;
+    a.iq = T <= kFusedMaxT ? ws + w.iq : nullptr;
     a.iq_on = 0;
+    a.fc = reinterpret_cast<FusedCtl*>(ws + w.ctrl + sizeof(Ctrl));
+    a.dn_done = reinterpret_cast<uint32_t*>(ws + w.tile_ctr);
+    a.hf = reinterpret_cast<float*>(ws + w.hf);
+    a.hq = ws + w.hq;
+    a.R16 = (T < kFusedMaxT ? T : kFusedMaxT) * (a.k + a.S);
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.h = reinterpret_cast<uint16_t*>(ws + w.h);
     a.ypart = reinterpret_cast<float*>(ws + w.ypart);
@@ -199,6 +298,8 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.nkp_gu = a.nkp_dn = 1;
     a.tile_ctr = reinterpret_cast<uint32_t*>(ws + w.tile_ctr);
     a.y = d_y;
+    a.y_f32 = ((int)path & MOE_OUT_F32) != 0;
+    path = (moe_path)((int)path & ~MOE_OUT_F32);
     a.num_ctas = sm_count();
     cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
     if (events)
@@ -208,12 +309,18 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     const bool tc_ok = a.H % 128 == 0 && (2 * a.I) % 128 == 0;
     if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
     const bool prefill = path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kSmallT && tc_ok);
-    if (!prefill) {
-        decode_kparts(shape, T, &a.nkp_gu, &a.nkp_dn);
-        a.iq_on = T <= kIqMaxT;
+    const bool fused = !prefill && T <= kFusedMaxT && a.E + a.S <= kMaxSlots;
+    cudaError_t err;
+    if (fused) {
+        // one kernel: the per-kernel events all follow it
+        err = launch_ffn_fused(a, s);
+        for (int i = 1; i < 3 && err == cudaSuccess; ++i)
+            if (ev[i]) err = record_event(ev[i], s);
+    } else {
+        if (!prefill) decode_kparts(shape, T, &a.nkp_gu, &a.nkp_dn);
+        err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
+                      : launch_ffn_decode(a, s, ev[1], ev[2]);
     }
-    cudaError_t err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
-                              : launch_ffn_decode(a, s, ev[1], ev[2]);
     if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
     if (ev[3] && record_event(ev[3], s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;

@@ -37,8 +37,25 @@ struct Ctrl {
     int32_t n_active;       // experts with tokens + shared experts, written by moe_route
     int32_t routed_T;       // T of the last moe_route
     uint32_t work[2];       // decode work counters (gate/up, down); zeroed by the router and the combine
-    uint32_t pad[56];
+    uint32_t test_stall;    // failure-path tests only: cycles of a wait nothing completes (0 = off)
+    uint32_t pad[55];
 };
+static_assert(sizeof(Ctrl) == 256, "control block layout");
+
+// Counters of the fused decode kernel, right after Ctrl in the control block.  Every
+// launch leaves them at zero again (the last warp to finish resets them); the
+// workspace initialisation zeroes them first.
+constexpr int kMaxSlots = 272;              // expert slots: shared experts, then routed (>= E + S)
+struct FusedCtl {
+    uint32_t work;          // next work unit to hand out
+    uint32_t ops_done;      // operand units finished
+    uint32_t warps_done;    // warps that have left the unit loop
+    uint32_t abort;         // set when a wait ran out: every warp stops working
+    uint32_t pad[12];
+    uint32_t gu_done[kMaxSlots];   // gate/up tiles finished per expert slot
+    uint32_t hq_done[kMaxSlots];   // shares of the down pass's h operands formed per slot
+};
+static_assert(256 + sizeof(FusedCtl) <= 4096, "control block size");
 
 // error detail codes
 enum : uint32_t {
@@ -46,11 +63,18 @@ enum : uint32_t {
     kDetWaitEmpty = 0x200,
     kDetDrain = 0x300,
     kDetHeader = 0x400,
+    kDetRoutedT = 0x500,    // moe_forward's T differs from the preceding moe_route's
+    kDetRange = 0x600,      // a token or an expert activation outside the fp16 range
+    kDetTestStall = 0x700,  // the failure-path test's wait ran out
+    kDetLoopCap = 0x800,    // a work loop reached its iteration cap
 };
 
 __device__ inline void report_error(Ctrl* c, uint32_t code, uint32_t detail) {
     if (atomicCAS(&c->err_code, 0u, code) == 0u) atomicExch(&c->err_detail, detail);
 }
+
+// |v| <= 65504, the largest finite fp16 value (false for NaN and infinities).
+__device__ inline bool in_f16_range(float v) { return fabsf(v) <= 65504.f; }
 
 // ---- PTX wrappers -----------------------------------------------------------------
 __device__ inline uint32_t smem_u32(const void* p) {

@@ -1,6 +1,8 @@
-// Expert FFN kernels of the decode path (gate/up + SwiGLU and down, routed and
-// shared experts) and the gate-weighted unpermute-combine: grouped skinny GEMMs over
-// the packed ternary / 2-bit / 3-bit experts, for few tokens per expert.
+// Expert FFN kernels of the decode path for 17 to 64 tokens (gate/up + SwiGLU and down,
+// routed and shared experts; up to 16 tokens the fused kernel of decode_fused.cu runs
+// instead) and the gate-weighted unpermute-combine used by the decode and prefill
+// paths: grouped skinny GEMMs over the packed ternary / 2-bit / 3-bit experts, for few
+// tokens per expert.
 //
 // Decode speed is set by the expert bytes moved per token (ossradar.top, Xolotl
 // README, "Fast mode (DeepSeek-V4.1)"), and each selected expert is read once for
@@ -39,10 +41,6 @@
 //      down: pairs are (c - o) exactly (one fp16x2 subtract); fp16 MMAs, h is fp16.
 //    Each group result is scaled by its fp16 scale into an fp32 accumulator.
 //    3-bit experts add an MMA per k-step for 4 * (third bit).
-//  * gate/up with at most 4 tokens, ternary and 2-bit experts: integer MMAs instead
-//    (u8 codes masked out of the code words against signed-byte digits of the tokens
-//    on a 12-bit grid per group; see "few-token gate/up on the integer tensor path"
-//    below), which halves the dequantiser's ALU work and the MMA chain per group.
 //  * gate/up: the 16 rows of a tile are 8 gate rows and the matching 8 up rows, which
 //    the MMA places in the same thread (rows g and g + 8), so with a single K part
 //    h = silu(gate) * up is formed in registers and stored as fp16; with several K
@@ -50,9 +48,11 @@
 //  * down: partial rows (fp32) per (K part, token, slot); the combine kernel then
 //    sums the parts, each token's k slots in slot order with the gates, adds the
 //    shared expert and writes y in bf16: deterministic, no floating-point atomics.
-// Every wait is bounded; a wait that runs out records an error in the workspace and
-// the warp carries on without waiting, so the kernel always terminates.
+// Every wait is bounded; a wait that runs out records an error in the workspace and the
+// warp gives up: it issues no more copies, waits (bounded) for those in flight and
+// leaves, so the kernel always terminates.
 #include "kernels.h"
+#include "dequant.cuh"
 
 namespace moe {
 namespace {
@@ -68,152 +68,7 @@ constexpr int NS = 2;                                  // stages per warp
 constexpr int TP = 8;                                  // tokens per pass (one n-tile)
 constexpr long long kWaitLimit = 4000000000LL;         // clock cycles (~2 s)
 
-// bf16 magic bases (exponent-only bit patterns) of the gate/up dequantiser
-constexpr uint32_t kMag128 = 0x43004300u, kMag32 = 0x42004200u, kMag8 = 0x41004100u, kMag64 = 0x42804280u,
-                   kMag16 = 0x41804180u, kMag512 = 0x44004400u, kMag256 = 0x43804380u;
-// fp16 magic bases of the down dequantiser
-constexpr uint32_t kH512 = 0x60006000u, kH256 = 0x5C005C00u, kH64 = 0x54005400u, kH16 = 0x4C004C00u,
-                   kH4 = 0x44004400u, kH4096 = 0x6C006C00u, kH2048 = 0x68006800u, kH1024 = 0x64006400u,
-                   kH128 = 0x58005800u, kH32 = 0x50005000u;
-
-// ---- dequantisers (code word: element 2p + h of its 16 at bits 16h + 2p .. +1) ----
-
-// bf16 pairs "base_p + c"; base per pair p: 128, 32, 8, 128, 32, 8, 128, 32 (a code
-// at mantissa bits 0-1 / 2-3 / 4-5 of 128 / 32 / 8 has weight exactly 1).
-__device__ __forceinline__ void raw_codes_bf16(uint32_t w, uint32_t (&pr)[8]) {
-    const uint32_t w6 = w >> 6, w12 = w >> 12;
-    pr[0] = lop3_and_or(w, 0x00030003u, kMag128);     // bits 0-1
-    pr[1] = lop3_and_or(w, 0x000C000Cu, kMag32);      // bits 2-3
-    pr[2] = lop3_and_or(w, 0x00300030u, kMag8);       // bits 4-5
-    pr[3] = lop3_and_or(w6, 0x00030003u, kMag128);    // bits 6-7 -> 0-1
-    pr[4] = lop3_and_or(w6, 0x000C000Cu, kMag32);     // bits 8-9 -> 2-3
-    pr[5] = lop3_and_or(w6, 0x00300030u, kMag8);      // bits 10-11 -> 4-5
-    pr[6] = lop3_and_or(w12, 0x00030003u, kMag128);   // bits 12-13 -> 0-1
-    pr[7] = lop3_and_or(w12, 0x000C000Cu, kMag32);    // bits 14-15 -> 2-3
-}
-
-// bf16 pairs "base_p + 4 * bit" of the third code bit (bits 0..7 of each half of u);
-// base per pair p: 512, 256, 128, 64, 32, 16, 8, 8.
-__device__ __forceinline__ void raw_hi_bf16(uint32_t u, uint32_t (&pr)[8]) {
-    pr[0] = lop3_and_or(u, 0x00010001u, kMag512);
-    pr[1] = lop3_and_or(u, 0x00020002u, kMag256);
-    pr[2] = lop3_and_or(u, 0x00040004u, kMag128);
-    pr[3] = lop3_and_or(u, 0x00080008u, kMag64);
-    pr[4] = lop3_and_or(u, 0x00100010u, kMag32);
-    pr[5] = lop3_and_or(u, 0x00200020u, kMag16);
-    pr[6] = lop3_and_or(u, 0x00400040u, kMag8);
-    pr[7] = lop3_and_or(u >> 1, 0x00400040u, kMag8);
-}
-
-// fp16 pairs (c - o), exact: the bases 512, 256, 64, 16, 4 have an ulp <= 1/2.
-__device__ __forceinline__ void exact_codes_f16(uint32_t w, const uint32_t (&sub)[5], uint32_t (&pr)[8]) {
-    const uint32_t w1 = w << 1, w8 = w >> 8;
-    pr[0] = f16x2_sub(lop3_and_or(w1, 0x00060006u, kH512), sub[0]);    // bits 0-1 -> 1-2
-    pr[1] = f16x2_sub(lop3_and_or(w, 0x000C000Cu, kH256), sub[1]);     // bits 2-3
-    pr[2] = f16x2_sub(lop3_and_or(w, 0x00300030u, kH64), sub[2]);      // bits 4-5
-    pr[3] = f16x2_sub(lop3_and_or(w, 0x00C000C0u, kH16), sub[3]);      // bits 6-7
-    pr[4] = f16x2_sub(lop3_and_or(w, 0x03000300u, kH4), sub[4]);       // bits 8-9
-    pr[5] = f16x2_sub(lop3_and_or(w8, 0x000C000Cu, kH256), sub[1]);    // bits 10-11 -> 2-3
-    pr[6] = f16x2_sub(lop3_and_or(w8, 0x00300030u, kH64), sub[2]);     // bits 12-13 -> 4-5
-    pr[7] = f16x2_sub(lop3_and_or(w8, 0x00C000C0u, kH16), sub[3]);     // bits 14-15 -> 6-7
-}
-
-// fp16 pairs 4 * (third bit), exact.
-__device__ __forceinline__ void exact_hi_f16(uint32_t u, uint32_t (&pr)[8]) {
-    pr[0] = f16x2_sub(lop3_and_or(u, 0x00010001u, kH4096), kH4096);
-    pr[1] = f16x2_sub(lop3_and_or(u, 0x00020002u, kH2048), kH2048);
-    pr[2] = f16x2_sub(lop3_and_or(u, 0x00040004u, kH1024), kH1024);
-    pr[3] = f16x2_sub(lop3_and_or(u, 0x00080008u, kH512), kH512);
-    pr[4] = f16x2_sub(lop3_and_or(u, 0x00100010u, kH256), kH256);
-    pr[5] = f16x2_sub(lop3_and_or(u, 0x00200020u, kH128), kH128);
-    pr[6] = f16x2_sub(lop3_and_or(u, 0x00400040u, kH64), kH64);
-    pr[7] = f16x2_sub(lop3_and_or(u, 0x00800080u, kH32), kH32);
-}
-
-// Rows g (wa) and g + 8 (wb) straight into MMA A-fragment order: k-step s uses
-// {pair 2s of wa, pair 2s of wb, pair 2s+1 of wa, pair 2s+1 of wb}.
-template <int MODE>
-__device__ __forceinline__ void dequant_rows(uint32_t wa, uint32_t wb, const uint32_t (&sub)[5], uint32_t (&pa)[8],
-                                             uint32_t (&pb)[8]) {
-    if (MODE == 0) {
-        raw_codes_bf16(wa, pa);
-        raw_codes_bf16(wb, pb);
-    } else {
-        exact_codes_f16(wa, sub, pa);
-        exact_codes_f16(wb, sub, pb);
-    }
-}
-
-template <int MODE>
-__device__ __forceinline__ void dequant_hi_rows(uint32_t ua, uint32_t ub, uint32_t (&pa)[8], uint32_t (&pb)[8]) {
-    if (MODE == 0) {
-        raw_hi_bf16(ua, pa);
-        raw_hi_bf16(ub, pb);
-    } else {
-        exact_hi_f16(ua, pa);
-        exact_hi_f16(ub, pb);
-    }
-}
-
-template <int MODE>
-__device__ __forceinline__ void mma_acc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                        uint32_t b0, uint32_t b1) {
-    if (MODE == 0)
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    else
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// The four k-steps of one 64-wide group of one tile against one n-tile (xb: the B
-// fragments of the group, pairs 0..7 of this lane's 16 elements).
-template <int MODE>
-__device__ __forceinline__ void mma_group(float (&d)[4], const uint32_t (&pa)[8], const uint32_t (&pb)[8],
-                                          const uint4& x0, const uint4& x1) {
-    mma_acc<MODE>(d, pa[0], pb[0], pa[1], pb[1], x0.x, x0.y);
-    mma_acc<MODE>(d, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
-    mma_acc<MODE>(d, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
-    mma_acc<MODE>(d, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
-}
-
-// The same four k-steps with a zero accumulator input (the group's sum starts at 0).
-template <int MODE>
-__device__ __forceinline__ void mma_group_first(float (&d)[4], const uint32_t (&pa)[8], const uint32_t (&pb)[8],
-                                                const uint4& x0, const uint4& x1) {
-    const float zero = 0.f;
-    if (MODE == 0)
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%10,%10,%10,%10};"
-            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-            : "r"(pa[0]), "r"(pb[0]), "r"(pa[1]), "r"(pb[1]), "r"(x0.x), "r"(x0.y), "f"(zero));
-    else
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%10,%10,%10,%10};"
-            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-            : "r"(pa[0]), "r"(pb[0]), "r"(pa[1]), "r"(pb[1]), "r"(x0.x), "r"(x0.y), "f"(zero));
-    mma_acc<MODE>(d, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
-    mma_acc<MODE>(d, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
-    mma_acc<MODE>(d, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
-}
-
-// acc += A B with A 16 x 8 fp16 (row-major fragment: rows g and g + 8, k = 2t, 2t+1)
-// and B 8 x 8 fp16 (k = 2t, 2t+1 of column g); fp32 accumulation.
-__device__ __forceinline__ void mma_f16_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-    asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(b0));
-}
-
-__device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w & 0xFFFFu))); }
-__device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half((uint16_t)(w >> 16))); }
-__device__ __forceinline__ const PackedEntry* entry(const uint8_t* packed, int e) {
-    return reinterpret_cast<const PackedEntry*>(packed + kHeaderBytes + (size_t)e * kEntryBytes);
-}
+using namespace dq;
 
 // ---- the CTA's copy of the schedule -------------------------------------------------
 constexpr int kMaxActive = 260;
@@ -221,6 +76,7 @@ constexpr int kPermSmem = 1024;                        // routed pairs staged in
 
 struct CtaSched {
     int ok;
+    uint32_t stall;            // failure-path tests: cycles of warp 0's wait on stall_bar (0 = off)
     int n_active;
     int n_units;
     int perm_in_smem;
@@ -288,9 +144,7 @@ __device__ __forceinline__ int src_token(const FfnArgs& p, const CtaSched& S, in
 struct UnitView {
     const uint16_t* b;         // B-operand row of token column g (+16t elements)
     const uint16_t* z;         // gate/up: -Z/16 (hi plane) of token column g, groups 2t, 2t+1
-    const uint4* bq;           // integer path: digit record of column g, lane t, group 0
-    const float* pq;           // integer path: factors p of token t, group 0
-    int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token); integer path: token t
+    int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token)
 };
 
 // Columns without a token read a valid row (the pass's first token); their MMA
@@ -329,7 +183,6 @@ __device__ __forceinline__ void make_view(const FfnArgs& p, const CtaSched& S, i
 struct LaneGeo {
     int g, t, cw_lane, g4, hw_lane, g2, sh;
     int zplane;                // elements from the hi to the lo plane of the Z table
-    int zplane_iq;             // the same for the integer path's offset planes
 };
 
 __device__ __forceinline__ uint32_t f16x2_mul16(uint32_t a, uint32_t b) {
@@ -464,147 +317,6 @@ __device__ __forceinline__ void chunk_partial(const uint8_t* stg, int c, int ng,
     }
 }
 
-// ---- few-token gate/up on the integer tensor path (ternary and 2-bit experts) ----
-// With at most kIqMaxT tokens a pass uses one n8 tile as two signed-byte digit
-// columns per token (column 2j + d: digit d of token j; route.cu writes the digit
-// records).  A code word w of row g gives four u8 A registers without any add:
-// w & 0x03030303 (the codes themselves), w & 0x0C0C0C0C (4 x the codes) and the same
-// of w >> 4; B carries 4q or q to match, so each group is two m16n8k32 u8 x s8 MMAs
-// with exact int32 sums.  The accumulator starts at the bit pattern of 1.5 * 2^23, so
-// the int32 result read as fp32 is 1.5 * 2^23 + D exactly (|D| < 2^17) and one
-// subtract recovers D.  Per group, acc += s p (D) with p = 2^-e / 4 of this lane's
-// token; the chunk's offsets are removed by the fp16 Z MMAs as on the bf16 path, with
-// the Z columns of the high digits zero.  Lane (g, t) ends with rows g, g + 8 of
-// token t: acc[.][0] + 256 acc[.][1] and acc[.][2] + 256 acc[.][3].
-constexpr uint32_t kIqMagic = 0x4B400000u;             // 1.5 * 2^23
-constexpr float kIqMagicF = 12582912.0f;
-
-__device__ __forceinline__ void imma_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                           uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(kIqMagic));
-}
-__device__ __forceinline__ void imma_acc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// One 64-group of one tile: wa, wb the code words of rows g and g + 8, b the lane's
-// digit record (MMA 0: b.x, b.y; MMA 1: b.z, b.w), s0, s1 the two rows' scales times p.
-__device__ __forceinline__ void group_iq_tile(uint32_t wa, uint32_t wb, const uint4& b, float s0, float s1,
-                                              float (&acc)[4]) {
-    const uint32_t wa4 = wa >> 4, wb4 = wb >> 4;
-    int d[4];
-    imma_first(d, wa & 0x03030303u, wb & 0x03030303u, wa & 0x0C0C0C0Cu, wb & 0x0C0C0C0Cu, b.x, b.y);
-    imma_acc(d, wa4 & 0x03030303u, wb4 & 0x03030303u, wa4 & 0x0C0C0C0Cu, wb4 & 0x0C0C0C0Cu, b.z, b.w);
-    acc[0] = fmaf(s0, __int_as_float(d[0]) - kIqMagicF, acc[0]);
-    acc[1] = fmaf(s0, __int_as_float(d[1]) - kIqMagicF, acc[1]);
-    acc[2] = fmaf(s1, __int_as_float(d[2]) - kIqMagicF, acc[2]);
-    acc[3] = fmaf(s1, __int_as_float(d[3]) - kIqMagicF, acc[3]);
-}
-
-// The chunk's offset correction on the integer path: the bf16 path's z_correction
-// with this lane's Z column (zero for the high-digit columns: v.z == nullptr).
-__device__ __forceinline__ void z_correction_iq(const uint8_t* stg, int c, const UnitView& v, const LaneGeo& L,
-                                                float (&acc)[NTL][4]) {
-    constexpr uint32_t kSixteen = 0x4C004C00u;
-    const uint32_t bhi = v.z ? __ldg(reinterpret_cast<const uint32_t*>(v.z + 8 * c)) : 0u;
-    const uint32_t blo = v.z ? __ldg(reinterpret_cast<const uint32_t*>(v.z + L.zplane_iq + 8 * c)) : 0u;
-#pragma unroll
-    for (int tl = 0; tl < NTL; ++tl) {
-        const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + tl * TSTAGE + OFF_SC);
-        const uint32_t a0 = f16x2_mul16(scw[4 * L.g + L.t], kSixteen);
-        const uint32_t a1 = f16x2_mul16(scw[4 * (L.g + 8) + L.t], kSixteen);
-        mma_f16_1688(acc[tl], a0, a1, bhi);
-        mma_f16_1688(acc[tl], a0, a1, blo);
-    }
-}
-
-template <int HI>
-__device__ __forceinline__ void group_iq(const uint8_t* stg, int gl, const uint4* bq, float pf, const LaneGeo& L,
-                                         const uint32_t (&s2)[NTL][2], float (&acc)[NTL][4]) {
-    const uint32_t* cw = reinterpret_cast<const uint32_t*>(stg);
-    const int cpos = L.cw_lane + ((4 * gl) ^ L.g4);
-    uint32_t w[NTL][2];
-#pragma unroll
-    for (int tl = 0; tl < NTL; ++tl) {
-        w[tl][0] = cw[cpos + tl * (TSTAGE / 4)];
-        w[tl][1] = cw[cpos + tl * (TSTAGE / 4) + 256];
-    }
-    const uint4 b = __ldg(bq + 8 * gl);
-#pragma unroll
-    for (int tl = 0; tl < NTL; ++tl) {
-        const float s0 = (HI ? half_hi(s2[tl][0]) : half_lo(s2[tl][0])) * pf;
-        const float s1 = (HI ? half_hi(s2[tl][1]) : half_lo(s2[tl][1])) * pf;
-        group_iq_tile(w[tl][0], w[tl][1], b, s0, s1, acc[tl]);
-    }
-}
-
-__device__ __forceinline__ void chunk_full_iq(const uint8_t* stg, int c, const UnitView& v, const LaneGeo& L,
-                                              float (&acc)[NTL][4]) {
-    const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + OFF_SC);
-    const uint4* bq = v.bq + c * (CG * 8);
-    const float2* pq = reinterpret_cast<const float2*>(v.pq + c * CG);
-    z_correction_iq(stg, c, v, L, acc);
-#pragma unroll 1
-    for (int gp = 0; gp < CG / 2; ++gp) {
-        uint32_t s2[NTL][2];
-#pragma unroll
-        for (int tl = 0; tl < NTL; ++tl) {
-            s2[tl][0] = scw[tl * (TSTAGE / 4) + 4 * L.g + gp];
-            s2[tl][1] = scw[tl * (TSTAGE / 4) + 4 * (L.g + 8) + gp];
-        }
-        const float2 pf = __ldg(pq + gp);
-        group_iq<0>(stg, 2 * gp, bq, pf.x, L, s2, acc);
-        group_iq<1>(stg, 2 * gp + 1, bq, pf.y, L, s2, acc);
-    }
-}
-
-__device__ __forceinline__ void chunk_partial_iq(const uint8_t* stg, int c, int ng, const UnitView& v,
-                                                 const LaneGeo& L, float (&acc)[NTL][4]) {
-    const int g = L.g, t = L.t;
-    z_correction_iq(stg, c, v, L, acc);
-    for (int gl = 0; gl < ng; ++gl) {
-        const uint4 b = __ldg(v.bq + c * (CG * 8) + 8 * gl);
-        const float pf = __ldg(v.pq + c * CG + gl);
-#pragma unroll
-        for (int tl = 0; tl < NTL; ++tl) {
-            const uint8_t* tb = stg + tl * TSTAGE;
-            const uint32_t* cw = reinterpret_cast<const uint32_t*>(tb);
-            const uint16_t* scs = reinterpret_cast<const uint16_t*>(tb + OFF_SC);
-            const float s0 = __half2float(__ushort_as_half(scs[g * 8 + gl])) * pf;
-            const float s1 = __half2float(__ushort_as_half(scs[(g + 8) * 8 + gl])) * pf;
-            group_iq_tile(cw[g * 4 * ng + 4 * gl + t], cw[(g + 8) * 4 * ng + 4 * gl + t], b, s0, s1, acc[tl]);
-        }
-    }
-}
-
-// View of an integer-path unit (one pass: cnt <= kIqMaxT).  B column g is digit g & 1
-// of the pass's token g >> 1; the outputs of this lane are token t's.  Columns and
-// outputs without a token read the pass's first token and are never stored.
-__device__ __forceinline__ void make_view_iq(const FfnArgs& p, const CtaSched& S, int a, int g, int t,
-                                             UnitView& v) {
-    const int e = S.e[a], f = S.fmt[a], nb = min(kIqMaxT, S.cnt[a]);
-    const bool routed = e < p.E;
-    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
-    const int ib = (g >> 1) < nb ? (g >> 1) : 0, it = t < nb ? t : 0;
-    const int tb = routed ? src_token(p, S, S.off[a] + ib) : ib;
-    const int tt = routed ? src_token(p, S, S.off[a] + it) : it;
-    v.bq = reinterpret_cast<const uint4*>(p.iq) + ((size_t)tb * G * 2 + (g & 1)) * 4 + t;
-    v.pq = reinterpret_cast<const float*>(p.iq + iq_pq_off(p.T, p.H)) + (size_t)tt * G8;
-    v.z = (g & 1) ? nullptr
-                  : reinterpret_cast<const uint16_t*>(p.iq + iq_zq_off(p.T, p.H)) + ((size_t)f * p.T + tb) * G8 + 2 * t;
-    v.orow[0] = t < nb ? (routed ? S.off[a] + t : p.T * p.k + (e - p.E) * p.T + t) : -1;
-    v.orow[1] = -1;
-}
-
 // Per-launch geometry of one expert pass (gate/up: K = H, rows 2I; down: K = I, rows H).
 struct Geo {
     int K, G, NC, blocks, nkp, cpk;
@@ -713,28 +425,6 @@ __device__ __forceinline__ void unit_epilogue(const FfnArgs& p, const Geo& geo, 
     }
 }
 
-// Integer-path unit end: combine the digit columns of token t and store as the bf16
-// path does (h directly, or this K part's gate and up sums).
-__device__ __forceinline__ void unit_epilogue_iq(const FfnArgs& p, const Geo& geo, const UnitPos& q,
-                                                 const UnitView& v, const LaneGeo& L, const float (&acc)[NTL][4]) {
-    const int orow = v.orow[0];
-    if (orow < 0) return;
-    const size_t R = (size_t)p.T * (p.k + p.S);
-#pragma unroll
-    for (int tl = 0; tl < NTL; ++tl) {
-        const int j = NTL * q.jb + tl;
-        const float gs = fmaf(256.f, acc[tl][1], acc[tl][0]);
-        const float us = fmaf(256.f, acc[tl][3], acc[tl][2]);
-        if (geo.nkp == 1) {
-            p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(silu_f(gs) * us);
-        } else {
-            float* dst = p.gpart + ((size_t)q.kp * R + orow) * (2 * p.I) + j * 16 + L.g;
-            dst[0] = gs;
-            dst[8] = us;
-        }
-    }
-}
-
 // Gate/up with few tokens: every SM reads the same token rows and Z values, so each CTA
 // pulls them into L1 at the start.  The token rows are the caller's input (ready before
 // the router ran); the Z values are the router's output and are prefetched only after
@@ -755,11 +445,11 @@ __device__ inline void warm_z(const FfnArgs& p) {
         prefetch_l1(reinterpret_cast<const uint8_t*>(p.zx) + i * 128);
 }
 
-// IQ (gate/up only): ternary and 2-bit experts take the integer path (T <= kIqMaxT).
-template <int MODE, bool IQ>
+template <int MODE>
 __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ CtaSched S;
+    __shared__ uint64_t stall_bar;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Geo geo;
     geo.K = MODE == 0 ? p.H : p.I;
@@ -783,9 +473,16 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     if (MODE == 0) warm_rows(p);
     griddep_wait();
     if (threadIdx.x == 0) {
-        if (!S.ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
-        S.n_active = p.ctrl->n_active;
+        if (!S.ok) {
+            report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
+        } else if (__ldcg(&p.ctrl->routed_T) != p.T) {
+            // the schedule in the workspace was routed for another T: do not read it
+            report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRoutedT | MODE);
+            S.ok = 0;
+        }
+        S.n_active = __ldcg(&p.ctrl->n_active);
         S.perm_in_smem = p.T * p.k <= kPermSmem;
+        S.stall = p.ctrl->test_stall;
     }
     __syncthreads();
     if (!S.ok) return;
@@ -816,6 +513,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     if (MODE == 0) warm_z(p);
     if (lane == 0)
         for (int s = 0; s < NS; ++s) mbar_init(&bar[s], 1);
+    if (threadIdx.x == 0) mbar_init(&stall_bar, 1);            // nothing ever arrives on it
     fence_mbar_init();
     __syncthreads();
     // Units come from the launch's work counter (zeroed by the router and by the
@@ -844,32 +542,48 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     L.g2 = 2 * (L.g >> 1);
     L.sh = 8 * (L.t & 1);
     L.zplane = 3 * p.T * (8 * ((p.H / 64 + 7) / 8));
-    L.zplane_iq = 2 * p.T * (8 * ((p.H / 64 + 7) / 8));
     bool aborted = false;
     int consumed = 0;
     // The chunk to consume is the one issued NS - 1 issues ago (hu / hc[NS - 1] after
     // the next issue).  A unit ends when the next chunk belongs to another unit.
     int unit = -1, view_a = -1, view_pass = -1;
-    bool q3 = false, iqu = false;                      // iqu: the current unit is on the integer path
+    bool q3 = false;
     UnitPos q;
     q.a = q.pass = q.jb = q.kp = 0;
     UnitView v;
     uint32_t sub[5] = {0, 0, 0, 0, 0};
     float acc[NTL][4];
-    while (true) {
+    // failure-path tests: warp 0 waits on a barrier nothing completes; the wait runs out
+    // and the warp takes the give-up path below
+    if (warp == 0 && S.stall) {
+        int done = 0;
+        if (lane == 0) done = mbar_wait_bounded(&stall_bar, 0, S.stall);
+        if (!__shfl_sync(0xffffffffu, done, 0)) {
+            aborted = true;
+            if (lane == 0) report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetTestStall | MODE);
+        }
+    }
+    // A warp consumes at most every chunk of every unit once, plus the empty issues at
+    // the end: a cap that consistent counters never reach.
+    const long long max_iters = (long long)S.n_units * geo.cpk + NS + 2;
+    long long iters = 0;
+    while (!aborted) {
+        if (++iters > max_iters) {
+            aborted = true;
+            if (lane == 0) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetLoopCap | MODE);
+            break;
+        }
         prod.issue(p, S, geo, per_ep, fkp, ctr, lane, ring, bar, pol);
         const int hu = prod.hu[NS - 1], c = prod.hc[NS - 1];
         if (hu < 0) {                                   // nothing left (or nothing at all)
             if (unit >= 0) {
-                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, acc);
-                else unit_epilogue<MODE>(p, geo, q, v, L, acc);
+                unit_epilogue<MODE>(p, geo, q, v, L, acc);
             }
             break;
         }
         if (hu != unit) {
             if (unit >= 0) {
-                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, acc);
-                else unit_epilogue<MODE>(p, geo, q, v, L, acc);
+                unit_epilogue<MODE>(p, geo, q, v, L, acc);
             }
             unit = hu;
             q = unit_pos(S, unit, per_ep, fkp);
@@ -877,9 +591,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
                 view_a = q.a;
                 view_pass = q.pass;
                 q3 = S.fmt[q.a] == MOE_FMT_Q3;
-                iqu = IQ && !q3;
-                if (IQ && iqu) make_view_iq(p, S, q.a, L.g, L.t, v);
-                else make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
+                make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
                 if (MODE == 1) {
                     const int f = S.fmt[q.a];
                     const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
@@ -894,16 +606,19 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
             for (int tl = 0; tl < NTL; ++tl) acc[tl][0] = acc[tl][1] = acc[tl][2] = acc[tl][3] = 0.f;
         }
         const int st = consumed % NS;
-        if (!aborted && !mbar_wait_bounded(&bar[st], (uint32_t)(consumed / NS) & 1, kWaitLimit)) {
-            aborted = true;
+        int ok = 1;
+        if (lane == 0 && !mbar_wait_bounded(&bar[st], (uint32_t)(consumed / NS) & 1, kWaitLimit)) {
+            ok = 0;
             report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | MODE);
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+            // give up: issue nothing more; the copies in flight are waited for below
+            aborted = true;
+            break;
         }
         const uint8_t* stg = ring + (size_t)st * STAGE;
         const int ng = min(CG, geo.G - c * CG);
-        if (IQ && iqu) {
-            if (ng == CG) chunk_full_iq(stg, c, v, L, acc);
-            else chunk_partial_iq(stg, c, ng, v, L, acc);
-        } else if (ng == CG) {
+        if (ng == CG) {
             if (q3) chunk_full<MODE, true>(stg, c, v, L, sub, acc);
             else chunk_full<MODE, false>(stg, c, v, L, sub, acc);
         } else {
@@ -976,6 +691,7 @@ __device__ __forceinline__ void add4(float4& a, const float4& b) {
 
 __global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
     griddep_wait();                                     // ypart comes from the down pass
+    if (__ldcg(&p.ctrl->routed_T) != p.T) return;       // inv_perm is another T's (reported by the FFN kernels)
     if (blockIdx.x == 0 && threadIdx.x == 0) {          // both expert passes are complete
         p.ctrl->work[0] = 0;
         p.ctrl->work[1] = 0;
@@ -1042,6 +758,10 @@ __global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
             }
         }
     }
+    if (p.y_f32) {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + (size_t)tok * p.H + c4) = acc;
+        return;
+    }
     uint2 o;
     o.x = (uint32_t)f32_to_bf16_bits(acc.x) | ((uint32_t)f32_to_bf16_bits(acc.y) << 16);
     o.y = (uint32_t)f32_to_bf16_bits(acc.z) | ((uint32_t)f32_to_bf16_bits(acc.w) << 16);
@@ -1052,6 +772,7 @@ __global__ void __launch_bounds__(128) combine_kernel(FfnArgs p) {
 // (two 16-byte loads per row and part), rows one after another.
 __global__ void __launch_bounds__(256) combine_rows_kernel(FfnArgs p) {
     griddep_wait();                                     // ypart comes from the down pass
+    if (__ldcg(&p.ctrl->routed_T) != p.T) return;       // inv_perm is another T's (reported by the FFN kernels)
     if (blockIdx.x == 0 && threadIdx.x == 0) {          // both expert passes are complete
         p.ctrl->work[0] = 0;
         p.ctrl->work[1] = 0;
@@ -1085,6 +806,12 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(FfnArgs p) {
             add4(a1, s1);
         }
     }
+    if (p.y_f32) {
+        float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + (size_t)tok * p.H + c8);
+        d[0] = a0;
+        d[1] = a1;
+        return;
+    }
     uint4 o;
     o.x = (uint32_t)f32_to_bf16_bits(a0.x) | ((uint32_t)f32_to_bf16_bits(a0.y) << 16);
     o.y = (uint32_t)f32_to_bf16_bits(a0.z) | ((uint32_t)f32_to_bf16_bits(a0.w) << 16);
@@ -1095,22 +822,17 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(FfnArgs p) {
 
 constexpr size_t kDynSmem = (size_t)NW * NS * STAGE + (size_t)NW * NS * 8;
 
-template <int MODE, bool IQ>
+template <int MODE>
 cudaError_t launch_mode(const FfnArgs& a, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_decode_kernel<MODE, IQ>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDynSmem);
-        if (err != cudaSuccess) return err;
-        attr = true;
-    }
-    return launch_pdl(ffn_decode_kernel<MODE, IQ>, dim3(a.num_ctas), dim3(NW * 32), kDynSmem, s, a);
+    const cudaError_t err = set_smem_limit(ffn_decode_kernel<MODE>, kDynSmem);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(ffn_decode_kernel<MODE>, dim3(a.num_ctas), dim3(NW * 32), kDynSmem, s, a);
 }
 
 }  // namespace
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down) {
-    cudaError_t err = a.iq_on && a.iq ? launch_mode<0, true>(a, s) : launch_mode<0, false>(a, s);
+    cudaError_t err = launch_mode<0>(a, s);
     if (err != cudaSuccess) return err;
     if (a.nkp_gu > 1) {
         const long long n = (long long)a.T * (a.k + a.S) * (a.I / 4);
@@ -1118,7 +840,7 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_g
         if (err != cudaSuccess) return err;
     }
     if (ev_gateup && (err = record_event(ev_gateup, s)) != cudaSuccess) return err;
-    err = launch_mode<1, false>(a, s);
+    err = launch_mode<1>(a, s);
     if (err != cudaSuccess) return err;
     if (ev_down && (err = record_event(ev_down, s)) != cudaSuccess) return err;
     return launch_combine(a, s);

@@ -1,0 +1,1076 @@
+// The decode forward for few tokens (1 <= T <= 16) as ONE persistent kernel: the
+// token operands, the gate/up + SwiGLU pass and the down pass of every selected expert
+// and of the shared expert, and the gate-weighted combine into y.
+//
+// Decode speed is set by the expert bytes moved per token (ossradar.top, Xolotl README,
+// "Fast mode (DeepSeek-V4.1)"), and each selected expert is read once for all of its
+// tokens (the same README, "Latest").  With one token, a step reads about 117 MB in
+// ~18 us at the HBM roofline, so the step cannot afford kernel boundaries (a launch,
+// a ramp and a tail each) between its phases; instead the phases are units of work in
+// one queue and wait on each other through counters in the workspace:
+//
+//   operands  (token, 64-wide group): the integer path's token digits and factors and
+//             the Z tables, formed from the bf16 tokens (operands.cuh)
+//   gate/up   (expert, 16-row tile of the fused gate/up matrix, all of K): needs the
+//             operands; h = silu(gate) * up in fp16
+//   down      (expert, 16-row tile of the down matrix, all of K): needs every gate/up
+//             tile of its expert; fp32 rows of y_e
+//   combine   the down unit that finishes a 16-row slice of y last for all experts
+//             sums the slice's rows, the routed ones weighted by their gates in slot
+//             order, plus the shared expert's, and stores bf16 (deterministic)
+//
+// Units are handed out in that order from one counter (one unit ahead of need), so
+// every wait is for a unit some running warp already holds: the queue cannot deadlock,
+// whatever the number of resident CTAs.  The shared expert does not depend on the
+// routing: its units come first and run while the router kernel, launched just
+// before with programmatic dependent launch, is still choosing the experts;
+// griddepcontrol.wait is executed only by warps that reach a routed unit.
+//
+// Inside a unit a warp streams its tile's 8-group chunks (codes, third bits, fp16
+// scales: contiguous blocks of the packed format) through its own ring of NS
+// shared-memory stages with 1-D bulk copies, and the ring runs ahead into the next
+// unit.  Gate/up of ternary and 2-bit experts runs on the integer tensor path (u8 codes
+// masked out of the code words against signed-byte token digits on a 12-bit grid per
+// token and group; passes of 4 tokens per n8 MMA tile); 3-bit experts use the bf16
+// dequantiser ("base + c" in the mantissa of a power of two, the offsets removed once
+// per chunk by a small MMA against the token's Z table; passes of 8 tokens); down
+// dequantises exact fp16 (c - o) against fp16 h.
+//
+// Every wait is bounded (mbarriers and counters); a wait that runs out records
+// MOE_ERR_TIMEOUT and raises an abort flag that makes every warp stop working, wait
+// (bounded) for its own copies in flight and leave.  The last warp to leave resets the
+// counters, so the next launch starts from zero.
+#include "kernels.h"
+#include "dequant.cuh"
+#include "operands.cuh"
+
+namespace moe {
+namespace {
+
+using namespace dq;
+
+constexpr int NW = 16;                           // warps per CTA (one CTA per SM)
+constexpr int NS = 3;                            // ring stages per warp
+constexpr int CG = 8;                            // 64-wide groups per chunk
+constexpr int OFF_HI = 2048;                     // stage: codes 16 rows x 32 words
+constexpr int OFF_SC = OFF_HI + 1024;            //        third bits 16 rows x 16 words
+constexpr int STAGE = OFF_SC + 256;              //        scales 16 rows x 8 halves
+constexpr int MAXP = 4;                          // integer passes per unit (4 tokens each)
+constexpr int MAXPB = 2;                         // bf16 / fp16 passes per unit (8 tokens each)
+constexpr long long kWaitLimit = 4000000000LL;   // clock cycles (~2 s)
+constexpr uint32_t kIqMagic = 0x4B400000u;       // 1.5 * 2^23
+constexpr float kIqMagicF = 12582912.0f;
+constexpr size_t kFusedSmem = (size_t)NW * NS * STAGE + (size_t)NW * NS * 8;
+
+static_assert(MAXP * 4 >= kFusedMaxT && MAXPB * 8 >= kFusedMaxT, "passes cover kFusedMaxT tokens");
+
+// ---- packed fp32 pairs (Blackwell f32x2 arithmetic) ---------------------------------
+__device__ __forceinline__ unsigned long long pk2(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 up2(unsigned long long v) {
+    float2 r;
+    asm("mov.b64 {%0,%1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// ---- global-memory synchronisation ---------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Lane 0 waits until *ctr >= target (or the launch aborts), bounded.  It polls with
+// relaxed loads and a growing sleep (an acquire load also drops the SM's L1 contents,
+// which the other warps on the SM are using), then makes one acquire load; the warp
+// barrier orders the other lanes' later loads after it.  Returns false if the wait ran
+// out or the launch aborted.
+__device__ __forceinline__ bool wait_counter(const uint32_t* ctr, uint32_t target, FusedCtl* fc, Ctrl* ctrl,
+                                             uint32_t detail, int lane) {
+    int ok = 1;
+    if (lane == 0) {
+        if (ld_relaxed(ctr) < target) {
+            const long long t0 = clock64();
+            uint32_t ns = 128;
+            while (true) {
+                __nanosleep(ns);
+                if (ns < 1024) ns *= 2;
+                if (ld_relaxed(ctr) >= target) break;
+                if (ld_relaxed(&fc->abort)) {
+                    ok = 0;
+                    break;
+                }
+                if (clock64() - t0 > kWaitLimit) {
+                    report_error(ctrl, MOE_ERR_TIMEOUT, detail);
+                    atomicExch(&fc->abort, 1u);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        if (ok) (void)ld_acquire(ctr);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// All lanes' stores of this unit happen-before the counter increment (release).
+__device__ __forceinline__ uint32_t signal_counter(uint32_t* ctr, int lane) {
+    __syncwarp();
+    uint32_t old = 0;
+    if (lane == 0) {
+        __threadfence();
+        old = atomicAdd(ctr, 1u);
+    }
+    return __shfl_sync(0xffffffffu, old, 0);
+}
+
+__device__ __forceinline__ const PackedEntry* pentry(const uint8_t* packed, int e) {
+    return reinterpret_cast<const PackedEntry*>(packed + kHeaderBytes + (size_t)e * kEntryBytes);
+}
+
+// ---- the work queue --------------------------------------------------------------------
+enum : int { U_NONE = 0, U_OPS = 1, U_GU = 2, U_DN = 3, U_PENDING = 4 };   // PENDING: not taken yet
+
+struct Layout {        // unit index ranges; the routed ones are known once routing is
+    int nops, nsgu, pre;        // operands, shared gate/up; pre = nops + nsgu
+    int tg, td;                 // 16-row tiles per expert: gate/up (2I/16), down (H/16)
+    int nch, nci;               // 8-group chunks per row: gate/up (K = H), down (K = I)
+    int nr;                     // routed experts with tokens (-1: not read yet)
+    int total;                  // all units (pre until routing is known)
+    bool t_ok;                  // the routing is for this call's T
+};
+
+// A unit is four integers; everything else about its expert comes from the CTA's slot
+// table in shared memory (a few registers per warp instead of a copy of it).
+struct Unit {
+    int kind, idx, slot, tile;
+};
+
+// Per expert slot (shared experts first, then the routed experts with tokens, in the
+// router's active order): table index, format, tokens, first row, and the packed
+// blocks of tile 0 of its gate/up and down matrices.
+struct SlotInfo {
+    const uint8_t* base[6];     // gate/up codes, third bits, scales; down codes, third bits, scales
+    int e, fmt, cnt, row0;
+};
+struct CtaState {
+    SlotInfo slot[kMaxSlots];
+    int routed;                 // 0: not read, 1: being read by one warp, 2: ready
+    int nr, t_ok;
+};
+
+__device__ __forceinline__ void fill_slot(SlotInfo& si, const FfnArgs& p, int e, int cnt, int row0) {
+    const PackedEntry* en = pentry(p.packed, e);
+    si.e = e;
+    si.fmt = (int)en->fmt;
+    si.cnt = cnt;
+    si.row0 = row0;
+    si.base[0] = p.packed + en->gu_codes;
+    si.base[1] = p.packed + en->gu_hi;
+    si.base[2] = p.packed + en->gu_scales;
+    si.base[3] = p.packed + en->dn_codes;
+    si.base[4] = p.packed + en->dn_hi;
+    si.base[5] = p.packed + en->dn_scales;
+}
+
+// The routing, once per CTA: every warp waits for the router grid (griddepcontrol.wait,
+// before it reads any router output); the first warp of the CTA to get here fills the
+// routed slots of the table, the others wait for it (bounded).  Returns the routed
+// expert count (-1 if that wait ran out; then the launch aborts) and whether the
+// routing is for this call's T.
+__device__ __noinline__ int read_routing(CtaState& cs, const FfnArgs& p, int lane, int* t_ok) {
+    griddep_wait();
+    int mine = 0;
+    if (lane == 0) mine = atomicCAS(&cs.routed, 0, 1) == 0;
+    mine = __shfl_sync(0xffffffffu, mine, 0);
+    int ok = 1;
+    if (mine) {
+        int nr = 0, tok = 1;
+        if (lane == 0) {
+            // from L2: this SM's L1 may hold the control block's line from before the
+            // router wrote it (the test-stall word shares the line)
+            tok = __ldcg(&p.ctrl->routed_T) == p.T;
+            nr = tok ? __ldcg(&p.ctrl->n_active) - p.S : 0;
+            if (!tok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRoutedT | 0x20);
+        }
+        nr = __shfl_sync(0xffffffffu, nr, 0);
+        tok = __shfl_sync(0xffffffffu, tok, 0);
+        for (int a = lane; a < nr; a += 32) {
+            const int e = __ldcg(p.active + a);
+            fill_slot(cs.slot[p.S + a], p, e, __ldcg(p.counts + e), __ldcg(p.offsets + e));
+        }
+        if (lane == 0) {
+            cs.nr = nr;
+            cs.t_ok = tok;
+        }
+        __syncwarp();
+        __threadfence_block();
+        if (lane == 0) *reinterpret_cast<volatile int*>(&cs.routed) = 2;
+        __syncwarp();
+    } else if (lane == 0) {
+        const long long t0 = clock64();
+        while (*reinterpret_cast<volatile int*>(&cs.routed) != 2) {
+            if (clock64() - t0 > kWaitLimit) {
+                report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | 0x24);
+                atomicExch(&p.fc->abort, 1u);
+                ok = 0;
+                break;
+            }
+            __nanosleep(100);
+        }
+        __threadfence_block();
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    *t_ok = ok && *reinterpret_cast<volatile int*>(&cs.t_ok) != 0;
+    return ok ? *reinterpret_cast<volatile int*>(&cs.nr) : -1;
+}
+
+// Unit u -> its kind, slot and tile.  Units at or past L.pre need the routing; until it
+// has been read they come back as U_NONE with idx = u.
+__device__ __forceinline__ Unit resolve(const FfnArgs& p, const Layout& L, int u) {
+    Unit U;
+    U.kind = U_NONE;
+    U.idx = u;
+    U.slot = 0;
+    U.tile = 0;
+    if (u < 0) return U;
+    if (u < L.nops) {
+        U.kind = U_OPS;
+        U.tile = u;
+        return U;
+    }
+    if (u < L.pre) {
+        const int v = u - L.nops;
+        U.kind = U_GU;
+        U.slot = v / L.tg;
+        U.tile = v - U.slot * L.tg;
+        return U;
+    }
+    if (L.nr < 0 || u >= L.total) return U;
+    int v = u - L.pre;
+    if (v < L.nr * L.tg) {
+        const int a = v / L.tg;
+        U.kind = U_GU;
+        U.tile = v - a * L.tg;
+        U.slot = p.S + a;
+    } else {
+        v -= L.nr * L.tg;
+        U.kind = U_DN;
+        U.slot = v / L.td;                  // shared experts first, then routed
+        U.tile = v - U.slot * L.td;
+    }
+    return U;
+}
+
+__device__ __forceinline__ bool streams(const Unit& U) { return U.kind == U_GU || U.kind == U_DN; }
+__device__ __forceinline__ int unit_nc(const Unit& U, const Layout& L) { return U.kind == U_DN ? L.nci : L.nch; }
+
+// The warp's next unit, taken from the launch's counter only when the ring is about to
+// need it (when the current unit's last chunks are being issued): a unit held early by a
+// warp that is still busy would hold back every unit that waits for it.
+struct Queue {
+    Unit nxt;
+};
+
+__device__ __forceinline__ void take_next(Queue& Q, const FfnArgs& p, const Layout& L, int lane) {
+    if (Q.nxt.kind != U_PENDING) return;
+    int u = 0;
+    if (lane == 0) u = (int)atomicAdd(&p.fc->work, 1u);
+    Q.nxt = resolve(p, L, __shfl_sync(0xffffffffu, u, 0));
+}
+
+// Source token of permuted row r of a slot's expert (routed: perm / k; shared: r - row0).
+__device__ __forceinline__ int row_token(const FfnArgs& p, int slot, int row0, int r) {
+    return slot < p.S ? r - row0 : __ldcg(p.perm + r) / p.k;
+}
+
+// ---- per-warp ring -------------------------------------------------------------------
+struct Ring {
+    uint8_t* base;
+    uint64_t* bar;
+    int issued, consumed;
+    int iw, ic;                // issue cursor: unit (0 = current, 1 = next) and chunk
+};
+
+// Issues the bulk copies of chunk c of unit U into the next stage (whole warp,
+// converged; one elected lane issues).
+__device__ __forceinline__ void issue_chunk(Ring& R, const CtaState& cs, const FfnArgs& p, const Unit& U, int c,
+                                            uint64_t pol) {
+    const int st = R.issued % NS;
+    const bool dn = U.kind == U_DN;
+    const SlotInfo& si = cs.slot[U.slot];
+    const int K = dn ? p.I : p.H, G = K / 64, NC = (G + CG - 1) / CG;
+    const int ng = min(CG, G - c * CG);
+    if (elect_one()) {
+        uint8_t* dst = R.base + (size_t)st * STAGE;
+        const uint32_t cb = 256 * ng, hb = si.fmt == MOE_FMT_Q3 ? 128 * ng : 0;
+        const int b = dn ? 3 : 0;
+        mbar_arrive_expect_tx(&R.bar[st], cb + hb + 256);
+        bulk_g2s_evict_first(dst, si.base[b] + (size_t)4 * K * U.tile + 2048 * (size_t)c, cb, &R.bar[st], pol);
+        bulk_g2s_evict_first(dst + OFF_SC, si.base[b + 2] + (size_t)256 * NC * U.tile + 256 * (size_t)c, 256,
+                             &R.bar[st], pol);
+        if (hb)
+            bulk_g2s_evict_first(dst + OFF_HI, si.base[b + 1] + (size_t)128 * G * U.tile + 1024 * (size_t)c, hb,
+                                 &R.bar[st], pol);
+    }
+    __syncwarp();
+    ++R.issued;
+}
+
+// Keeps up to NS chunks in flight: the current unit's, then the next unit's (if it is
+// known and streams).  Stops issuing after an abort.
+__device__ __forceinline__ void top_up(Ring& R, const CtaState& cs, const Unit& cur, Queue& Q, bool stop,
+                                       uint64_t pol, int lane, const FfnArgs& p, const Layout& L) {
+    if (stop) return;
+    while (R.issued - R.consumed < NS) {
+        if (R.iw == 0) {
+            if (streams(cur) && R.ic < unit_nc(cur, L)) {
+                issue_chunk(R, cs, p, cur, R.ic++, pol);
+                continue;
+            }
+            R.iw = 1;
+            R.ic = 0;
+            take_next(Q, p, L, lane);
+        }
+        if (streams(Q.nxt) && R.ic < unit_nc(Q.nxt, L)) {
+            issue_chunk(R, cs, p, Q.nxt, R.ic++, pol);
+            continue;
+        }
+        break;
+    }
+}
+
+// Waits for the stage of the next chunk to consume; false if the wait ran out (then
+// the abort flag is raised).
+__device__ __forceinline__ bool wait_stage(Ring& R, FusedCtl* fc, Ctrl* ctrl, int lane) {
+    const int st = R.consumed % NS;
+    int ok = 1;
+    if (lane == 0 && !mbar_wait_bounded(&R.bar[st], (uint32_t)(R.consumed / NS) & 1, kWaitLimit)) {
+        report_error(ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | 0x20);
+        atomicExch(&fc->abort, 1u);
+        ok = 0;
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// ---- stage readers ---------------------------------------------------------------------
+// code word (r, wl) and third-bit word (r, vl) of a stage (swizzled when the chunk is full)
+__device__ __forceinline__ int cw_idx(int r, int wl, bool full, int ng) {
+    return full ? r * 32 + (wl ^ (4 * (r & 7))) : r * 4 * ng + wl;
+}
+__device__ __forceinline__ int hw_idx(int r, int vl, bool full, int ng) {
+    return full ? r * 16 + (vl ^ (2 * ((r & 7) >> 1))) : r * 2 * ng + vl;
+}
+__device__ __forceinline__ float scale_of(const uint8_t* stg, int r, int gl) {
+    return __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(stg + OFF_SC)[r * 8 + gl]));
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul16(uint32_t a) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(0x4C004C00u));
+    return r;
+}
+
+// The chunk's offset correction, C += sum_gl 16 s[row][gl] * (-Z[col][gl] / 16) as two
+// m16n8k8 fp16 MMAs (hi and lo halves of -Z / 16): A = this lane's scale words of rows
+// g, g + 8 for groups 2t, 2t + 1 (x 16, exact), B = the halves of column g at groups
+// 2t, 2t + 1 (zero pointer: a column without correction).
+__device__ __forceinline__ void zcorr(const uint8_t* stg, const uint16_t* zhi, int zplane, int c, int g, int t,
+                                      float (&d)[4]) {
+    const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + OFF_SC);
+    const uint32_t a0 = f16x2_mul16(scw[4 * g + t]), a1 = f16x2_mul16(scw[4 * (g + 8) + t]);
+    const uint32_t bhi = zhi ? *reinterpret_cast<const uint32_t*>(zhi + 8 * c) : 0u;
+    const uint32_t blo = zhi ? *reinterpret_cast<const uint32_t*>(zhi + zplane + 8 * c) : 0u;
+    mma_f16_1688(d, a0, a1, bhi);
+    mma_f16_1688(d, a0, a1, blo);
+}
+
+// ---- gate/up on the integer path (ternary, 2-bit) ----------------------------------------
+// Pass q holds tokens 4q .. 4q + 3 of the expert.  B column g = digit (g & 1) of token
+// 4q + (g >> 1); lane (g, t) ends with rows g (gate) and g + 8 (up) of token 4q + t.
+// Offsets (32-bit, to keep registers): bq in 16-byte units from the digit records, pq in
+// floats from the factors, zq in halves from the offset planes (-1: no correction).
+template <int NP>
+struct IqView {
+    uint32_t bq[NP];     // digit record of column g, lane t, group 0 (16-byte units)
+    uint32_t pq[NP];     // pair {p, sum q} of token 4q + t, group 0
+    int orow[NP];        // h row of token 4q + t (-1: none)
+};
+
+struct IqBase {
+    const uint4* bq;     // digit records
+    const float2* pq;    // pairs
+};
+
+__device__ __forceinline__ void imma2(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                      uint32_t a5, uint32_t a6, uint32_t a7, const uint4& b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%10,%11};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y), "r"(kIqMagic), "r"(0));
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a4), "r"(a5), "r"(a6), "r"(a7), "r"(b.z), "r"(b.w));
+}
+
+// o4 = 4 o: 4 for ternary codes, 6 for 2-bit codes (the offset removed exactly, in the
+// integer sums: sum 4 (c - o) q = D - o4 sum q).
+template <int NP, bool FULL>
+__device__ __forceinline__ void chunk_gu_iq(const uint8_t* stg, int c, int ng, const IqView<NP>& v, const IqBase& B,
+                                            int np, int o4, int g, int t, unsigned long long (&acc)[NP]) {
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(stg);
+#pragma unroll 2
+    for (int gl = 0; gl < (FULL ? CG : ng); ++gl) {
+        const uint32_t w0 = cw[cw_idx(g, 4 * gl + t, FULL, ng)], w1 = cw[cw_idx(g + 8, 4 * gl + t, FULL, ng)];
+        const uint32_t w0s = w0 >> 4, w1s = w1 >> 4;
+        const uint32_t m0 = w0 & 0x03030303u, m1 = w1 & 0x03030303u, n0 = w0 & 0x0C0C0C0Cu, n1 = w1 & 0x0C0C0C0Cu;
+        const uint32_t m0s = w0s & 0x03030303u, m1s = w1s & 0x03030303u, n0s = w0s & 0x0C0C0C0Cu,
+                       n1s = w1s & 0x0C0C0C0Cu;
+        const unsigned long long sv = pk2(scale_of(stg, g, gl), scale_of(stg, g + 8, gl));
+        const int grp = c * CG + gl;
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            if (q < np) {
+                const uint4 b = B.bq[v.bq[q] + grp * 8];
+                const float2 pr = B.pq[v.pq[q] + grp];
+                const float pf = pr.x;
+                const int corr = o4 * __float_as_int(pr.y);
+                int d[4];
+                imma2(d, m0, m1, n0, n1, m0s, m1s, n0s, n1s, b);
+                const unsigned long long D =
+                    add2(pk2(__int_as_float(d[0] + 256 * d[1] - corr), __int_as_float(d[2] + 256 * d[3] - corr)),
+                         pk2(-kIqMagicF, -kIqMagicF));
+                acc[q] = fma2(mul2(sv, pk2(pf, pf)), D, acc[q]);
+            }
+        }
+    }
+}
+
+// The same for a full chunk (8 groups), with the addressing hoisted: the swizzled
+// position of this lane's code word for group gl is sw ^ (16 gl) bytes into the stage
+// (sw = 128 g + 16 (g mod 8) + 4 t; the row's 128-byte block keeps bits 4-6 free for
+// the XOR), row g + 8 is 1024 bytes further; the digit records and the pairs of the
+// chunk are at fixed offsets from one pointer each; the scales of the chunk come in
+// with one 16-byte load per row; and the code offset is folded into the accumulator's
+// start value, M - o4 sum q, so the low digit's sum comes out already corrected.
+template <int NP>
+__device__ __forceinline__ void chunk_iq_full(const uint8_t* stg, int c, const IqView<NP>& v, const IqBase& B, int np,
+                                              int o4, int sw, int g, unsigned long long (&acc)[NP]) {
+    const uint4 sg4 = *reinterpret_cast<const uint4*>(stg + OFF_SC + 16 * g);
+    const uint4 su4 = *reinterpret_cast<const uint4*>(stg + OFF_SC + 16 * (g + 8));
+    const uint32_t sg[4] = {sg4.x, sg4.y, sg4.z, sg4.w}, su[4] = {su4.x, su4.y, su4.z, su4.w};
+    const uint4* rec[NP];
+    const float2* prs[NP];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+        rec[q] = B.bq + v.bq[q] + 64 * c;
+        prs[q] = B.pq + v.pq[q] + CG * c;
+    }
+#pragma unroll(NP == 1 ? 8 : 2)
+    for (int gl = 0; gl < CG; ++gl) {
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(stg + (sw ^ (16 * gl)));
+        const uint32_t w0 = wp[0], w1 = wp[256];
+        const uint32_t w0s = w0 >> 4, w1s = w1 >> 4;
+        const uint32_t m0 = w0 & 0x03030303u, m1 = w1 & 0x03030303u, n0 = w0 & 0x0C0C0C0Cu, n1 = w1 & 0x0C0C0C0Cu;
+        const uint32_t m0s = w0s & 0x03030303u, m1s = w1s & 0x03030303u, n0s = w0s & 0x0C0C0C0Cu,
+                       n1s = w1s & 0x0C0C0C0Cu;
+        const uint32_t hg = (gl & 1) ? sg[gl >> 1] >> 16 : sg[gl >> 1] & 0xFFFFu;
+        const uint32_t hu = (gl & 1) ? su[gl >> 1] >> 16 : su[gl >> 1] & 0xFFFFu;
+        const unsigned long long sv = pk2(__half2float(__ushort_as_half((uint16_t)hg)),
+                                          __half2float(__ushort_as_half((uint16_t)hu)));
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            if (NP == 1 || q < np) {
+                const uint4 b = rec[q][8 * gl];
+                const float2 pr = prs[q][gl];
+                const int c0 = (int)kIqMagic - o4 * __float_as_int(pr.y);
+                int d[4];
+                asm volatile(
+                    "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                    "{%10,%11,%10,%11};"
+                    : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+                    : "r"(m0), "r"(m1), "r"(n0), "r"(n1), "r"(b.x), "r"(b.y), "r"(c0), "r"(0));
+                asm volatile(
+                    "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                    "{%0,%1,%2,%3};"
+                    : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                    : "r"(m0s), "r"(m1s), "r"(n0s), "r"(n1s), "r"(b.z), "r"(b.w));
+                const unsigned long long D =
+                    add2(pk2(__int_as_float(d[0] + 256 * d[1]), __int_as_float(d[2] + 256 * d[3])),
+                         pk2(-kIqMagicF, -kIqMagicF));
+                acc[q] = fma2(mul2(sv, pk2(pr.x, pr.x)), D, acc[q]);
+            }
+        }
+    }
+}
+
+// ---- gate/up on the bf16 path (3-bit) and down on the exact fp16 path ---------------------
+// Pass q holds tokens (gate/up) or rows (down) 8q .. 8q + 7 of the expert: B column g is
+// 8q + g; lane (g, t) ends with rows g, g + 8 of columns 8q + 2t, 8q + 2t + 1.
+template <int NP>
+struct BfView {
+    uint32_t b[NP];      // B row of column g (+ 16 t elements), elements from x (gate/up) or h (down)
+    int z[NP];           // gate/up: -Z/16 (hi plane, 3-bit) of column g, group 2t, in halves
+    int orow[NP][2];     // output rows of columns 2t, 2t + 1 (-1: none)
+};
+
+template <int MODE, bool Q3, bool FULL, int NP>
+__device__ __forceinline__ void chunk_bf(const uint8_t* stg, int c, int ng, const BfView<NP>& v, const uint16_t* bbase,
+                                         const uint16_t* zbase, int zplane, int np, const uint32_t (&sub)[5], int g,
+                                         int t, float (&acc)[NP][4]) {
+    if (MODE == 0) {
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+            if (q < np) zcorr(stg, zbase + v.z[q], zplane, c, g, t, acc[q]);
+    }
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(stg);
+    const uint32_t* hw = reinterpret_cast<const uint32_t*>(stg + OFF_HI);
+    const int sh = 8 * (t & 1);
+#pragma unroll 1
+    for (int gl = 0; gl < (FULL ? CG : ng); ++gl) {
+        uint32_t pa[8], pb[8], ha[8], hb[8];
+        dequant_rows<MODE>(cw[cw_idx(g, 4 * gl + t, FULL, ng)], cw[cw_idx(g + 8, 4 * gl + t, FULL, ng)], sub, pa, pb);
+        if (Q3)
+            dequant_hi_rows<MODE>(hw[hw_idx(g, 2 * gl + (t >> 1), FULL, ng)] >> sh,
+                                  hw[hw_idx(g + 8, 2 * gl + (t >> 1), FULL, ng)] >> sh, ha, hb);
+        const float s0 = scale_of(stg, g, gl), s1 = scale_of(stg, g + 8, gl);
+        const int grp = c * CG + gl;
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            if (q < np) {
+                const uint4* bp = reinterpret_cast<const uint4*>(bbase + v.b[q] + 64 * grp);
+                const uint4 x0 = bp[0], x1 = bp[1];
+                float d[4];
+                mma_group_first<MODE>(d, pa, pb, x0, x1);
+                if (Q3) mma_group<MODE>(d, ha, hb, x0, x1);
+                acc[q][0] = fmaf(s0, d[0], acc[q][0]);
+                acc[q][1] = fmaf(s0, d[1], acc[q][1]);
+                acc[q][2] = fmaf(s1, d[2], acc[q][2]);
+                acc[q][3] = fmaf(s1, d[3], acc[q][3]);
+            }
+        }
+    }
+}
+
+// chunk_bf for a full chunk, with the addressing hoisted as in chunk_iq_full: code word
+// of group gl at cw_sw ^ (16 gl) (row g + 8: 1024 bytes on), third-bit word at
+// hw_sw ^ (8 gl) (row g + 8: 512 bytes on; hw_sw = 64 g + 8 ((g mod 8) / 2) + 4 (t / 2)),
+// the chunk's scales in one 16-byte load per row, the B rows from one pointer per pass.
+template <int MODE, bool Q3, int NP>
+__device__ __forceinline__ void chunk_bf_full(const uint8_t* stg, int c, const BfView<NP>& v, const uint16_t* bbase,
+                                              const uint16_t* zbase, int zplane, int np, const uint32_t (&sub)[5],
+                                              int cw_sw, int hw_sw, int g, int t, float (&acc)[NP][4]) {
+    if (MODE == 0) {
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+            if (NP == 1 || q < np) zcorr(stg, zbase + v.z[q], zplane, c, g, t, acc[q]);
+    }
+    const uint4 sg4 = *reinterpret_cast<const uint4*>(stg + OFF_SC + 16 * g);
+    const uint4 su4 = *reinterpret_cast<const uint4*>(stg + OFF_SC + 16 * (g + 8));
+    const uint32_t sg[4] = {sg4.x, sg4.y, sg4.z, sg4.w}, su[4] = {su4.x, su4.y, su4.z, su4.w};
+    const int sh = 8 * (t & 1);
+    const uint4* bp[NP];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) bp[q] = reinterpret_cast<const uint4*>(bbase + v.b[q] + 64 * CG * c);
+#pragma unroll 2
+    for (int gl = 0; gl < CG; ++gl) {
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(stg + (cw_sw ^ (16 * gl)));
+        uint32_t pa[8], pb[8], ha[8], hb[8];
+        dequant_rows<MODE>(wp[0], wp[256], sub, pa, pb);
+        if (Q3) {
+            const uint32_t* hp = reinterpret_cast<const uint32_t*>(stg + OFF_HI + (hw_sw ^ (8 * gl)));
+            dequant_hi_rows<MODE>(hp[0] >> sh, hp[128] >> sh, ha, hb);
+        }
+        const uint32_t hg = (gl & 1) ? sg[gl >> 1] >> 16 : sg[gl >> 1] & 0xFFFFu;
+        const uint32_t hu = (gl & 1) ? su[gl >> 1] >> 16 : su[gl >> 1] & 0xFFFFu;
+        const float s0 = __half2float(__ushort_as_half((uint16_t)hg)), s1 = __half2float(__ushort_as_half((uint16_t)hu));
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            if (NP == 1 || q < np) {
+                const uint4 x0 = bp[q][8 * gl], x1 = bp[q][8 * gl + 1];
+                float d[4];
+                mma_group_first<MODE>(d, pa, pb, x0, x1);
+                if (Q3) mma_group<MODE>(d, ha, hb, x0, x1);
+                acc[q][0] = fmaf(s0, d[0], acc[q][0]);
+                acc[q][1] = fmaf(s0, d[1], acc[q][1]);
+                acc[q][2] = fmaf(s1, d[2], acc[q][2]);
+                acc[q][3] = fmaf(s1, d[3], acc[q][3]);
+            }
+        }
+    }
+}
+
+// The next chunk's stage of the current unit (the ring topped up first, into the next
+// unit if the current one is all issued), once its copies have landed; nullptr if
+// nothing is in flight (after an abort).  A wait that runs out raises stop.
+__device__ __forceinline__ const uint8_t* next_stage(Ring& R, const CtaState& cs, const Unit& cur, Queue& Q,
+                                                     bool& stop, FusedCtl* fc, Ctrl* ctrl, int lane, uint64_t pol,
+                                                     const FfnArgs& p, const Layout& L) {
+    top_up(R, cs, cur, Q, stop, pol, lane, p, L);
+    if (R.consumed >= R.issued) return nullptr;
+    if (!wait_stage(R, fc, ctrl, lane)) stop = true;
+    return R.base + (size_t)(R.consumed % NS) * STAGE;
+}
+
+// Every lane is done with the stage: it may be refilled.
+__device__ __forceinline__ void release_stage(Ring& R) {
+    __syncwarp();
+    ++R.consumed;
+}
+
+// A tile of a ternary or 2-bit expert on the integer path, with NP passes of 4 rows.
+// MODE 0 (gate/up): B = the tokens' digit records, output h = silu(gate) * up in fp32
+// (hf, quantised later for the down pass); MODE 1 (down): B = the expert's h rows'
+// digit records, output fp32 rows of y_e (ypart).
+template <int MODE, int NP>
+__device__ __forceinline__ void unit_iq(const FfnArgs& p, const Layout& L, const CtaState& cs, const Unit& cur,
+                                        Queue& Q, Ring& R, bool& stop, bool ready, const IqBase& B, int G, int G8,
+                                        FusedCtl* fc, uint64_t pol, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int cnt = cs.slot[cur.slot].cnt, row0 = cs.slot[cur.slot].row0;
+    const int np = (cnt + 3) / 4;
+    IqView<NP> v;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+        const int ib = 4 * q + (g >> 1), it = 4 * q + t;
+        const int rb = row0 + (ib < cnt ? ib : 0), rt = row0 + (it < cnt ? it : 0);
+        const int tb = MODE == 0 ? row_token(p, cur.slot, row0, rb) : rb;   // record row: token, or h row
+        const int tk = MODE == 0 ? row_token(p, cur.slot, row0, rt) : rt;
+        v.bq[q] = (uint32_t)(((size_t)tb * G * 2 + (g & 1)) * 4 + t);
+        v.pq[q] = (uint32_t)((size_t)tk * G8);
+        v.orow[q] = it < cnt ? row0 + it : -1;
+    }
+    const int o4 = cs.slot[cur.slot].fmt == MOE_FMT_TERNARY ? 4 : 6;
+    const int K = MODE == 0 ? p.H : p.I, NC = (K / 64 + CG - 1) / CG, GK = K / 64;
+    const int sw = 128 * g + 16 * (g & 7) + 4 * t;       // this lane's word of group 0, swizzled
+    unsigned long long acc[NP];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) acc[q] = 0ull;
+    for (int c = 0; c < NC; ++c) {
+        const uint8_t* stg = next_stage(R, cs, cur, Q, stop, fc, p.ctrl, lane, pol, p, L);
+        if (!stg) break;
+        const int ng = min(CG, GK - c * CG);
+        if (ready && !stop) {
+            if (ng == CG) chunk_iq_full<NP>(stg, c, v, B, np, o4, sw, g, acc);
+            else chunk_gu_iq<NP, false>(stg, c, ng, v, B, np, o4, g, t, acc);
+        }
+        release_stage(R);
+    }
+    if (MODE == 0) {
+        // h = silu(gate) * up in fp32 for the down pass's quantisation; a value outside
+        // the fp16 range is reported (the range the layer is defined for)
+        bool range_ok = true;
+        if (ready && !stop) {
+            const int hcol = cur.tile * 8 + g;
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                if (q < np && v.orow[q] >= 0) {
+                    const float2 a = up2(acc[q]);
+                    const float hv = silu_f(a.x) * a.y;
+                    range_ok &= in_f16_range(hv);
+                    p.hf[(size_t)v.orow[q] * p.I + hcol] = hv;
+                }
+            }
+        }
+        if (!__all_sync(0xffffffffu, range_ok) && lane == 0)
+            report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 0x20);
+    } else if (ready && !stop) {
+        // rows 16 tile + g and 16 tile + g + 8 of y_e for token 4q + t, fp32
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            if (q < np && v.orow[q] >= 0) {
+                const float2 a = up2(acc[q]);
+                float* dst = p.ypart + (size_t)v.orow[q] * p.H + cur.tile * 16 + g;
+                dst[0] = a.x;
+                dst[8] = a.y;
+            }
+        }
+    }
+}
+
+// The down pass's integer operands of expert slot `cur.slot`: groups gq = tile,
+// tile + td, ... of every h row of the expert (its cnt tokens), each on its own 12-bit
+// grid (iq_group).  Groups past I (padding to whole chunks) get a zero pair.
+__device__ __forceinline__ void quantise_h_share(const FfnArgs& p, const CtaState& cs, const Unit& cur, int td,
+                                                 int lane) {
+    const int GI = p.I / 64, GI8 = 8 * ((GI + 7) / 8);
+    const int cnt = cs.slot[cur.slot].cnt, row0 = cs.slot[cur.slot].row0;
+    float2* pairs = reinterpret_cast<float2*>(p.hq + iq_pair_off(p.R16, p.I));
+    for (int gq = cur.tile; gq < GI8; gq += td) {
+        for (int r = 0; r < cnt; ++r) {
+            const int row = row0 + r;
+            if (gq >= GI) {
+                if (lane == 0) pairs[(size_t)row * GI8 + gq] = make_float2(0.f, 0.f);
+                continue;
+            }
+            const float2 hv = *reinterpret_cast<const float2*>(p.hf + (size_t)row * p.I + gq * 64 + 2 * lane);
+            iq_group(hv.x, hv.y, lane, p.hq + ((size_t)row * GI + gq) * 128, pairs + (size_t)row * GI8 + gq);
+        }
+    }
+}
+
+// A gate/up tile of a 3-bit expert (MODE 0: bf16 path, B = tokens) or a down tile of any
+// expert (MODE 1: exact fp16 path, B = h), with NP passes of 8 columns.
+template <int MODE, bool Q3, int NP>
+__device__ __forceinline__ void unit_bf(const FfnArgs& p, const Layout& L, const CtaState& cs, const Unit& cur,
+                                        Queue& Q, Ring& R, bool& stop, bool ready, const uint16_t* zq3,
+                                        int zplane_q3, int G8, FusedCtl* fc, uint64_t pol, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int cnt = cs.slot[cur.slot].cnt, row0 = cs.slot[cur.slot].row0, fmt = cs.slot[cur.slot].fmt;
+    const int np = (cnt + 7) / 8;
+    const int K = MODE == 0 ? p.H : p.I, NC = (K / 64 + CG - 1) / CG, GK = K / 64;
+    BfView<NP> v;
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+        const int ib = 8 * q + g;
+        const int rb = row0 + (ib < cnt ? ib : 0);
+        if (MODE == 0) {
+            const int tb = row_token(p, cur.slot, row0, rb);
+            v.b[q] = (uint32_t)((size_t)tb * p.H + 16 * t);
+            v.z[q] = (int)((size_t)tb * G8 + 2 * t);
+        } else {
+            v.b[q] = (uint32_t)((size_t)rb * p.I + 16 * t);
+            v.z[q] = 0;
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int col = 8 * q + 2 * t + cc;
+            v.orow[q][cc] = col < cnt ? row0 + col : -1;
+        }
+    }
+    uint32_t sub[5] = {0, 0, 0, 0, 0};
+    if (MODE == 1) {
+        const float o = fmt == MOE_FMT_TERNARY ? 1.f : (fmt == MOE_FMT_Q2 ? 1.5f : 3.5f);
+        sub[0] = f16x2_bits_of(512.f + o);
+        sub[1] = f16x2_bits_of(256.f + o);
+        sub[2] = f16x2_bits_of(64.f + o);
+        sub[3] = f16x2_bits_of(16.f + o);
+        sub[4] = f16x2_bits_of(4.f + o);
+    }
+    const uint16_t* bbase = MODE == 0 ? p.x : p.h;
+    const int cw_sw = 128 * g + 16 * (g & 7) + 4 * t;                 // swizzled word offsets of group 0
+    const int hw_sw = 64 * g + 8 * ((g & 7) >> 1) + 4 * (t >> 1);
+    float acc[NP][4];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+    for (int c = 0; c < NC; ++c) {
+        const uint8_t* stg = next_stage(R, cs, cur, Q, stop, fc, p.ctrl, lane, pol, p, L);
+        if (!stg) break;
+        const int ng = min(CG, GK - c * CG);
+        if (ready && !stop) {
+            if (ng == CG)
+                chunk_bf_full<MODE, Q3, NP>(stg, c, v, bbase, zq3, zplane_q3, np, sub, cw_sw, hw_sw, g, t, acc);
+            else chunk_bf<MODE, Q3, false, NP>(stg, c, ng, v, bbase, zq3, zplane_q3, np, sub, g, t, acc);
+        }
+        release_stage(R);
+    }
+    if (!ready || stop) return;
+    if (MODE == 0) {
+        bool range_ok = true;
+        const int hcol = cur.tile * 8 + g;
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc)
+                if (q < np && v.orow[q][cc] >= 0) {
+                    const float hv = silu_f(acc[q][cc]) * acc[q][2 + cc];
+                    range_ok &= in_f16_range(hv);
+                    p.h[(size_t)v.orow[q][cc] * p.I + hcol] = f32_to_f16_bits(hv);
+                }
+        if (!__all_sync(0xffffffffu, range_ok) && lane == 0)
+            report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 0x20);
+    } else {
+        // rows 16 tile + g and 16 tile + g + 8 of y_e for this lane's columns, fp32
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc)
+                if (q < np && v.orow[q][cc] >= 0) {
+                    float* dst = p.ypart + (size_t)v.orow[q][cc] * p.H + cur.tile * 16 + g;
+                    dst[0] = acc[q][cc];
+                    dst[8] = acc[q][2 + cc];
+                }
+    }
+}
+
+// y[t][16 tile + r] for every token t and r < 16: the routed rows weighted by their gates
+// in slot order, then the shared rows, summed in fp32 and stored as bf16.  Loads go out
+// four rows at a time.
+__device__ __forceinline__ void combine_slice(const FfnArgs& p, int tile, int lane) {
+    const int nrows = p.k + p.S;
+    for (int i = lane; i < p.T * 16; i += 32) {
+        const int tok = i >> 4, col = tile * 16 + (i & 15);
+        float y = 0.f;
+        for (int r0 = 0; r0 < nrows; r0 += 4) {
+            float v[4], gw[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = r0 + u;
+                int row = -1;
+                gw[u] = 1.f;
+                if (r < p.k) {
+                    row = __ldcg(p.inv_perm + (size_t)tok * p.k + r);
+                    gw[u] = __ldcg(p.topk_w + (size_t)tok * p.k + r);
+                } else if (r < nrows) {
+                    row = p.T * p.k + (r - p.k) * p.T + tok;
+                }
+                v[u] = row >= 0 ? __ldcg(p.ypart + (size_t)row * p.H + col) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = r0 + u;
+                if (r < p.k) y = fmaf(gw[u], v[u], y);
+                else if (r < nrows) y += v[u];
+            }
+        }
+        if (p.y_f32) reinterpret_cast<float*>(p.y)[(size_t)tok * p.H + col] = y;
+        else p.y[(size_t)tok * p.H + col] = f32_to_bf16_bits(y);
+    }
+}
+
+// ---- the kernel ---------------------------------------------------------------------
+__global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_constant__ FfnArgs p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t stall_bar;
+    __shared__ CtaState cs;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    FusedCtl* fc = p.fc;
+    Ctrl* ctrl = p.ctrl;
+    // No griddepcontrol.launch_dependents here: a following forward on the same
+    // workspace must not start before this launch has reset the counters it shares.
+
+    Ring R;
+    R.base = smem + (size_t)warp * NS * STAGE;
+    R.bar = reinterpret_cast<uint64_t*>(smem + (size_t)NW * NS * STAGE) + warp * NS;
+    R.issued = R.consumed = 0;
+    R.iw = 0;
+    R.ic = 0;
+    if (lane == 0)
+        for (int s = 0; s < NS; ++s) mbar_init(&R.bar[s], 1);
+    __shared__ int hdr_ok;
+    if (threadIdx.x == 0) {
+        mbar_init(&stall_bar, 1);                               // nothing ever arrives on it
+        cs.routed = 0;
+        // every CTA checks the packed buffer's header before it reads the expert table
+        const uint32_t* hd = reinterpret_cast<const uint32_t*>(p.packed);
+        hdr_ok = hd[0] == kMagic && hd[1] == kVersion && (int)hd[2] == p.H && (int)hd[3] == p.I &&
+                 (int)hd[4] == p.E && (int)hd[5] == p.S && hd[6] == 64u && hd[7] == (uint32_t)kInterleave;
+        if (!hdr_ok) {
+            report_error(ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
+            atomicExch(&fc->abort, 1u);
+        }
+    }
+    __syncthreads();
+    if (hdr_ok && warp == 0 && lane < p.S)                      // the shared experts' slots
+        fill_slot(cs.slot[lane], p, p.E + lane, p.T, p.T * p.k + lane * p.T);
+    fence_mbar_init();
+    __syncthreads();
+
+    // failure-path tests: one warp per CTA waits on a barrier nothing completes; the
+    // wait runs out and the launch takes its abort path
+    if (warp == 0 && ctrl->test_stall) {
+        int done = 0;
+        if (lane == 0) done = mbar_wait_bounded(&stall_bar, 0, ctrl->test_stall);
+        if (!__shfl_sync(0xffffffffu, done, 0) && lane == 0) {
+            report_error(ctrl, MOE_ERR_TIMEOUT, kDetTestStall | 0x20);
+            atomicExch(&fc->abort, 1u);
+        }
+        __syncwarp();
+    }
+
+    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
+    Layout L;
+    L.nops = p.T * G8;                            // one operand unit per (token, group)
+    L.tg = 2 * p.I / 16;
+    L.td = p.H / 16;
+    L.nch = (p.H / 64 + CG - 1) / CG;
+    L.nci = (p.I / 64 + CG - 1) / CG;
+    L.nsgu = p.S * L.tg;
+    L.pre = L.nops + L.nsgu;
+    L.nr = -1;
+    L.total = L.pre;
+    L.t_ok = true;
+    const OperandArgs oa{p.T, p.H, p.x, const_cast<float*>(p.zx), const_cast<uint8_t*>(p.iq), ctrl};
+    const int zplane_q3 = 3 * p.T * G8;          // hi -> lo plane of the Z tables (elements)
+    const uint16_t* zq3 = reinterpret_cast<const uint16_t*>(p.zx) + (size_t)2 * p.T * G8;   // format 2 plane
+    IqBase IB;                                    // the tokens' integer operands (gate/up)
+    IB.bq = reinterpret_cast<const uint4*>(p.iq);
+    IB.pq = reinterpret_cast<const float2*>(p.iq + iq_pair_off(p.T, p.H));
+    const int GI = p.I / 64, GI8 = 8 * ((GI + 7) / 8);
+    IqBase HB;                                    // the h rows' integer operands (down)
+    HB.bq = reinterpret_cast<const uint4*>(p.hq);
+    HB.pq = reinterpret_cast<const float2*>(p.hq + iq_pair_off(p.R16, p.I));
+    const uint64_t pol = l2_policy_evict_first();
+
+    auto grab = [&]() -> int {
+        int u = 0;
+        if (lane == 0) u = (int)atomicAdd(&fc->work, 1u);
+        return __shfl_sync(0xffffffffu, u, 0);
+    };
+    bool stop = !hdr_ok || ld_relaxed(&fc->abort) != 0;
+    bool ops_seen = false;
+    Unit cur = resolve(p, L, grab());
+    Queue Q;
+    Q.nxt.kind = U_PENDING;
+    Q.nxt.idx = -1;
+    int iters = 0;
+    while (true) {
+        if (cur.kind == U_NONE && cur.idx >= L.pre) {
+            if (L.nr < 0) {                       // routed range: the routing is needed
+                int tok = 0;
+                const int nr = read_routing(cs, p, lane, &tok);
+                if (nr < 0) stop = true;
+                L.nr = nr < 0 ? 0 : nr;
+                L.t_ok = tok != 0;
+                L.total = L.pre + L.nr * L.tg + p.S * L.td + L.nr * L.td;
+                cur = resolve(p, L, cur.idx);
+                if (Q.nxt.kind == U_NONE) Q.nxt = resolve(p, L, Q.nxt.idx);
+            }
+        }
+        if (cur.kind == U_NONE) break;            // the queue is empty
+        if (++iters > L.total + 2) {              // cannot happen with consistent counters
+            if (lane == 0) {
+                report_error(ctrl, MOE_ERR_DEVICE_CHECK, kDetLoopCap | 0x20);
+                atomicExch(&fc->abort, 1u);
+            }
+            break;
+        }
+        stop = stop || ld_relaxed(&fc->abort) != 0;
+        top_up(R, cs, cur, Q, stop, pol, lane, p, L);
+
+        if (cur.kind == U_OPS) {
+            // ---------------- operands of token tt, group Gi ---------------------------
+            if (!stop) {
+                const int tt = cur.tile / G8, Gi = cur.tile - tt * G8;
+                compute_z(oa, tt, Gi, lane);
+                compute_iq(oa, tt, Gi, lane);
+            }
+            signal_counter(&fc->ops_done, lane);
+        } else {
+            // ---------------- a gate/up or down tile ----------------------------------
+            const bool dn = cur.kind == U_DN;
+            const int cnt = cs.slot[cur.slot].cnt;
+            const bool q3 = cs.slot[cur.slot].fmt == MOE_FMT_Q3;
+            bool ready = !stop;
+            if (ready && !dn && !ops_seen) {
+                // the operands are written once per launch: one acquire per warp suffices
+                ready = wait_counter(&fc->ops_done, (uint32_t)L.nops, fc, ctrl, kDetWaitFull | 0x21, lane);
+                ops_seen = ready;
+            }
+            if (ready && dn) ready = wait_counter(&fc->gu_done[cur.slot], (uint32_t)L.tg, fc, ctrl, kDetWaitFull | 0x22, lane);
+            if (dn && !q3) {
+                // integer down pass: h of this expert on a 12-bit grid per 64-group, formed
+                // by the expert's first down tiles (a share each), waited for by all
+                const int shares = min(L.td, GI8);
+                if (cur.tile < shares) {
+                    if (ready) quantise_h_share(p, cs, cur, L.td, lane);
+                    signal_counter(&fc->hq_done[cur.slot], lane);
+                }
+                if (ready) ready = wait_counter(&fc->hq_done[cur.slot], (uint32_t)shares, fc, ctrl, kDetWaitFull | 0x23, lane);
+            }
+            if (!dn && !q3) {
+                if (cnt <= 4) unit_iq<0, 1>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
+                else if (cnt <= 8) unit_iq<0, 2>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
+                else unit_iq<0, 4>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
+            } else if (dn && !q3) {
+                if (cnt <= 4) unit_iq<1, 1>(p, L, cs, cur, Q, R, stop, ready, HB, GI, GI8, fc, pol, lane);
+                else if (cnt <= 8) unit_iq<1, 2>(p, L, cs, cur, Q, R, stop, ready, HB, GI, GI8, fc, pol, lane);
+                else unit_iq<1, 4>(p, L, cs, cur, Q, R, stop, ready, HB, GI, GI8, fc, pol, lane);
+            } else if (!dn) {
+                if (cnt <= 8) unit_bf<0, true, 1>(p, L, cs, cur, Q, R, stop, ready, zq3, zplane_q3, G8, fc, pol, lane);
+                else unit_bf<0, true, 2>(p, L, cs, cur, Q, R, stop, ready, zq3, zplane_q3, G8, fc, pol, lane);
+            } else {
+                if (cnt <= 8) unit_bf<1, true, 1>(p, L, cs, cur, Q, R, stop, ready, zq3, 0, G8, fc, pol, lane);
+                else unit_bf<1, true, 2>(p, L, cs, cur, Q, R, stop, ready, zq3, 0, G8, fc, pol, lane);
+            }
+            stop = stop || !ready;
+            if (!dn) {
+                signal_counter(&fc->gu_done[cur.slot], lane);
+            } else {
+                const uint32_t n_slots = (uint32_t)(L.nr + p.S);
+                const uint32_t old = signal_counter(&p.dn_done[cur.tile], lane);
+                if (old == n_slots - 1 && !stop && L.t_ok) {
+                    // the last expert of this 16-row slice: combine it (slot order, fixed)
+                    (void)ld_acquire(&p.dn_done[cur.tile]);
+                    combine_slice(p, cur.tile, lane);
+                }
+            }
+        }
+        // next unit: the issue cursor moves from "next" to "current"
+        if (R.iw == 1) R.iw = 0;
+        else R.ic = 0;
+        take_next(Q, p, L, lane);
+        cur = Q.nxt;
+        if (cur.kind == U_NONE && cur.idx >= L.pre && L.nr >= 0) cur = resolve(p, L, cur.idx);
+        Q.nxt.kind = U_PENDING;
+    }
+
+    // copies still in flight (only after an abort): wait for them, bounded
+    if (lane == 0)
+        for (int qd = R.consumed; qd < R.issued; ++qd)
+            if (!mbar_wait_bounded(&R.bar[qd % NS], (uint32_t)(qd / NS) & 1, kWaitLimit)) {
+                report_error(ctrl, MOE_ERR_TIMEOUT, kDetDrain | 0x20);
+                break;
+            }
+    __syncwarp();
+    // the last warp of the launch resets the counters for the next one
+    const uint32_t n_warps = gridDim.x * NW;
+    if (signal_counter(&fc->warps_done, lane) == n_warps - 1) {
+        (void)ld_acquire(&fc->warps_done);
+        for (int i = lane; i < kMaxSlots; i += 32) {
+            fc->gu_done[i] = 0;
+            fc->hq_done[i] = 0;
+        }
+        for (int i = lane; i < p.H / 16; i += 32) p.dn_done[i] = 0;
+        __syncwarp();
+        if (lane == 0) {
+            fc->work = 0;
+            fc->ops_done = 0;
+            fc->abort = 0;
+            __threadfence();
+            fc->warps_done = 0;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_fused(const FfnArgs& a, cudaStream_t s) {
+    if (a.T < 1 || a.T > kFusedMaxT || a.E + a.S > kMaxSlots) return cudaErrorInvalidConfiguration;
+    const cudaError_t err = set_smem_limit(ffn_fused_kernel, kFusedSmem);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(ffn_fused_kernel, dim3(a.num_ctas), dim3(NW * 32), kFusedSmem, s, a);
+}
+
+}  // namespace moe

@@ -20,7 +20,10 @@ struct RouteArgs {
     int32_t* hist;      // ws [ceil(T/kChunk)][E]
     int32_t* active;    // ws [E+S]
     float* zx;          // ws fp16 planes [2][3][T][G8] of -Z/16, hi and lo (see route.cu)
-    uint8_t* iq;        // ws integer gate/up operands for T <= kIqMaxT (see route.cu), else null
+    uint8_t* iq;        // ws integer operands of the tokens (T <= kFusedMaxT), else null
+    int ops;            // form the decode operands (Z tables, integer operands) here
+    const int32_t* fixed_ids;   // moe_route_fixed: the caller's expert ids [T][k] (else null)
+    const float* fixed_w;       // moe_route_fixed: the caller's gates [T][k]
     Ctrl* ctrl;
     moe_routing r;
 };
@@ -36,7 +39,7 @@ struct FfnArgs {
     const float* topk_w;
     const int32_t* active;   // ws
     const float* zx;         // ws fp16 planes [2][3][T][G8] of -Z/16, hi and lo
-    const uint8_t* iq;       // ws integer gate/up operands (T <= kIqMaxT), else null
+    const uint8_t* iq;       // ws integer operands of the tokens (T <= kFusedMaxT), else null
     int iq_on;               // gate/up of ternary / 2-bit experts on the integer path
     Ctrl* ctrl;
     uint16_t* h;             // ws fp16 [T*(k+S)][I]
@@ -44,34 +47,51 @@ struct FfnArgs {
     float* gpart;            // ws f32 [nkp_gu][T*(k+S)][2I] (aliases ypart; decode, nkp_gu > 1)
     int nkp_gu, nkp_dn;      // K parts of the decode gate/up and down passes (1 on the prefill path)
     uint32_t* tile_ctr;      // ws [H/16]
-    uint16_t* y;             // bf16 [T][H]
+    uint16_t* y;             // bf16 [T][H], or fp32 [T][H] when y_f32
+    int y_f32;               // the combine stores fp32 (MOE_OUT_F32)
     int num_ctas;
+    FusedCtl* fc;            // ws: counters of the fused decode kernel
+    uint32_t* dn_done;       // ws [H/16]: down tiles finished per 16-row slice of y (fused kernel)
+    float* hf;               // ws fp32 [R16][I]: h of ternary / 2-bit experts (fused kernel)
+    uint8_t* hq;             // ws integer operands of those h rows (iq_size(R16, I))
+    int R16;                 // rows those two regions hold: min(T, kFusedMaxT) (k + S)
 };
 
 // Workspace layout for T tokens (api.cu).  The control block, tile counters and the
 // active-expert list sit at fixed offsets (independent of T).
 struct Ws {
-    size_t ctrl, tile_ctr, active, logits, hist, zx, iq, h, ypart, total;
+    size_t ctrl, tile_ctr, active, logits, hist, zx, iq, hf, hq, h, ypart, total;
 };
 
-// Few-token gate/up on the integer tensor path (decode_ffn.cu, route.cu): up to
-// kIqMaxT tokens, each as two signed-byte digit columns of one n8 MMA tile.  The
-// region holds, per token t and 64-group g (G groups, G8 = G padded to whole chunks):
-//   digit records  [T][G][2 digits][4 lanes] x 16 bytes          (offset 0)
-//   factors p      fp32 [T][G8]                                   (iq_pq_off)
-//   offset planes  fp16 [2 hi/lo][2 formats][T][G8] of -o sum x / 16  (iq_zq_off)
-constexpr int kIqMaxT = 4;
-__host__ __device__ inline size_t iq_pq_off(int64_t T, int64_t H) { return (size_t)T * (H / 64) * 128; }
-__host__ __device__ inline size_t iq_zq_off(int64_t T, int64_t H) {
-    return iq_pq_off(T, H) + (size_t)4 * T * (8 * ((H / 64 + 7) / 8));
+// Integer-path operands of the fused decode kernel (operands.cuh, decode_fused.cu): per
+// row (a token, or an h row of the down pass) and 64-group g (G groups, G8 = G padded to
+// whole chunks), a 128-byte digit record [2 digits][4 lanes] x 16 bytes of the row's
+// values on a 12-bit grid, then per (row, group) the pair {p = 2^-e / 4 (fp32),
+// sum of q (int32)}:
+//   digit records  [R][G] x 128 bytes         (offset 0)
+//   pairs          [R][G8] x 8 bytes          (iq_pair_off)
+// The fused decode kernel (decode_fused.cu) serves up to kFusedMaxT tokens.
+constexpr int kFusedMaxT = 16;
+__host__ __device__ inline size_t iq_pair_off(int64_t R, int64_t K) { return (size_t)R * (K / 64) * 128; }
+__host__ __device__ inline size_t iq_size(int64_t R, int64_t K) {
+    return iq_pair_off(R, K) + (size_t)8 * R * (8 * ((K / 64 + 7) / 8));
 }
-// Reserved for min(T, kIqMaxT) tokens at every T >= 1, so that the workspace size
-// never shrinks as T grows; used only when T <= kIqMaxT.
+// Token operands, reserved for min(T, kFusedMaxT) tokens at every T >= 1 so that the
+// workspace size never shrinks as T grows; used only when T <= kFusedMaxT.
 inline size_t iq_bytes(int64_t T, int64_t H) {
-    const int64_t t = T < kIqMaxT ? T : kIqMaxT;
-    return t >= 1 ? iq_zq_off(t, H) + (size_t)2 * 2 * 2 * t * (8 * ((H / 64 + 7) / 8)) : 0;
+    const int64_t t = T < kFusedMaxT ? T : kFusedMaxT;
+    return t >= 1 ? iq_size(t, H) : 0;
 }
 Ws ws_layout(const moe_shape* s, int64_t T);
+
+// Host-side argument checks of moe_route and moe_forward (api.cu); they enqueue nothing,
+// so an entry point can run all of them before its first launch.
+bool shape_ok(const moe_shape* s);
+moe_status check_route_args(const moe_shape* shape, int32_t T, const uint16_t* d_x, const float* d_router_w,
+                            const moe_routing* out, const void* d_ws, size_t ws_bytes);
+moe_status check_forward_args(const moe_shape* shape, int32_t T, const void* d_packed, const uint16_t* d_x,
+                              const moe_routing* r, const uint16_t* d_y, moe_path path, const void* d_ws,
+                              size_t ws_bytes);
 
 // K parts of the decode-path expert passes for T tokens.  With few tokens only a few
 // experts are active and their 32-row blocks are fewer than the warps of the GPU, so
@@ -97,14 +117,36 @@ inline void decode_kparts(const moe_shape* s, int64_t T, int* nkp_gu, int* nkp_d
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+// the routing of caller-given expert ids and gates (a.fixed_ids): histogram, scan,
+// permutation, active list and (if a.ops) the decode operands
+cudaError_t launch_route_fixed(const RouteArgs& a, cudaStream_t s);
 // decode-path expert kernels + combine; ev_gateup / ev_down (may be null) are recorded
 // after the gate/up and the down kernel
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down);
+// the whole decode forward (operands, gate/up, down, combine) as one persistent kernel,
+// for 1 <= T <= kFusedMaxT
+cudaError_t launch_ffn_fused(const FfnArgs& a, cudaStream_t s);
 // prefill-path expert kernels (tcgen05) + combine; x16: fp16 scratch of T*(k+S)*H
 cudaError_t launch_ffn_prefill(const FfnArgs& a, uint16_t* x16, cudaStream_t s, cudaEvent_t ev_gateup,
                                cudaEvent_t ev_down);
+// expert-parallel row kernels (ep.cu): dst[i] = src[index[i] / div] (bf16 rows); y[t] =
+// sum_j g[t][j] rows[inv_perm[t k + j]] + shared[t] (fp32 rows, bf16 y); bad indices are
+// reported in ctrl
+cudaError_t launch_gather_rows(int n, int H, const uint16_t* src, const int32_t* index, int div, int n_src,
+                               uint16_t* dst, Ctrl* ctrl, cudaStream_t s);
+cudaError_t launch_combine_pairs(int T, int k, int H, int n_rows, const float* rows, const int32_t* inv_perm,
+                                 const float* gates, const float* shared, uint16_t* y, Ctrl* ctrl, cudaStream_t s);
 // gate-weighted unpermute-combine of the partial rows into y
 cudaError_t launch_combine(const FfnArgs& a, cudaStream_t s);
+
+// Raises a kernel's dynamic shared memory limit on the current device.  The attribute
+// belongs to the device's context, so it is set before every launch rather than once
+// per process: a host-side call that enqueues nothing, cheap, and correct whichever
+// device is current and from any number of host threads.
+template <typename... KArgs>
+inline cudaError_t set_smem_limit(void (*kern)(KArgs...), size_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
 
 // Launches kern<<<grid, block, smem, s>>>(args...) with programmatic stream
 // serialization: the kernel may begin while its predecessor in s is still running and

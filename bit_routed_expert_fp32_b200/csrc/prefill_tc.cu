@@ -194,7 +194,8 @@ __device__ inline const PackedEntry* entry(const uint8_t* packed, int e) {
 struct TcSched {
     int ok, n_active, n_tiles, abort_flag;
     uint32_t tmem;
-    int pad[3];
+    uint32_t stall;  // failure-path tests: cycles of the MMA issuer's wait on stall_bar (0 = off)
+    int pad[2];
     int e[260];
     int fmt[260];
     int cnt[260];
@@ -243,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
     extern __shared__ uint8_t smem_raw[];
     __shared__ TcSched S;
     __shared__ __align__(8) uint64_t full_a[NSTG], full_b[NSTG], empty_[NSTG], acc_full[2], acc_empty[2], mma_done,
-        pk_full[kDqWarps][NP];
+        pk_full[kDqWarps][NP], stall_bar;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = MODE == 0 ? p.H : p.I;
@@ -258,12 +259,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
     griddep_wait();
     if (threadIdx.x == 0) {
         const uint32_t* hd = reinterpret_cast<const uint32_t*>(p.packed);
-        const bool ok = hd[0] == kMagic && hd[1] == kVersion && (int)hd[2] == p.H && (int)hd[3] == p.I &&
-                        (int)hd[4] == p.E && (int)hd[5] == p.S && hd[6] == 64u && hd[7] == (uint32_t)kInterleave;
-        S.ok = ok;
+        const bool hdr_ok = hd[0] == kMagic && hd[1] == kVersion && (int)hd[2] == p.H && (int)hd[3] == p.I &&
+                            (int)hd[4] == p.E && (int)hd[5] == p.S && hd[6] == 64u &&
+                            hd[7] == (uint32_t)kInterleave;
+        // the schedule in the workspace must be the one routed for these T tokens
+        const bool t_ok = p.ctrl->routed_T == p.T;
+        S.ok = hdr_ok && t_ok;
         S.abort_flag = 0;
-        if (!ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
+        if (!hdr_ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetHeader);
+        else if (!t_ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRoutedT | 0x10 | MODE);
         S.n_active = p.ctrl->n_active;
+        S.stall = p.ctrl->test_stall;
     }
     __syncthreads();
     if (!S.ok) return;
@@ -301,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
             mbar_init(&acc_empty[i], 4 * 32);
         }
         mbar_init(&mma_done, 1);
+        mbar_init(&stall_bar, 1);                       // nothing ever arrives on it
         fence_mbar_init();
     }
     if (warp == kMmaWarp) tmem_alloc(&S.tmem, 512);
@@ -505,6 +512,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         int slot = 0, tc = 0;
         uint32_t phase = 0;
         bool ok = true;
+        if (S.stall) {
+            // failure-path tests: a bounded wait on a barrier that nothing completes; it
+            // runs out and the CTA takes the give-up path below (as for any wait)
+            bool done = false;
+            if (lane == 0) done = mbar_wait_bounded(&stall_bar, 0, S.stall);
+            if (!__shfl_sync(0xffffffffu, done, 0)) {
+                if (lane == 0) {
+                    st_volatile(S.abort_flag, 1);
+                    report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetTestStall | 0x10 | MODE);
+                }
+                ok = false;
+            }
+            __syncwarp();
+        }
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
             const int buf = tc & 1;
@@ -574,12 +595,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
                     // shared memory into one 16-byte store per lane
                     const bool gate_lane = (lane & 15) < 8;
                     const int lc = ((lane >> 4) << 3) | (lane & 7);    // h column within the warp
+                    bool range_ok = true;
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const float a = __uint_as_float(v[u]);
                         const float b = __shfl_down_sync(0xffffffffu, a, 8);
-                        if (gate_lane) stg[u * 16 + lc] = f32_to_f16_bits(silu_fast(a) * b);
+                        const float hv = silu_fast(a) * b;
+                        range_ok &= !gate_lane || c0 + u >= ti.N || in_f16_range(hv);
+                        if (gate_lane) stg[u * 16 + lc] = f32_to_f16_bits(hv);
                     }
+                    // h outside the fp16 range: reported, not carried on (see moe_forward)
+                    if (!__all_sync(0xffffffffu, range_ok) && lane == 0)
+                        report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 0x10);
                     __syncwarp();
                     const int u = lane >> 1, half = lane & 1;
                     if (c0 + u < ti.N)
@@ -608,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
 // One block per row, threads over 8-element column chunks.
 __global__ void __launch_bounds__(256) gather_x16_kernel(FfnArgs p, uint16_t* x16) {
     griddep_wait();                     // perm comes from the router
+    if (p.ctrl->routed_T != p.T) return;   // another T was routed: perm may point past x (reported by the GEMM)
     const int r = blockIdx.x;
     const int tk = p.T * p.k;
     const int tok = r < tk ? __ldg(p.perm + r) / p.k : (r - tk) % p.T;
@@ -617,11 +645,15 @@ __global__ void __launch_bounds__(256) gather_x16_kernel(FfnArgs p, uint16_t* x1
         const uint4 v = __ldg(src + c);
         const uint32_t in[4] = {v.x, v.y, v.z, v.w};
         uint32_t out[4];
+        bool ok = true;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const float lo = __uint_as_float(in[u] << 16), hi = __uint_as_float(in[u] & 0xFFFF0000u);
+            ok &= in_f16_range(lo) && in_f16_range(hi);
             out[u] = (uint32_t)f32_to_f16_bits(lo) | ((uint32_t)f32_to_f16_bits(hi) << 16);
         }
+        // a token outside the fp16 range is reported, not carried on (see moe_forward)
+        if (!ok) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 1);
         dst[c] = make_uint4(out[0], out[1], out[2], out[3]);
     }
 }
@@ -661,13 +693,8 @@ bool make_maps(BMaps* b, const void* base, long long rows, int K) {
 
 template <int MODE>
 cudaError_t launch_tc(const FfnArgs& a, const BMaps& maps, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t err =
-            cudaFuncSetAttribute(tc_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
-        if (err != cudaSuccess) return err;
-        attr = true;
-    }
+    const cudaError_t err = set_smem_limit(tc_gemm_kernel<MODE>, kTcSmem);
+    if (err != cudaSuccess) return err;
     return launch_pdl(tc_gemm_kernel<MODE>, dim3(a.num_ctas), dim3(kThreads), kTcSmem, s, a, maps);
 }
 

@@ -16,12 +16,19 @@
 // Ordering inside an expert is token ascending, made deterministic by processing the
 // flattened (token, slot) pairs in order with warp match/ballot ranks.
 #include "kernels.h"
+#include "operands.cuh"
 
 namespace moe {
 namespace {
 
 __device__ inline float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ inline float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ inline double warp_sum_f64(double v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
 
 __device__ inline float warp_sum(float v) {
 #pragma unroll
@@ -109,13 +116,17 @@ __device__ void warp_scan_counts(const int* s_cnt, int* s_off, int E, int lane) 
 
 // Ranks the flattened pairs [0, n) (ids in s_ids) into positions starting at
 // s_run[e]; writes perm / inv_perm.  One warp; pair order = (token, slot) order.
+// An id outside [0, E) (only possible with caller-given routing, which reports it) takes
+// no position; its pair's inv_perm entry is set to 0 so that readers stay in bounds.
 __device__ void warp_scatter(const int32_t* ids, int pair0, int n, int* s_run, int32_t* perm, int32_t* inv_perm,
-                             int lane) {
+                             int lane, int E) {
     const unsigned lt = (1u << lane) - 1u;
     for (int base = 0; base < n; base += 32) {
         int i = base + lane;
-        bool valid = i < n;
-        int e = valid ? ids[i] : -1 - lane;
+        int e = i < n ? ids[i] : -1;
+        if (i < n && (e < 0 || e >= E)) inv_perm[pair0 + i] = 0;
+        bool valid = i < n && e >= 0 && e < E;
+        if (!valid) e = -1 - lane;
         unsigned mask = __match_any_sync(0xffffffffu, e);
         int rank = __popc(mask & lt);
         int first = valid ? s_run[e] : 0;
@@ -147,100 +158,6 @@ __device__ void warp_active(const int* s_cnt, int E, int S, int32_t* active, Ctr
     }
 }
 
-// ---------------------------------------------------------------- Z tables
-// The gate/up expert kernel feeds the MMA with "base + c" values straight out of the
-// code words (no per-pair subtraction), so each 64-wide group's MMA yields
-// sum (base + c) x, and the kernel subtracts Z once per 8-group chunk with a small MMA
-// of the scales against Z.  For token t and group G (elements x_e, e = 0..63):
-//   Bx = sum_e lo_base(e) x_e,  Hx = sum_e hi_base(e) x_e,  Sx = sum_e x_e,
-// with lo_base / hi_base the magic bases the expert kernel uses for the pair that
-// holds element e (pair p = (e % 16) / 2):  lo 128,32,8,128,32,8,128,32 and
-// hi 512,256,128,64,32,16,8,8.  Then for code offset o:
-//   Z_ternary = Bx + Sx,  Z_q2 = Bx + 1.5 Sx,  Z_q3 = Bx + Hx + 3.5 Sx.
-// Stored as -Z / 16 split exactly into two fp16 halves (hi = the rounding, lo = the
-// rounding of what is left), in planes z16[hl][format][T][G8] with the group count
-// padded to whole chunks (G8 = 8 ceil(G / 8); the padding is zero): the B fragments of
-// the correction MMA.  The 1/16 keeps Z inside the fp16 range; the kernel scales the
-// A side (the fp16 scales) by 16, exactly.
-__device__ void compute_z(const RouteArgs& p, int t, int Gi, int lane) {
-    constexpr float kLo[8] = {128.f, 32.f, 8.f, 128.f, 32.f, 8.f, 128.f, 32.f};
-    constexpr float kHi[8] = {512.f, 256.f, 128.f, 64.f, 32.f, 16.f, 8.f, 8.f};
-    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
-    float z[3] = {0.f, 0.f, 0.f};
-    if (Gi < G) {
-        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * p.H + Gi * 64) + lane);
-        const float x0 = bf16lo(v), x1 = bf16hi(v);
-        const float bl = kLo[lane & 7], bh = kHi[lane & 7];
-        float bx = fmaf(bl, x0, bl * x1), hx = fmaf(bh, x0, bh * x1), sx = x0 + x1;
-        bx = warp_sum(bx);
-        hx = warp_sum(hx);
-        sx = warp_sum(sx);
-        z[0] = bx + sx;
-        z[1] = fmaf(1.5f, sx, bx);
-        z[2] = fmaf(3.5f, sx, bx + hx);
-    }
-    if (lane < 3) {
-        const float zs = -0.0625f * (lane == 0 ? z[0] : (lane == 1 ? z[1] : z[2]));
-        const __half hi = __float2half_rn(zs);
-        const __half lo = __float2half_rn(zs - __half2float(hi));
-        uint16_t* z16 = reinterpret_cast<uint16_t*>(p.zx);
-        const size_t i = ((size_t)lane * p.T + t) * G8 + Gi, plane = (size_t)3 * p.T * G8;
-        z16[i] = __half_as_ushort(hi);
-        z16[plane + i] = __half_as_ushort(lo);
-    }
-}
-
-// Integer operands of the few-token gate/up pass (T <= kIqMaxT; ternary and 2-bit
-// experts, decode_ffn.cu).  Per token t and 64-group Gi: e = 11 - floor(log2 max |x|)
-// puts the group on a 12-bit grid, q = rint(x 2^e) (exact for every x above 2^-4 of
-// the group maximum).  The kernel masks each code word into four byte classes c (two
-// per MMA): classes 0 and 2 hold the code, 1 and 3 four times the code, so B = 4q for
-// even c and q for odd c makes every product 4 c q.  Element k of the group sits in
-// lane k / 16 of the record, class c = (k mod 8) / 2, byte 2 (k mod 2) + (k mod 16) / 8
-// (the inverse of the code word's element order); B is split into signed bytes
-// lo + 256 hi, one record per digit.  p = 2^-e / 4 turns the integer sums into x
-// units; the offset planes hold -o sum(q 2^-e) / 16 as fp16 hi + lo for o = 1 and 1.5.
-__device__ void compute_iq(const RouteArgs& p, int t, int Gi, int lane) {
-    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
-    float* pq = reinterpret_cast<float*>(p.iq + iq_pq_off(p.T, p.H));
-    uint16_t* zq = reinterpret_cast<uint16_t*>(p.iq + iq_zq_off(p.T, p.H));
-    const size_t zplane = (size_t)2 * p.T * G8;
-    if (Gi >= G) {                                      // padding of the last chunk
-        if (lane == 0) pq[(size_t)t * G8 + Gi] = 0.f;
-        if (lane < 4) zq[(lane >> 1) * zplane + ((size_t)(lane & 1) * p.T + t) * G8 + Gi] = 0;
-        return;
-    }
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * p.H + Gi * 64) + lane);
-    const float x[2] = {bf16lo(v), bf16hi(v)};
-    const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fabsf(x[0]), fabsf(x[1])))));
-    const int e = m > 0.f ? 11 - ilogbf(m) : 0;
-    uint8_t* rec = p.iq + ((size_t)t * G + Gi) * 128;
-    int qsum = 0;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int q = (int)rintf(ldexpf(x[h], e));
-        qsum += q;
-        const int k = 2 * lane + h, lt = k >> 4, off = k & 15;
-        const int c = (off & 7) >> 1, b = 2 * (off & 1) + (off >> 3);
-        const int bv = (c & 1) ? q : 4 * q;
-        const int lo = (int)(int8_t)(uint8_t)(bv & 0xFF), hi = (bv - lo) >> 8;
-        const int pos = 16 * lt + 4 * c + b;
-        rec[pos] = (uint8_t)lo;
-        rec[64 + pos] = (uint8_t)hi;
-    }
-    qsum = (int)__reduce_add_sync(0xffffffffu, (uint32_t)qsum);
-    if (lane == 0) pq[(size_t)t * G8 + Gi] = ldexpf(0.25f, -e);
-    if (lane < 2) {
-        const float sx = ldexpf((float)qsum, -e);
-        const float zs = -0.0625f * (lane == 0 ? sx : 1.5f * sx);
-        const __half hi = __float2half_rn(zs);
-        const __half lo = __float2half_rn(zs - __half2float(hi));
-        const size_t i = ((size_t)lane * p.T + t) * G8 + Gi;
-        zq[i] = __half_as_ushort(hi);
-        zq[zplane + i] = __half_as_ushort(lo);
-    }
-}
-
 __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {          // no expert pass of this workspace runs now
         p.ctrl->work[0] = 0;
@@ -248,9 +165,10 @@ __global__ void __launch_bounds__(256) route_xz_kernel(RouteArgs p) {
     }
     const int G8 = 8 * ((p.H / 64 + 7) / 8);
     const int warp = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (warp < p.T * G8) {
-        compute_z(p, warp / G8, warp % G8, lane);
-        if (p.iq) compute_iq(p, warp / G8, warp % G8, lane);
+    if (p.ops && warp < p.T * G8) {
+        const OperandArgs o{p.T, p.H, p.x, p.zx, p.iq, p.ctrl};
+        compute_z(o, warp / G8, warp % G8, lane);
+        if (p.iq) compute_iq(o, warp / G8, warp % G8, lane);
     }
 }
 
@@ -321,7 +239,10 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
         p.ctrl->work[0] = 0;
         p.ctrl->work[1] = 0;
     }
-    __shared__ float s_part[8][kSmallT];
+    // fp64 accumulation: each product of an fp32 weight and a bf16 token is exact in
+    // fp64, so the logit is the exact sum rounded once to fp32 (tokens with large
+    // outliers make fp32 partial sums lose the bits that separate close logits)
+    __shared__ double s_part[8][kSmallT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x;
     const int n4 = p.H / 4;                                        // float4 per row
@@ -334,7 +255,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
             w[u] = i < n4 ? __ldg(w4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         for (int tb = 0; tb < p.T; tb += 8) {
-            float acc[8];
+            double acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 acc[j] = 0.f;
@@ -345,33 +266,34 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
                     const int i = i0 + threadIdx.x + 256 * u;
                     if (i < n4) {
                         const uint2 xv = __ldg(xr + i);
-                        acc[j] = fmaf(w[u].x, bf16lo(xv.x), acc[j]);
-                        acc[j] = fmaf(w[u].y, bf16hi(xv.x), acc[j]);
-                        acc[j] = fmaf(w[u].z, bf16lo(xv.y), acc[j]);
-                        acc[j] = fmaf(w[u].w, bf16hi(xv.y), acc[j]);
+                        acc[j] = fma((double)w[u].x, (double)bf16lo(xv.x), acc[j]);
+                        acc[j] = fma((double)w[u].y, (double)bf16hi(xv.x), acc[j]);
+                        acc[j] = fma((double)w[u].z, (double)bf16lo(xv.y), acc[j]);
+                        acc[j] = fma((double)w[u].w, (double)bf16hi(xv.y), acc[j]);
                     }
                 }
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 if (tb + j >= p.T) break;
-                const float v = warp_sum(acc[j]);
-                if (lane == 0) s_part[warp][tb + j] = (i0 == 0 ? 0.f : s_part[warp][tb + j]) + v;
+                const double v = warp_sum_f64(acc[j]);
+                if (lane == 0) s_part[warp][tb + j] = (i0 == 0 ? 0.0 : s_part[warp][tb + j]) + v;
             }
         }
     }
     __syncthreads();
     for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
-        float v = 0.f;
+        double v = 0.0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) v += s_part[w][t];
-        p.logits[(size_t)t * p.E + e] = v + (p.bias ? p.bias[e] : 0.f);
+        p.logits[(size_t)t * p.E + e] = (float)(v + (p.bias ? (double)p.bias[e] : 0.0));
     }
-    {
+    if (p.ops) {
         const int G8 = 8 * ((p.H / 64 + 7) / 8);
         for (int pr = blockIdx.x * 8 + warp; pr < p.T * G8; pr += gridDim.x * 8) {
-            compute_z(p, pr / G8, pr % G8, lane);
-            if (p.iq) compute_iq(p, pr / G8, pr % G8, lane);
+            const OperandArgs o{p.T, p.H, p.x, p.zx, p.iq, p.ctrl};
+            compute_z(o, pr / G8, pr % G8, lane);
+            if (p.iq) compute_iq(o, pr / G8, pr % G8, lane);
         }
     }
     __shared__ int s_last;
@@ -410,7 +332,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
         if (lane == 0) p.r.offsets[p.E] = s_off[p.E];
         __syncwarp();
         // s_off doubles as the running position per expert
-        warp_scatter(s_ids, 0, p.T * p.k, s_off, p.r.perm, p.r.inv_perm, lane);
+        warp_scatter(s_ids, 0, p.T * p.k, s_off, p.r.perm, p.r.inv_perm, lane, p.E);
         if (lane == 0) p.ctrl->route_ticket = 0;
     } else if (warp == 1) {
         warp_active(s_cnt, p.E, p.S, p.active, p.ctrl, p.T, lane);
@@ -444,7 +366,7 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = blockIdx.x * RBM, e0 = blockIdx.y * RBN;
     const int wm = warp >> 1, wn = warp & 1;            // warp tile: tokens 32wm.., experts 32wn..
-    float acc[2][4][4];
+    double acc[2][4][4];        // K-tile partials added in fp64 (see the decode router)
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -544,7 +466,7 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][b][c] += part[a][b][c];
+                for (int c = 0; c < 4; ++c) acc[a][b][c] += (double)part[a][b][c];
         if (kt + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
@@ -560,7 +482,8 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
                 for (int c = 0; c < 2; ++c) {
                     const int e = e0 + 32 * wn + 8 * nt + 2 * t4 + c;
                     if (t < p.T && e < p.E)
-                        p.logits[(size_t)t * p.E + e] = acc[mt][nt][2 * h + c] + (p.bias ? p.bias[e] : 0.f);
+                        p.logits[(size_t)t * p.E + e] =
+                            (float)(acc[mt][nt][2 * h + c] + (p.bias ? (double)p.bias[e] : 0.0));
                 }
             }
 }
@@ -574,6 +497,19 @@ __global__ void __launch_bounds__(256) route_topk_kernel(RouteArgs p) {
     __syncthreads();
     const int tend = min(p.T, (c + 1) * kChunk);
     for (int t = c * kChunk + warp; t < tend; t += 8) {
+        if (p.fixed_ids) {
+            // caller-given routing: copied; an id outside [0, E) is reported and counted
+            // nowhere (its pair is left out of the permutation's expert ranges)
+            if (lane < p.k) {
+                const size_t i = (size_t)t * p.k + lane;
+                const int id = __ldg(p.fixed_ids + i);
+                p.r.topk_ids[i] = id;
+                p.r.topk_w[i] = __ldg(p.fixed_w + i);
+                if (id >= 0 && id < p.E) atomicAdd(&s_cnt[id], 1);
+                else report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 2);
+            }
+            continue;
+        }
         float v[8];
         load_logits_row(p.logits + (size_t)t * p.E, p.E, lane, v);
         warp_topk(v, p.k, lane, p.r.topk_ids + (size_t)t * p.k, p.r.topk_w + (size_t)t * p.k);
@@ -623,10 +559,22 @@ __global__ void __launch_bounds__(32) route_scatter_kernel(RouteArgs p) {
     for (int e = lane; e < p.E; e += 32) s_run[e] = p.hist[(size_t)c * p.E + e];
     __syncwarp();
     const int t0 = c * kChunk, t1 = min(p.T, t0 + kChunk);
-    warp_scatter(p.r.topk_ids + (size_t)t0 * p.k, t0 * p.k, (t1 - t0) * p.k, s_run, p.r.perm, p.r.inv_perm, lane);
+    warp_scatter(p.r.topk_ids + (size_t)t0 * p.k, t0 * p.k, (t1 - t0) * p.k, s_run, p.r.perm, p.r.inv_perm, lane,
+                 p.E);
 }
 
 }  // namespace
+
+cudaError_t launch_route_fixed(const RouteArgs& a, cudaStream_t s) {
+    if (a.ops) {
+        const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);
+        route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
+    }
+    const int nchunks = (a.T + kChunk - 1) / kChunk;
+    route_topk_kernel<<<nchunks, 256, 0, s>>>(a);
+    route_scatter_kernel<<<nchunks, 32, 0, s>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     if (a.T <= kSmallT) {
@@ -635,13 +583,8 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     }
     const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);
     route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t err = cudaFuncSetAttribute(route_logits_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kRouteMmaSmem);
-        if (err != cudaSuccess) return err;
-        attr = true;
-    }
+    cudaError_t err = set_smem_limit(route_logits_mma_kernel, kRouteMmaSmem);
+    if (err != cudaSuccess) return err;
     dim3 g1((a.T + RBM - 1) / RBM, (a.E + RBN - 1) / RBN);
     route_logits_mma_kernel<<<g1, 256, kRouteMmaSmem, s>>>(a);
     const int nchunks = (a.T + kChunk - 1) / kChunk;

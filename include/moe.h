@@ -59,6 +59,11 @@ typedef enum { MOE_FMT_TERNARY = 0, MOE_FMT_Q2 = 1, MOE_FMT_Q3 = 2 } moe_format;
  * the same function; they differ only in kernels and rounding of intermediates. */
 typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_DECODE = 1, MOE_PATH_PREFILL = 2 } moe_path;
 
+/* OR-ed into moe_forward's path: d_y is fp32 [T][H] instead of bf16 (the sums are not
+ * rounded to bf16; the expert-parallel layer returns expert outputs this way, so that
+ * its gate-weighted combine rounds once, as the single-GPU layer does). */
+#define MOE_OUT_F32 0x10
+
 /* Layer shape.  hidden and inter must be positive multiples of 64; 1 <= top_k <= 16;
  * top_k <= n_experts <= 256; n_shared in {0, 1}. */
 typedef struct {
@@ -188,6 +193,28 @@ moe_status moe_workspace_size(const moe_shape* shape, int32_t max_tokens, size_t
  * Every later call leaves the counters cleared again. */
 moe_status moe_workspace_init(void* d_ws, size_t ws_bytes, void* stream);
 
+/* For tests of the failure path only (the pages have no counterpart).  cycles > 0
+ * makes every expert kernel of the following moe_forward calls on this workspace first
+ * wait, for at most `cycles` SM clock cycles, on a barrier that nothing completes.  The
+ * wait runs out; the kernel records MOE_ERR_TIMEOUT with detail MOE_DETAIL_TEST_STALL
+ * (low byte: which kernel), then takes the path every kernel takes when one of its
+ * bounded waits runs out: it issues no further copies, waits (bounded) for the copies
+ * it has in flight, releases its tensor memory and returns; d_y is then unspecified.
+ * cycles = 0 (or moe_workspace_init) switches the stall off.  Enqueued on stream. */
+moe_status moe_workspace_set_test_stall(void* d_ws, size_t ws_bytes, uint32_t cycles, void* stream);
+
+/* Detail codes that moe_get_error returns beside MOE_ERR_TIMEOUT or
+ * MOE_ERR_DEVICE_CHECK: the high bits say what happened, the low byte in which
+ * kernel or wait. */
+#define MOE_DETAIL_WAIT_FULL 0x100u   /* a wait for data (a copy, a stage) ran out        */
+#define MOE_DETAIL_WAIT_EMPTY 0x200u  /* a wait for a free stage ran out                  */
+#define MOE_DETAIL_DRAIN 0x300u       /* the wait for in-flight copies after a give-up    */
+#define MOE_DETAIL_HEADER 0x400u      /* the packed buffer's header does not match        */
+#define MOE_DETAIL_ROUTED_T 0x500u    /* moe_forward's T differs from moe_route's T       */
+#define MOE_DETAIL_RANGE 0x600u       /* a token or expert activation outside fp16 range  */
+#define MOE_DETAIL_TEST_STALL 0x700u  /* moe_workspace_set_test_stall's wait ran out      */
+#define MOE_DETAIL_LOOP_CAP 0x800u    /* a work loop reached its iteration cap            */
+
 /* Route T tokens: fp32 router logits, softmax + top-k + renormalised gates,
  * per-expert histogram, prefix sum and permutation.
  *   d_x        bf16 bit patterns [T][H], row-major
@@ -196,20 +223,95 @@ moe_status moe_workspace_init(void* d_ws, size_t ws_bytes, void* stream);
  *   out        caller-allocated device arrays (see moe_routing)
  * Also leaves in d_ws the expert schedule that moe_forward reads, so moe_forward
  * must be given the same d_ws and T.  T = 0 is a no-op returning MOE_OK.
- * Tokens, router weights and bias must be finite: a NaN or infinity gives
- * unspecified routing and outputs (the few-token integer path does not carry a NaN
- * token through to y); nothing checks this on the device. */
+ * Router weights and bias must be finite (a NaN or infinity there gives unspecified
+ * routing; nothing checks this).  Tokens must be finite with every |x| <= 65504: the
+ * router checks each element and records MOE_ERR_DEVICE_CHECK with
+ * MOE_DETAIL_RANGE | 1 for moe_get_error otherwise (routing and outputs are then
+ * unspecified). */
 moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x,
                      const float* d_router_w, const float* d_router_b, const moe_routing* out,
                      void* d_ws, size_t ws_bytes, void* stream);
+
+/* moe_route with the expert choice given instead of computed: for callers that route
+ * elsewhere, such as the expert-parallel layer, whose GPUs each run only their own
+ * experts on the token rows sent to them (every row with one expert, gate 1).  Writes
+ * the routing arrays (ids and gates copied from d_ids / d_gates, [T][k] each; counts,
+ * offsets, perm, inv_perm computed as moe_route does) and the schedule in d_ws that
+ * moe_forward reads.  Same argument rules and errors as moe_route; d_ids and d_gates
+ * are device pointers.  An id outside [0, E) is recorded as MOE_ERR_DEVICE_CHECK
+ * (MOE_DETAIL_RANGE | 2) and its pair is left out of every expert's rows. */
+moe_status moe_route_fixed(const moe_shape* shape, int32_t T, const uint16_t* d_x, const int32_t* d_ids,
+                           const float* d_gates, const moe_routing* out, void* d_ws, size_t ws_bytes,
+                           void* stream);
+
+/* Expert-parallel row helpers (the layer's experts split over several GPUs; the pages
+ * run their engine on more than one consumer GPU: molayo1419.me, "Delta Inference
+ * Engine", the multi-GPU paragraph).  Both only enqueue one kernel on `stream` and
+ * record bad indices in the control block of d_ws (moe_get_error), never faulting.
+ *   moe_gather_rows:   d_dst[i][:] = d_src[d_index[i] / divisor][:] for i < n; bf16 rows
+ *                      of `hidden` elements; d_src has n_src rows.  With d_index = perm
+ *                      and divisor = top_k it builds the dispatch buffer (token rows in
+ *                      expert-major order).  An index past d_src: MOE_DETAIL_RANGE | 3,
+ *                      the row is zeroed.
+ *   moe_combine_pairs: d_y[t][:] = sum_j d_gates[t][j] * d_rows[d_inv_perm[t k + j]][:]
+ *                      (j ascending) + d_shared[t][:] (if not NULL), fp32 rows and sums
+ *                      (moe_forward's MOE_OUT_F32 output), stored as bf16, for t < T;
+ *                      d_rows has n_rows rows.  A row index past d_rows:
+ *                      MOE_DETAIL_RANGE | 4, left out of the sum.
+ * MOE_ERR_INVALID_ARG: a null pointer, hidden not a positive multiple of 64, a negative
+ * count, divisor < 1, top_k outside 1..16. */
+moe_status moe_gather_rows(int32_t n, int32_t hidden, const uint16_t* d_src, int32_t n_src,
+                           const int32_t* d_index, int32_t divisor, uint16_t* d_dst, void* d_ws,
+                           size_t ws_bytes, void* stream);
+moe_status moe_combine_pairs(int32_t T, int32_t top_k, int32_t hidden, const float* d_rows, int32_t n_rows,
+                             const int32_t* d_inv_perm, const float* d_gates, const float* d_shared,
+                             uint16_t* d_y, void* d_ws, size_t ws_bytes, void* stream);
+
+/* Host-tiered experts.  The engine on the pages keeps the experts that do not fit its
+ * GPU in a pinned host-RAM arena and brings the ones a layer needs into GPU memory ahead
+ * of use (ossradar.top, Xolotl README, "How it works, in one paragraph").  These calls
+ * let a layer run from a device cache of n_slots expert slots in front of a packed
+ * buffer h_packed in host memory (page-locked, so that the copies are asynchronous).
+ * The cache d_cache is itself a packed buffer: the layer's header and expert table,
+ * then the slots; pass it to moe_forward as d_packed.  Every expert the routing selects,
+ * and the shared expert, must have been loaded into some slot first; which expert goes
+ * to which slot (and when) is the caller's choice.
+ *   moe_cache_size: bytes of the cache for n_slots slots (each as large as the largest
+ *                   expert's span of the host buffer).
+ *   moe_cache_init: writes the header and table (every entry pointing into slot 0 until
+ *                   its expert is loaded); enqueued on stream.
+ *   moe_cache_load: for i < n copies expert h_experts[i]'s span (its gate/up and down
+ *                   arrays, contiguous in the packer's layout) into slot h_slots[i] and
+ *                   points its table entry there: one cudaMemcpyAsync per expert and a
+ *                   one-thread kernel for the entry, enqueued on stream (a prefetch
+ *                   stream, with an event before the forward, overlaps it with compute).
+ * MOE_ERR_INVALID_ARG: a null pointer, n_slots < 1, an expert or slot index out of
+ * range, or a host buffer whose header does not describe the shape; MOE_ERR_WORKSPACE:
+ * cache_bytes too small; MOE_ERR_CUDA: a copy or launch failed. */
+moe_status moe_cache_size(const moe_shape* shape, const uint8_t* h_packed, int32_t n_slots, size_t* bytes);
+moe_status moe_cache_init(const moe_shape* shape, const uint8_t* h_packed, int32_t n_slots, void* d_cache,
+                          size_t cache_bytes, void* stream);
+moe_status moe_cache_load(const moe_shape* shape, const uint8_t* h_packed, int32_t n_slots, void* d_cache,
+                          size_t cache_bytes, const int32_t* h_experts, const int32_t* h_slots, int32_t n,
+                          void* stream);
 
 /* Expert FFNs of the routed and shared experts and the gate-weighted combine,
  * using the routing of the preceding moe_route on the same d_ws.
  *   d_packed  packed experts (format above), device memory
  *   d_x       bf16 [T][H] (the same tokens as routed)
  *   r         the routing moe_route wrote
- *   d_y       bf16 [T][H] output, written in full
- * T = 0 is a no-op.  T > 64 with MOE_PATH_DECODE is allowed (slower). */
+ *   d_y       bf16 [T][H] output, written in full (fp32 with path | MOE_OUT_F32)
+ * T = 0 is a no-op.  T > 64 with MOE_PATH_DECODE is allowed (slower).
+ * Checked on the device (recorded for moe_get_error; d_y is then unspecified):
+ *   - T must be the T of the preceding moe_route on d_ws; otherwise the expert
+ *     kernels return without reading the routing (MOE_ERR_DEVICE_CHECK,
+ *     MOE_DETAIL_ROUTED_T).
+ *   - Range: the kernels hold tokens (prefill) and the expert activations
+ *     h = silu(Wg x) * (Wu x) (both paths) in fp16, so they compute the layer for
+ *     tokens with every |x| <= 65504 whose activations have every |h| <= 65504.  A
+ *     token or an activation outside that range is reported as MOE_ERR_DEVICE_CHECK
+ *     with MOE_DETAIL_RANGE (the router reports tokens, low byte 1; the gate/up
+ *     kernels activations). */
 moe_status moe_forward(const moe_shape* shape, int32_t T, const void* d_packed,
                        const uint16_t* d_x, const moe_routing* r, uint16_t* d_y, moe_path path,
                        void* d_ws, size_t ws_bytes, void* stream);
@@ -238,19 +340,32 @@ moe_status moe_get_error(void* d_ws, size_t ws_bytes, void* stream, uint32_t* de
  * instead of a caller-given workspace it uses a scratch array that the library holds
  * in device memory: MOE_STATIC_WS_BYTES (8 MiB), held by every GPU that loads the
  * library until the process exits.  It allocates nothing itself.
+ *   - Every argument check of moe_route and moe_forward runs before anything is
+ *     enqueued; a rejected call leaves the scratch array and d_y untouched.
  *   - If the workspace T tokens need (moe_workspace_size) exceeds MOE_STATIC_WS_BYTES
- *     it returns MOE_ERR_WORKSPACE and enqueues nothing; with the full-size layer
- *     (H 7168, I 2048, E 256, k 8, S 1) that allows up to 27 tokens per call.
- *   - The first call on each device looks up the scratch array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call before
- *     any stream capture.  Later calls only enqueue work.
- *   - All calls share the one array, and each call first clears its control block.
- *     Calls that overlap on the GPU (other streams, other host threads, other
- *     devices' calls do not overlap) race on the array: serialise them. */
+ *     it returns MOE_ERR_WORKSPACE; with the full-size layer (H 7168, I 2048, E 256,
+ *     k 8, S 1) that allows up to 21 tokens per call.
+ *   - The first call on each device (and the first after a cudaDeviceReset) looks up
+ *     the scratch array's device address (cudaGetSymbolAddress) with that device
+ *     current; make that first call before any stream capture.  Later calls only
+ *     enqueue work.
+ *   - All calls share the one array, and each call first clears its counters.
+ *     Calls that overlap on the GPU (other streams, other host threads; other
+ *     devices' calls do not overlap) race on the array: serialise them.
+ *   - Problems found on the device (a bounded wait that ran out, a corrupt packed
+ *     header) are recorded in the array and kept across later calls until
+ *     moe_decode_static_get_error reads and clears them. */
 #define MOE_STATIC_WS_BYTES ((size_t)8 << 20)
 moe_status moe_decode_static(const moe_shape* shape, int32_t T, const uint16_t* d_x,
                              const float* d_router_w, const float* d_router_b, const void* d_packed,
                              const moe_routing* out, uint16_t* d_y, void* stream);
+
+/* moe_get_error for the scratch array of moe_decode_static on the current device:
+ * synchronises the stream, returns the first problem recorded by any
+ * moe_decode_static call since the last read (MOE_OK, MOE_ERR_TIMEOUT or
+ * MOE_ERR_DEVICE_CHECK; *detail, if not NULL, the detail code) and clears it.
+ * MOE_ERR_CUDA if the array's address cannot be looked up or the copy fails. */
+moe_status moe_decode_static_get_error(void* stream, uint32_t* detail);
 
 /* Records a caller-created CUDA event (cudaEvent_t, passed as void*) on a stream.
  * While the stream is being captured into a CUDA graph the record is captured as an

@@ -33,13 +33,19 @@ class Case:
     extra: dict = field(default_factory=dict)
 
 
-def make_case(cfg, layer_idx=0, step=0, T=None, bias=None, router_w=None, threads=None) -> Case:
+def make_case(cfg, layer_idx=0, step=0, T=None, bias=None, router_w=None, threads=None,
+              transform=None) -> Case:
+    """transform(x, rows) (optional) rewrites the listed token rows of x in place after
+    they are drawn or redrawn (e.g. to plant outliers); the near-tie guard then runs on
+    the rewritten tokens."""
     layer = synth.Layer(cfg, layer_idx)
     if router_w is not None:
         layer.router_w = router_w
     if bias is not None:
         layer.router_b = bias
     x = synth.tokens(cfg, layer_idx, step, T)
+    if transform is not None:
+        transform(x, np.arange(x.shape[0]))
     redrawn = 0
     for rnd in range(20):
         L = oracle.logits(x, layer.router_w, threads)
@@ -48,6 +54,8 @@ def make_case(cfg, layer_idx=0, step=0, T=None, bias=None, router_w=None, thread
             break
         redrawn += bad.size
         synth.redraw_tokens(cfg, x, bad, layer_idx, step, rnd)
+        if transform is not None:
+            transform(x, bad)
     else:
         raise RuntimeError("could not remove near-ties")
     ids, gates = oracle.select(L, layer.router_b, cfg.k)
@@ -97,7 +105,7 @@ def pack(case: Case, threads=None) -> np.ndarray:
     return buf
 
 
-def run_gpu(case: Case, packed_host=None, path=0, gpu_layer=None):
+def run_gpu(case: Case, packed_host=None, path=0, gpu_layer=None, check_error=True):
     """Route + forward on the GPU; returns (routing dict of numpy arrays, y uint16)."""
     import torch
     import bit_routed_expert_fp32_b200 as moe
@@ -110,8 +118,9 @@ def run_gpu(case: Case, packed_host=None, path=0, gpu_layer=None):
     gpu_layer.route(x)
     gpu_layer.forward(x, y, path=path)
     torch.cuda.synchronize()
-    st, det = moe.moe_get_error(gpu_layer.ws)
-    assert st == 0, f"device error {moe.STATUS[st]} detail {det:#x}"
+    if check_error:
+        st, det = moe.moe_get_error(gpu_layer.ws)
+        assert st == 0, f"device error {moe.STATUS[st]} detail {det:#x}"
     rt = {n: t.cpu().numpy() for n, t in gpu_layer.rt.items()}
     return rt, moe.bf16_to_host(y)
 
@@ -124,21 +133,44 @@ def check_routing(case: Case, rt: dict):
     np.testing.assert_array_equal(rt["offsets"], case.offsets)
     np.testing.assert_array_equal(rt["perm"][:T * cfg.k], case.perm)
     np.testing.assert_array_equal(rt["inv_perm"][:T * cfg.k], case.inv_perm)
-    np.testing.assert_allclose(rt["topk_w"][:T].astype(np.float64), case.gates, rtol=GATE_RTOL, atol=0)
+    # The router's logits are fp32 values (the layer's router is fp32), so a gate
+    # g_j = exp(L_j - L_max) / sum is exact only up to the rounding of L_j and L_max to
+    # fp32: |dg / g| <= ulp(max |L|) beyond the fixed 1e-5.  For N(0,1) tokens max |L| is
+    # a few units (ulp ~ 5e-7); tokens with 1000x outliers reach hundreds (ulp ~ 6e-5).
+    Lb = case.L + (0.0 if case.layer.router_b is None else case.layer.router_b.astype(np.float64))
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(Lb).max(axis=1), 1e-30))) - 23)
+    rtol = GATE_RTOL + ulp[:, None]
+    g = rt["topk_w"][:T].astype(np.float64)
+    bad = np.abs(g - case.gates) > rtol * np.abs(case.gates)
+    assert not bad.any(), (f"gates differ beyond 1e-5 + ulp(max |L|) at {np.argwhere(bad)[:5].tolist()}: "
+                           f"{g[bad][:5]} vs {case.gates[bad][:5]}")
 
 
 def oracle_outputs(case: Case, tokens, threads=None) -> np.ndarray:
     return oracle.forward_tokens(case.layer, case.x, case.ids, case.gates, tokens, threads)
 
 
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 values (8 significant bits) at |v|: the error of rounding
+    the exact value to the output format."""
+    a = np.maximum(np.abs(v), np.finfo(np.float32).tiny)
+    return np.exp2(np.floor(np.log2(a)) - 8)
+
+
 def check_outputs(y_gpu_bits: np.ndarray, y_ref: np.ndarray):
+    """The parity bar.  The layer's output is bf16, so the max-abs bound applies to the
+    error beyond the rounding of the exact value to bf16 (half an ulp at |y|): an output
+    of 8x rms has a rounding error of ~2 % of rms by itself, more than the bound, even
+    from exact arithmetic.  The Frobenius bound applies to the whole error."""
     y = synth.bf16_bits_to_f32(y_gpu_bits).astype(np.float64)
     assert np.all(np.isfinite(y))
     diff = y - y_ref
     rms = np.sqrt(np.mean(y_ref ** 2))
-    max_err = np.abs(diff).max()
+    excess = np.maximum(np.abs(diff) - bf16_half_ulp(y_ref), 0.0)
+    max_err = excess.max()
     frob = np.linalg.norm(diff) / np.linalg.norm(y_ref)
-    assert max_err <= ATOL_RMS * rms, f"max |err| {max_err:.3e} > {ATOL_RMS} * rms {rms:.3e}"
+    assert max_err <= ATOL_RMS * rms, (f"max |err| beyond bf16 rounding {max_err:.3e} > {ATOL_RMS} * rms {rms:.3e} "
+                                       f"(raw max |err| {np.abs(diff).max():.3e})")
     assert frob <= FROB, f"relative Frobenius error {frob:.3e} > {FROB}"
     return max_err / rms, frob
 

@@ -56,8 +56,13 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
 
 
 def test_paths_and_launch_counts():
-    c2, c4 = synth.CONFIGS[2], synth.CONFIGS[4]
-    # one token: 9 active experts, so gate/up K is split into parts and reduced by one more kernel
-    assert bench.decode_kparts(c2) == (7, 4)
-    assert bench.path_of(c2) == "decode" and bench.launches_per_step(c2) == 1 + 4
+    import dataclasses
+    c2, c3, c4 = synth.CONFIGS[2], synth.CONFIGS[3], synth.CONFIGS[4]
+    # up to 16 tokens: the router, then the whole forward as one kernel
+    assert bench.path_of(c2) == "fused" and bench.launches_per_step(c2) == 1 + 1
+    assert bench.path_of(c3) == "fused" and bench.launches_per_step(c3) == 1 + 1
+    # 17 to 64 tokens: the decode kernels; with 24 tokens K is split for neither pass
+    c24 = dataclasses.replace(c2, T=24)
+    assert bench.path_of(c24) == "decode"
+    assert bench.launches_per_step(c24) == 1 + 3 + (1 if bench.decode_kparts(c24)[0] > 1 else 0)
     assert bench.path_of(c4) == "prefill" and bench.launches_per_step(c4) == 4 + 4

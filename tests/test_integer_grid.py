@@ -1,12 +1,15 @@
-"""Bounds the few-token integer gate/up path relies on (host-side arithmetic, no GPU).
+"""Bounds the integer MMA path of the fused decode kernel relies on (host-side
+arithmetic, no GPU).
 
-The path puts each 64-group of a token on a 12-bit grid, q = rint(x 2^e) with
-e = 11 - floor(log2 max|x|), stores B = 4q or q as two signed bytes lo + 256 hi, and
-sums 64 products A B per group in an int32 accumulator that starts at the bit pattern
-of 1.5 * 2^23, reading the result back as fp32.  These tests check, from those
-definitions alone, that the digits fit their bytes, that the worst-case group sum
-stays inside the window where the fp32 reinterpretation is exact, and how far the grid
-moves bf16 tokens.
+The path puts each 64-group of a row (a token, or an h row) on a 12-bit grid,
+q = rint(v 2^e) with e = 11 - floor(log2 max|v|), stores B = 4q or q as two signed
+bytes lo + 256 hi, and sums 64 products A B per group and digit in int32 (the low
+digit's accumulator starting at the bit pattern of 1.5 * 2^23); the two digit sums are
+joined as d0 + 256 d1, the code offset is removed exactly as D - 4 o sum q, and the
+result is read back as fp32.  These tests check, from those definitions alone, that the
+digits fit their bytes, that the joined and corrected group sum stays inside the window
+where the fp32 reinterpretation is exact, that the steps give exactly
+sum 4 (c - o) q, and how far the grid moves bf16 values.
 """
 import numpy as np
 
@@ -62,3 +65,31 @@ def test_grid_moves_bf16_tokens_by_about_1e_4_rms():
         err.append(xt - g)
     rel = np.sqrt(np.mean(np.square(err))) / np.sqrt(np.mean(np.square(x)))
     assert 5e-5 < rel < 2e-4
+
+
+def test_joined_and_corrected_sum_is_exact_and_inside_the_window():
+    rng = np.random.default_rng(1)
+    magic = 0x4B400000
+    for o4, cmax in ((4, 2), (6, 3)):                        # ternary (o = 1), 2-bit (o = 1.5)
+        for trial in range(200):
+            c = rng.integers(0, cmax + 1, 64)
+            if trial == 0:
+                q = np.full(64, 4096)                         # the extreme group
+                c = np.full(64, cmax if o4 == 6 else 2)
+            else:
+                q = rng.integers(-4096, 4097, 64)
+            # class of element k: c = (k mod 8) / 2; odd classes hold 4 c with B = q,
+            # even classes hold c with B = 4 q: every product is 4 c q
+            cls = (np.arange(64) % 8) // 2
+            a = np.where(cls % 2 == 1, 4 * c, c)
+            b = np.where(cls % 2 == 1, q, 4 * q)
+            lo = ((b & 0xFF) ^ 0x80) - 0x80
+            hi = (b - lo) >> 8
+            d0 = magic + int(np.sum(a * lo))
+            d1 = int(np.sum(a * hi))
+            joined = d0 + 256 * d1 - o4 * int(np.sum(q))
+            D = joined - magic
+            assert D == int(np.sum(4 * c * q)) - o4 * int(np.sum(q))
+            assert abs(D) < 2 ** 22
+            f = np.array([joined], np.uint32).view(np.float32)[0]
+            assert float(f) - 12582912.0 == D

@@ -71,6 +71,31 @@ def test_argument_errors_are_synchronous():
     assert L.moe_forward(ctypes.byref(sh), 0, fake, fake, ctypes.byref(r), fake, 0, fake, need, None) == 0
 
 
+def test_static_entry_point_checks_everything_before_any_cuda_call():
+    """moe_decode_static runs every argument check of moe_route and moe_forward before
+    it touches the device (no GPU here: any CUDA call would fail with MOE_ERR_CUDA)."""
+    L = moe.lib()
+    fake = ctypes.c_void_p(0x1000)
+    r = moe.Routing(*([0x1000] * 6))
+    r0 = moe.Routing(0x1000, 0x1000, 0, 0x1000, 0x1000, 0x1000)
+    sh = _shape()
+    assert L.moe_decode_static(None, 4, fake, fake, None, fake, ctypes.byref(r), fake, None) == 1
+    assert L.moe_decode_static(ctypes.byref(_shape(k=5)), 4, fake, fake, None, fake, ctypes.byref(r), fake,
+                               None) == 1                                  # k > E
+    bad_s = moe.Shape(128, 64, 4, 2, -1)                                      # negative n_shared
+    assert L.moe_decode_static(ctypes.byref(bad_s), 4, fake, fake, None, fake, ctypes.byref(r), fake, None) == 1
+    assert L.moe_decode_static(ctypes.byref(sh), -1, fake, fake, None, fake, ctypes.byref(r), fake, None) == 1
+    assert L.moe_decode_static(ctypes.byref(sh), 4, None, fake, None, fake, ctypes.byref(r), fake, None) == 1
+    assert L.moe_decode_static(ctypes.byref(sh), 4, fake, None, None, fake, ctypes.byref(r), fake, None) == 1
+    assert L.moe_decode_static(ctypes.byref(sh), 4, fake, fake, None, None, ctypes.byref(r), fake, None) == 1
+    assert L.moe_decode_static(ctypes.byref(sh), 4, fake, fake, None, fake, ctypes.byref(r0), fake, None) == 1
+    assert L.moe_decode_static(ctypes.byref(sh), 4, fake, fake, None, fake, ctypes.byref(r), None, None) == 1
+    big = moe.Shape(7168, 2048, 256, 8, 1)                                   # 64 tokens need ~19 MB
+    assert L.moe_decode_static(ctypes.byref(big), 64, fake, fake, None, fake, ctypes.byref(r), fake, None) == 3
+    assert L.moe_decode_static(ctypes.byref(sh), 0, fake, fake, None, fake, ctypes.byref(r), fake, None) == 0
+    assert L.moe_workspace_set_test_stall(None, 1 << 20, 100, None) == 1
+
+
 def test_workspace_size_never_shrinks_as_tokens_grow():
     # A workspace sized for max_tokens must serve every smaller T: the K-part split
     # of the decode passes and the few-token integer operands must not make a smaller
@@ -78,9 +103,9 @@ def test_workspace_size_never_shrinks_as_tokens_grow():
     for cfg in (synth.CONFIGS[2], synth.micro(T=8, H=256, E=8, k=2, I=128, S=0)):
         sizes = [moe.moe_workspace_size(cfg, T) for T in range(0, 97)]
         assert all(b >= a for a, b in zip(sizes, sizes[1:]))
-    # the full-size layer: the library's static scratch holds 27 tokens, not 28
+    # the full-size layer: the library's static scratch holds 21 tokens, not 22
     cfg = synth.CONFIGS[2]
-    assert moe.moe_workspace_size(cfg, 27) <= moe.STATIC_WS_BYTES < moe.moe_workspace_size(cfg, 28)
+    assert moe.moe_workspace_size(cfg, 21) <= moe.STATIC_WS_BYTES < moe.moe_workspace_size(cfg, 22)
 
 
 @pytest.mark.parametrize("H,I,formats", [(128, 64, "mixed"), (192, 128, "q3"), (256, 64, "ternary"),
