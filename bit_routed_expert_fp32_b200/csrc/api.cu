@@ -25,8 +25,8 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     size_t off = 0;
     w.ctrl = off;
     off += 4096;
-    w.tile_ctr = off;
-    off = align256(off + 4 * (size_t)(H / 16));
+    w.tile_ctr = off;                                   // [H/16] down, then [2I/16] gate/up
+    off = align256(off + 4 * (size_t)(H / 16 + 2 * I / 16));
     w.active = off;
     off = align256(off + 4 * (size_t)(E + S));
     w.logits = off;
@@ -43,12 +43,20 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     off = align256(off + 4 * (size_t)(r16 * I));
     w.hq = off;
     off = align256(off + (r16 > 0 ? iq_size(r16, I) : 0));
+    // the fused kernel's need of the ypart region (its K-part sums) for every token
+    // count up to min(T, kFusedMaxT)
+    size_t yfused = 0;
+    for (int64_t t = 1; t <= T && t <= kFusedMaxT; ++t) {
+        const size_t y = fused_ypart_floats(s, t);
+        yfused = yfused > y ? yfused : y;
+    }
     w.h = off;
     off = align256(off + 2 * (size_t)(T * (k + S) * I));
     // ypart, and the decode gate/up partial sums that alias it: the largest need of any
     // token count up to T (the split into K parts shrinks as T grows), so a workspace
     // sized for T tokens serves every smaller T.
     size_t yfl = (size_t)(T * (k + S) * H);
+    yfl = yfl > yfused ? yfl : yfused;
     for (int64_t t = 1; t <= T && t <= kSmallT; ++t) {
         int ngu = 1, ndn = 1;
         decode_kparts(s, t, &ngu, &ndn);
@@ -291,9 +299,13 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.hf = reinterpret_cast<float*>(ws + w.hf);
     a.hq = ws + w.hq;
     a.R16 = (T < kFusedMaxT ? T : kFusedMaxT) * (a.k + a.S);
+    a.gp_done = a.dn_done + a.H / 16;
+    a.fpg = a.fpd = 1;
+    if (T >= 1 && T <= kFusedMaxT) fused_kparts(shape, T, &a.fpg, &a.fpd);
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.h = reinterpret_cast<uint16_t*>(ws + w.h);
     a.ypart = reinterpret_cast<float*>(ws + w.ypart);
+    a.gsh = a.ypart + (size_t)a.fpd * T * (a.k + a.S) * a.H;
     a.gpart = a.ypart;
     a.nkp_gu = a.nkp_dn = 1;
     a.tile_ctr = reinterpret_cast<uint32_t*>(ws + w.tile_ctr);

@@ -162,6 +162,10 @@ struct Layout {        // unit index ranges; the routed ones are known once rout
     int nops, nsgu, pre;        // operands, shared gate/up; pre = nops + nsgu
     int tg, td;                 // 16-row tiles per expert: gate/up (2I/16), down (H/16)
     int nch, nci;               // 8-group chunks per row: gate/up (K = H), down (K = I)
+    int S;                      // shared experts (their slots come first)
+    int pg, pd;                 // K parts: shared experts' gate/up tiles, every down tile
+    int cpg, cpd;               // chunks per part
+    int shares;                 // down tiles per expert that form the h operands (integer path)
     int nr;                     // routed experts with tokens (-1: not read yet)
     int total;                  // all units (pre until routing is known)
     bool t_ok;                  // the routing is for this call's T
@@ -170,7 +174,7 @@ struct Layout {        // unit index ranges; the routed ones are known once rout
 // A unit is four integers; everything else about its expert comes from the CTA's slot
 // table in shared memory (a few registers per warp instead of a copy of it).
 struct Unit {
-    int kind, idx, slot, tile;
+    int kind, idx, slot, tile, part;
 };
 
 // Per expert slot (shared experts first, then the routed experts with tokens, in the
@@ -261,17 +265,20 @@ __device__ __forceinline__ Unit resolve(const FfnArgs& p, const Layout& L, int u
     U.idx = u;
     U.slot = 0;
     U.tile = 0;
+    U.part = 0;
     if (u < 0) return U;
     if (u < L.nops) {
         U.kind = U_OPS;
         U.tile = u;
         return U;
     }
-    if (u < L.pre) {
-        const int v = u - L.nops;
+    if (u < L.pre) {                        // shared gate/up: (slot, tile, K part), part fastest
+        const int v = u - L.nops, per = L.tg * L.pg;
         U.kind = U_GU;
-        U.slot = v / L.tg;
-        U.tile = v - U.slot * L.tg;
+        U.slot = v / per;
+        const int r = v - U.slot * per;
+        U.tile = r / L.pg;
+        U.part = r - U.tile * L.pg;
         return U;
     }
     if (L.nr < 0 || u >= L.total) return U;
@@ -281,17 +288,43 @@ __device__ __forceinline__ Unit resolve(const FfnArgs& p, const Layout& L, int u
         U.kind = U_GU;
         U.tile = v - a * L.tg;
         U.slot = p.S + a;
-    } else {
-        v -= L.nr * L.tg;
-        U.kind = U_DN;
-        U.slot = v / L.td;                  // shared experts first, then routed
-        U.tile = v - U.slot * L.td;
+        return U;
     }
+    // down: every slot's first `shares` tiles (they form the h operands) before the rest;
+    // within each, slots in order (shared first), tiles ascending, K parts fastest
+    v -= L.nr * L.tg;
+    U.kind = U_DN;
+    const int n_slots = p.S + L.nr;
+    const int b1 = L.shares * L.pd, rest = (L.td - L.shares) * L.pd;
+    int r;
+    if (v < n_slots * b1) {
+        U.slot = v / b1;
+        r = v - U.slot * b1;
+    } else {
+        v -= n_slots * b1;
+        U.slot = v / rest;
+        r = v - U.slot * rest + b1;
+    }
+    U.tile = r / L.pd;
+    U.part = r - U.tile * L.pd;
     return U;
 }
 
 __device__ __forceinline__ bool streams(const Unit& U) { return U.kind == U_GU || U.kind == U_DN; }
-__device__ __forceinline__ int unit_nc(const Unit& U, const Layout& L) { return U.kind == U_DN ? L.nci : L.nch; }
+// The unit's chunks: [c0, c0 + n) of its matrix's K (one K part of it, if split; the
+// routed experts' gate/up tiles are not split and have part 0).
+__device__ __forceinline__ int unit_c0(const Unit& U, const Layout& L) {
+    return U.part * (U.kind == U_DN ? L.cpd : L.cpg);
+}
+__device__ __forceinline__ int unit_nc(const Unit& U, const Layout& L) {
+    const int c0 = unit_c0(U, L);
+    if (U.kind == U_DN) return min(L.nci, c0 + L.cpd) - c0;
+    return U.slot < L.S ? min(L.nch, c0 + L.cpg) - c0 : L.nch;
+}
+// A shared expert's gate/up tile split into K parts: the parts' sums go to gsh.
+__device__ __forceinline__ bool gu_split(const Unit& U, const Layout& L) {
+    return U.kind == U_GU && U.slot < L.S && L.pg > 1;
+}
 
 // The warp's next unit, taken from the launch's counter only when the ring is about to
 // need it (when the current unit's last chunks are being issued): a unit held early by a
@@ -353,7 +386,7 @@ __device__ __forceinline__ void top_up(Ring& R, const CtaState& cs, const Unit& 
     while (R.issued - R.consumed < NS) {
         if (R.iw == 0) {
             if (streams(cur) && R.ic < unit_nc(cur, L)) {
-                issue_chunk(R, cs, p, cur, R.ic++, pol);
+                issue_chunk(R, cs, p, cur, unit_c0(cur, L) + R.ic++, pol);
                 continue;
             }
             R.iw = 1;
@@ -361,7 +394,7 @@ __device__ __forceinline__ void top_up(Ring& R, const CtaState& cs, const Unit& 
             take_next(Q, p, L, lane);
         }
         if (streams(Q.nxt) && R.ic < unit_nc(Q.nxt, L)) {
-            issue_chunk(R, cs, p, Q.nxt, R.ic++, pol);
+            issue_chunk(R, cs, p, Q.nxt, unit_c0(Q.nxt, L) + R.ic++, pol);
             continue;
         }
         break;
@@ -649,6 +682,16 @@ __device__ __forceinline__ void release_stage(Ring& R) {
     ++R.consumed;
 }
 
+// Where a unit's fp32 results go: a split shared gate/up tile's {gate, up} sums of K part
+// U.part (gsh, rows of the shared experts only), and a down tile's rows of y_e for K part
+// U.part (ypart [part][T (k + S)][H]).
+__device__ __forceinline__ float2* gsh_at(const FfnArgs& p, const Unit& U, int orow, int hcol) {
+    return reinterpret_cast<float2*>(p.gsh) + ((size_t)U.part * p.S * p.T + (orow - p.T * p.k)) * p.I + hcol;
+}
+__device__ __forceinline__ float* ypart_at(const FfnArgs& p, const Unit& U, int orow, int col) {
+    return p.ypart + ((size_t)U.part * p.T * (p.k + p.S) + orow) * p.H + col;
+}
+
 // A tile of a ternary or 2-bit expert on the integer path, with NP passes of 4 rows.
 // MODE 0 (gate/up): B = the tokens' digit records, output h = silu(gate) * up in fp32
 // (hf, quantised later for the down pass); MODE 1 (down): B = the expert's h rows'
@@ -672,12 +715,13 @@ __device__ __forceinline__ void unit_iq(const FfnArgs& p, const Layout& L, const
         v.orow[q] = it < cnt ? row0 + it : -1;
     }
     const int o4 = cs.slot[cur.slot].fmt == MOE_FMT_TERNARY ? 4 : 6;
-    const int K = MODE == 0 ? p.H : p.I, NC = (K / 64 + CG - 1) / CG, GK = K / 64;
+    const int K = MODE == 0 ? p.H : p.I, GK = K / 64;
     const int sw = 128 * g + 16 * (g & 7) + 4 * t;       // this lane's word of group 0, swizzled
     unsigned long long acc[NP];
 #pragma unroll
     for (int q = 0; q < NP; ++q) acc[q] = 0ull;
-    for (int c = 0; c < NC; ++c) {
+    const int c0 = unit_c0(cur, L), c1 = c0 + unit_nc(cur, L);
+    for (int c = c0; c < c1; ++c) {
         const uint8_t* stg = next_stage(R, cs, cur, Q, stop, fc, p.ctrl, lane, pol, p, L);
         if (!stg) break;
         const int ng = min(CG, GK - c * CG);
@@ -693,13 +737,18 @@ __device__ __forceinline__ void unit_iq(const FfnArgs& p, const Layout& L, const
         bool range_ok = true;
         if (ready && !stop) {
             const int hcol = cur.tile * 8 + g;
+            const bool split = gu_split(cur, L);
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
                 if (q < np && v.orow[q] >= 0) {
                     const float2 a = up2(acc[q]);
-                    const float hv = silu_f(a.x) * a.y;
-                    range_ok &= in_f16_range(hv);
-                    p.hf[(size_t)v.orow[q] * p.I + hcol] = hv;
+                    if (split) {
+                        *gsh_at(p, cur, v.orow[q], hcol) = a;
+                    } else {
+                        const float hv = silu_f(a.x) * a.y;
+                        range_ok &= in_f16_range(hv);
+                        p.hf[(size_t)v.orow[q] * p.I + hcol] = hv;
+                    }
                 }
             }
         }
@@ -711,7 +760,7 @@ __device__ __forceinline__ void unit_iq(const FfnArgs& p, const Layout& L, const
         for (int q = 0; q < NP; ++q) {
             if (q < np && v.orow[q] >= 0) {
                 const float2 a = up2(acc[q]);
-                float* dst = p.ypart + (size_t)v.orow[q] * p.H + cur.tile * 16 + g;
+                float* dst = ypart_at(p, cur, v.orow[q], cur.tile * 16 + g);
                 dst[0] = a.x;
                 dst[8] = a.y;
             }
@@ -749,7 +798,7 @@ __device__ __forceinline__ void unit_bf(const FfnArgs& p, const Layout& L, const
     const int g = lane >> 2, t = lane & 3;
     const int cnt = cs.slot[cur.slot].cnt, row0 = cs.slot[cur.slot].row0, fmt = cs.slot[cur.slot].fmt;
     const int np = (cnt + 7) / 8;
-    const int K = MODE == 0 ? p.H : p.I, NC = (K / 64 + CG - 1) / CG, GK = K / 64;
+    const int K = MODE == 0 ? p.H : p.I, GK = K / 64;
     BfView<NP> v;
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
@@ -784,7 +833,8 @@ __device__ __forceinline__ void unit_bf(const FfnArgs& p, const Layout& L, const
     float acc[NP][4];
 #pragma unroll
     for (int q = 0; q < NP; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
-    for (int c = 0; c < NC; ++c) {
+    const int c0 = unit_c0(cur, L), c1 = c0 + unit_nc(cur, L);
+    for (int c = c0; c < c1; ++c) {
         const uint8_t* stg = next_stage(R, cs, cur, Q, stop, fc, p.ctrl, lane, pol, p, L);
         if (!stg) break;
         const int ng = min(CG, GK - c * CG);
@@ -799,14 +849,19 @@ __device__ __forceinline__ void unit_bf(const FfnArgs& p, const Layout& L, const
     if (MODE == 0) {
         bool range_ok = true;
         const int hcol = cur.tile * 8 + g;
+        const bool split = gu_split(cur, L);
 #pragma unroll
         for (int q = 0; q < NP; ++q)
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc)
                 if (q < np && v.orow[q][cc] >= 0) {
-                    const float hv = silu_f(acc[q][cc]) * acc[q][2 + cc];
-                    range_ok &= in_f16_range(hv);
-                    p.h[(size_t)v.orow[q][cc] * p.I + hcol] = f32_to_f16_bits(hv);
+                    if (split) {
+                        *gsh_at(p, cur, v.orow[q][cc], hcol) = make_float2(acc[q][cc], acc[q][2 + cc]);
+                    } else {
+                        const float hv = silu_f(acc[q][cc]) * acc[q][2 + cc];
+                        range_ok &= in_f16_range(hv);
+                        p.h[(size_t)v.orow[q][cc] * p.I + hcol] = f32_to_f16_bits(hv);
+                    }
                 }
         if (!__all_sync(0xffffffffu, range_ok) && lane == 0)
             report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 0x20);
@@ -817,18 +872,47 @@ __device__ __forceinline__ void unit_bf(const FfnArgs& p, const Layout& L, const
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc)
                 if (q < np && v.orow[q][cc] >= 0) {
-                    float* dst = p.ypart + (size_t)v.orow[q][cc] * p.H + cur.tile * 16 + g;
+                    float* dst = ypart_at(p, cur, v.orow[q][cc], cur.tile * 16 + g);
                     dst[0] = acc[q][cc];
                     dst[8] = acc[q][2 + cc];
                 }
     }
 }
 
+// The last K part of a split shared gate/up tile: h = silu(gate) * up of its 8 columns
+// for the shared expert's rows, from the parts' sums added in part order; fp16 h for a
+// 3-bit expert (the bf16 path's down operand), fp32 hf for the integer path.
+__device__ __forceinline__ void finish_shared_gu(const FfnArgs& p, const Layout& L, const CtaState& cs,
+                                                 const Unit& cur, int lane) {
+    const int cnt = cs.slot[cur.slot].cnt, row0 = cs.slot[cur.slot].row0;
+    const bool q3 = cs.slot[cur.slot].fmt == MOE_FMT_Q3;
+    const size_t part_stride = (size_t)p.S * p.T * p.I;
+    bool range_ok = true;
+    for (int i = lane; i < cnt * 8; i += 32) {
+        const int orow = row0 + (i >> 3), hcol = cur.tile * 8 + (i & 7);
+        Unit u0 = cur;
+        u0.part = 0;
+        const float2* src = gsh_at(p, u0, orow, hcol);
+        float gs = 0.f, us = 0.f;
+        for (int part = 0; part < L.pg; ++part) {
+            const float2 v = __ldcg(src + part * part_stride);
+            gs += v.x;
+            us += v.y;
+        }
+        const float hv = silu_f(gs) * us;
+        range_ok &= in_f16_range(hv);
+        if (q3) p.h[(size_t)orow * p.I + hcol] = f32_to_f16_bits(hv);
+        else p.hf[(size_t)orow * p.I + hcol] = hv;
+    }
+    if (!__all_sync(0xffffffffu, range_ok) && lane == 0) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 0x20);
+}
+
 // y[t][16 tile + r] for every token t and r < 16: the routed rows weighted by their gates
-// in slot order, then the shared rows, summed in fp32 and stored as bf16.  Loads go out
-// four rows at a time.
-__device__ __forceinline__ void combine_slice(const FfnArgs& p, int tile, int lane) {
+// in slot order, then the shared rows, summed in fp32 and stored as bf16.  A row's value
+// is the sum of its pd K parts, in part order.  Loads go out four rows at a time.
+__device__ __forceinline__ void combine_slice(const FfnArgs& p, int tile, int pd, int lane) {
     const int nrows = p.k + p.S;
+    const size_t part_stride = (size_t)p.T * (p.k + p.S) * p.H;
     for (int i = lane; i < p.T * 16; i += 32) {
         const int tok = i >> 4, col = tile * 16 + (i & 15);
         float y = 0.f;
@@ -845,7 +929,12 @@ __device__ __forceinline__ void combine_slice(const FfnArgs& p, int tile, int la
                 } else if (r < nrows) {
                     row = p.T * p.k + (r - p.k) * p.T + tok;
                 }
-                v[u] = row >= 0 ? __ldcg(p.ypart + (size_t)row * p.H + col) : 0.f;
+                v[u] = 0.f;
+                if (row >= 0) {
+                    const float* src = p.ypart + (size_t)row * p.H + col;
+                    v[u] = __ldcg(src);
+                    for (int part = 1; part < pd; ++part) v[u] += __ldcg(src + part * part_stride);
+                }
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -916,7 +1005,13 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
     L.td = p.H / 16;
     L.nch = (p.H / 64 + CG - 1) / CG;
     L.nci = (p.I / 64 + CG - 1) / CG;
-    L.nsgu = p.S * L.tg;
+    L.S = p.S;
+    // K parts (no empty part: the part count is re-derived from the chunks per part)
+    L.cpg = (L.nch + max(1, p.fpg) - 1) / max(1, p.fpg);
+    L.pg = (L.nch + L.cpg - 1) / L.cpg;
+    L.cpd = (L.nci + max(1, p.fpd) - 1) / max(1, p.fpd);
+    L.pd = (L.nci + L.cpd - 1) / L.cpd;
+    L.nsgu = p.S * L.tg * L.pg;
     L.pre = L.nops + L.nsgu;
     L.nr = -1;
     L.total = L.pre;
@@ -928,6 +1023,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
     IB.bq = reinterpret_cast<const uint4*>(p.iq);
     IB.pq = reinterpret_cast<const float2*>(p.iq + iq_pair_off(p.T, p.H));
     const int GI = p.I / 64, GI8 = 8 * ((GI + 7) / 8);
+    L.shares = min(L.td, GI8);
     IqBase HB;                                    // the h rows' integer operands (down)
     HB.bq = reinterpret_cast<const uint4*>(p.hq);
     HB.pq = reinterpret_cast<const float2*>(p.hq + iq_pair_off(p.R16, p.I));
@@ -953,7 +1049,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
                 if (nr < 0) stop = true;
                 L.nr = nr < 0 ? 0 : nr;
                 L.t_ok = tok != 0;
-                L.total = L.pre + L.nr * L.tg + p.S * L.td + L.nr * L.td;
+                L.total = L.pre + L.nr * L.tg + (p.S + L.nr) * L.td * L.pd;
                 cur = resolve(p, L, cur.idx);
                 if (Q.nxt.kind == U_NONE) Q.nxt = resolve(p, L, Q.nxt.idx);
             }
@@ -991,13 +1087,13 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
             if (ready && dn) ready = wait_counter(&fc->gu_done[cur.slot], (uint32_t)L.tg, fc, ctrl, kDetWaitFull | 0x22, lane);
             if (dn && !q3) {
                 // integer down pass: h of this expert on a 12-bit grid per 64-group, formed
-                // by the expert's first down tiles (a share each), waited for by all
-                const int shares = min(L.td, GI8);
-                if (cur.tile < shares) {
+                // by K part 0 of the expert's first down tiles (a share each), waited for by all
+                if (cur.tile < L.shares && cur.part == 0) {
                     if (ready) quantise_h_share(p, cs, cur, L.td, lane);
                     signal_counter(&fc->hq_done[cur.slot], lane);
                 }
-                if (ready) ready = wait_counter(&fc->hq_done[cur.slot], (uint32_t)shares, fc, ctrl, kDetWaitFull | 0x23, lane);
+                if (ready)
+                    ready = wait_counter(&fc->hq_done[cur.slot], (uint32_t)L.shares, fc, ctrl, kDetWaitFull | 0x23, lane);
             }
             if (!dn && !q3) {
                 if (cnt <= 4) unit_iq<0, 1>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
@@ -1015,15 +1111,23 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
                 else unit_bf<1, true, 2>(p, L, cs, cur, Q, R, stop, ready, zq3, 0, G8, fc, pol, lane);
             }
             stop = stop || !ready;
-            if (!dn) {
+            if (!dn && gu_split(cur, L)) {
+                // the last K part of a shared gate/up tile forms its h
+                uint32_t* ctr = &p.gp_done[cur.slot * L.tg + cur.tile];
+                if (signal_counter(ctr, lane) == (uint32_t)L.pg - 1) {
+                    (void)ld_acquire(ctr);
+                    if (!stop) finish_shared_gu(p, L, cs, cur, lane);
+                    signal_counter(&fc->gu_done[cur.slot], lane);
+                }
+            } else if (!dn) {
                 signal_counter(&fc->gu_done[cur.slot], lane);
             } else {
-                const uint32_t n_slots = (uint32_t)(L.nr + p.S);
+                const uint32_t n_parts = (uint32_t)((L.nr + p.S) * L.pd);
                 const uint32_t old = signal_counter(&p.dn_done[cur.tile], lane);
-                if (old == n_slots - 1 && !stop && L.t_ok) {
-                    // the last expert of this 16-row slice: combine it (slot order, fixed)
+                if (old == n_parts - 1 && !stop && L.t_ok) {
+                    // the last expert part of this 16-row slice: combine it (fixed order)
                     (void)ld_acquire(&p.dn_done[cur.tile]);
-                    combine_slice(p, cur.tile, lane);
+                    combine_slice(p, cur.tile, L.pd, lane);
                 }
             }
         }
@@ -1053,6 +1157,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
             fc->hq_done[i] = 0;
         }
         for (int i = lane; i < p.H / 16; i += 32) p.dn_done[i] = 0;
+        for (int i = lane; i < L.tg; i += 32) p.gp_done[i] = 0;
         __syncwarp();
         if (lane == 0) {
             fc->work = 0;

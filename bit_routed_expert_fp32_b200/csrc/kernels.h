@@ -55,6 +55,10 @@ struct FfnArgs {
     float* hf;               // ws fp32 [R16][I]: h of ternary / 2-bit experts (fused kernel)
     uint8_t* hq;             // ws integer operands of those h rows (iq_size(R16, I))
     int R16;                 // rows those two regions hold: min(T, kFusedMaxT) (k + S)
+    float* gsh;              // ws fp32 pairs [fpg][S*T][I] x {gate, up}: the shared experts'
+                             // gate/up K-part sums (fused kernel, fpg > 1; in the ypart region)
+    uint32_t* gp_done;       // ws [2I/16]: K parts finished per shared gate/up tile (fused kernel)
+    int fpg, fpd;            // fused kernel K parts: shared gate/up tiles, every down tile
 };
 
 // Workspace layout for T tokens (api.cu).  The control block, tile counters and the
@@ -114,6 +118,25 @@ inline void decode_kparts(const moe_shape* s, int64_t T, int* nkp_gu, int* nkp_d
     };
     *nkp_gu = pick(s->hidden, 2 * s->inter);
     *nkp_dn = pick(s->inter, s->hidden);
+}
+
+// K parts of the fused decode kernel (T <= kFusedMaxT).  The shared expert's gate/up
+// tiles are split into fpg parts so that they finish with the routed experts' (one
+// shared tile has all T tokens, a routed tile one or two); every down tile into fpd
+// parts at one or two tokens, so that the down pass (nine experts x H/16 tiles) fills
+// the GPU in more, shorter waves.  The parts are summed in a fixed order.  Their sums
+// live in the ypart region: the down parts [fpd][T (k + S)][H] fp32, then the shared
+// gate/up parts [fpg][S T][I] x {gate, up} fp32 (fused_ypart_floats in all).
+inline void fused_kparts(const moe_shape* s, int64_t T, int* fpg, int* fpd) {
+    const int nch = (int)((s->hidden / 64 + 7) / 8), nci = (int)((s->inter / 64 + 7) / 8);
+    *fpg = s->n_shared ? (nch < 4 ? nch : 4) : 1;
+    *fpd = T <= 2 && nci >= 2 ? 2 : 1;
+}
+inline size_t fused_ypart_floats(const moe_shape* s, int64_t T) {
+    int fpg = 1, fpd = 1;
+    fused_kparts(s, T, &fpg, &fpd);
+    const size_t dn = (size_t)fpd * T * (s->top_k + s->n_shared) * s->hidden;
+    return dn + (fpg > 1 ? (size_t)fpg * s->n_shared * T * 2 * s->inter : 0);
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
