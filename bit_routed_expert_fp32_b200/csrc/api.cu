@@ -25,8 +25,8 @@ Ws ws_layout(const moe_shape* s, int64_t T) {
     size_t off = 0;
     w.ctrl = off;
     off += 4096;
-    w.tile_ctr = off;                                   // [H/16] down, then [2I/16] gate/up
-    off = align256(off + 4 * (size_t)(H / 16 + 2 * I / 16));
+    w.tile_ctr = off;                         // [H/16] down, then the gate/up part counters
+    off = align256(off + 4 * (size_t)(H / 16 + fused_gp_counters(s)));
     w.active = off;
     off = align256(off + 4 * (size_t)(E + S));
     w.logits = off;
@@ -206,8 +206,8 @@ moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x, con
     a.zx = reinterpret_cast<float*>(ws + w.zx);
     // The decode operands are formed by the router only for the decode kernels that do
     // not form them themselves (more than kFusedMaxT tokens).
-    a.ops = T > kFusedMaxT;
-    a.iq = nullptr;
+    a.ops = 1;                                            // the decode operands
+    a.iq = T <= kFusedMaxT ? ws + w.iq : nullptr;         // and the integer records
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.r = *out;
     if (launch_route(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -234,8 +234,8 @@ moe_status moe_route_fixed(const moe_shape* shape, int32_t T, const uint16_t* d_
     a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
     a.active = reinterpret_cast<int32_t*>(ws + w.active);
     a.zx = reinterpret_cast<float*>(ws + w.zx);
-    a.ops = T > kFusedMaxT;
-    a.iq = nullptr;
+    a.ops = 1;                                            // the decode operands
+    a.iq = T <= kFusedMaxT ? ws + w.iq : nullptr;         // and the integer records
     a.fixed_ids = d_ids;
     a.fixed_w = d_gates;
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
@@ -300,12 +300,11 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.hq = ws + w.hq;
     a.R16 = (T < kFusedMaxT ? T : kFusedMaxT) * (a.k + a.S);
     a.gp_done = a.dn_done + a.H / 16;
-    a.fpg = a.fpd = 1;
-    if (T >= 1 && T <= kFusedMaxT) fused_kparts(shape, T, &a.fpg, &a.fpd);
+    a.fk = fused_kparts(shape, T >= 1 && T <= kFusedMaxT ? T : 1);
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.h = reinterpret_cast<uint16_t*>(ws + w.h);
     a.ypart = reinterpret_cast<float*>(ws + w.ypart);
-    a.gsh = a.ypart + (size_t)a.fpd * T * (a.k + a.S) * a.H;
+    a.gsh = a.ypart + (size_t)a.fk.pd * T * (a.k + a.S) * a.H;
     a.gpart = a.ypart;
     a.nkp_gu = a.nkp_dn = 1;
     a.tile_ctr = reinterpret_cast<uint32_t*>(ws + w.tile_ctr);

@@ -48,7 +48,7 @@ static_assert(sizeof(Ctrl) == 256, "control block layout");
 constexpr int kMaxSlots = 272;              // expert slots: shared experts, then routed (>= E + S)
 struct FusedCtl {
     uint32_t work;          // next work unit to hand out
-    uint32_t ops_done;      // operand units finished
+    uint32_t spare;
     uint32_t warps_done;    // warps that have left the unit loop
     uint32_t abort;         // set when a wait ran out: every warp stops working
     uint32_t pad[12];

@@ -1,6 +1,6 @@
 // The decode forward for few tokens (1 <= T <= 16) as ONE persistent kernel: the
-// token operands, the gate/up + SwiGLU pass and the down pass of every selected expert
-// and of the shared expert, and the gate-weighted combine into y.
+// gate/up + SwiGLU pass and the down pass of every selected expert and of the shared
+// expert, and the gate-weighted combine into y.
 //
 // Decode speed is set by the expert bytes moved per token (ossradar.top, Xolotl README,
 // "Fast mode (DeepSeek-V4.1)"), and each selected expert is read once for all of its
@@ -9,22 +9,23 @@
 // a ramp and a tail each) between its phases; instead the phases are units of work in
 // one queue and wait on each other through counters in the workspace:
 //
-//   operands  (token, 64-wide group): the integer path's token digits and factors and
-//             the Z tables, formed from the bf16 tokens (operands.cuh)
-//   gate/up   (expert, 16-row tile of the fused gate/up matrix, all of K): needs the
-//             operands; h = silu(gate) * up in fp16
-//   down      (expert, 16-row tile of the down matrix, all of K): needs every gate/up
-//             tile of its expert; fp32 rows of y_e
+//   gate/up   (expert, 16-row tile of the fused gate/up matrix, all of K or one of
+//             its K parts): h = silu(gate) * up (fp16 for the bf16 down path, fp32
+//             for the integer one); a split tile's last part sums the parts in order
+//   down      (expert, 16-row tile of the down matrix, all of K or one K part): needs
+//             every gate/up tile of its expert (and, on the integer path, the expert's
+//             h operands, formed by its first down units); fp32 rows of y_e
 //   combine   the down unit that finishes a 16-row slice of y last for all experts
-//             sums the slice's rows, the routed ones weighted by their gates in slot
-//             order, plus the shared expert's, and stores bf16 (deterministic)
+//             and parts sums the slice's rows, the routed ones weighted by their gates
+//             in slot order, plus the shared expert's, and stores bf16 (deterministic)
 //
 // Units are handed out in that order from one counter (one unit ahead of need), so
 // every wait is for a unit some running warp already holds: the queue cannot deadlock,
-// whatever the number of resident CTAs.  The shared expert does not depend on the
-// routing: its units come first and run while the router kernel, launched just
-// before with programmatic dependent launch, is still choosing the experts;
-// griddepcontrol.wait is executed only by warps that reach a routed unit.
+// whatever the number of resident CTAs.  The shared expert's gate/up tiles come
+// first (every token's chain runs through them), split into K parts when the gate/up
+// tiles of all experts do not fit in one wave of warps.  The token operands (the integer path's digit records, the Z tables) are formed by the
+// router launch this kernel follows (programmatic dependent launch: the prologue
+// overlaps the router's tail, griddepcontrol.wait comes before the first unit).
 //
 // Inside a unit a warp streams its tile's 8-group chunks (codes, third bits, fp16
 // scales: contiguous blocks of the packed format) through its own ring of NS
@@ -42,7 +43,7 @@
 // counters, so the next launch starts from zero.
 #include "kernels.h"
 #include "dequant.cuh"
-#include "operands.cuh"
+#include "operands.cuh"      // iq_group: the down pass forms its h operands
 
 namespace moe {
 namespace {
@@ -61,6 +62,15 @@ constexpr long long kWaitLimit = 4000000000LL;   // clock cycles (~2 s)
 constexpr uint32_t kIqMagic = 0x4B400000u;       // 1.5 * 2^23
 constexpr float kIqMagicF = 12582912.0f;
 constexpr size_t kFusedSmem = (size_t)NW * NS * STAGE + (size_t)NW * NS * 8;
+// At up to kStageMaxT tokens the tokens' integer records and pairs (iq_size(T, H): 15 KB
+// a token at H = 7168) are copied once per CTA into shared memory behind the rings:
+// every routed gate/up tile of the launch reads the same few tokens, and shared-memory
+// loads have a short, fixed latency where L1 hits do not (and an acquire load clears L1).
+#ifndef MOE_STAGE_TOKENS
+#define MOE_STAGE_TOKENS 1
+#endif
+constexpr int kStageMaxT = MOE_STAGE_TOKENS ? 2 : 0;
+inline size_t fused_smem_bytes(int T, int H) { return kFusedSmem + (T <= kStageMaxT ? iq_size(T, H) : 0); }
 
 static_assert(MAXP * 4 >= kFusedMaxT && MAXPB * 8 >= kFusedMaxT, "passes cover kFusedMaxT tokens");
 
@@ -156,18 +166,18 @@ __device__ __forceinline__ const PackedEntry* pentry(const uint8_t* packed, int 
 }
 
 // ---- the work queue --------------------------------------------------------------------
-enum : int { U_NONE = 0, U_OPS = 1, U_GU = 2, U_DN = 3, U_PENDING = 4 };   // PENDING: not taken yet
+enum : int { U_NONE = 0, U_GU = 2, U_DN = 3, U_PENDING = 4 };   // PENDING: not taken yet
 
-struct Layout {        // unit index ranges; the routed ones are known once routing is
-    int nops, nsgu, pre;        // operands, shared gate/up; pre = nops + nsgu
+struct Layout {        // unit index ranges (resolve)
+    int nsgu;                   // shared gate/up units (tiles x K parts)
     int tg, td;                 // 16-row tiles per expert: gate/up (2I/16), down (H/16)
     int nch, nci;               // 8-group chunks per row: gate/up (K = H), down (K = I)
     int S;                      // shared experts (their slots come first)
-    int pg, pd;                 // K parts: shared experts' gate/up tiles, every down tile
-    int cpg, cpd;               // chunks per part
+    int pg, pr, pd;             // K parts: shared gate/up tiles, routed gate/up tiles, down tiles
+    int cpg, cpr, cpd;          // chunks per part
     int shares;                 // down tiles per expert that form the h operands (integer path)
-    int nr;                     // routed experts with tokens (-1: not read yet)
-    int total;                  // all units (pre until routing is known)
+    int nr;                     // routed experts with tokens
+    int total;                  // all units
     bool t_ok;                  // the routing is for this call's T
 };
 
@@ -257,8 +267,12 @@ __device__ __noinline__ int read_routing(CtaState& cs, const FfnArgs& p, int lan
     return ok ? *reinterpret_cast<volatile int*>(&cs.nr) : -1;
 }
 
-// Unit u -> its kind, slot and tile.  Units at or past L.pre need the routing; until it
-// has been read they come back as U_NONE with idx = u.
+// Unit u -> its kind, slot, tile and K part (U_NONE past the last unit).  The order:
+// the shared experts' gate/up tiles (K parts fastest; every token goes through them,
+// so they are the longest chain), the routed experts' gate/up tiles (slot order),
+// then the down tiles: every slot's first `shares` tiles (they form the integer
+// path's h operands) before the rest, slots in order (the shared ones first), tiles
+// ascending, K parts fastest.
 __device__ __forceinline__ Unit resolve(const FfnArgs& p, const Layout& L, int u) {
     Unit U;
     U.kind = U_NONE;
@@ -266,14 +280,10 @@ __device__ __forceinline__ Unit resolve(const FfnArgs& p, const Layout& L, int u
     U.slot = 0;
     U.tile = 0;
     U.part = 0;
-    if (u < 0) return U;
-    if (u < L.nops) {
-        U.kind = U_OPS;
-        U.tile = u;
-        return U;
-    }
-    if (u < L.pre) {                        // shared gate/up: (slot, tile, K part), part fastest
-        const int v = u - L.nops, per = L.tg * L.pg;
+    if (u < 0 || u >= L.total) return U;
+    int v = u;
+    if (v < L.nsgu) {
+        const int per = L.tg * L.pg;
         U.kind = U_GU;
         U.slot = v / per;
         const int r = v - U.slot * per;
@@ -281,49 +291,50 @@ __device__ __forceinline__ Unit resolve(const FfnArgs& p, const Layout& L, int u
         U.part = r - U.tile * L.pg;
         return U;
     }
-    if (L.nr < 0 || u >= L.total) return U;
-    int v = u - L.pre;
-    if (v < L.nr * L.tg) {
-        const int a = v / L.tg;
+    v -= L.nsgu;
+    if (v < L.nr * L.tg * L.pr) {
+        const int per = L.tg * L.pr, a = v / per;
+        const int r = v - a * per;
         U.kind = U_GU;
-        U.tile = v - a * L.tg;
         U.slot = p.S + a;
+        U.tile = r / L.pr;
+        U.part = r - U.tile * L.pr;
         return U;
     }
-    // down: every slot's first `shares` tiles (they form the h operands) before the rest;
-    // within each, slots in order (shared first), tiles ascending, K parts fastest
-    v -= L.nr * L.tg;
+    v -= L.nr * L.tg * L.pr;
     U.kind = U_DN;
     const int n_slots = p.S + L.nr;
     const int b1 = L.shares * L.pd, rest = (L.td - L.shares) * L.pd;
-    int r;
+    int d, r;
     if (v < n_slots * b1) {
-        U.slot = v / b1;
-        r = v - U.slot * b1;
+        d = v / b1;
+        r = v - d * b1;
     } else {
         v -= n_slots * b1;
-        U.slot = v / rest;
-        r = v - U.slot * rest + b1;
+        d = v / rest;
+        r = v - d * rest + b1;
     }
+    U.slot = d;
     U.tile = r / L.pd;
     U.part = r - U.tile * L.pd;
     return U;
 }
 
 __device__ __forceinline__ bool streams(const Unit& U) { return U.kind == U_GU || U.kind == U_DN; }
-// The unit's chunks: [c0, c0 + n) of its matrix's K (one K part of it, if split; the
-// routed experts' gate/up tiles are not split and have part 0).
-__device__ __forceinline__ int unit_c0(const Unit& U, const Layout& L) {
-    return U.part * (U.kind == U_DN ? L.cpd : L.cpg);
+// The unit's chunks: [c0, c0 + n) of its matrix's K (one K part of it, if split).
+__device__ __forceinline__ int unit_cpp(const Unit& U, const Layout& L) {      // chunks per part
+    return U.kind == U_DN ? L.cpd : (U.slot < L.S ? L.cpg : L.cpr);
 }
+__device__ __forceinline__ int unit_c0(const Unit& U, const Layout& L) { return U.part * unit_cpp(U, L); }
 __device__ __forceinline__ int unit_nc(const Unit& U, const Layout& L) {
     const int c0 = unit_c0(U, L);
-    if (U.kind == U_DN) return min(L.nci, c0 + L.cpd) - c0;
-    return U.slot < L.S ? min(L.nch, c0 + L.cpg) - c0 : L.nch;
+    return min(U.kind == U_DN ? L.nci : L.nch, c0 + unit_cpp(U, L)) - c0;
 }
-// A shared expert's gate/up tile split into K parts: the parts' sums go to gsh.
+// K parts of a gate/up tile of this unit's slot
+__device__ __forceinline__ int gu_parts(const Unit& U, const Layout& L) { return U.slot < L.S ? L.pg : L.pr; }
+// A gate/up tile split into K parts: the parts' sums go to gsh, the last part forms h.
 __device__ __forceinline__ bool gu_split(const Unit& U, const Layout& L) {
-    return U.kind == U_GU && U.slot < L.S && L.pg > 1;
+    return U.kind == U_GU && gu_parts(U, L) > 1;
 }
 
 // The warp's next unit, taken from the launch's counter only when the ring is about to
@@ -379,9 +390,12 @@ __device__ __forceinline__ void issue_chunk(Ring& R, const CtaState& cs, const F
 }
 
 // Keeps up to NS chunks in flight: the current unit's, then the next unit's (if it is
-// known and streams).  Stops issuing after an abort.
+// known and streams).  The next unit is taken only once the current one has passed its
+// waits (allow_next): a warp waiting on a dependency holds one unit, not two.  Stops
+// issuing after an abort.
 __device__ __forceinline__ void top_up(Ring& R, const CtaState& cs, const Unit& cur, Queue& Q, bool stop,
-                                       uint64_t pol, int lane, const FfnArgs& p, const Layout& L) {
+                                       uint64_t pol, int lane, const FfnArgs& p, const Layout& L,
+                                       bool allow_next = true) {
     if (stop) return;
     while (R.issued - R.consumed < NS) {
         if (R.iw == 0) {
@@ -389,6 +403,7 @@ __device__ __forceinline__ void top_up(Ring& R, const CtaState& cs, const Unit& 
                 issue_chunk(R, cs, p, cur, unit_c0(cur, L) + R.ic++, pol);
                 continue;
             }
+            if (!allow_next) break;
             R.iw = 1;
             R.ic = 0;
             take_next(Q, p, L, lane);
@@ -465,16 +480,27 @@ struct IqBase {
 
 __device__ __forceinline__ void imma2(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
                                       uint32_t a5, uint32_t a6, uint32_t a7, const uint4& b) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%10,%11,%10,%11};"
         : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y), "r"(kIqMagic), "r"(0));
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a4), "r"(a5), "r"(a6), "r"(a7), "r"(b.z), "r"(b.w));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float2 lds64f(uint32_t a) {
+    float2 v;
+    asm("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
 }
 
 // o4 = 4 o: 4 for ternary codes, 6 for 2-bit codes (the offset removed exactly, in the
@@ -517,7 +543,9 @@ __device__ __forceinline__ void chunk_gu_iq(const uint8_t* stg, int c, int ng, c
 // chunk are at fixed offsets from one pointer each; the scales of the chunk come in
 // with one 16-byte load per row; and the code offset is folded into the accumulator's
 // start value, M - o4 sum q, so the low digit's sum comes out already corrected.
-template <int NP>
+// STG: the records and pairs are in shared memory (B points there; read with ld.shared,
+// which never changes during the launch once staged).
+template <int NP, bool STG>
 __device__ __forceinline__ void chunk_iq_full(const uint8_t* stg, int c, const IqView<NP>& v, const IqBase& B, int np,
                                               int o4, int sw, int g, unsigned long long (&acc)[NP]) {
     const uint4 sg4 = *reinterpret_cast<const uint4*>(stg + OFF_SC + 16 * g);
@@ -525,10 +553,15 @@ __device__ __forceinline__ void chunk_iq_full(const uint8_t* stg, int c, const I
     const uint32_t sg[4] = {sg4.x, sg4.y, sg4.z, sg4.w}, su[4] = {su4.x, su4.y, su4.z, su4.w};
     const uint4* rec[NP];
     const float2* prs[NP];
+    uint32_t rec_s[NP], prs_s[NP];
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
         rec[q] = B.bq + v.bq[q] + 64 * c;
         prs[q] = B.pq + v.pq[q] + CG * c;
+        if (STG) {
+            rec_s[q] = (uint32_t)__cvta_generic_to_shared(rec[q]);
+            prs_s[q] = (uint32_t)__cvta_generic_to_shared(prs[q]);
+        }
     }
 #pragma unroll(NP == 1 ? 8 : 2)
     for (int gl = 0; gl < CG; ++gl) {
@@ -545,16 +578,16 @@ __device__ __forceinline__ void chunk_iq_full(const uint8_t* stg, int c, const I
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
             if (NP == 1 || q < np) {
-                const uint4 b = rec[q][8 * gl];
-                const float2 pr = prs[q][gl];
+                const uint4 b = STG ? lds128(rec_s[q] + 128 * gl) : rec[q][8 * gl];
+                const float2 pr = STG ? lds64f(prs_s[q] + 8 * gl) : prs[q][gl];
                 const int c0 = (int)kIqMagic - o4 * __float_as_int(pr.y);
                 int d[4];
-                asm volatile(
+                asm(
                     "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
                     "{%10,%11,%10,%11};"
                     : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
                     : "r"(m0), "r"(m1), "r"(n0), "r"(n1), "r"(b.x), "r"(b.y), "r"(c0), "r"(0));
-                asm volatile(
+                asm(
                     "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
                     "{%0,%1,%2,%3};"
                     : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -685,8 +718,8 @@ __device__ __forceinline__ void release_stage(Ring& R) {
 // Where a unit's fp32 results go: a split shared gate/up tile's {gate, up} sums of K part
 // U.part (gsh, rows of the shared experts only), and a down tile's rows of y_e for K part
 // U.part (ypart [part][T (k + S)][H]).
-__device__ __forceinline__ float2* gsh_at(const FfnArgs& p, const Unit& U, int orow, int hcol) {
-    return reinterpret_cast<float2*>(p.gsh) + ((size_t)U.part * p.S * p.T + (orow - p.T * p.k)) * p.I + hcol;
+__device__ __forceinline__ float2* gsh_at(const FfnArgs& p, int part, int orow, int hcol) {
+    return reinterpret_cast<float2*>(p.gsh) + ((size_t)part * p.fk.gsh_rows + (orow - p.fk.gsh_row0)) * p.I + hcol;
 }
 __device__ __forceinline__ float* ypart_at(const FfnArgs& p, const Unit& U, int orow, int col) {
     return p.ypart + ((size_t)U.part * p.T * (p.k + p.S) + orow) * p.H + col;
@@ -696,7 +729,7 @@ __device__ __forceinline__ float* ypart_at(const FfnArgs& p, const Unit& U, int 
 // MODE 0 (gate/up): B = the tokens' digit records, output h = silu(gate) * up in fp32
 // (hf, quantised later for the down pass); MODE 1 (down): B = the expert's h rows'
 // digit records, output fp32 rows of y_e (ypart).
-template <int MODE, int NP>
+template <int MODE, int NP, bool STG = false>
 __device__ __forceinline__ void unit_iq(const FfnArgs& p, const Layout& L, const CtaState& cs, const Unit& cur,
                                         Queue& Q, Ring& R, bool& stop, bool ready, const IqBase& B, int G, int G8,
                                         FusedCtl* fc, uint64_t pol, int lane) {
@@ -726,7 +759,7 @@ __device__ __forceinline__ void unit_iq(const FfnArgs& p, const Layout& L, const
         if (!stg) break;
         const int ng = min(CG, GK - c * CG);
         if (ready && !stop) {
-            if (ng == CG) chunk_iq_full<NP>(stg, c, v, B, np, o4, sw, g, acc);
+            if (ng == CG) chunk_iq_full<NP, STG>(stg, c, v, B, np, o4, sw, g, acc);
             else chunk_gu_iq<NP, false>(stg, c, ng, v, B, np, o4, g, t, acc);
         }
         release_stage(R);
@@ -743,7 +776,7 @@ __device__ __forceinline__ void unit_iq(const FfnArgs& p, const Layout& L, const
                 if (q < np && v.orow[q] >= 0) {
                     const float2 a = up2(acc[q]);
                     if (split) {
-                        *gsh_at(p, cur, v.orow[q], hcol) = a;
+                        *gsh_at(p, cur.part, v.orow[q], hcol) = a;
                     } else {
                         const float hv = silu_f(a.x) * a.y;
                         range_ok &= in_f16_range(hv);
@@ -856,7 +889,7 @@ __device__ __forceinline__ void unit_bf(const FfnArgs& p, const Layout& L, const
             for (int cc = 0; cc < 2; ++cc)
                 if (q < np && v.orow[q][cc] >= 0) {
                     if (split) {
-                        *gsh_at(p, cur, v.orow[q][cc], hcol) = make_float2(acc[q][cc], acc[q][2 + cc]);
+                        *gsh_at(p, cur.part, v.orow[q][cc], hcol) = make_float2(acc[q][cc], acc[q][2 + cc]);
                     } else {
                         const float hv = silu_f(acc[q][cc]) * acc[q][2 + cc];
                         range_ok &= in_f16_range(hv);
@@ -879,22 +912,21 @@ __device__ __forceinline__ void unit_bf(const FfnArgs& p, const Layout& L, const
     }
 }
 
-// The last K part of a split shared gate/up tile: h = silu(gate) * up of its 8 columns
-// for the shared expert's rows, from the parts' sums added in part order; fp16 h for a
-// 3-bit expert (the bf16 path's down operand), fp32 hf for the integer path.
-__device__ __forceinline__ void finish_shared_gu(const FfnArgs& p, const Layout& L, const CtaState& cs,
-                                                 const Unit& cur, int lane) {
+// The last K part of a split gate/up tile: h = silu(gate) * up of its 8 columns for
+// the expert's rows, from the parts' sums added in part order; fp16 h for a 3-bit
+// expert (the bf16 path's down operand), fp32 hf for the integer path.
+__device__ __forceinline__ void finish_gu(const FfnArgs& p, const Layout& L, const CtaState& cs, const Unit& cur,
+                                          int lane) {
     const int cnt = cs.slot[cur.slot].cnt, row0 = cs.slot[cur.slot].row0;
     const bool q3 = cs.slot[cur.slot].fmt == MOE_FMT_Q3;
-    const size_t part_stride = (size_t)p.S * p.T * p.I;
+    const size_t part_stride = (size_t)p.fk.gsh_rows * p.I;
+    const int parts = gu_parts(cur, L);
     bool range_ok = true;
     for (int i = lane; i < cnt * 8; i += 32) {
         const int orow = row0 + (i >> 3), hcol = cur.tile * 8 + (i & 7);
-        Unit u0 = cur;
-        u0.part = 0;
-        const float2* src = gsh_at(p, u0, orow, hcol);
+        const float2* src = gsh_at(p, 0, orow, hcol);
         float gs = 0.f, us = 0.f;
-        for (int part = 0; part < L.pg; ++part) {
+        for (int part = 0; part < parts; ++part) {
             const float2 v = __ldcg(src + part * part_stride);
             gs += v.x;
             us += v.y;
@@ -909,40 +941,38 @@ __device__ __forceinline__ void finish_shared_gu(const FfnArgs& p, const Layout&
 
 // y[t][16 tile + r] for every token t and r < 16: the routed rows weighted by their gates
 // in slot order, then the shared rows, summed in fp32 and stored as bf16.  A row's value
-// is the sum of its pd K parts, in part order.  Loads go out four rows at a time.
+// is the sum of its pd K parts, in part order.  The loads of an output go out in two
+// rounds: the row indices and gates of eight slots (and the shared rows' values), then
+// those slots' values.
+__device__ __forceinline__ float ypart_row(const FfnArgs& p, int row, int col, int pd, size_t part_stride) {
+    const float* src = p.ypart + (size_t)row * p.H + col;
+    float v = __ldcg(src);
+    for (int part = 1; part < pd; ++part) v += __ldcg(src + part * part_stride);
+    return v;
+}
+
 __device__ __forceinline__ void combine_slice(const FfnArgs& p, int tile, int pd, int lane) {
-    const int nrows = p.k + p.S;
     const size_t part_stride = (size_t)p.T * (p.k + p.S) * p.H;
     for (int i = lane; i < p.T * 16; i += 32) {
         const int tok = i >> 4, col = tile * 16 + (i & 15);
+        const float ysh = p.S ? ypart_row(p, p.T * p.k + tok, col, pd, part_stride) : 0.f;   // S <= 1
         float y = 0.f;
-        for (int r0 = 0; r0 < nrows; r0 += 4) {
-            float v[4], gw[4];
+        for (int r0 = 0; r0 < p.k; r0 += 8) {
+            int row[8];
+            float gw[8], v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = r0 + u;
-                int row = -1;
-                gw[u] = 1.f;
-                if (r < p.k) {
-                    row = __ldcg(p.inv_perm + (size_t)tok * p.k + r);
-                    gw[u] = __ldcg(p.topk_w + (size_t)tok * p.k + r);
-                } else if (r < nrows) {
-                    row = p.T * p.k + (r - p.k) * p.T + tok;
-                }
-                v[u] = 0.f;
-                if (row >= 0) {
-                    const float* src = p.ypart + (size_t)row * p.H + col;
-                    v[u] = __ldcg(src);
-                    for (int part = 1; part < pd; ++part) v[u] += __ldcg(src + part * part_stride);
-                }
+            for (int u = 0; u < 8; ++u) {
+                const bool on = r0 + u < p.k;
+                row[u] = on ? __ldcg(p.inv_perm + (size_t)tok * p.k + r0 + u) : -1;
+                gw[u] = on ? __ldcg(p.topk_w + (size_t)tok * p.k + r0 + u) : 0.f;
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = r0 + u;
-                if (r < p.k) y = fmaf(gw[u], v[u], y);
-                else if (r < nrows) y += v[u];
-            }
+            for (int u = 0; u < 8; ++u) v[u] = row[u] >= 0 ? ypart_row(p, row[u], col, pd, part_stride) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (r0 + u < p.k) y = fmaf(gw[u], v[u], y);
         }
+        y += ysh;
         if (p.y_f32) reinterpret_cast<float*>(p.y)[(size_t)tok * p.H + col] = y;
         else p.y[(size_t)tok * p.H + col] = f32_to_bf16_bits(y);
     }
@@ -1000,23 +1030,19 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
 
     const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
     Layout L;
-    L.nops = p.T * G8;                            // one operand unit per (token, group)
     L.tg = 2 * p.I / 16;
     L.td = p.H / 16;
     L.nch = (p.H / 64 + CG - 1) / CG;
     L.nci = (p.I / 64 + CG - 1) / CG;
     L.S = p.S;
     // K parts (no empty part: the part count is re-derived from the chunks per part)
-    L.cpg = (L.nch + max(1, p.fpg) - 1) / max(1, p.fpg);
+    L.cpg = (L.nch + max(1, p.fk.pg) - 1) / max(1, p.fk.pg);
     L.pg = (L.nch + L.cpg - 1) / L.cpg;
-    L.cpd = (L.nci + max(1, p.fpd) - 1) / max(1, p.fpd);
+    L.cpr = (L.nch + max(1, p.fk.pr) - 1) / max(1, p.fk.pr);
+    L.pr = (L.nch + L.cpr - 1) / L.cpr;
+    L.cpd = (L.nci + max(1, p.fk.pd) - 1) / max(1, p.fk.pd);
     L.pd = (L.nci + L.cpd - 1) / L.cpd;
     L.nsgu = p.S * L.tg * L.pg;
-    L.pre = L.nops + L.nsgu;
-    L.nr = -1;
-    L.total = L.pre;
-    L.t_ok = true;
-    const OperandArgs oa{p.T, p.H, p.x, const_cast<float*>(p.zx), const_cast<uint8_t*>(p.iq), ctrl};
     const int zplane_q3 = 3 * p.T * G8;          // hi -> lo plane of the Z tables (elements)
     const uint16_t* zq3 = reinterpret_cast<const uint16_t*>(p.zx) + (size_t)2 * p.T * G8;   // format 2 plane
     IqBase IB;                                    // the tokens' integer operands (gate/up)
@@ -1029,31 +1055,35 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
     HB.pq = reinterpret_cast<const float2*>(p.hq + iq_pair_off(p.R16, p.I));
     const uint64_t pol = l2_policy_evict_first();
 
-    auto grab = [&]() -> int {
-        int u = 0;
-        if (lane == 0) u = (int)atomicAdd(&fc->work, 1u);
-        return __shfl_sync(0xffffffffu, u, 0);
-    };
+    // The routing and the token operands (Z tables, integer records) come from the
+    // router launch this one follows: wait for it, then every unit is known.
     bool stop = !hdr_ok || ld_relaxed(&fc->abort) != 0;
-    bool ops_seen = false;
-    Unit cur = resolve(p, L, grab());
+    {
+        int tok = 0;
+        const int nr = read_routing(cs, p, lane, &tok);
+        if (nr < 0) stop = true;
+        L.nr = nr < 0 ? 0 : nr;
+        L.t_ok = tok != 0;
+        L.total = L.nsgu + L.nr * L.tg * L.pr + (p.S + L.nr) * L.td * L.pd;
+    }
+    const bool staged = p.T <= kStageMaxT;
+    IqBase IBs = IB;
+    if (staged) {                                 // every warp of the CTA is here
+        uint4* dst = reinterpret_cast<uint4*>(smem + kFusedSmem);
+        const uint4* src = reinterpret_cast<const uint4*>(p.iq);
+        const int n16 = (int)(iq_size(p.T, p.H) / 16);
+        for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = __ldcg(src + i);
+        IBs.bq = dst;
+        IBs.pq = reinterpret_cast<const float2*>(smem + kFusedSmem + iq_pair_off(p.T, p.H));
+        __syncthreads();
+    }
     Queue Q;
     Q.nxt.kind = U_PENDING;
-    Q.nxt.idx = -1;
+    take_next(Q, p, L, lane);
+    Unit cur = Q.nxt;
+    Q.nxt.kind = U_PENDING;
     int iters = 0;
     while (true) {
-        if (cur.kind == U_NONE && cur.idx >= L.pre) {
-            if (L.nr < 0) {                       // routed range: the routing is needed
-                int tok = 0;
-                const int nr = read_routing(cs, p, lane, &tok);
-                if (nr < 0) stop = true;
-                L.nr = nr < 0 ? 0 : nr;
-                L.t_ok = tok != 0;
-                L.total = L.pre + L.nr * L.tg + (p.S + L.nr) * L.td * L.pd;
-                cur = resolve(p, L, cur.idx);
-                if (Q.nxt.kind == U_NONE) Q.nxt = resolve(p, L, Q.nxt.idx);
-            }
-        }
         if (cur.kind == U_NONE) break;            // the queue is empty
         if (++iters > L.total + 2) {              // cannot happen with consistent counters
             if (lane == 0) {
@@ -1063,27 +1093,13 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
             break;
         }
         stop = stop || ld_relaxed(&fc->abort) != 0;
-        top_up(R, cs, cur, Q, stop, pol, lane, p, L);
-
-        if (cur.kind == U_OPS) {
-            // ---------------- operands of token tt, group Gi ---------------------------
-            if (!stop) {
-                const int tt = cur.tile / G8, Gi = cur.tile - tt * G8;
-                compute_z(oa, tt, Gi, lane);
-                compute_iq(oa, tt, Gi, lane);
-            }
-            signal_counter(&fc->ops_done, lane);
-        } else {
+        top_up(R, cs, cur, Q, stop, pol, lane, p, L, false);
+        {
             // ---------------- a gate/up or down tile ----------------------------------
             const bool dn = cur.kind == U_DN;
             const int cnt = cs.slot[cur.slot].cnt;
             const bool q3 = cs.slot[cur.slot].fmt == MOE_FMT_Q3;
             bool ready = !stop;
-            if (ready && !dn && !ops_seen) {
-                // the operands are written once per launch: one acquire per warp suffices
-                ready = wait_counter(&fc->ops_done, (uint32_t)L.nops, fc, ctrl, kDetWaitFull | 0x21, lane);
-                ops_seen = ready;
-            }
             if (ready && dn) ready = wait_counter(&fc->gu_done[cur.slot], (uint32_t)L.tg, fc, ctrl, kDetWaitFull | 0x22, lane);
             if (dn && !q3) {
                 // integer down pass: h of this expert on a 12-bit grid per 64-group, formed
@@ -1096,7 +1112,8 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
                     ready = wait_counter(&fc->hq_done[cur.slot], (uint32_t)L.shares, fc, ctrl, kDetWaitFull | 0x23, lane);
             }
             if (!dn && !q3) {
-                if (cnt <= 4) unit_iq<0, 1>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
+                if (staged) unit_iq<0, 1, true>(p, L, cs, cur, Q, R, stop, ready, IBs, G, G8, fc, pol, lane);
+                else if (cnt <= 4) unit_iq<0, 1>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
                 else if (cnt <= 8) unit_iq<0, 2>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
                 else unit_iq<0, 4>(p, L, cs, cur, Q, R, stop, ready, IB, G, G8, fc, pol, lane);
             } else if (dn && !q3) {
@@ -1112,11 +1129,11 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
             }
             stop = stop || !ready;
             if (!dn && gu_split(cur, L)) {
-                // the last K part of a shared gate/up tile forms its h
+                // the last K part of a gate/up tile forms its h
                 uint32_t* ctr = &p.gp_done[cur.slot * L.tg + cur.tile];
-                if (signal_counter(ctr, lane) == (uint32_t)L.pg - 1) {
+                if (signal_counter(ctr, lane) == (uint32_t)gu_parts(cur, L) - 1) {
                     (void)ld_acquire(ctr);
-                    if (!stop) finish_shared_gu(p, L, cs, cur, lane);
+                    if (!stop) finish_gu(p, L, cs, cur, lane);
                     signal_counter(&fc->gu_done[cur.slot], lane);
                 }
             } else if (!dn) {
@@ -1136,7 +1153,6 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
         else R.ic = 0;
         take_next(Q, p, L, lane);
         cur = Q.nxt;
-        if (cur.kind == U_NONE && cur.idx >= L.pre && L.nr >= 0) cur = resolve(p, L, cur.idx);
         Q.nxt.kind = U_PENDING;
     }
 
@@ -1157,11 +1173,11 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
             fc->hq_done[i] = 0;
         }
         for (int i = lane; i < p.H / 16; i += 32) p.dn_done[i] = 0;
-        for (int i = lane; i < L.tg; i += 32) p.gp_done[i] = 0;
+        const int n_ctr = (L.pr > 1 ? p.S + L.nr : p.S) * L.tg;
+        for (int i = lane; i < n_ctr; i += 32) p.gp_done[i] = 0;
         __syncwarp();
         if (lane == 0) {
             fc->work = 0;
-            fc->ops_done = 0;
             fc->abort = 0;
             __threadfence();
             fc->warps_done = 0;
@@ -1173,9 +1189,10 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
 
 cudaError_t launch_ffn_fused(const FfnArgs& a, cudaStream_t s) {
     if (a.T < 1 || a.T > kFusedMaxT || a.E + a.S > kMaxSlots) return cudaErrorInvalidConfiguration;
-    const cudaError_t err = set_smem_limit(ffn_fused_kernel, kFusedSmem);
+    const size_t smem = fused_smem_bytes(a.T, a.H);
+    const cudaError_t err = set_smem_limit(ffn_fused_kernel, smem);
     if (err != cudaSuccess) return err;
-    return launch_pdl(ffn_fused_kernel, dim3(a.num_ctas), dim3(NW * 32), kFusedSmem, s, a);
+    return launch_pdl(ffn_fused_kernel, dim3(a.num_ctas), dim3(NW * 32), smem, s, a);
 }
 
 }  // namespace moe

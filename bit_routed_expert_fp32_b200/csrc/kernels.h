@@ -28,6 +28,12 @@ struct RouteArgs {
     moe_routing r;
 };
 
+// K parts of the fused decode kernel (fused_kparts below)
+struct FusedParts {
+    int pg, pr, pd;
+    int gsh_row0, gsh_rows;      // first row and number of rows with gate/up part sums
+};
+
 struct FfnArgs {
     int T, H, I, E, k, S;
     const uint8_t* packed;
@@ -55,10 +61,10 @@ struct FfnArgs {
     float* hf;               // ws fp32 [R16][I]: h of ternary / 2-bit experts (fused kernel)
     uint8_t* hq;             // ws integer operands of those h rows (iq_size(R16, I))
     int R16;                 // rows those two regions hold: min(T, kFusedMaxT) (k + S)
-    float* gsh;              // ws fp32 pairs [fpg][S*T][I] x {gate, up}: the shared experts'
-                             // gate/up K-part sums (fused kernel, fpg > 1; in the ypart region)
-    uint32_t* gp_done;       // ws [2I/16]: K parts finished per shared gate/up tile (fused kernel)
-    int fpg, fpd;            // fused kernel K parts: shared gate/up tiles, every down tile
+    float* gsh;              // ws fp32 pairs [max(pg, pr)][gsh_rows][I] x {gate, up}: gate/up
+                             // K-part sums (fused kernel; in the ypart region)
+    uint32_t* gp_done;       // ws [fused_gp_counters]: K parts finished per split gate/up tile
+    FusedParts fk;           // fused kernel K parts
 };
 
 // Workspace layout for T tokens (api.cu).  The control block, tile counters and the
@@ -120,23 +126,39 @@ inline void decode_kparts(const moe_shape* s, int64_t T, int* nkp_gu, int* nkp_d
     *nkp_dn = pick(s->inter, s->hidden);
 }
 
-// K parts of the fused decode kernel (T <= kFusedMaxT).  The shared expert's gate/up
-// tiles are split into fpg parts so that they finish with the routed experts' (one
-// shared tile has all T tokens, a routed tile one or two); every down tile into fpd
-// parts at one or two tokens, so that the down pass (nine experts x H/16 tiles) fills
-// the GPU in more, shorter waves.  The parts are summed in a fixed order.  Their sums
-// live in the ypart region: the down parts [fpd][T (k + S)][H] fp32, then the shared
-// gate/up parts [fpg][S T][I] x {gate, up} fp32 (fused_ypart_floats in all).
-inline void fused_kparts(const moe_shape* s, int64_t T, int* fpg, int* fpd) {
+// K parts of the fused decode kernel (T <= kFusedMaxT).  A gate/up tile of a shared
+// expert has all T tokens against a routed tile's one or two, so the shared expert's
+// chain (which every token goes through) is split into pg K parts, unless the gate/up
+// tiles of all experts fit in one wave of warps (148 SMs x 16); at one or two tokens
+// the routed gate/up tiles (pr parts) and every down tile (pd parts) are split too, so
+// that the work comes in shorter units that fill the GPU in several waves.  The last
+// part of a split gate/up tile sums the parts in part order (gp_done counts them);
+// the down parts are summed in part order by the combine.  The sums live in the ypart
+// region: the down parts [pd][T (k + S)][H] fp32, then the gate/up parts
+// [max(pg, pr)][gsh rows][I] x {gate, up} fp32, whose rows are every expert row when
+// routed tiles are split and the shared rows only otherwise.
+// gate/up part counters kept in the workspace: every expert slot's tiles at two tokens
+// if that stays small, else the shared experts' only
+inline int64_t fused_gp_counters(const moe_shape* s) {
+    const int64_t tg = 2 * s->inter / 16, all = (2 * s->top_k + s->n_shared) * tg;
+    return all <= 8192 ? all : s->n_shared * tg;
+}
+inline FusedParts fused_kparts(const moe_shape* s, int64_t T) {
+    FusedParts f = {1, 1, 1, 0, 0};
     const int nch = (int)((s->hidden / 64 + 7) / 8), nci = (int)((s->inter / 64 + 7) / 8);
-    *fpg = s->n_shared ? (nch < 4 ? nch : 4) : 1;
-    *fpd = T <= 2 && nci >= 2 ? 2 : 1;
+    const int64_t tg = 2 * s->inter / 16, gu_tiles = (T * s->top_k + s->n_shared) * tg;
+    if (T <= 2 && gu_tiles <= fused_gp_counters(s)) f.pr = nch < 2 ? nch : 2;
+    if (s->n_shared && (gu_tiles > 148 * 16 || f.pr > 1)) f.pg = nch < 4 ? nch : 4;
+    if (T <= 2 && nci >= 2) f.pd = 2;
+    f.gsh_row0 = f.pr > 1 ? 0 : (int)(T * s->top_k);
+    f.gsh_rows = (int)(f.pr > 1 ? T * (s->top_k + s->n_shared) : T * s->n_shared);
+    return f;
 }
 inline size_t fused_ypart_floats(const moe_shape* s, int64_t T) {
-    int fpg = 1, fpd = 1;
-    fused_kparts(s, T, &fpg, &fpd);
-    const size_t dn = (size_t)fpd * T * (s->top_k + s->n_shared) * s->hidden;
-    return dn + (fpg > 1 ? (size_t)fpg * s->n_shared * T * 2 * s->inter : 0);
+    const FusedParts f = fused_kparts(s, T);
+    const size_t dn = (size_t)f.pd * T * (s->top_k + s->n_shared) * s->hidden;
+    const int pmax = f.pg > f.pr ? f.pg : f.pr;
+    return dn + (pmax > 1 ? (size_t)pmax * f.gsh_rows * 2 * s->inter : 0);
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);

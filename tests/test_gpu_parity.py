@@ -175,6 +175,21 @@ def test_few_token_integer_gate_up_full_chunks(T, shared_format):
     _full_check(cfg, PATHS["decode"])
 
 
+@pytest.mark.parametrize("T,shared_format", [(1, synth.FMT_Q2), (2, synth.FMT_TERNARY), (2, synth.FMT_Q2),
+                                             (2, synth.FMT_Q3), (5, synth.FMT_Q2)])
+def test_shared_gate_up_and_down_in_k_parts(T, shared_format):
+    """Inter 2048 with eight experts a token: at one or two tokens the fused kernel
+    splits every gate/up tile into K parts (their sums added in part order by the last
+    part, which forms h in fp32 for the integer down pass or fp16 for the bf16 one) and
+    every down tile into two; at five tokens the gate/up tiles of all experts exceed
+    one wave of warps and only the shared expert's are split.  Shared expert in each
+    format."""
+    import dataclasses
+    cfg = synth.micro(T=T, H=1024, E=16, k=8, I=2048, S=1, formats="mixed", seed=80 + T)
+    cfg = dataclasses.replace(cfg, shared_format=shared_format)
+    _full_check(cfg, PATHS["decode"])
+
+
 @pytest.mark.parametrize("formats,T,path", [("q2", 1, "decode"), ("mixed", 12, "decode"), ("mixed", 96, "prefill")])
 def test_fast_mode_copy(formats, T, path):
     """The fast mode's second buffer (every 3-bit expert replaced by its 2-bit copy)
