@@ -19,7 +19,7 @@ MOE_OK = 0
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_DEVICE_CHECK"}
 FMT_TERNARY, FMT_Q2, FMT_Q3 = 0, 1, 2
-PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_DECODE_FUSED = 0, 1, 2, 3
 OUT_F32 = 0x10          # OR into a path: moe_forward writes fp32 y
 
 # every symbol include/moe.h declares
@@ -31,7 +31,8 @@ EXPORTS = ["moe_packed_size", "moe_pack_experts", "moe_requantize_q3_to_q2", "mo
            "moe_cache_load"]
 # detail codes beside MOE_ERR_TIMEOUT / MOE_ERR_DEVICE_CHECK (high bits: what; low byte: where)
 DETAIL = {"WAIT_FULL": 0x100, "WAIT_EMPTY": 0x200, "DRAIN": 0x300, "HEADER": 0x400, "ROUTED_T": 0x500,
-          "RANGE": 0x600, "TEST_STALL": 0x700, "LOOP_CAP": 0x800}
+          "RANGE": 0x600, "TEST_STALL": 0x700, "LOOP_CAP": 0x800, "FORMAT": 0x900}
+FMT_TERNARY_DENSE = 3       # storage form of ternary experts (five codes per byte), see moe.h
 STATIC_WS_BYTES = 8 << 20
 
 

@@ -97,6 +97,10 @@ int sm_count() {
     return n;
 }
 
+// The kernels load tokens, router rows, weights and workspace regions in 16-byte
+// pieces (vector loads, bulk copies): every such base pointer must be 16-byte aligned.
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 bool routing_ok(const moe_routing* r) {
     return r && r->topk_ids && r->topk_w && r->counts && r->offsets && r->perm && r->inv_perm;
 }
@@ -116,6 +120,7 @@ moe_status check_route_args(const moe_shape* shape, int32_t T, const uint16_t* d
     const moe_status st = check_common(shape, T, d_ws, ws_bytes);
     if (st != MOE_OK) return st;
     if (!d_x || !d_router_w || !routing_ok(out)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(d_x) || !aligned16(d_router_w) || !aligned16(d_ws)) return MOE_ERR_INVALID_ARG;
     if (ws_fixed_prefix(shape) > 4096 + 65536) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
@@ -126,8 +131,11 @@ moe_status check_forward_args(const moe_shape* shape, int32_t T, const void* d_p
     const moe_status st = check_common(shape, T, d_ws, ws_bytes);
     if (st != MOE_OK) return st;
     if (!d_packed || !d_x || !d_y || !routing_ok(r)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(d_packed) || !aligned16(d_x) || !aligned16(d_y) || !aligned16(d_ws)) return MOE_ERR_INVALID_ARG;
     const int base = (int)path & ~MOE_OUT_F32;
-    if (base != MOE_PATH_AUTO && base != MOE_PATH_DECODE && base != MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+    if (base != MOE_PATH_AUTO && base != MOE_PATH_DECODE && base != MOE_PATH_PREFILL && base != MOE_PATH_DECODE_FUSED)
+        return MOE_ERR_INVALID_ARG;
+    if (base == MOE_PATH_DECODE_FUSED && T > kFusedMaxT) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
@@ -320,7 +328,10 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     const bool tc_ok = a.H % 128 == 0 && (2 * a.I) % 128 == 0;
     if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
     const bool prefill = path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kSmallT && tc_ok);
-    const bool fused = !prefill && T <= kFusedMaxT && a.E + a.S <= kMaxSlots;
+    // the fused decode kernel where it is the faster decode choice (kFusedAutoMinT ..
+    // kFusedAutoMaxT tokens, measured on the full-size layer), or when asked for
+    const bool fused = !prefill && T <= kFusedMaxT && a.E + a.S <= kMaxSlots &&
+                       (path == MOE_PATH_DECODE_FUSED || (T >= kFusedAutoMinT && T <= kFusedAutoMaxT));
     cudaError_t err;
     if (fused) {
         // one kernel: the per-kernel events all follow it

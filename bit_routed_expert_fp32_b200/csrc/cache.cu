@@ -13,6 +13,13 @@
 // (cudaMemcpyAsync, one per expert, and a one-thread kernel for the entry).
 // moe_forward then reads the cache buffer like any packed buffer; which experts must be
 // resident (those the routing selected, and the shared expert) is the caller's choice.
+//
+// A ternary expert may be stored in the host buffer in the dense storage form (five
+// codes per byte: 1.625 bits per weight against 2, i.e. ~18 % fewer bytes to move
+// over PCIe for the expert with its scales).  Its span is copied into a staging area
+// behind the slots and expanded there on the GPU into the kernels' 2-bit ternary
+// layout (one thread per code word; the scales, blocked the same way in both forms,
+// are copied as they are); its table entry then says MOE_FMT_TERNARY.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -45,7 +52,41 @@ struct HostLayer {
     int n;                                 // expert tables (E + S)
     size_t total;                          // bytes of the host buffer
     std::vector<uint64_t> start, end;      // each expert's contiguous span
+    std::vector<uint32_t> fmt;
 };
+
+// Offsets, from the start of an expert's span, of its arrays in the kernels' layout
+// (the packer's order: gate/up scales, codes, third bits; down scales, codes, third
+// bits; each 256-byte aligned), and the span's size.
+struct SpanLayout {
+    uint64_t gs, gc, gh, ds, dc, dh, bytes;
+};
+SpanLayout span_layout(const moe_shape* s, uint32_t fmt) {
+    const uint64_t H = s->hidden, I = s->inter, nch = (H / 64 + 7) / 8, nci = (I / 64 + 7) / 8;
+    SpanLayout L = {};
+    uint64_t off = 0;
+    L.gs = off;
+    off = align256(off + (2 * I / 16) * 256 * nch);
+    L.gc = off;
+    off += 2 * I * H / 4;
+    if (fmt == MOE_FMT_Q3) {
+        off = align256(off);
+        L.gh = off;
+        off += 2 * I * H / 8;
+    }
+    off = align256(off);
+    L.ds = off;
+    off = align256(off + (H / 16) * 256 * nci);
+    L.dc = off;
+    off += H * I / 4;
+    if (fmt == MOE_FMT_Q3) {
+        off = align256(off);
+        L.dh = off;
+        off += H * I / 8;
+    }
+    L.bytes = off;
+    return L;
+}
 
 // Reads the header and expert table of a host packed buffer (format version 2) and
 // finds each expert's span: from its first array to the next expert's first array (or
@@ -60,9 +101,12 @@ bool parse(const moe_shape* s, const uint8_t* h, HostLayer* L) {
     L->total = rd64(h + 32);
     L->start.resize(n);
     L->end.resize(n);
+    L->fmt.resize(n);
     std::vector<std::pair<uint64_t, int>> order(n);
     for (int e = 0; e < n; ++e) {
         const uint8_t* ent = h + kHeaderBytes + (size_t)e * kEntryBytes;
+        L->fmt[e] = rd32(ent);
+        if (L->fmt[e] > MOE_FMT_TERNARY_DENSE) return false;
         uint64_t lo = UINT64_MAX;
         for (int i = 1; i < 7; ++i) {
             const uint64_t v = rd64(ent + 8 * i);
@@ -79,10 +123,69 @@ bool parse(const moe_shape* s, const uint8_t* h, HostLayer* L) {
 
 size_t table_bytes(int n) { return align256((size_t)kHeaderBytes + (size_t)kEntryBytes * n); }
 
-size_t slot_bytes(const HostLayer& L) {
+// A slot holds any expert in the kernels' layout (a dense ternary one once expanded).
+size_t slot_bytes(const moe_shape* s, const HostLayer& L) {
     uint64_t m = 0;
-    for (int e = 0; e < L.n; ++e) m = std::max(m, L.end[e] - L.start[e]);
+    for (int e = 0; e < L.n; ++e)
+        m = std::max(m, L.fmt[e] == MOE_FMT_TERNARY_DENSE ? span_layout(s, MOE_FMT_TERNARY).bytes : L.end[e] - L.start[e]);
     return align256(m);
+}
+
+// The staging area for dense experts' spans (behind the slots; 0 if there are none).
+size_t staging_bytes(const HostLayer& L) {
+    uint64_t m = 0;
+    for (int e = 0; e < L.n; ++e)
+        if (L.fmt[e] == MOE_FMT_TERNARY_DENSE) m = std::max(m, L.end[e] - L.start[e]);
+    return align256(m);
+}
+
+size_t cache_total(const moe_shape* s, const HostLayer& L, int n_slots) {
+    return table_bytes(L.n) + (size_t)n_slots * slot_bytes(s, L) + staging_bytes(L);
+}
+
+// The 7 table words of expert e placed at byte `at` of the cache: as in the host
+// buffer, rebased; a dense ternary expert in its expanded layout, as MOE_FMT_TERNARY.
+void entry_words(const moe_shape* s, const uint8_t* h, const HostLayer& L, int e, uint64_t at, uint64_t w[7]) {
+    if (L.fmt[e] == MOE_FMT_TERNARY_DENSE) {
+        const SpanLayout X = span_layout(s, MOE_FMT_TERNARY);
+        const uint64_t v[7] = {MOE_FMT_TERNARY, at + X.gs, at + X.gc, 0, at + X.ds, at + X.dc, 0};
+        for (int i = 0; i < 7; ++i) w[i] = v[i];
+        return;
+    }
+    const uint8_t* ent = h + kHeaderBytes + (size_t)e * kEntryBytes;
+    w[0] = rd64(ent);
+    for (int i = 1; i < 7; ++i) {
+        const uint64_t v = rd64(ent + 8 * i);
+        w[i] = v ? v - L.start[e] + at : 0;
+    }
+}
+
+// Dense ternary codes of one matrix (rows packed rows of ceil(K/5) bytes) -> the
+// kernels' blocked 2-bit code words: one thread per word (16 codes of a packed row).
+__global__ void expand_ternary_kernel(const uint8_t* __restrict__ src, int rows, int K, uint8_t* __restrict__ dst) {
+    const int wpr = K / 16;                                   // words per row
+    const size_t w = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (w >= (size_t)rows * wpr) return;
+    const int pr = (int)(w / wpr), q16 = (int)(w % wpr);
+    const int G = K / 64, g = q16 / 4, c = g / 8, gl = g % 8, wl = 4 * gl + q16 % 4;
+    const int ng = G - 8 * c < 8 ? G - 8 * c : 8;
+    const int j = pr / 16, r = pr % 16;
+    const int pos = ng == 8 ? r * 32 + (wl ^ (4 * (r % 8))) : r * 4 * ng + wl;
+    const uint8_t* row = src + (size_t)pr * ((K + 4) / 5);
+    uint32_t word = 0;
+    for (int e = 0; e < 16; ++e) {
+        const int k = 16 * q16 + e;
+        uint32_t b = row[k / 5];
+        for (int d = k % 5; d > 0; --d) b /= 3;
+        word |= (b % 3) << (16 * (e & 1) + 2 * (e >> 1));
+    }
+    *reinterpret_cast<uint32_t*>(dst + (size_t)4 * K * j + 2048 * (size_t)c + 4 * (size_t)pos) = word;
+}
+
+cudaError_t expand_matrix(const uint8_t* src, int rows, int K, uint8_t* dst, cudaStream_t s) {
+    const size_t words = (size_t)rows * (K / 16);
+    expand_ternary_kernel<<<(unsigned)((words + 255) / 256), 256, 0, s>>>(src, rows, K, dst);
+    return cudaGetLastError();
 }
 
 // The eight 64-bit words of an expert table entry (format; six array offsets; zero).
@@ -105,7 +208,7 @@ extern "C" moe_status moe_cache_size(const moe_shape* shape, const uint8_t* h_pa
     HostLayer L;
     if (!moe::shape_ok(shape) || !h_packed || !bytes || n_slots < 1) return MOE_ERR_INVALID_ARG;
     if (!parse(shape, h_packed, &L)) return MOE_ERR_INVALID_ARG;
-    *bytes = table_bytes(L.n) + (size_t)n_slots * slot_bytes(L);
+    *bytes = cache_total(shape, L, n_slots);
     return MOE_OK;
 }
 
@@ -114,7 +217,7 @@ extern "C" moe_status moe_cache_init(const moe_shape* shape, const uint8_t* h_pa
     HostLayer L;
     if (!moe::shape_ok(shape) || !h_packed || !d_cache || n_slots < 1) return MOE_ERR_INVALID_ARG;
     if (!parse(shape, h_packed, &L)) return MOE_ERR_INVALID_ARG;
-    if (cache_bytes < table_bytes(L.n) + (size_t)n_slots * slot_bytes(L)) return MOE_ERR_WORKSPACE;
+    if (cache_bytes < cache_total(shape, L, n_slots)) return MOE_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // header and table as in the host buffer; every entry is rebased onto slot 0 so that
     // it points into the cache buffer even before its expert is loaded
@@ -125,13 +228,8 @@ extern "C" moe_status moe_cache_init(const moe_shape* shape, const uint8_t* h_pa
     // entries go in by kernel arguments
     const size_t base = table_bytes(L.n);
     for (int e = 0; e < L.n; ++e) {
-        const uint8_t* ent = h_packed + kHeaderBytes + (size_t)e * kEntryBytes;
         uint64_t w[7];
-        w[0] = rd64(ent);
-        for (int i = 1; i < 7; ++i) {
-            const uint64_t v = rd64(ent + 8 * i);
-            w[i] = v ? v - L.start[e] + base : 0;
-        }
+        entry_words(shape, h_packed, L, e, base, w);
         write_entry_kernel<<<1, 1, 0, s>>>(reinterpret_cast<uint64_t*>(d + kHeaderBytes + (size_t)e * kEntryBytes),
                                            w[0], w[1], w[2], w[3], w[4], w[5], w[6]);
     }
@@ -145,26 +243,42 @@ extern "C" moe_status moe_cache_load(const moe_shape* shape, const uint8_t* h_pa
     if (!moe::shape_ok(shape) || !h_packed || !d_cache || n_slots < 1 || n < 0) return MOE_ERR_INVALID_ARG;
     if (n > 0 && (!h_experts || !h_slots)) return MOE_ERR_INVALID_ARG;
     if (!parse(shape, h_packed, &L)) return MOE_ERR_INVALID_ARG;
-    const size_t sb = slot_bytes(L), base = table_bytes(L.n);
-    if (cache_bytes < base + (size_t)n_slots * sb) return MOE_ERR_WORKSPACE;
+    const size_t sb = slot_bytes(shape, L), base = table_bytes(L.n);
+    if (cache_bytes < cache_total(shape, L, n_slots)) return MOE_ERR_WORKSPACE;
     for (int i = 0; i < n; ++i)
         if (h_experts[i] < 0 || h_experts[i] >= L.n || h_slots[i] < 0 || h_slots[i] >= n_slots)
             return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* d = static_cast<uint8_t*>(d_cache);
+    uint8_t* staging = d + base + (size_t)n_slots * sb;
+    const int H = shape->hidden, I = shape->inter;
     for (int i = 0; i < n; ++i) {
         const int e = h_experts[i];
-        const size_t slot0 = base + (size_t)h_slots[i] * sb;
-        if (cudaMemcpyAsync(d + slot0, h_packed + L.start[e], L.end[e] - L.start[e], cudaMemcpyHostToDevice, s) !=
-            cudaSuccess)
-            return MOE_ERR_CUDA;
-        const uint8_t* ent = h_packed + kHeaderBytes + (size_t)e * kEntryBytes;
-        uint64_t w[7];
-        w[0] = rd64(ent);
-        for (int k = 1; k < 7; ++k) {
-            const uint64_t v = rd64(ent + 8 * k);
-            w[k] = v ? v - L.start[e] + slot0 : 0;
+        const size_t slot0 = base + (size_t)h_slots[i] * sb, span = L.end[e] - L.start[e];
+        if (L.fmt[e] != MOE_FMT_TERNARY_DENSE) {
+            if (cudaMemcpyAsync(d + slot0, h_packed + L.start[e], span, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        } else {
+            // the dense span into the staging area (stream order serialises its reuse),
+            // then scales copied and codes expanded into the slot's 2-bit layout
+            if (cudaMemcpyAsync(staging, h_packed + L.start[e], span, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            const uint8_t* ent = h_packed + kHeaderBytes + (size_t)e * kEntryBytes;
+            const uint64_t hs_gs = rd64(ent + 8) - L.start[e], hs_gc = rd64(ent + 16) - L.start[e];
+            const uint64_t hs_ds = rd64(ent + 32) - L.start[e], hs_dc = rd64(ent + 40) - L.start[e];
+            const SpanLayout X = span_layout(shape, MOE_FMT_TERNARY);
+            const uint64_t nch = (H / 64 + 7) / 8, nci = (I / 64 + 7) / 8;
+            if (cudaMemcpyAsync(d + slot0 + X.gs, staging + hs_gs, (size_t)(2 * I / 16) * 256 * nch,
+                                cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+                cudaMemcpyAsync(d + slot0 + X.ds, staging + hs_ds, (size_t)(H / 16) * 256 * nci,
+                                cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            if (expand_matrix(staging + hs_gc, 2 * I, H, d + slot0 + X.gc, s) != cudaSuccess ||
+                expand_matrix(staging + hs_dc, H, I, d + slot0 + X.dc, s) != cudaSuccess)
+                return MOE_ERR_CUDA;
         }
+        uint64_t w[7];
+        entry_words(shape, h_packed, L, e, slot0, w);
         write_entry_kernel<<<1, 1, 0, s>>>(reinterpret_cast<uint64_t*>(d + kHeaderBytes + (size_t)e * kEntryBytes),
                                            w[0], w[1], w[2], w[3], w[4], w[5], w[6]);
     }

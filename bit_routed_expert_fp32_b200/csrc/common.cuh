@@ -67,6 +67,7 @@ enum : uint32_t {
     kDetRange = 0x600,      // a token or an expert activation outside the fp16 range
     kDetTestStall = 0x700,  // the failure-path test's wait ran out
     kDetLoopCap = 0x800,    // a work loop reached its iteration cap
+    kDetFormat = 0x900,     // an expert's format is not one the kernels read (a storage form)
 };
 
 __device__ inline void report_error(Ctrl* c, uint32_t code, uint32_t detail) {

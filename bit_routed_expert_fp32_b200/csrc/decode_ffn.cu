@@ -493,10 +493,15 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         S.fmt[a] = (int)entry(p.packed, e)->fmt;
         S.cnt[a] = e < p.E ? p.counts[e] : p.T;
         S.off[a] = e < p.E ? p.offsets[e] : 0;
+        if (S.fmt[a] > MOE_FMT_Q3) {            // a storage form (dense ternary): not read here
+            if (blockIdx.x == 0) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetFormat | MODE);
+            S.ok = 0;
+        }
     }
     if (S.perm_in_smem)
         for (int r = threadIdx.x; r < p.T * p.k; r += blockDim.x) S.tok[r] = p.perm[r] / p.k;
     __syncthreads();
+    if (!S.ok) return;
     if (threadIdx.x == 0) {
         int run = 0, one = 1;
         for (int a = 0; a < nA; ++a) {

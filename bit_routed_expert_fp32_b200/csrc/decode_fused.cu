@@ -150,15 +150,19 @@ __device__ __forceinline__ bool wait_counter(const uint32_t* ctr, uint32_t targe
     return ok != 0;
 }
 
-// All lanes' stores of this unit happen-before the counter increment (release).
+// All lanes' stores of this unit happen-before the counter increment: the warp barrier
+// orders them before lane 0's increment, which is a release at GPU scope (cumulative
+// over what lane 0 has observed).  signal_counter returns the old value; post_counter
+// does not wait for it.
 __device__ __forceinline__ uint32_t signal_counter(uint32_t* ctr, int lane) {
     __syncwarp();
     uint32_t old = 0;
-    if (lane == 0) {
-        __threadfence();
-        old = atomicAdd(ctr, 1u);
-    }
+    if (lane == 0) asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
     return __shfl_sync(0xffffffffu, old, 0);
+}
+__device__ __forceinline__ void post_counter(uint32_t* ctr, int lane) {
+    __syncwarp();
+    if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
 
 __device__ __forceinline__ const PackedEntry* pentry(const uint8_t* packed, int e) {
@@ -204,6 +208,13 @@ __device__ __forceinline__ void fill_slot(SlotInfo& si, const FfnArgs& p, int e,
     const PackedEntry* en = pentry(p.packed, e);
     si.e = e;
     si.fmt = (int)en->fmt;
+    if (si.fmt > MOE_FMT_Q3) {
+        // a storage form (dense ternary) the kernels do not read: the launch aborts
+        // before any unit is taken (every warp reads the routing first)
+        report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetFormat | 0x20);
+        atomicExch(&p.fc->abort, 1u);
+        si.fmt = MOE_FMT_Q2;
+    }
     si.cnt = cnt;
     si.row0 = row0;
     si.base[0] = p.packed + en->gu_codes;
@@ -1057,11 +1068,11 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
 
     // The routing and the token operands (Z tables, integer records) come from the
     // router launch this one follows: wait for it, then every unit is known.
-    bool stop = !hdr_ok || ld_relaxed(&fc->abort) != 0;
+    bool stop = !hdr_ok;
     {
         int tok = 0;
         const int nr = read_routing(cs, p, lane, &tok);
-        if (nr < 0) stop = true;
+        stop = stop || nr < 0 || ld_relaxed(&fc->abort) != 0;
         L.nr = nr < 0 ? 0 : nr;
         L.t_ok = tok != 0;
         L.total = L.nsgu + L.nr * L.tg * L.pr + (p.S + L.nr) * L.td * L.pd;
@@ -1106,7 +1117,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
                 // by K part 0 of the expert's first down tiles (a share each), waited for by all
                 if (cur.tile < L.shares && cur.part == 0) {
                     if (ready) quantise_h_share(p, cs, cur, L.td, lane);
-                    signal_counter(&fc->hq_done[cur.slot], lane);
+                    post_counter(&fc->hq_done[cur.slot], lane);
                 }
                 if (ready)
                     ready = wait_counter(&fc->hq_done[cur.slot], (uint32_t)L.shares, fc, ctrl, kDetWaitFull | 0x23, lane);
@@ -1134,10 +1145,10 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_fused_kernel(const __grid_cons
                 if (signal_counter(ctr, lane) == (uint32_t)gu_parts(cur, L) - 1) {
                     (void)ld_acquire(ctr);
                     if (!stop) finish_gu(p, L, cs, cur, lane);
-                    signal_counter(&fc->gu_done[cur.slot], lane);
+                    post_counter(&fc->gu_done[cur.slot], lane);
                 }
             } else if (!dn) {
-                signal_counter(&fc->gu_done[cur.slot], lane);
+                post_counter(&fc->gu_done[cur.slot], lane);
             } else {
                 const uint32_t n_parts = (uint32_t)((L.nr + p.S) * L.pd);
                 const uint32_t old = signal_counter(&p.dn_done[cur.tile], lane);

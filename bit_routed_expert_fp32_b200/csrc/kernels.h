@@ -82,6 +82,11 @@ struct Ws {
 //   pairs          [R][G8] x 8 bytes          (iq_pair_off)
 // The fused decode kernel (decode_fused.cu) serves up to kFusedMaxT tokens.
 constexpr int kFusedMaxT = 16;
+// token counts for which MOE_PATH_AUTO / MOE_PATH_DECODE take the fused decode kernel:
+// there it beat the separate decode launches on the full-size layer (one to two tokens:
+// 97-135 against 102-147 us per step; four to eight: 187-309 against 204-332; sixteen:
+// 525 against 535, and 440 against 554 with mixed formats and skewed routing)
+constexpr int kFusedAutoMinT = 3, kFusedAutoMaxT = 8;
 __host__ __device__ inline size_t iq_pair_off(int64_t R, int64_t K) { return (size_t)R * (K / 64) * 128; }
 __host__ __device__ inline size_t iq_size(int64_t R, int64_t K) {
     return iq_pair_off(R, K) + (size_t)8 * R * (8 * ((K / 64 + 7) / 8));

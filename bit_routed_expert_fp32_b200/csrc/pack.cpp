@@ -1,5 +1,6 @@
 // Host-side packer: interchange-form codes and fp16 scales -> packed format v2
-// (layout documented in include/moe.h).  Pure host code, no CUDA calls.
+// (layout documented in include/moe.h), including the dense ternary storage form.
+// Pure host code, no CUDA calls.
 #include <stdint.h>
 #include <string.h>
 
@@ -31,12 +32,14 @@ struct ExpertLayout {
     MatLayout gu, dn;
 };
 
+// bytes of a dense ternary row: five codes per byte
+inline size_t dense_row_bytes(int K) { return (size_t)(K + 4) / 5; }
 size_t mat_bytes(int rows, int K, uint32_t fmt, MatLayout* m, size_t off) {
     off = align256(off);
     m->scales = off;
     off = align256(off + (size_t)(rows / 16) * 256 * n_chunks(K));
     m->codes = off;
-    off += (size_t)rows * (K / 4);
+    off += fmt == MOE_FMT_TERNARY_DENSE ? (size_t)rows * dense_row_bytes(K) : (size_t)rows * (K / 4);
     if (fmt == MOE_FMT_Q3) {
         off = align256(off);
         m->hi = off;
@@ -99,17 +102,30 @@ inline void store_u32(uint8_t* p, uint32_t v) {
 // matrix, in the tile/chunk-blocked, swizzled layout documented in moe.h.
 bool pack_row(const moe_matrix_src& src, int sr, int K, uint32_t fmt, uint8_t* base, const MatLayout& m, int dr) {
     const uint8_t* codes = src.codes + (size_t)sr * (K / 4);
-    if (fmt == MOE_FMT_TERNARY) {
+    if (fmt == MOE_FMT_TERNARY || fmt == MOE_FMT_TERNARY_DENSE) {
         for (int b = 0; b < K / 4; ++b)
             if (codes[b] & (codes[b] >> 1) & 0x55) return false;   // a field equal to 3
     }
     const int G = K / 64, NC = n_chunks(K), j = dr / 16, r = dr % 16;
     const uint16_t* ssrc = src.scales + (size_t)sr * G;
     const uint8_t* hi = fmt == MOE_FMT_Q3 ? src.hi + (size_t)sr * (K / 8) : nullptr;
+    if (fmt == MOE_FMT_TERNARY_DENSE) {
+        // packed row dr: byte i = sum over j < 5 of c(5i + j) 3^j (codes past K are 0)
+        uint8_t* drow = base + m.codes + (size_t)dr * dense_row_bytes(K);
+        for (size_t i = 0; i < dense_row_bytes(K); ++i) {
+            uint32_t v = 0;
+            for (int d = 4; d >= 0; --d) {
+                const int k = 5 * (int)i + d;
+                const uint32_t c = k < K ? (codes[k / 4] >> (2 * (k % 4))) & 3u : 0u;
+                v = 3 * v + c;
+            }
+            drow[i] = (uint8_t)v;
+        }
+    }
     for (int c = 0; c < NC; ++c) {
         const int ng = G - 8 * c < 8 ? G - 8 * c : 8;
         uint8_t* cblk = base + m.codes + (size_t)4 * K * j + 2048 * (size_t)c;
-        for (int wl = 0; wl < 4 * ng; ++wl) {
+        for (int wl = 0; wl < 4 * ng && fmt != MOE_FMT_TERNARY_DENSE; ++wl) {
             const int pos = ng == 8 ? r * 32 + (wl ^ (4 * (r % 8))) : r * 4 * ng + wl;
             store_u32(cblk + 4 * pos, code_word(load_u32(codes + 4 * (32 * c + wl))));
         }
@@ -155,7 +171,7 @@ void write_header(const moe_shape* s, const std::vector<ExpertLayout>& L, size_t
 extern "C" moe_status moe_packed_size(const moe_shape* shape, const uint8_t* h_fmt, size_t* bytes) {
     if (!shape_ok(shape) || !h_fmt || !bytes) return MOE_ERR_INVALID_ARG;
     for (int e = 0; e < shape->n_experts + shape->n_shared; ++e)
-        if (h_fmt[e] > MOE_FMT_Q3) return MOE_ERR_INVALID_ARG;
+        if (h_fmt[e] > MOE_FMT_TERNARY_DENSE) return MOE_ERR_INVALID_ARG;
     *bytes = layout(shape, h_fmt, nullptr);
     return MOE_OK;
 }
@@ -166,7 +182,7 @@ extern "C" moe_status moe_pack_experts(const moe_shape* shape, const uint8_t* h_
     const int n = shape->n_experts + shape->n_shared;
     if (first < 0 || count < 0 || first + count > n) return MOE_ERR_INVALID_ARG;
     for (int e = 0; e < n; ++e)
-        if (h_fmt[e] > MOE_FMT_Q3) return MOE_ERR_INVALID_ARG;
+        if (h_fmt[e] > MOE_FMT_TERNARY_DENSE) return MOE_ERR_INVALID_ARG;
     std::vector<ExpertLayout> L;
     const size_t total = layout(shape, h_fmt, &L);
     if (h_dst_bytes < total) return MOE_ERR_WORKSPACE;

@@ -285,8 +285,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         S.cnt[a] = c;
         S.nt[a] = nt;
         S.nb[a] = nb;
+        if (S.fmt[a] > MOE_FMT_Q3) {            // a storage form (dense ternary): not read here
+            if (blockIdx.x == 0) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetFormat | 0x10 | MODE);
+            S.ok = 0;
+        }
     }
     __syncthreads();
+    if (!S.ok) return;
     if (threadIdx.x == 0) {
         int run = 0;
         for (int a = 0; a < nA; ++a) {

@@ -24,9 +24,39 @@ namespace {
 __device__ inline float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ inline float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-__device__ inline double warp_sum_f64(double v) {
+// Double-float sums (a value is hi + lo, two fp32 numbers) with the exact two-sum
+// (Knuth: s = a + b and the rounding error of that addition, both in fp32): the
+// relative error of a sum of n terms is about n 2^-48 of the sum of their magnitudes.
+// The decode router forms each thread's share of a logit (28 products of an fp32
+// weight and a bf16 token) with fp32 fmas and adds the shares across the CTA in
+// double-float, so the logit carries the rounding of 28-term partial sums only, at
+// fp32 arithmetic rates (the fp64 units of this part are a small fraction of its fp32
+// ones, and a double-float product costs a dozen fp32 operations).
+struct Df {
+    float hi, lo;
+};
+// (explicitly rounded operations: the compiler must not fuse or reorder them)
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& err) {
+    s = __fadd_rn(a, b);
+    const float bp = __fsub_rn(s, a);
+    err = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bp)), __fsub_rn(b, bp));
+}
+__device__ __forceinline__ Df df_add(Df a, Df b) {
+    Df r;
+    float err;
+    two_sum(a.hi, b.hi, r.hi, err);
+    r.lo = __fadd_rn(__fadd_rn(a.lo, b.lo), err);
+    return r;
+}
+// every lane ends with the same sum (the exact two-sum is symmetric in its arguments)
+__device__ inline Df warp_sum_df(Df v) {
 #pragma unroll
-    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = 16; o; o >>= 1) {
+        Df w;
+        w.hi = __shfl_xor_sync(0xffffffffu, v.hi, o);
+        w.lo = __shfl_xor_sync(0xffffffffu, v.lo, o);
+        v = df_add(v, w);
+    }
     return v;
 }
 
@@ -228,10 +258,15 @@ __device__ void warp_topk_redux(const float (&v)[8], int k, int lane, int32_t* i
 }
 
 // One CTA per expert row: 8 warps hold the whole fp32 row in registers (one load
-// each, all in flight at once) and form its logit for every token; then the Z
-// tables; the last CTA to finish (atomic ticket) does top-k, histogram, scan and the
-// permutation.
+// each, all in flight at once) and form its logit for every token, the tokens staged
+// kRouteTB at a time in shared memory (one coalesced load of all of them, then
+// shared-memory reads: a token's elements reach every thread without a chain of
+// global-memory round trips); then the Z tables; the last CTA to finish (atomic
+// ticket) does top-k, histogram, scan and the permutation.
 constexpr int kRouteVec = 7;                           // float4 of the row per thread (H <= 7168)
+constexpr int kRouteTB = 4;                            // tokens staged per round
+constexpr int kRouteSlice = 256 * kRouteVec * 4;       // row elements per pass (7168)
+constexpr size_t kRouteSmem = (size_t)kRouteTB * kRouteSlice * 2;   // 57,344 B
 
 __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
     griddep_launch_dependents();        // one wave of CTAs: the expert pass may start launching
@@ -239,10 +274,12 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
         p.ctrl->work[0] = 0;
         p.ctrl->work[1] = 0;
     }
-    // fp64 accumulation: each product of an fp32 weight and a bf16 token is exact in
-    // fp64, so the logit is the exact sum rounded once to fp32 (tokens with large
-    // outliers make fp32 partial sums lose the bits that separate close logits)
-    __shared__ double s_part[8][kSmallT];
+    // fp32 fma partial sums of 28 products per thread, added across the CTA in
+    // double-float (Df): the logit carries only the partial sums' rounding (tokens with
+    // large outliers make long fp32 sums lose the bits that separate close logits)
+    extern __shared__ __align__(16) uint8_t route_smem[];
+    uint2* xs = reinterpret_cast<uint2*>(route_smem);   // [kRouteTB][kRouteSlice / 4]
+    __shared__ Df s_part[8][kSmallT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x;
     const int n4 = p.H / 4;                                        // float4 per row
@@ -254,47 +291,61 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs p) {
             const int i = i0 + threadIdx.x + 256 * u;
             w[u] = i < n4 ? __ldg(w4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        for (int tb = 0; tb < p.T; tb += 8) {
-            double acc[8];
+        if (i0 == 0 && p.ops) {
+            // the decode operands of (token, group) pairs, one per warp: formed while the
+            // router row's loads are in flight
+            const int G8 = 8 * ((p.H / 64 + 7) / 8);
+            for (int pr = blockIdx.x * 8 + warp; pr < p.T * G8; pr += gridDim.x * 8) {
+                const OperandArgs o{p.T, p.H, p.x, p.zx, p.iq, p.ctrl};
+                compute_z(o, pr / G8, pr % G8, lane);
+                if (p.iq) compute_iq(o, pr / G8, pr % G8, lane);
+            }
+        }
+        const int n_el = min(kRouteSlice, p.H - 4 * i0);            // elements of this pass
+        for (int tb = 0; tb < p.T; tb += kRouteTB) {
+            const int nt = min(kRouteTB, p.T - tb);
+            // stage tokens tb .. tb+nt-1, elements 4 i0 .. 4 i0 + n_el (8 per uint4)
+            for (int q = threadIdx.x; q < nt * (n_el / 8); q += 256) {
+                const int j = q / (n_el / 8), c = q - j * (n_el / 8);
+                reinterpret_cast<uint4*>(xs)[j * (kRouteSlice / 8) + c] =
+                    __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)(tb + j) * p.H + 4 * i0) + c);
+            }
+            __syncthreads();
+            float acc[kRouteTB];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                acc[j] = 0.f;
-                if (tb + j >= p.T) continue;
-                const uint2* xr = reinterpret_cast<const uint2*>(p.x + (size_t)(tb + j) * p.H);
+            for (int j = 0; j < kRouteTB; ++j) acc[j] = 0.f;
 #pragma unroll
-                for (int u = 0; u < kRouteVec; ++u) {
-                    const int i = i0 + threadIdx.x + 256 * u;
-                    if (i < n4) {
-                        const uint2 xv = __ldg(xr + i);
-                        acc[j] = fma((double)w[u].x, (double)bf16lo(xv.x), acc[j]);
-                        acc[j] = fma((double)w[u].y, (double)bf16hi(xv.x), acc[j]);
-                        acc[j] = fma((double)w[u].z, (double)bf16lo(xv.y), acc[j]);
-                        acc[j] = fma((double)w[u].w, (double)bf16hi(xv.y), acc[j]);
+            for (int u = 0; u < kRouteVec; ++u) {
+                const int il = threadIdx.x + 256 * u;                // float4 index within the pass
+                if (i0 + il < n4) {
+#pragma unroll
+                    for (int j = 0; j < kRouteTB; ++j) {
+                        if (j < nt) {
+                            const uint2 xv = xs[j * (kRouteSlice / 4) + il];
+                            acc[j] = __fmaf_rn(w[u].x, bf16lo(xv.x), acc[j]);
+                            acc[j] = __fmaf_rn(w[u].y, bf16hi(xv.x), acc[j]);
+                            acc[j] = __fmaf_rn(w[u].z, bf16lo(xv.y), acc[j]);
+                            acc[j] = __fmaf_rn(w[u].w, bf16hi(xv.y), acc[j]);
+                        }
                     }
                 }
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (tb + j >= p.T) break;
-                const double v = warp_sum_f64(acc[j]);
-                if (lane == 0) s_part[warp][tb + j] = (i0 == 0 ? 0.0 : s_part[warp][tb + j]) + v;
+            for (int j = 0; j < kRouteTB; ++j) {
+                if (j >= nt) break;
+                const Df v = warp_sum_df(Df{acc[j], 0.f});
+                if (lane == 0) s_part[warp][tb + j] = i0 == 0 ? v : df_add(s_part[warp][tb + j], v);
             }
+            __syncthreads();                                         // xs is refilled next round
         }
     }
     __syncthreads();
     for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
-        double v = 0.0;
+        Df v = s_part[0][t];
 #pragma unroll
-        for (int w = 0; w < 8; ++w) v += s_part[w][t];
-        p.logits[(size_t)t * p.E + e] = (float)(v + (p.bias ? (double)p.bias[e] : 0.0));
-    }
-    if (p.ops) {
-        const int G8 = 8 * ((p.H / 64 + 7) / 8);
-        for (int pr = blockIdx.x * 8 + warp; pr < p.T * G8; pr += gridDim.x * 8) {
-            const OperandArgs o{p.T, p.H, p.x, p.zx, p.iq, p.ctrl};
-            compute_z(o, pr / G8, pr % G8, lane);
-            if (p.iq) compute_iq(o, pr / G8, pr % G8, lane);
-        }
+        for (int w = 1; w < 8; ++w) v = df_add(v, s_part[w][t]);
+        // the bias and the one final rounding (a few fp64 operations per logit)
+        p.logits[(size_t)t * p.E + e] = (float)((double)v.hi + (double)v.lo + (p.bias ? (double)p.bias[e] : 0.0));
     }
     __shared__ int s_last;
     __threadfence();
@@ -366,11 +417,13 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = blockIdx.x * RBM, e0 = blockIdx.y * RBN;
     const int wm = warp >> 1, wn = warp & 1;            // warp tile: tokens 32wm.., experts 32wn..
-    double acc[2][4][4];        // K-tile partials added in fp64 (see the decode router)
+    Df acc[2][4][4];            // K-tile partials added in double-float (see the decode router)
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = acc[a][b][2] = acc[a][b][3] = 0.f;
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][b][c] = Df{0.f, 0.f};
 
     // loaders: x tile 128 x 32 bf16 = 512 x 16 B (2 per thread); w tile 64 x 32 fp32 (8 floats per thread)
     uint4 xr[2];
@@ -466,7 +519,7 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][b][c] += (double)part[a][b][c];
+                for (int c = 0; c < 4; ++c) acc[a][b][c] = df_add(acc[a][b][c], Df{part[a][b][c], 0.f});
         if (kt + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
@@ -483,7 +536,8 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
                     const int e = e0 + 32 * wn + 8 * nt + 2 * t4 + c;
                     if (t < p.T && e < p.E)
                         p.logits[(size_t)t * p.E + e] =
-                            (float)(acc[mt][nt][2 * h + c] + (p.bias ? (double)p.bias[e] : 0.0));
+                            (float)((double)acc[mt][nt][2 * h + c].hi + (double)acc[mt][nt][2 * h + c].lo +
+                                    (p.bias ? (double)p.bias[e] : 0.0));
                 }
             }
 }
@@ -578,7 +632,9 @@ cudaError_t launch_route_fixed(const RouteArgs& a, cudaStream_t s) {
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     if (a.T <= kSmallT) {
-        route_small_kernel<<<a.E, 256, 0, s>>>(a);
+        const cudaError_t err = set_smem_limit(route_small_kernel, kRouteSmem);
+        if (err != cudaSuccess) return err;
+        route_small_kernel<<<a.E, 256, kRouteSmem, s>>>(a);
         return cudaGetLastError();
     }
     const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);

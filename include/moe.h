@@ -53,16 +53,29 @@ typedef enum {
     MOE_ERR_DEVICE_CHECK = 6   /* the device found bad data, e.g. a packed header     */
 } moe_status;
 
-typedef enum { MOE_FMT_TERNARY = 0, MOE_FMT_Q2 = 1, MOE_FMT_Q3 = 2 } moe_format;
+/* MOE_FMT_TERNARY_DENSE is a storage form of ternary experts (five codes per byte,
+ * 1.625 bits per weight against 2): the packer writes it, the expert cache
+ * (moe_cache_load) copies it from host memory and expands it on the GPU into
+ * MOE_FMT_TERNARY, and no expert kernel reads it (moe_forward on a buffer that holds
+ * it records MOE_ERR_DEVICE_CHECK with detail MOE_DETAIL_FORMAT and computes nothing). */
+typedef enum { MOE_FMT_TERNARY = 0, MOE_FMT_Q2 = 1, MOE_FMT_Q3 = 2, MOE_FMT_TERNARY_DENSE = 3 } moe_format;
 
-/* MOE_PATH_AUTO picks DECODE for T <= 64 and PREFILL otherwise.  Both paths compute
- * the same function; they differ only in kernels and rounding of intermediates. */
-typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_DECODE = 1, MOE_PATH_PREFILL = 2 } moe_path;
+/* MOE_PATH_AUTO picks DECODE for T <= 64 and PREFILL otherwise.  DECODE runs the decode
+ * kernels: for 3 <= T <= 8 the whole forward as one persistent kernel (the fused
+ * decode kernel), otherwise separate gate/up, down and combine launches (the faster
+ * choice at each T on the full-size layer).  MOE_PATH_DECODE_FUSED asks for the fused
+ * decode kernel at any T <= 16 (MOE_ERR_UNSUPPORTED above).  All paths compute the
+ * same function; they differ only in kernels and rounding of intermediates. */
+typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_DECODE = 1, MOE_PATH_PREFILL = 2, MOE_PATH_DECODE_FUSED = 3 } moe_path;
 
 /* OR-ed into moe_forward's path: d_y is fp32 [T][H] instead of bf16 (the sums are not
  * rounded to bf16; the expert-parallel layer returns expert outputs this way, so that
  * its gate-weighted combine rounds once, as the single-GPU layer does). */
 #define MOE_OUT_F32 0x10
+
+/* Device pointers.  The token, output, router-weight, packed-expert and workspace
+ * pointers given to moe_route and moe_forward must be 16-byte aligned (allocations from
+ * cudaMalloc and the CUDA caching allocators are); others are MOE_ERR_INVALID_ARG. */
 
 /* Layer shape.  hidden and inter must be positive multiples of 64; 1 <= top_k <= 16;
  * top_k <= n_experts <= 256; n_shared in {0, 1}. */
@@ -116,6 +129,11 @@ typedef struct {
  *   q2       (c - 1.5) * s,  c in 0..3
  *   q3       (c - 3.5) * s,  c = lo + 4*hi in 0..7
  * with s the fp16 scale of the element's group (64 consecutive k).
+ * MOE_FMT_TERNARY_DENSE (a storage form): the ternary values as above, but the codes
+ * array of a matrix holds ceil(K/5) bytes per packed row (rows in the same order as
+ * the blocked arrays: packed row pr from byte pr*ceil(K/5)), element k in byte k/5 as
+ * base-3 digit k%5 (byte i = sum over j < 5 of c(5i + j) 3^j, codes past K zero, at
+ * most 242); the scales blocked as below; no third bits.
  *
  * Blocking.  A matrix W[N][K] (N a multiple of 16, K of 64) has G = K/64 groups per
  * row, cut into NC = ceil(G/8) chunks; chunk c holds groups 8c .. 8c+ng-1 with
@@ -214,6 +232,7 @@ moe_status moe_workspace_set_test_stall(void* d_ws, size_t ws_bytes, uint32_t cy
 #define MOE_DETAIL_RANGE 0x600u       /* a token or expert activation outside fp16 range  */
 #define MOE_DETAIL_TEST_STALL 0x700u  /* moe_workspace_set_test_stall's wait ran out      */
 #define MOE_DETAIL_LOOP_CAP 0x800u    /* a work loop reached its iteration cap            */
+#define MOE_DETAIL_FORMAT 0x900u      /* an expert in a storage form (dense ternary)      */
 
 /* Route T tokens: fp32 router logits, softmax + top-k + renormalised gates,
  * per-expert histogram, prefix sum and permutation.

@@ -233,6 +233,10 @@ static uint64_t rd64(const uint8_t* p) { return (uint64_t)rd32(p) | ((uint64_t)r
  *   hi     at 128*G*j + 1024*c; word vl = 2*gl + half at r*16 + (vl ^ 2*((r%8)/2)) when
  *          ng == 8, else r*2*ng + vl; element 32v+16q+2p+h at bit 16h+8q+p;
  *   scales at 256*NC*j + 256*c; scale of group 8c+gl of row r at half r*8 + gl.
+ * Format 3 (ternary, five codes per byte, a storage form): the scales as above; the
+ * codes of physical row pr (the fused gate/up row order) in ceil(K/5) bytes from
+ * pr*ceil(K/5), element k in byte k/5 as base-3 digit k%5 (the byte is the sum of
+ * c_{5i+j} 3^j, at most 242); no third bits.
  * Returns 0 or a negative error. */
 int oracle_unpack(const uint8_t* buf, size_t bytes, int table, int which, int8_t* codes,
                   uint16_t* scales, int* fmt) {
@@ -268,6 +272,15 @@ int oracle_unpack(const uint8_t* buf, size_t bytes, int table, int which, int8_t
             uint32_t word = rd32(buf + off_c + (size_t)4 * K * j + 2048 * (size_t)c + 4 * (size_t)pos);
             int i = k % 16, p = i / 2, h = i % 2;
             int code = (int)((word >> (16 * h + 2 * p)) & 3u);
+            if (f == 3) {
+                /* dense ternary: physical row pr holds ceil(K/5) bytes, element k in
+                   byte k/5 as base-3 digit k%5 (byte = sum of c_{5i+j} 3^j) */
+                size_t rb = (size_t)(K + 4) / 5;
+                int v = buf[off_c + (size_t)pr * rb + (size_t)(k / 5)];
+                if (v > 242) return -4;
+                for (int d = 0; d < k % 5; ++d) v /= 3;
+                code = v % 3;
+            }
             if (f == 2) {
                 int vl = 2 * gl + (k % 64) / 32;
                 int hpos = ng == 8 ? r * 16 + (vl ^ (2 * ((r % 8) / 2))) : r * 2 * ng + vl;

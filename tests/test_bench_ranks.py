@@ -58,10 +58,15 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
 def test_paths_and_launch_counts():
     import dataclasses
     c2, c3, c4 = synth.CONFIGS[2], synth.CONFIGS[3], synth.CONFIGS[4]
-    # up to 16 tokens: the router, then the whole forward as one kernel
-    assert bench.path_of(c2) == "fused" and bench.launches_per_step(c2) == 1 + 1
-    assert bench.path_of(c3) == "fused" and bench.launches_per_step(c3) == 1 + 1
-    # 17 to 64 tokens: the decode kernels; with 24 tokens K is split for neither pass
+    # one token: the router, gate/up (K in parts), the K-part reduction, down, combine
+    assert bench.path_of(c2) == "decode" and bench.decode_kparts(c2)[0] > 1
+    assert bench.launches_per_step(c2) == 1 + 3 + 1
+    # 3 to 8 tokens: the router, then the whole forward as one kernel
+    for T in (3, 5, 8):
+        c = dataclasses.replace(c2, T=T)
+        assert bench.path_of(c) == "fused" and bench.launches_per_step(c) == 1 + 1
+    # 16 and 24 tokens: the separate decode kernels
+    assert bench.path_of(c3) == "decode"
     c24 = dataclasses.replace(c2, T=24)
     assert bench.path_of(c24) == "decode"
     assert bench.launches_per_step(c24) == 1 + 3 + (1 if bench.decode_kparts(c24)[0] > 1 else 0)

@@ -25,7 +25,7 @@ from tests import harness as H
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"decode": 1, "prefill": 2}
+PATHS = {"decode": 1, "prefill": 2, "fused": 3}
 
 
 def plant_outliers(factor, seed, every=1, base=1.0):
@@ -71,7 +71,8 @@ OUTLIERS = {"100x_every_group": (100.0, 1, 0.1), "1000x_every_group": (1000.0, 1
 
 
 @pytest.mark.parametrize("kind", sorted(OUTLIERS))
-@pytest.mark.parametrize("T,path", [(1, "decode"), (2, "decode"), (4, "decode"), (16, "decode"), (96, "prefill")])
+@pytest.mark.parametrize("T,path", [(1, "decode"), (1, "fused"), (2, "fused"), (4, "decode"), (16, "decode"),
+                                    (16, "fused"), (96, "prefill")])
 def test_outlier_tokens_full_size(mixed_layer, kind, T, path):
     cfg, layer = mixed_layer
     factor, every, base = OUTLIERS[kind]
@@ -88,9 +89,10 @@ def test_outlier_tokens_all_q2_integer_path():
     cfg = synth.CONFIGS[2]
     case = H.make_case(cfg, T=1, transform=plant_outliers(1000.0, seed=7, every=1, base=0.02))
     packed = H.pack(case)
-    rt, y = H.run_gpu(case, packed, path=PATHS["decode"])
-    H.check_routing(case, rt)
-    H.check_outputs(y, H.oracle_outputs(case, [0]))
+    for path in ("decode", "fused"):
+        rt, y = H.run_gpu(case, packed, path=PATHS[path])
+        H.check_routing(case, rt)
+        H.check_outputs(y, H.oracle_outputs(case, [0]))
     del packed
     torch.cuda.empty_cache()
 
@@ -160,7 +162,7 @@ def test_forward_with_another_T_than_routed_is_reported(t_route, t_fwd, path):
     H.check_outputs(y2, H.oracle_outputs(case, list(range(cfg.T))))
 
 
-@pytest.mark.parametrize("T,path", [(1, "decode"), (8, "decode"), (24, "decode"), (96, "prefill")])
+@pytest.mark.parametrize("T,path", [(1, "decode"), (1, "fused"), (8, "decode"), (24, "decode"), (96, "prefill")])
 def test_wait_that_runs_out_is_reported_and_the_next_call_is_correct(T, path):
     """Each expert kernel waits (test-only, 20,000 SM cycles at most) on a barrier that
     nothing completes; the wait runs out, the kernel takes its give-up path and returns.

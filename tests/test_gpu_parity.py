@@ -13,7 +13,7 @@ from tests import harness as H
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"decode": 1, "prefill": 2}
+PATHS = {"decode": 1, "prefill": 2, "fused": 3}
 
 
 def _full_check(cfg, path, bias=None, router_w=None, T=None):
@@ -152,27 +152,29 @@ def test_full_size_few_tokens_and_determinism():
     layer = moe.MoeLayer(base, packed, case1.layer.router_w, case1.layer.router_b, 16)
     for T in (1, 2, 3, 4, 16):
         case = case1 if T == 1 else H.make_case(base, step=T, T=T)
-        rt, y = H.run_gpu(case, None, path=1, gpu_layer=layer)
-        H.check_routing(case, rt)
-        H.check_outputs(y, H.oracle_outputs(case, list(range(T))))
-        if T in (1, 16):
-            _, y_again = H.run_gpu(case, None, path=1, gpu_layer=layer)
-            np.testing.assert_array_equal(y, y_again)
+        ref = H.oracle_outputs(case, list(range(T)))
+        for path in (1, 3):              # the decode choice for T, and the fused decode kernel
+            rt, y = H.run_gpu(case, None, path=path, gpu_layer=layer)
+            H.check_routing(case, rt)
+            H.check_outputs(y, ref)
+            if T in (1, 16):
+                _, y_again = H.run_gpu(case, None, path=path, gpu_layer=layer)
+                np.testing.assert_array_equal(y, y_again)
     del layer, packed
     torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("T,shared_format", [(1, synth.FMT_TERNARY), (2, synth.FMT_Q2), (4, synth.FMT_TERNARY)])
 def test_few_token_integer_gate_up_full_chunks(T, shared_format):
-    """Gate/up with at most 4 tokens runs ternary and 2-bit experts on integer MMAs:
-    hidden 1024 gives whole 8-group chunks (the micro shapes above only reach the
-    partial-chunk code), all routed experts ternary exercises the o = 1 offset plane,
-    and a ternary or 2-bit shared expert takes the integer path's shared-expert rows
-    (every other workload's shared expert is 3-bit, which stays on the bf16 path)."""
+    """The fused decode kernel runs gate/up and down of ternary and 2-bit experts on
+    integer MMAs: hidden 1024 gives whole 8-group chunks (the micro shapes above only
+    reach the partial-chunk code), all routed experts ternary exercises the o = 1
+    offset, and a ternary or 2-bit shared expert takes the integer path's shared-expert
+    rows (every other workload's shared expert is 3-bit, which stays on the bf16 path)."""
     import dataclasses
     cfg = synth.micro(T=T, H=1024, E=16, k=8, I=128, S=1, formats="ternary", seed=40 + T)
     cfg = dataclasses.replace(cfg, shared_format=shared_format)
-    _full_check(cfg, PATHS["decode"])
+    _full_check(cfg, PATHS["fused"])
 
 
 @pytest.mark.parametrize("T,shared_format", [(1, synth.FMT_Q2), (2, synth.FMT_TERNARY), (2, synth.FMT_Q2),
@@ -187,7 +189,7 @@ def test_shared_gate_up_and_down_in_k_parts(T, shared_format):
     import dataclasses
     cfg = synth.micro(T=T, H=1024, E=16, k=8, I=2048, S=1, formats="mixed", seed=80 + T)
     cfg = dataclasses.replace(cfg, shared_format=shared_format)
-    _full_check(cfg, PATHS["decode"])
+    _full_check(cfg, PATHS["fused"])
 
 
 @pytest.mark.parametrize("formats,T,path", [("q2", 1, "decode"), ("mixed", 12, "decode"), ("mixed", 96, "prefill")])

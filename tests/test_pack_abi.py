@@ -52,7 +52,7 @@ def test_argument_errors_are_synchronous():
     assert L.moe_packed_size(ctypes.byref(bad), fmt.ctypes.data, ctypes.byref(sz)) == 1
     assert L.moe_workspace_size(ctypes.byref(_shape(k=5)), 4, ctypes.byref(sz)) == 1       # k > E
     assert L.moe_workspace_size(ctypes.byref(_shape()), -1, ctypes.byref(sz)) == 1
-    fmt_bad = np.array([1, 1, 3, 1, 1], np.uint8)
+    fmt_bad = np.array([1, 1, 4, 1, 1], np.uint8)                 # 3 is the dense ternary storage form
     assert L.moe_packed_size(ctypes.byref(_shape()), fmt_bad.ctypes.data, ctypes.byref(sz)) == 1
     sh = _shape()
     fake = ctypes.c_void_p(0x1000)
