@@ -47,12 +47,12 @@ METRIC = "routed-MoE layer tokens/s; decode weight-stream GB/s vs HBM peak (1 B2
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # gate/up kernel of each path and the sources its ncu traffic record is tied to
 PATHS = {
-    "fused": ("ffn_fused_kernel (the whole decode forward: token operands, gate/up + SwiGLU, down and the "
-              "combine, one persistent launch; integer MMAs for ternary / 2-bit gate/up)",
+    "fused": ("ffn_fused_kernel (the whole decode forward: gate/up + SwiGLU, down and the combine, one "
+              "persistent launch; integer MMAs for ternary / 2-bit experts)",
               ["bit_routed_expert_fp32_b200/csrc/decode_fused.cu", "bit_routed_expert_fp32_b200/csrc/dequant.cuh",
                "bit_routed_expert_fp32_b200/csrc/operands.cuh", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
-    "decode": ("ffn_decode_kernel<0, *> (gate/up + SwiGLU; integer MMAs for ternary / 2-bit experts at <= 4 "
-               "tokens; interval includes the K-part reduction when K is split)",
+    "decode": ("ffn_decode_kernel<0> (gate/up + SwiGLU; interval includes the K-part reduction when K is "
+               "split)",
                ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "prefill": ("tc_gemm_kernel<0> (gate/up + SwiGLU, tcgen05; interval includes the token gather)",
                 ["bit_routed_expert_fp32_b200/csrc/prefill_tc.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
@@ -117,6 +117,18 @@ def max_over_ranks(x: float, world: int, device) -> float:
 def throughput(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
     """Whole-job tokens/s: every rank's tokens over the slowest rank's device time."""
     return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), for the CPU baseline's record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def peaks():
@@ -287,8 +299,8 @@ def run_reference(args, cfg):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_dict(cfg, world),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": f"{per_step} token(s) of the workload per step, routed and run through "
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "cpu": cpu_model(),
+                             "kind": "oracle", "sample": f"{per_step} token(s) of the workload per step, routed and run through "
                                        f"all selected experts and the shared expert in fp64 (expert weights "
                                        f"drawn before timing)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -486,21 +498,28 @@ def run_ours(args, cfg):
     x_pin = torch.from_numpy(xs_host.view(np.int16)).pin_memory()
     y_pin = torch.empty((total, T, cfg.H), dtype=torch.int16).pin_memory()
     x_stage = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    # (eager calls, as a caller without a graph makes them; two more events split off the
+    # copies so that the gap to the graph-replayed device time can be attributed)
     e2e_ms = []
     for s in range(total):
         flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a, c1, c2, b = (torch.cuda.Event(enable_timing=True) for _ in range(4))
         a.record(stream)
         x_stage.view(torch.int16).copy_(x_pin[s], non_blocking=True)
+        c1.record(stream)
         lay = layers[s % n_layers]
         lay.route(x_stage)
         lay.forward(x_stage, y)
+        c2.record(stream)
         y_pin[s].copy_(y.view(torch.int16), non_blocking=True)
         b.record(stream)
         if s >= args.warmup:
-            e2e_ms.append((a, b))
+            e2e_ms.append((a, b, c1, c2))
     torch.cuda.synchronize(dev)
-    e2e_total = sum(a.elapsed_time(b) for a, b in e2e_ms)
+    e2e_total = sum(a.elapsed_time(b) for a, b, _, _ in e2e_ms)
+    e2e_h2d_us = 1e3 * float(np.mean([a.elapsed_time(c1) for a, _, c1, _ in e2e_ms]))
+    e2e_d2h_us = 1e3 * float(np.mean([c2.elapsed_time(b) for _, b, _, c2 in e2e_ms]))
+    e2e_calls_us = 1e3 * float(np.mean([c1.elapsed_time(c2) for _, _, c1, c2 in e2e_ms]))
     e2e_value = throughput(world, T, args.steps, max_over_ranks(e2e_total, world, dev))
     st, det = moe.moe_get_error(layers[0].ws)
     if st != 0:
@@ -526,7 +545,9 @@ def run_ours(args, cfg):
                                "step_with_events_between_kernels": 1e3 * float(np.mean(step_serial_ms)),
                                "measured": "second pass over the same steps with an event between kernels"}),
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.H * 2,
-                        "d2h_bytes_per_step": T * cfg.H * 2},
+                        "d2h_bytes_per_step": T * cfg.H * 2, "launch": "eager calls (no graph)",
+                        "us_per_step": {"h2d_copy": e2e_h2d_us, "route_and_forward": e2e_calls_us,
+                                        "d2h_copy": e2e_d2h_us}},
                 "gpu_launches": launches_per_step(cfg) * args.steps,
                 "path": path,
                 "wall_s_timed_region": wall,
@@ -535,7 +556,8 @@ def run_ours(args, cfg):
             L0 = synth.Layer(cfg, 0)
             sample = [xs_host[i][: max(1, min(T, 4))] for i in range(min(8, total))]
             v, n, dt, cores = oracle_tokens_per_s(cfg, L0, sample, args.cpu_budget, 64)
-            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "cpu": cpu_model(),
+                                    "kind": "oracle",
                                     "sample": f"{n} token(s) of this workload ({dt:.1f} s), routed and run "
                                               f"through every selected expert and the shared expert in fp64 "
                                               f"(expert weights drawn before timing)"}

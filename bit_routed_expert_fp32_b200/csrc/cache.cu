@@ -15,7 +15,7 @@
 // resident (those the routing selected, and the shared expert) is the caller's choice.
 //
 // A ternary expert may be stored in the host buffer in the dense storage form (five
-// codes per byte: 1.625 bits per weight against 2, i.e. ~18 % fewer bytes to move
+// codes per byte: 1.6 bits per weight against 2, i.e. ~18 % fewer bytes to move
 // over PCIe for the expert with its scales).  Its span is copied into a staging area
 // behind the slots and expanded there on the GPU into the kernels' 2-bit ternary
 // layout (one thread per code word; the scales, blocked the same way in both forms,

@@ -54,7 +54,7 @@ typedef enum {
 } moe_status;
 
 /* MOE_FMT_TERNARY_DENSE is a storage form of ternary experts (five codes per byte,
- * 1.625 bits per weight against 2): the packer writes it, the expert cache
+ * 1.6 bits per weight against 2): the packer writes it, the expert cache
  * (moe_cache_load) copies it from host memory and expands it on the GPU into
  * MOE_FMT_TERNARY, and no expert kernel reads it (moe_forward on a buffer that holds
  * it records MOE_ERR_DEVICE_CHECK with detail MOE_DETAIL_FORMAT and computes nothing). */

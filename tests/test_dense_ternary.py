@@ -2,7 +2,7 @@
 
 Ternary experts are in the pages' mix (ossradar.top, Xolotl README, "Get a model") and
 the bytes moved per token set the speed (the same README, "Fast mode (DeepSeek-V4.1)");
-five base-3 codes fit a byte (3^5 = 243 <= 256), 1.625 bits per weight against the 2 of
+five base-3 codes fit a byte (3^5 = 243 <= 256), 1.6 bits per weight against the 2 of
 the kernels' ternary layout.  The form is a storage one: the packer writes it, the
 expert cache moves it from host memory and expands it on the GPU, no expert kernel
 reads it.
