@@ -92,10 +92,10 @@ def decode_kparts(cfg):
 
 
 def launches_per_step(cfg) -> int:
-    """Kernels one step launches: routing (one fused kernel up to 64 tokens, else four)
+    """Kernels one step launches: routing (one fused kernel up to 64 tokens, else three)
     plus gate/up, down and combine, plus the token gather on the prefill path and the
     K-part reduction of gate/up on the decode path when K is split."""
-    route = 1 if cfg.T <= 64 else 4
+    route = 1 if cfg.T <= 64 else 3
     if path_of(cfg) == "prefill":
         return route + 4
     if path_of(cfg) == "fused":
@@ -570,6 +570,50 @@ def run_ours(args, cfg):
     return 0
 
 
+def run_host_tier(args):
+    """--host-tier: loads of experts from page-locked host memory into the device expert
+    cache (moe_cache_load), the 2-bit ternary layout against the dense ternary storage
+    form (five codes per byte, expanded on the GPU).  Full-size experts (hidden 7168,
+    ffn 2048), 32 routed ternary experts + a ternary shared one, 16 slots; every timed
+    round loads 8 experts (a one-token step's) into slots that held others, on one
+    stream, timed with CUDA events.  One JSON line; not the benchmark's main line."""
+    import dataclasses
+    import torch
+    import bit_routed_expert_fp32_b200 as moe
+    from bit_routed_expert_fp32_b200.cache import ExpertCache
+    cfg = synth.micro(T=1, H=7168, E=32, k=8, I=2048, S=1, formats="ternary", seed=7)
+    cfg = dataclasses.replace(cfg, shared_format=synth.FMT_TERNARY, name="host_tier_H7168_I2048_ternary")
+    layer = synth.Layer(cfg, 0)
+    fmt_dense = np.full(cfg.E + cfg.S, moe.FMT_TERNARY_DENSE, np.uint8)
+    out = {"metric": "host-tier expert load: host bytes and device time per expert", "config": {
+        "workload": cfg.name, "experts": cfg.E, "slots": 16, "experts_per_round": 8, "rounds": args.steps}}
+    stream = torch.cuda.current_stream()
+    for name, fmt in (("ternary_2bit", layer.fmt), ("ternary_dense", fmt_dense)):
+        host = moe.pack_layer(cfg, np.asarray(fmt, np.uint8), layer.expert)
+        cache = ExpertCache(cfg, host, n_slots=16)
+        ms = []
+        for r in range(args.warmup + args.steps):
+            ids = [(8 * r + j) % cfg.E for j in range(8)]
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            cache.ensure(ids)
+            b.record(stream)
+            if r >= args.warmup:
+                ms.append((a, b))
+        torch.cuda.synchronize()
+        loads = [a.elapsed_time(b) for a, b in ms]
+        ent = host[256:256 + 64 * (cfg.E + cfg.S)].view(np.uint64).reshape(-1, 8)
+        starts = sorted(int(v) for v in ent[:, 1])
+        span = (starts[1] - starts[0]) if len(starts) > 1 else 0        # one expert's host bytes
+        us = 1e3 * float(np.mean(loads)) / 8
+        out[name] = {"host_bytes_per_expert": span, "us_per_expert": us,
+                     "host_gb_per_s": span / (us * 1e-6) / 1e9}
+        del cache
+    out["bytes_saved"] = 1 - out["ternary_dense"]["host_bytes_per_expert"] / out["ternary_2bit"]["host_bytes_per_expert"]
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -584,6 +628,8 @@ def main():
                     help="override the routed expert count (profiling: the same per-step work on a smaller layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every call eagerly instead of replaying graphs")
+    ap.add_argument("--host-tier", action="store_true",
+                    help="time expert loads from host memory into the expert cache (2-bit vs dense ternary)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -594,6 +640,8 @@ def main():
     if args.experts:
         import dataclasses
         cfg = dataclasses.replace(cfg, E=args.experts, name=f"{cfg.name}_E{args.experts}")
+    if args.host_tier:
+        return run_host_tier(args)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

@@ -214,7 +214,8 @@ moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x, con
     a.zx = reinterpret_cast<float*>(ws + w.zx);
     // The decode operands are formed by the router only for the decode kernels that do
     // not form them themselves (more than kFusedMaxT tokens).
-    a.ops = 1;                                            // the decode operands
+    a.ops = T <= kSmallT;                                 // the decode operands (the decode
+                                                          // path forms them itself above)
     a.iq = T <= kFusedMaxT ? ws + w.iq : nullptr;         // and the integer records
     a.ctrl = reinterpret_cast<Ctrl*>(ws + w.ctrl);
     a.r = *out;
@@ -242,7 +243,8 @@ moe_status moe_route_fixed(const moe_shape* shape, int32_t T, const uint16_t* d_
     a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
     a.active = reinterpret_cast<int32_t*>(ws + w.active);
     a.zx = reinterpret_cast<float*>(ws + w.zx);
-    a.ops = 1;                                            // the decode operands
+    a.ops = T <= kSmallT;                                 // the decode operands (the decode
+                                                          // path forms them itself above)
     a.iq = T <= kFusedMaxT ? ws + w.iq : nullptr;         // and the integer records
     a.fixed_ids = d_ids;
     a.fixed_w = d_gates;
@@ -339,6 +341,17 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
         for (int i = 1; i < 3 && err == cudaSuccess; ++i)
             if (ev[i]) err = record_event(ev[i], s);
     } else {
+        if (!prefill && T > kSmallT) {
+            // the decode kernels' token operands (the router forms them up to kSmallT tokens)
+            RouteArgs ra = {};
+            ra.T = T;
+            ra.H = a.H;
+            ra.x = d_x;
+            ra.zx = reinterpret_cast<float*>(ws + w.zx);
+            ra.ctrl = a.ctrl;
+            ra.ops = 1;
+            if (launch_decode_operands(ra, s) != cudaSuccess) return MOE_ERR_CUDA;
+        }
         if (!prefill) decode_kparts(shape, T, &a.nkp_gu, &a.nkp_dn);
         err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
                       : launch_ffn_decode(a, s, ev[1], ev[2]);

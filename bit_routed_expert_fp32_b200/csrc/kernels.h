@@ -9,7 +9,7 @@
 namespace moe {
 
 constexpr int kSmallT = 64;        // decode router / decode path threshold
-constexpr int kChunk = 128;        // tokens per chunk of the large-T router
+constexpr int kChunk = 64;         // tokens per chunk of the large-T router (one CTA each)
 
 struct RouteArgs {
     int T, H, E, k, S;
@@ -167,6 +167,8 @@ inline size_t fused_ypart_floats(const moe_shape* s, int64_t T) {
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+// the decode operands (Z tables) of a.T tokens, for the decode path above kSmallT tokens
+cudaError_t launch_decode_operands(const RouteArgs& a, cudaStream_t s);
 // the routing of caller-given expert ids and gates (a.fixed_ids): histogram, scan,
 // permutation, active list and (if a.ops) the decode operands
 cudaError_t launch_route_fixed(const RouteArgs& a, cudaStream_t s);

@@ -29,9 +29,9 @@
 //  * MMA issuer (warp 13, one elected lane): per stage four tcgen05.mma.kind::f16
 //    (K = 16 each) with A from tensor memory and B from shared memory, fp32
 //    accumulation in TMEM; tcgen05.commit releases the stage to the producers and,
-//    after the last stage, hands the accumulator to the epilogue.  Two accumulators of
-//    192 columns alternate between tiles, so the epilogue of one tile overlaps the main
-//    loop of the next.
+//    after the last stage, hands the accumulator to the epilogue (gate/up: two
+//    accumulators of 192 columns alternate between tiles, so the epilogue of one tile
+//    overlaps the main loop of the next; down: one of 256 columns, see TcCfg).
 //  * Epilogue (warps 8-11, TMEM lanes 32q..32q+31): tcgen05.ld 16 columns at a time.
 //    gate/up: rows 16b..16b+7 are gate rows and 16b+8..16b+15 the matching up rows,
 //    i.e. TMEM lanes l and l+8 of the same warp: h = silu(gate) * up is formed with
@@ -48,31 +48,46 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128;                       // weight rows per tile (UMMA M)
-constexpr int BN = 192;                       // max tokens per tile (UMMA N)
 constexpr int BK = 64;                        // K per stage (one scale group)
-constexpr int NSTG = 4;                       // pipeline stages
-constexpr int B_BYTES = BN * BK * 2;          // 24 KB: a stage's shared memory is its B tile
-constexpr int STG_BYTES = B_BYTES;
-// Tensor memory (512 columns x 128 lanes x 32 bit): two fp32 accumulators of BN
-// columns, then NSTG A stages of 32 columns (128 rows x 64 fp16, two per column).
-constexpr uint32_t kACol0 = 2 * BN;
-static_assert(kACol0 + 32 * NSTG <= 512, "TMEM columns");
+constexpr int kDqWarps = 8, kEpiWarp0 = 8, kTmaWarp = 12, kMmaWarp = 13;   // warps 8-11: epilogue
+constexpr int kPkwBytes = 2 * 3328;          // a dequantiser warp's packed ring (below)
+// Per pass: the token tile (UMMA N, at most BN tokens; an expert with more tokens is split
+// into equal N tiles), the fp32 accumulators in tensor memory that the tiles use in
+// turn, and the pipeline stages.  Gate/up keeps two accumulators of 192 columns, so the
+// epilogue of one tile overlaps the main loop of the next.  Down has a quarter of the
+// gate/up FLOPs per weight byte, so the weight re-reads of a second N tile cost it more
+// than its epilogue: one accumulator of 256 columns (an expert of up to 256 tokens is one
+// tile) and three stages, the same shared memory in all.
+template <int MODE>
+struct TcCfg {
+    static constexpr int BN = MODE == 0 ? 192 : 256;
+    static constexpr int NACC = MODE == 0 ? 2 : 1;
+    static constexpr int NSTG = MODE == 0 ? 4 : 3;
+    static constexpr int STG_BYTES = BN * BK * 2;          // a stage's shared memory is its B tile
+    // Tensor memory (512 columns x 128 lanes x 32 bit): NACC fp32 accumulators of BN
+    // columns, then NSTG A stages of 32 columns (128 rows x 64 fp16, two per column).
+    static constexpr uint32_t kACol0 = NACC * BN;
+    static constexpr size_t SMEM = (size_t)NSTG * STG_BYTES + (size_t)kDqWarps * 2 * kPkwBytes + 4 * 512 + 1024;
+};
+static_assert(TcCfg<0>::kACol0 + 32 * TcCfg<0>::NSTG <= 512 && TcCfg<1>::kACol0 + 32 * TcCfg<1>::NSTG <= 512,
+              "TMEM columns");
+static_assert(TcCfg<0>::BN % 16 == 0 && TcCfg<1>::BN % 16 == 0 && TcCfg<1>::BN <= 256, "UMMA N");
 // Per-warp packed ring: each dequantiser warp streams the two 16-row blocks of its TMEM
 // lane quarter, one 8-group chunk (codes, third bits, scales of the packed format) of
 // both per slot.
 constexpr int NP = 2;
 constexpr int PK_CODES = 0, PK_HI = 2048, PK_SC = 3072, PK_BYTES = 3328, PKW_BYTES = 2 * PK_BYTES;
+static_assert(PKW_BYTES == kPkwBytes, "packed ring size");
 constexpr int kThreads = 448;                 // 14 warps
-constexpr int kDqWarps = 8, kEpiWarp0 = 8, kTmaWarp = 12, kMmaWarp = 13;   // warps 8-11: epilogue
 
 // B tiles: one tensor-map load per stage, from the map whose box (64, 128 or 256 token
 // rows) is the smallest that covers the tile's tokens.  A single thread issues bulk
 // loads at a limited rate, so one large box beats several small ones.
 struct BMaps {
-    CUtensorMap m[3];   // box rows 64, 128, BN
+    CUtensorMap m[3];   // box rows 64, 128, BN of the pass
 };
 __device__ inline int box_index(int n) { return n <= 64 ? 0 : (n <= 128 ? 1 : 2); }
-__host__ __device__ constexpr int box_rows(int i) { return i == 0 ? 64 : (i == 1 ? 128 : BN); }
+__host__ __device__ constexpr int box_rows(int i, int bn) { return i == 0 ? 64 : (i == 1 ? 128 : bn); }
 constexpr long long kWaitLimit = 4000000000LL;
 
 constexpr uint32_t kH512 = 0x60006000u, kH256 = 0x5C005C00u, kH64 = 0x54005400u, kH16 = 0x4C004C00u,
@@ -241,9 +256,12 @@ __device__ bool wait_or_flag(TcSched& S, uint64_t* bar, uint32_t parity, const F
 
 template <int MODE>   // 0: gate/up (B = gathered tokens, K = H); 1: down (B = h, K = I)
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const __grid_constant__ BMaps bmaps) {
+    constexpr int BN = TcCfg<MODE>::BN, NACC = TcCfg<MODE>::NACC, NSTG = TcCfg<MODE>::NSTG;
+    constexpr int STG_BYTES = TcCfg<MODE>::STG_BYTES;
+    constexpr uint32_t kACol0 = TcCfg<MODE>::kACol0;
     extern __shared__ uint8_t smem_raw[];
     __shared__ TcSched S;
-    __shared__ __align__(8) uint64_t full_a[NSTG], full_b[NSTG], empty_[NSTG], acc_full[2], acc_empty[2], mma_done,
+    __shared__ __align__(8) uint64_t full_a[NSTG], full_b[NSTG], empty_[NSTG], acc_full[NACC], acc_empty[NACC], mma_done,
         pk_full[kDqWarps][NP], stall_bar;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         }
         for (int w = 0; w < kDqWarps; ++w)
             for (int i = 0; i < NP; ++i) mbar_init(&pk_full[w][i], 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NACC; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 4 * 32);
         }
@@ -476,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
             const int bx = box_index(ti.N);
-            const uint32_t bbytes = (uint32_t)box_rows(bx) * BK * 2;
+            const uint32_t bbytes = (uint32_t)box_rows(bx, BN) * BK * 2;
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 if (!mbar_try_wait(&empty_[slot], eph))
                     wait_or_flag(S, &empty_[slot], eph, p, kDetWaitEmpty | 0x20 | MODE);
@@ -533,11 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         }
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
-            const int buf = tc & 1;
+            const int buf = tc % NACC;
+            const uint32_t acc_par = (uint32_t)(tc / NACC) & 1;
             const int n16 = (ti.N + 15) & ~15;
             const uint32_t idesc = instr_desc(n16);
-            if (!mbar_try_wait(&acc_empty[buf], ((tc >> 1) & 1) ^ 1))
-                ok &= wait_or_flag(S, &acc_empty[buf], ((tc >> 1) & 1) ^ 1, p, kDetWaitEmpty | 0x30 | MODE);
+            if (!mbar_try_wait(&acc_empty[buf], acc_par ^ 1))
+                ok &= wait_or_flag(S, &acc_empty[buf], acc_par ^ 1, p, kDetWaitEmpty | 0x30 | MODE);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
             const uint32_t d_tmem = tmem + buf * BN;
@@ -579,11 +598,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(FfnArgs p, const _
         int tc = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
             const TileInfo ti = tile_info(S, p, tile, mtiles);
-            const int buf = tc & 1;
+            const int buf = tc % NACC;
+            const uint32_t acc_par = (uint32_t)(tc / NACC) & 1;
             // a long wait (a whole tile's main loop): poll slowly to leave the issue slots
             // to the dequantisers on this sub-partition
-            if (!mbar_try_wait(&acc_full[buf], (tc >> 1) & 1) && !ld_volatile(S.abort_flag) &&
-                !mbar_wait_bounded_backoff(&acc_full[buf], (tc >> 1) & 1, kWaitLimit, 256)) {
+            if (!mbar_try_wait(&acc_full[buf], acc_par) && !ld_volatile(S.abort_flag) &&
+                !mbar_wait_bounded_backoff(&acc_full[buf], acc_par, kWaitLimit, 256)) {
                 st_volatile(S.abort_flag, 1);
                 report_error(p.ctrl, MOE_ERR_TIMEOUT, kDetWaitFull | 0x30 | MODE);
             }
@@ -689,18 +709,17 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_r
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kTcSmem = (size_t)NSTG * STG_BYTES + (size_t)kDqWarps * NP * PKW_BYTES + 4 * 512 + 1024;
-
-bool make_maps(BMaps* b, const void* base, long long rows, int K) {
-    return make_map(&b->m[0], base, rows, K, box_rows(0)) && make_map(&b->m[1], base, rows, K, box_rows(1)) &&
-           make_map(&b->m[2], base, rows, K, box_rows(2));
+bool make_maps(BMaps* b, const void* base, long long rows, int K, int bn) {
+    return make_map(&b->m[0], base, rows, K, box_rows(0, bn)) && make_map(&b->m[1], base, rows, K, box_rows(1, bn)) &&
+           make_map(&b->m[2], base, rows, K, box_rows(2, bn));
 }
 
 template <int MODE>
 cudaError_t launch_tc(const FfnArgs& a, const BMaps& maps, cudaStream_t s) {
-    const cudaError_t err = set_smem_limit(tc_gemm_kernel<MODE>, kTcSmem);
+    constexpr size_t smem = TcCfg<MODE>::SMEM;
+    const cudaError_t err = set_smem_limit(tc_gemm_kernel<MODE>, smem);
     if (err != cudaSuccess) return err;
-    return launch_pdl(tc_gemm_kernel<MODE>, dim3(a.num_ctas), dim3(kThreads), kTcSmem, s, a, maps);
+    return launch_pdl(tc_gemm_kernel<MODE>, dim3(a.num_ctas), dim3(kThreads), smem, s, a, maps);
 }
 
 }  // namespace
@@ -713,7 +732,8 @@ cudaError_t launch_ffn_prefill(const FfnArgs& a, uint16_t* x16, cudaStream_t s, 
     cudaError_t err = launch_pdl(gather_x16_kernel, dim3((unsigned)rows), dim3(256), 0, s, a, x16);
     if (err != cudaSuccess) return err;
     BMaps mx, mh;
-    if (!make_maps(&mx, x16, rows, a.H) || !make_maps(&mh, a.h, rows, a.I)) return cudaErrorInvalidConfiguration;
+    if (!make_maps(&mx, x16, rows, a.H, TcCfg<0>::BN) || !make_maps(&mh, a.h, rows, a.I, TcCfg<1>::BN))
+        return cudaErrorInvalidConfiguration;
     err = launch_tc<0>(a, mx, s);
     if (err != cudaSuccess) return err;
     if (ev_gateup && (err = record_event(ev_gateup, s)) != cudaSuccess) return err;

@@ -48,6 +48,14 @@ __device__ __forceinline__ Df df_add(Df a, Df b) {
     r.lo = __fadd_rn(__fadd_rn(a.lo, b.lo), err);
     return r;
 }
+// Kahan's compensated sum: a.hi the sum, a.lo minus the compensation (the low-order
+// part the next addition must still add).
+__device__ __forceinline__ void kahan_add(Df& a, float v) {
+    const float y = __fadd_rn(v, a.lo);
+    const float t = __fadd_rn(a.hi, y);
+    a.lo = __fsub_rn(y, __fsub_rn(t, a.hi));
+    a.hi = t;
+}
 // every lane ends with the same sum (the exact two-sum is symmetric in its arguments)
 __device__ inline Df warp_sum_df(Df v) {
 #pragma unroll
@@ -417,7 +425,10 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = blockIdx.x * RBM, e0 = blockIdx.y * RBN;
     const int wm = warp >> 1, wn = warp & 1;            // warp tile: tokens 32wm.., experts 32wn..
-    Df acc[2][4][4];            // K-tile partials added in double-float (see the decode router)
+    // K-tile partials added with Kahan's compensated summation (hi, and lo = minus the
+    // running compensation): four fp32 operations a partial instead of the eight of a
+    // full two-sum, with an error ~2^-48 of the sum of the partials' magnitudes
+    Df acc[2][4][4];
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -519,7 +530,7 @@ __global__ void __launch_bounds__(256) route_logits_mma_kernel(RouteArgs p) {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][b][c] = df_add(acc[a][b][c], Df{part[a][b][c], 0.f});
+                for (int c = 0; c < 4; ++c) kahan_add(acc[a][b][c], part[a][b][c]);
         if (kt + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
@@ -578,16 +589,20 @@ __global__ void __launch_bounds__(256) route_topk_kernel(RouteArgs p) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    // last CTA: per-expert exclusive scan over chunks, totals, offsets, chunk bases
+    // last CTA: per-expert totals over the chunks, the exclusive scan over experts, then
+    // each chunk's base in each expert's range (offset + the expert's rows in earlier
+    // chunks).  A thread reads its expert's column 16 chunks at a time (independent
+    // loads, one L2 round trip per 16 chunks).
     const int nchunks = gridDim.x;
     __shared__ int s_off[257];
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
         int run = 0;
-        for (int q = 0; q < nchunks; ++q) {
-            int* h = p.hist + (size_t)q * p.E + e;
-            int v = __ldcg(h);
-            *h = run;
-            run += v;
+        for (int q0 = 0; q0 < nchunks; q0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = q0 + u < nchunks ? __ldcg(p.hist + (size_t)(q0 + u) * p.E + e) : 0;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) run += v[u];
         }
         s_cnt[e] = run;
     }
@@ -597,7 +612,17 @@ __global__ void __launch_bounds__(256) route_topk_kernel(RouteArgs p) {
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
         p.r.counts[e] = s_cnt[e];
         p.r.offsets[e] = s_off[e];
-        for (int q = 0; q < nchunks; ++q) p.hist[(size_t)q * p.E + e] += s_off[e];
+        int run = s_off[e];
+        for (int q0 = 0; q0 < nchunks; q0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = q0 + u < nchunks ? __ldcg(p.hist + (size_t)(q0 + u) * p.E + e) : 0;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                if (q0 + u < nchunks) p.hist[(size_t)(q0 + u) * p.E + e] = run;
+                run += v[u];
+            }
+        }
     }
     if (threadIdx.x == 0) p.r.offsets[p.E] = s_off[p.E];
     if (warp == 0) {
@@ -619,6 +644,12 @@ __global__ void __launch_bounds__(32) route_scatter_kernel(RouteArgs p) {
 
 }  // namespace
 
+cudaError_t launch_decode_operands(const RouteArgs& a, cudaStream_t s) {
+    const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);
+    route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_route_fixed(const RouteArgs& a, cudaStream_t s) {
     if (a.ops) {
         const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);
@@ -637,8 +668,10 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
         route_small_kernel<<<a.E, 256, kRouteSmem, s>>>(a);
         return cudaGetLastError();
     }
-    const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);
-    route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
+    if (a.ops) {
+        const int zwarps = a.T * 8 * ((a.H / 64 + 7) / 8);
+        route_xz_kernel<<<(zwarps + 7) / 8, 256, 0, s>>>(a);
+    }
     cudaError_t err = set_smem_limit(route_logits_mma_kernel, kRouteMmaSmem);
     if (err != cudaSuccess) return err;
     dim3 g1((a.T + RBM - 1) / RBM, (a.E + RBN - 1) / RBN);

@@ -70,4 +70,4 @@ def test_paths_and_launch_counts():
     c24 = dataclasses.replace(c2, T=24)
     assert bench.path_of(c24) == "decode"
     assert bench.launches_per_step(c24) == 1 + 3 + (1 if bench.decode_kparts(c24)[0] > 1 else 0)
-    assert bench.path_of(c4) == "prefill" and bench.launches_per_step(c4) == 4 + 4
+    assert bench.path_of(c4) == "prefill" and bench.launches_per_step(c4) == 3 + 4
