@@ -50,7 +50,8 @@ PATHS = {
     "fused": ("ffn_fused_kernel (the whole decode forward: gate/up + SwiGLU, down and the combine, one "
               "persistent launch; integer MMAs for ternary / 2-bit experts)",
               ["bit_routed_expert_fp32_b200/csrc/decode_fused.cu", "bit_routed_expert_fp32_b200/csrc/dequant.cuh",
-               "bit_routed_expert_fp32_b200/csrc/operands.cuh", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
+               "bit_routed_expert_fp32_b200/csrc/operands.cuh", "bit_routed_expert_fp32_b200/csrc/iqmma.cuh",
+               "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "decode": ("ffn_decode_kernel<0> (gate/up + SwiGLU; interval includes the K-part reduction when K is "
                "split)",
                ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),

@@ -23,7 +23,7 @@ CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-I", INCLUDE]
 
 CU = ["route.cu", "decode_ffn.cu", "decode_fused.cu", "prefill_tc.cu", "ep.cu", "cache.cu", "api.cu", "static_ws.cu"]
 CPP = ["pack.cpp"]
-HEADERS = ["common.cuh", "kernels.h", "dequant.cuh", "operands.cuh"]
+HEADERS = ["common.cuh", "kernels.h", "dequant.cuh", "operands.cuh", "iqmma.cuh"]
 
 
 def _newer(src_list, target):

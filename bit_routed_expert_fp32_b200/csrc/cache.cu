@@ -160,32 +160,80 @@ void entry_words(const moe_shape* s, const uint8_t* h, const HostLayer& L, int e
     }
 }
 
-// Dense ternary codes of one matrix (rows packed rows of ceil(K/5) bytes) -> the
-// kernels' blocked 2-bit code words: one thread per word (16 codes of a packed row).
-__global__ void expand_ternary_kernel(const uint8_t* __restrict__ src, int rows, int K, uint8_t* __restrict__ dst) {
+// One dense ternary expert -> the kernels' layout of its slot, in one launch: the code
+// words of both matrices (one thread per 32-bit word: 16 codes of a packed row, read
+// from the about four bytes that hold them through a table of each byte value's five
+// base-3 digits, built in shared memory by every CTA), then the scales, copied in
+// 16-byte pieces (the same blocked layout in both forms).
+struct ExpandArgs {
+    const uint8_t* gc_src;      // dense codes, packed rows of ceil(K/5) bytes
+    const uint8_t* dc_src;
+    const uint4* gs_src;        // blocked scales
+    const uint4* ds_src;
+    uint8_t* gc_dst;            // blocked 2-bit code words
+    uint8_t* dc_dst;
+    uint4* gs_dst;
+    uint4* ds_dst;
+    int H, I;
+    unsigned long long n_gw, n_dw, n_gs, n_ds;   // words of each code array, 16-byte pieces of each scale array
+};
+
+__device__ __forceinline__ uint32_t expand_word(const uint8_t* __restrict__ src, int K, unsigned long long w,
+                                                const uint16_t* tab) {
     const int wpr = K / 16;                                   // words per row
-    const size_t w = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (w >= (size_t)rows * wpr) return;
+    const int pr = (int)(w / wpr), q16 = (int)(w % wpr);
+    const uint8_t* row = src + (size_t)pr * ((K + 4) / 5);
+    const int k0 = 16 * q16, b0 = k0 / 5;
+    uint32_t d[4];                                            // digits of the (up to) four bytes
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = b0 + i < (K + 4) / 5 ? tab[row[b0 + i]] : 0u;
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const int k = k0 + e, bi = k / 5 - b0, di = k % 5;
+        word |= ((d[bi] >> (2 * di)) & 3u) << (16 * (e & 1) + 2 * (e >> 1));
+    }
+    return word;
+}
+
+__device__ __forceinline__ size_t word_pos(int K, unsigned long long w) {
+    const int wpr = K / 16;
     const int pr = (int)(w / wpr), q16 = (int)(w % wpr);
     const int G = K / 64, g = q16 / 4, c = g / 8, gl = g % 8, wl = 4 * gl + q16 % 4;
     const int ng = G - 8 * c < 8 ? G - 8 * c : 8;
     const int j = pr / 16, r = pr % 16;
     const int pos = ng == 8 ? r * 32 + (wl ^ (4 * (r % 8))) : r * 4 * ng + wl;
-    const uint8_t* row = src + (size_t)pr * ((K + 4) / 5);
-    uint32_t word = 0;
-    for (int e = 0; e < 16; ++e) {
-        const int k = 16 * q16 + e;
-        uint32_t b = row[k / 5];
-        for (int d = k % 5; d > 0; --d) b /= 3;
-        word |= (b % 3) << (16 * (e & 1) + 2 * (e >> 1));
-    }
-    *reinterpret_cast<uint32_t*>(dst + (size_t)4 * K * j + 2048 * (size_t)c + 4 * (size_t)pos) = word;
+    return (size_t)4 * K * j + 2048 * (size_t)c + 4 * (size_t)pos;
 }
 
-cudaError_t expand_matrix(const uint8_t* src, int rows, int K, uint8_t* dst, cudaStream_t s) {
-    const size_t words = (size_t)rows * (K / 16);
-    expand_ternary_kernel<<<(unsigned)((words + 255) / 256), 256, 0, s>>>(src, rows, K, dst);
-    return cudaGetLastError();
+__global__ void __launch_bounds__(256) expand_ternary_kernel(const __grid_constant__ ExpandArgs a) {
+    __shared__ uint16_t tab[256];                             // byte value -> digits at bits 2d
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+        uint32_t v = b, t = 0;
+        for (int dd = 0; dd < 5; ++dd) {
+            t |= (v % 3) << (2 * dd);
+            v /= 3;
+        }
+        tab[b] = (uint16_t)t;
+    }
+    __syncthreads();
+    unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < a.n_gw) {
+        *reinterpret_cast<uint32_t*>(a.gc_dst + word_pos(a.H, i)) = expand_word(a.gc_src, a.H, i, tab);
+        return;
+    }
+    i -= a.n_gw;
+    if (i < a.n_dw) {
+        *reinterpret_cast<uint32_t*>(a.dc_dst + word_pos(a.I, i)) = expand_word(a.dc_src, a.I, i, tab);
+        return;
+    }
+    i -= a.n_dw;
+    if (i < a.n_gs) {
+        a.gs_dst[i] = a.gs_src[i];
+        return;
+    }
+    i -= a.n_gs;
+    if (i < a.n_ds) a.ds_dst[i] = a.ds_src[i];
 }
 
 // The eight 64-bit words of an expert table entry (format; six array offsets; zero).
@@ -268,14 +316,24 @@ extern "C" moe_status moe_cache_load(const moe_shape* shape, const uint8_t* h_pa
             const uint64_t hs_ds = rd64(ent + 32) - L.start[e], hs_dc = rd64(ent + 40) - L.start[e];
             const SpanLayout X = span_layout(shape, MOE_FMT_TERNARY);
             const uint64_t nch = (H / 64 + 7) / 8, nci = (I / 64 + 7) / 8;
-            if (cudaMemcpyAsync(d + slot0 + X.gs, staging + hs_gs, (size_t)(2 * I / 16) * 256 * nch,
-                                cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
-                cudaMemcpyAsync(d + slot0 + X.ds, staging + hs_ds, (size_t)(H / 16) * 256 * nci,
-                                cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-                return MOE_ERR_CUDA;
-            if (expand_matrix(staging + hs_gc, 2 * I, H, d + slot0 + X.gc, s) != cudaSuccess ||
-                expand_matrix(staging + hs_dc, H, I, d + slot0 + X.dc, s) != cudaSuccess)
-                return MOE_ERR_CUDA;
+            ExpandArgs ea;
+            ea.gc_src = staging + hs_gc;
+            ea.dc_src = staging + hs_dc;
+            ea.gs_src = reinterpret_cast<const uint4*>(staging + hs_gs);
+            ea.ds_src = reinterpret_cast<const uint4*>(staging + hs_ds);
+            ea.gc_dst = d + slot0 + X.gc;
+            ea.dc_dst = d + slot0 + X.dc;
+            ea.gs_dst = reinterpret_cast<uint4*>(d + slot0 + X.gs);
+            ea.ds_dst = reinterpret_cast<uint4*>(d + slot0 + X.ds);
+            ea.H = H;
+            ea.I = I;
+            ea.n_gw = (unsigned long long)(2 * I) * (H / 16);
+            ea.n_dw = (unsigned long long)H * (I / 16);
+            ea.n_gs = (unsigned long long)(2 * I / 16) * 256 * nch / 16;
+            ea.n_ds = (unsigned long long)(H / 16) * 256 * nci / 16;
+            const unsigned long long n = ea.n_gw + ea.n_dw + ea.n_gs + ea.n_ds;
+            expand_ternary_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ea);
+            if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
         }
         uint64_t w[7];
         entry_words(shape, h_packed, L, e, slot0, w);
