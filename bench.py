@@ -54,7 +54,8 @@ PATHS = {
                "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "decode": ("ffn_decode_kernel<0> (gate/up + SwiGLU; interval includes the K-part reduction when K is "
                "split)",
-               ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
+               ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/dequant.cuh",
+                "bit_routed_expert_fp32_b200/csrc/iqmma.cuh", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "prefill": ("tc_gemm_kernel<0> (gate/up + SwiGLU, tcgen05; interval includes the token gather)",
                 ["bit_routed_expert_fp32_b200/csrc/prefill_tc.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
 }

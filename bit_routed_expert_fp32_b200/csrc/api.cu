@@ -303,7 +303,7 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.active = reinterpret_cast<const int32_t*>(ws + w.active);
     a.zx = reinterpret_cast<const float*>(ws + w.zx);
     a.iq = T <= kFusedMaxT ? ws + w.iq : nullptr;
-    a.iq_on = 0;
+    a.iq_on = T <= kIqMaxT && T <= kFusedMaxT;          // the router wrote the records
     a.fc = reinterpret_cast<FusedCtl*>(ws + w.ctrl + sizeof(Ctrl));
     a.dn_done = reinterpret_cast<uint32_t*>(ws + w.tile_ctr);
     a.hf = reinterpret_cast<float*>(ws + w.hf);

@@ -1,8 +1,8 @@
-// Expert FFN kernels of the decode path for 17 to 64 tokens (gate/up + SwiGLU and down,
-// routed and shared experts; up to 16 tokens the fused kernel of decode_fused.cu runs
-// instead) and the gate-weighted unpermute-combine used by the decode and prefill
-// paths: grouped skinny GEMMs over the packed ternary / 2-bit / 3-bit experts, for few
-// tokens per expert.
+// Expert FFN kernels of the decode path (gate/up + SwiGLU and down, routed and shared
+// experts; at one, two and 9 to 64 tokens, while from 3 to 8 tokens the fused kernel of
+// decode_fused.cu runs instead) and the gate-weighted unpermute-combine used by the
+// decode and prefill paths: grouped skinny GEMMs over the packed ternary / 2-bit / 3-bit
+// experts, for few tokens per expert.
 //
 // Decode speed is set by the expert bytes moved per token (ossradar.top, Xolotl
 // README, "Fast mode (DeepSeek-V4.1)"), and each selected expert is read once for
@@ -41,6 +41,11 @@
 //      down: pairs are (c - o) exactly (one fp16x2 subtract); fp16 MMAs, h is fp16.
 //    Each group result is scaled by its fp16 scale into an fp32 accumulator.
 //    3-bit experts add an MMA per k-step for 4 * (third bit).
+//  * gate/up with at most 4 tokens, ternary and 2-bit experts: integer MMAs instead
+//    (u8 codes masked out of the code words against signed-byte digits of the tokens
+//    on a 12-bit grid per group, the code offset removed exactly in the integer sums;
+//    "few-token gate/up on the integer tensor path" below), which halves the
+//    dequantiser's ALU work and the MMA chain per group.
 //  * gate/up: the 16 rows of a tile are 8 gate rows and the matching 8 up rows, which
 //    the MMA places in the same thread (rows g and g + 8), so with a single K part
 //    h = silu(gate) * up is formed in registers and stored as fp16; with several K
@@ -53,6 +58,7 @@
 // leaves, so the kernel always terminates.
 #include "kernels.h"
 #include "dequant.cuh"
+#include "iqmma.cuh"
 
 namespace moe {
 namespace {
@@ -144,7 +150,10 @@ __device__ __forceinline__ int src_token(const FfnArgs& p, const CtaSched& S, in
 struct UnitView {
     const uint16_t* b;         // B-operand row of token column g (+16t elements)
     const uint16_t* z;         // gate/up: -Z/16 (hi plane) of token column g, groups 2t, 2t+1
-    int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token)
+    const uint4* bq;           // integer path: digit record of column g, lane t, group 0
+    const float2* pq;          // integer path: pairs {p, sum q} of token t, group 0
+    int o4;                    // integer path: 4 o (4 ternary, 6 two-bit)
+    int orow[2];               // output rows of columns 2t, 2t+1 (-1: no token); integer path: token t
 };
 
 // Columns without a token read a valid row (the pass's first token); their MMA
@@ -397,6 +406,133 @@ struct Producer {
     }
 };
 
+// ---- few-token gate/up on the integer tensor path (ternary and 2-bit experts) ----
+// With at most kIqMaxT tokens a pass uses one n8 tile as two signed-byte digit columns
+// per token (column 2j + d: digit d of token j; the router writes the digit records and
+// pairs, operands.cuh).  The four u8 A registers of a code word need no add (iqmma.cuh),
+// the accumulator of the low digit starts at 1.5 x 2^23 - 4 o sum q, so the joined int32
+// sum read as fp32 is 1.5 x 2^23 + the offset-corrected dot product exactly; per group
+// acc += s p (that sum) with p = 2^-e / 4 of this lane's token.  The record and the pair
+// of a group are loaded once and serve both tiles of the block.  Lane (g, t) ends with
+// rows g (gate) and g + 8 (up) of token t, packed as one fp32 pair per tile.
+__device__ __forceinline__ void iq_tile(uint32_t w0, uint32_t w1, const uint4& b, int c0, unsigned long long spf,
+                                        unsigned long long& acc) {
+    const uint32_t w0s = w0 >> 4, w1s = w1 >> 4;
+    int d[4];
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%10,%11};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(w0 & 0x03030303u), "r"(w1 & 0x03030303u), "r"(w0 & 0x0C0C0C0Cu), "r"(w1 & 0x0C0C0C0Cu), "r"(b.x),
+          "r"(b.y), "r"(c0), "r"(0));
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(w0s & 0x03030303u), "r"(w1s & 0x03030303u), "r"(w0s & 0x0C0C0C0Cu), "r"(w1s & 0x0C0C0C0Cu),
+          "r"(b.z), "r"(b.w));
+    const unsigned long long D = iq::add2(iq::pk2(__int_as_float(d[0] + 256 * d[1]), __int_as_float(d[2] + 256 * d[3])),
+                                          iq::pk2(-iq::kIqMagicF, -iq::kIqMagicF));
+    acc = iq::fma2(spf, D, acc);
+}
+
+__device__ __forceinline__ unsigned long long scale_pair(uint32_t wg, uint32_t wu, bool hi) {
+    const uint16_t hg = (uint16_t)(hi ? wg >> 16 : wg), hu = (uint16_t)(hi ? wu >> 16 : wu);
+    return iq::pk2(__half2float(__ushort_as_half(hg)), __half2float(__ushort_as_half(hu)));
+}
+
+// A full chunk (8 groups, swizzled code words: this lane's word of group gl is at byte
+// sw ^ 16 gl of the tile's stage, row g + 8 1024 bytes on), in group pairs so that the
+// scale words stay in registers with static indices.
+__device__ __forceinline__ void chunk_full_iq(const uint8_t* stg, int c, const UnitView& v, const LaneGeo& L,
+                                              unsigned long long (&ia)[NTL]) {
+    const uint4* rec = v.bq + 64 * c;
+    const float4* prs = reinterpret_cast<const float4*>(v.pq + CG * c);     // two pairs per load
+    const int sw = 128 * L.g + 16 * (L.g & 7) + 4 * L.t;
+#pragma unroll 1
+    for (int gp = 0; gp < CG / 2; ++gp) {
+        uint32_t sg[NTL], su[NTL];
+#pragma unroll
+        for (int tl = 0; tl < NTL; ++tl) {
+            const uint32_t* scw = reinterpret_cast<const uint32_t*>(stg + tl * TSTAGE + OFF_SC);
+            sg[tl] = scw[4 * L.g + gp];
+            su[tl] = scw[4 * (L.g + 8) + gp];
+        }
+        const float4 pr = __ldg(prs + gp);
+        const uint4 b0 = __ldg(rec + 16 * gp), b1 = __ldg(rec + 16 * gp + 8);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int gl = 2 * gp + h;
+            const float pf = h ? pr.z : pr.x;
+            const int c0 = (int)iq::kIqMagic - v.o4 * __float_as_int(h ? pr.w : pr.y);
+#pragma unroll
+            for (int tl = 0; tl < NTL; ++tl) {
+                const uint32_t* wp = reinterpret_cast<const uint32_t*>(stg + tl * TSTAGE + (sw ^ (16 * gl)));
+                iq_tile(wp[0], wp[256], h ? b1 : b0, c0, iq::mul2(scale_pair(sg[tl], su[tl], h), iq::pk2(pf, pf)),
+                        ia[tl]);
+            }
+        }
+    }
+}
+
+// A partial chunk (ng < 8 groups, code words unswizzled: 4 ng words per row).
+__device__ __forceinline__ void chunk_partial_iq(const uint8_t* stg, int c, int ng, const UnitView& v,
+                                                 const LaneGeo& L, unsigned long long (&ia)[NTL]) {
+    for (int gl = 0; gl < ng; ++gl) {
+        const uint4 b = __ldg(v.bq + 64 * c + 8 * gl);
+        const float2 pr = __ldg(v.pq + CG * c + gl);
+        const int c0 = (int)iq::kIqMagic - v.o4 * __float_as_int(pr.y);
+#pragma unroll
+        for (int tl = 0; tl < NTL; ++tl) {
+            const uint8_t* tb = stg + tl * TSTAGE;
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(tb);
+            const unsigned long long sv = iq::pk2(iq::iq_scale_of(tb, L.g, gl), iq::iq_scale_of(tb, L.g + 8, gl));
+            iq_tile(cw[L.g * 4 * ng + 4 * gl + L.t], cw[(L.g + 8) * 4 * ng + 4 * gl + L.t], b, c0,
+                    iq::mul2(sv, iq::pk2(pr.x, pr.x)), ia[tl]);
+        }
+    }
+}
+
+// View of an integer-path unit (T <= kIqMaxT: one pass of at most four tokens).  B
+// column g is digit g & 1 of the pass's token g >> 1; the outputs of this lane are token
+// t's.  Columns and outputs without a token read the pass's first token and are never
+// stored.
+__device__ __forceinline__ void make_view_iq(const FfnArgs& p, const CtaSched& S, int a, int g, int t, UnitView& v) {
+    const int e = S.e[a], nb = min(kIqMaxT, S.cnt[a]);
+    const bool routed = e < p.E;
+    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
+    const int ib = (g >> 1) < nb ? (g >> 1) : 0, it = t < nb ? t : 0;
+    const int tb = routed ? src_token(p, S, S.off[a] + ib) : ib;
+    const int tt = routed ? src_token(p, S, S.off[a] + it) : it;
+    // records [T][G][2 digits][4 lanes] of 16 bytes; pairs [T][G8]
+    v.bq = reinterpret_cast<const uint4*>(p.iq) + ((size_t)tb * G * 8 + 4 * (g & 1) + t);
+    v.pq = reinterpret_cast<const float2*>(p.iq + iq_pair_off(p.T, p.H)) + (size_t)tt * G8;
+    v.o4 = S.fmt[a] == MOE_FMT_TERNARY ? 4 : 6;
+    v.b = nullptr;
+    v.z = nullptr;
+    v.orow[0] = t < nb ? (routed ? S.off[a] + t : p.T * p.k + (e - p.E) * p.T + t) : -1;
+    v.orow[1] = -1;
+}
+
+// Integer-path unit end: h directly, or this K part's gate and up sums.
+__device__ __forceinline__ void unit_epilogue_iq(const FfnArgs& p, const Geo& geo, const UnitPos& q,
+                                                 const UnitView& v, const LaneGeo& L,
+                                                 const unsigned long long (&ia)[NTL]) {
+    const int orow = v.orow[0];
+    if (orow < 0) return;
+    const size_t R = (size_t)p.T * (p.k + p.S);
+#pragma unroll
+    for (int tl = 0; tl < NTL; ++tl) {
+        const int j = NTL * q.jb + tl;
+        const float2 gu = iq::up2(ia[tl]);
+        if (geo.nkp == 1) {
+            p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(silu_f(gu.x) * gu.y);
+        } else {
+            float* dst = p.gpart + ((size_t)q.kp * R + orow) * (2 * p.I) + j * 16 + L.g;
+            dst[0] = gu.x;
+            dst[8] = gu.y;
+        }
+    }
+}
+
 // The output of one finished unit: tile j = NTL jb + tl, rows g (gate / first half) and
 // g + 8 (up / second half) of this lane's token columns.
 template <int MODE>
@@ -445,7 +581,8 @@ __device__ inline void warm_z(const FfnArgs& p) {
         prefetch_l1(reinterpret_cast<const uint8_t*>(p.zx) + i * 128);
 }
 
-template <int MODE>
+// IQ (gate/up only): ternary and 2-bit experts take the integer path (T <= kIqMaxT).
+template <int MODE, bool IQ>
 __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ CtaSched S;
@@ -558,6 +695,8 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     UnitView v;
     uint32_t sub[5] = {0, 0, 0, 0, 0};
     float acc[NTL][4];
+    unsigned long long ia[NTL];                        // integer path: (gate, up) of token t per tile
+    bool iqu = false;                                  // the current unit is on the integer path
     // failure-path tests: warp 0 waits on a barrier nothing completes; the wait runs out
     // and the warp takes the give-up path below
     if (warp == 0 && S.stall) {
@@ -582,13 +721,15 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         const int hu = prod.hu[NS - 1], c = prod.hc[NS - 1];
         if (hu < 0) {                                   // nothing left (or nothing at all)
             if (unit >= 0) {
-                unit_epilogue<MODE>(p, geo, q, v, L, acc);
+                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, ia);
+                else unit_epilogue<MODE>(p, geo, q, v, L, acc);
             }
             break;
         }
         if (hu != unit) {
             if (unit >= 0) {
-                unit_epilogue<MODE>(p, geo, q, v, L, acc);
+                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, ia);
+                else unit_epilogue<MODE>(p, geo, q, v, L, acc);
             }
             unit = hu;
             q = unit_pos(S, unit, per_ep, fkp);
@@ -596,7 +737,9 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
                 view_a = q.a;
                 view_pass = q.pass;
                 q3 = S.fmt[q.a] == MOE_FMT_Q3;
-                make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
+                iqu = IQ && !q3;
+                if (IQ && iqu) make_view_iq(p, S, q.a, L.g, L.t, v);
+                else make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
                 if (MODE == 1) {
                     const int f = S.fmt[q.a];
                     const float o = f == MOE_FMT_TERNARY ? 1.f : (f == MOE_FMT_Q2 ? 1.5f : 3.5f);
@@ -608,7 +751,10 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
                 }
             }
 #pragma unroll
-            for (int tl = 0; tl < NTL; ++tl) acc[tl][0] = acc[tl][1] = acc[tl][2] = acc[tl][3] = 0.f;
+            for (int tl = 0; tl < NTL; ++tl) {
+                acc[tl][0] = acc[tl][1] = acc[tl][2] = acc[tl][3] = 0.f;
+                ia[tl] = 0ull;                          // the fp32 pair (0, 0)
+            }
         }
         const int st = consumed % NS;
         int ok = 1;
@@ -623,7 +769,10 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         }
         const uint8_t* stg = ring + (size_t)st * STAGE;
         const int ng = min(CG, geo.G - c * CG);
-        if (ng == CG) {
+        if (IQ && iqu) {
+            if (ng == CG) chunk_full_iq(stg, c, v, L, ia);
+            else chunk_partial_iq(stg, c, ng, v, L, ia);
+        } else if (ng == CG) {
             if (q3) chunk_full<MODE, true>(stg, c, v, L, sub, acc);
             else chunk_full<MODE, false>(stg, c, v, L, sub, acc);
         } else {
@@ -827,17 +976,17 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(FfnArgs p) {
 
 constexpr size_t kDynSmem = (size_t)NW * NS * STAGE + (size_t)NW * NS * 8;
 
-template <int MODE>
+template <int MODE, bool IQ>
 cudaError_t launch_mode(const FfnArgs& a, cudaStream_t s) {
-    const cudaError_t err = set_smem_limit(ffn_decode_kernel<MODE>, kDynSmem);
+    const cudaError_t err = set_smem_limit(ffn_decode_kernel<MODE, IQ>, kDynSmem);
     if (err != cudaSuccess) return err;
-    return launch_pdl(ffn_decode_kernel<MODE>, dim3(a.num_ctas), dim3(NW * 32), kDynSmem, s, a);
+    return launch_pdl(ffn_decode_kernel<MODE, IQ>, dim3(a.num_ctas), dim3(NW * 32), kDynSmem, s, a);
 }
 
 }  // namespace
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down) {
-    cudaError_t err = launch_mode<0>(a, s);
+    cudaError_t err = a.iq_on && a.iq ? launch_mode<0, true>(a, s) : launch_mode<0, false>(a, s);
     if (err != cudaSuccess) return err;
     if (a.nkp_gu > 1) {
         const long long n = (long long)a.T * (a.k + a.S) * (a.I / 4);
@@ -845,7 +994,7 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_g
         if (err != cudaSuccess) return err;
     }
     if (ev_gateup && (err = record_event(ev_gateup, s)) != cudaSuccess) return err;
-    err = launch_mode<1>(a, s);
+    err = launch_mode<1, false>(a, s);
     if (err != cudaSuccess) return err;
     if (ev_down && (err = record_event(ev_down, s)) != cudaSuccess) return err;
     return launch_combine(a, s);

@@ -82,11 +82,15 @@ struct Ws {
 //   pairs          [R][G8] x 8 bytes          (iq_pair_off)
 // The fused decode kernel (decode_fused.cu) serves up to kFusedMaxT tokens.
 constexpr int kFusedMaxT = 16;
-// token counts for which MOE_PATH_AUTO / MOE_PATH_DECODE take the fused decode kernel:
-// there it beat the separate decode launches on the full-size layer (one to two tokens:
-// 97-135 against 102-147 us per step; four to eight: 187-309 against 204-332; sixteen:
-// 525 against 535, and 440 against 554 with mixed formats and skewed routing)
+// token counts for which MOE_PATH_AUTO / MOE_PATH_DECODE take the fused decode kernel,
+// from the per-step times on the full-size layer, separate launches against the fused
+// kernel: one token 92.7 against 101.7 us, two 125.7 against 147.2, three 150.5 against
+// 151.2, four 188.5 against 183.4, eight 331.9 against 308.9, sixteen 525 against 535
+// (451 against 562 with mixed formats and skewed routing)
 constexpr int kFusedAutoMinT = 3, kFusedAutoMaxT = 8;
+// token counts up to which the separate gate/up launch runs ternary and 2-bit experts on
+// integer MMAs (two signed-byte digit columns per token fill one n8 tile at four tokens)
+constexpr int kIqMaxT = 4;
 __host__ __device__ inline size_t iq_pair_off(int64_t R, int64_t K) { return (size_t)R * (K / 64) * 128; }
 __host__ __device__ inline size_t iq_size(int64_t R, int64_t K) {
     return iq_pair_off(R, K) + (size_t)8 * R * (8 * ((K / 64 + 7) / 8));

@@ -44,6 +44,8 @@ def test_token_counts_around_the_path_switch(T):
     dict(T=5, H=320, E=8, k=1, I=192, S=0, formats="q3"),          # k = 1, 3-bit only
     dict(T=17, H=128, E=12, k=12, I=64, S=1, formats="ternary"),   # k = E: every expert
     dict(T=3, H=128, E=40, k=16, I=64, S=0, formats="mixed"),      # k = 16
+    dict(T=2, H=192, E=8, k=2, I=64, S=1, formats="mixed"),        # integer gate/up, partial chunk only
+    dict(T=2, H=576, E=8, k=4, I=128, S=1, formats="ternary"),     # integer gate/up, full + partial chunk
 ])
 def test_micro_shapes(kw):
     import bit_routed_expert_fp32_b200 as moe
@@ -164,32 +166,38 @@ def test_full_size_few_tokens_and_determinism():
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("T,shared_format", [(1, synth.FMT_TERNARY), (2, synth.FMT_Q2), (4, synth.FMT_TERNARY)])
-def test_few_token_integer_gate_up_full_chunks(T, shared_format):
+@pytest.mark.parametrize("T,shared_format,path", [(1, synth.FMT_TERNARY, "fused"), (2, synth.FMT_Q2, "fused"),
+                                                  (4, synth.FMT_TERNARY, "fused"), (1, synth.FMT_TERNARY, "decode"),
+                                                  (2, synth.FMT_Q2, "decode"), (1, synth.FMT_Q2, "decode")])
+def test_few_token_integer_gate_up_full_chunks(T, shared_format, path):
     """The fused decode kernel runs gate/up and down of ternary and 2-bit experts on
-    integer MMAs: hidden 1024 gives whole 8-group chunks (the micro shapes above only
-    reach the partial-chunk code), all routed experts ternary exercises the o = 1
-    offset, and a ternary or 2-bit shared expert takes the integer path's shared-expert
-    rows (every other workload's shared expert is 3-bit, which stays on the bf16 path)."""
+    integer MMAs, the separate gate/up launch (one and two tokens) gate/up: hidden 1024
+    gives whole 8-group chunks (the micro shapes above only reach the partial-chunk
+    code), all routed experts ternary exercises the o = 1 offset, and a ternary or 2-bit
+    shared expert takes the integer path's shared-expert rows (every other workload's
+    shared expert is 3-bit, which stays on the bf16 path)."""
     import dataclasses
     cfg = synth.micro(T=T, H=1024, E=16, k=8, I=128, S=1, formats="ternary", seed=40 + T)
     cfg = dataclasses.replace(cfg, shared_format=shared_format)
-    _full_check(cfg, PATHS["fused"])
+    _full_check(cfg, PATHS[path])
 
 
-@pytest.mark.parametrize("T,shared_format", [(1, synth.FMT_Q2), (2, synth.FMT_TERNARY), (2, synth.FMT_Q2),
-                                             (2, synth.FMT_Q3), (5, synth.FMT_Q2)])
-def test_shared_gate_up_and_down_in_k_parts(T, shared_format):
+@pytest.mark.parametrize("T,shared_format,path", [(1, synth.FMT_Q2, "fused"), (2, synth.FMT_TERNARY, "fused"),
+                                                  (2, synth.FMT_Q2, "fused"), (2, synth.FMT_Q3, "fused"),
+                                                  (5, synth.FMT_Q2, "fused"), (1, synth.FMT_Q2, "decode"),
+                                                  (2, synth.FMT_TERNARY, "decode")])
+def test_shared_gate_up_and_down_in_k_parts(T, shared_format, path):
     """Inter 2048 with eight experts a token: at one or two tokens the fused kernel
     splits every gate/up tile into K parts (their sums added in part order by the last
     part, which forms h in fp32 for the integer down pass or fp16 for the bf16 one) and
     every down tile into two; at five tokens the gate/up tiles of all experts exceed
     one wave of warps and only the shared expert's are split.  Shared expert in each
-    format."""
+    format.  The separate launches at one and two tokens split gate/up in K parts too
+    (the integer path's partial sums, added in part order by the K-part reduction)."""
     import dataclasses
     cfg = synth.micro(T=T, H=1024, E=16, k=8, I=2048, S=1, formats="mixed", seed=80 + T)
     cfg = dataclasses.replace(cfg, shared_format=shared_format)
-    _full_check(cfg, PATHS["fused"])
+    _full_check(cfg, PATHS[path])
 
 
 @pytest.mark.parametrize("formats,T,path", [("q2", 1, "decode"), ("mixed", 12, "decode"), ("mixed", 96, "prefill")])
