@@ -12,7 +12,7 @@ replica on its own token stream (the layer is data-parallel: no collective on th
 data path) and the time is the max over ranks.
 
 The roofline object describes the dominant launch.  On the decode path the library
-runs the whole forward as one kernel (ffn_fused_kernel) for 3 to 8 tokens: against the
+runs the whole forward as one kernel (ffn_fused_kernel) for 5 to 8 tokens: against the
 measured HBM copy bandwidth, with algorithmic bytes = the packed gate/up and down bytes
 of every selected expert and the shared expert, each read once.  At other decode token
 counts (the default workload's one token among them) it runs separate gate/up, down
@@ -55,13 +55,14 @@ PATHS = {
     "decode": ("ffn_decode_kernel<0> (gate/up + SwiGLU; interval includes the K-part reduction when K is "
                "split)",
                ["bit_routed_expert_fp32_b200/csrc/decode_ffn.cu", "bit_routed_expert_fp32_b200/csrc/dequant.cuh",
-                "bit_routed_expert_fp32_b200/csrc/iqmma.cuh", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
+                "bit_routed_expert_fp32_b200/csrc/iqmma.cuh", "bit_routed_expert_fp32_b200/csrc/operands.cuh",
+                "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
     "prefill": ("tc_gemm_kernel<0> (gate/up + SwiGLU, tcgen05; interval includes the token gather)",
                 ["bit_routed_expert_fp32_b200/csrc/prefill_tc.cu", "bit_routed_expert_fp32_b200/csrc/common.cuh"]),
 }
 
 
-FUSED_AUTO_T = (3, 8)  # token counts for which the library's decode choice is the fused kernel
+FUSED_AUTO_T = (5, 8)  # token counts for which the library's decode choice is the fused kernel
 
 
 def path_of(cfg) -> str:

@@ -1,5 +1,5 @@
 // Expert FFN kernels of the decode path (gate/up + SwiGLU and down, routed and shared
-// experts; at one, two and 9 to 64 tokens, while from 3 to 8 tokens the fused kernel of
+// experts; at 1 to 4 and 9 to 64 tokens, while from 5 to 8 tokens the fused kernel of
 // decode_fused.cu runs instead) and the gate-weighted unpermute-combine used by the
 // decode and prefill paths: grouped skinny GEMMs over the packed ternary / 2-bit / 3-bit
 // experts, for few tokens per expert.
@@ -59,6 +59,7 @@
 #include "kernels.h"
 #include "dequant.cuh"
 #include "iqmma.cuh"
+#include "operands.cuh"      // iq_group: the K-part reduction forms h's integer operands
 
 namespace moe {
 namespace {
@@ -73,6 +74,7 @@ constexpr int NW = 16;                                 // warps per CTA
 constexpr int NS = 2;                                  // stages per warp
 constexpr int TP = 8;                                  // tokens per pass (one n-tile)
 constexpr long long kWaitLimit = 4000000000LL;         // clock cycles (~2 s)
+constexpr uint32_t kRangeDecode = 0x40;                // detail low byte: an activation of these kernels
 
 using namespace dq;
 
@@ -492,27 +494,40 @@ __device__ __forceinline__ void chunk_partial_iq(const uint8_t* stg, int c, int 
 }
 
 // View of an integer-path unit (T <= kIqMaxT: one pass of at most four tokens).  B
-// column g is digit g & 1 of the pass's token g >> 1; the outputs of this lane are token
-// t's.  Columns and outputs without a token read the pass's first token and are never
-// stored.
+// column g is digit g & 1 of the pass's token g >> 1 (gate/up: the router's records of
+// the token; down: the K-part reduction's records of the token's h row); the outputs of
+// this lane are token t's.  Columns and outputs without a token read the pass's first
+// token and are never stored.
+template <int MODE>
 __device__ __forceinline__ void make_view_iq(const FfnArgs& p, const CtaSched& S, int a, int g, int t, UnitView& v) {
     const int e = S.e[a], nb = min(kIqMaxT, S.cnt[a]);
     const bool routed = e < p.E;
-    const int G = p.H / 64, G8 = 8 * ((G + 7) / 8);
+    const int G = (MODE == 0 ? p.H : p.I) / 64, G8 = 8 * ((G + 7) / 8);
     const int ib = (g >> 1) < nb ? (g >> 1) : 0, it = t < nb ? t : 0;
-    const int tb = routed ? src_token(p, S, S.off[a] + ib) : ib;
-    const int tt = routed ? src_token(p, S, S.off[a] + it) : it;
-    // records [T][G][2 digits][4 lanes] of 16 bytes; pairs [T][G8]
-    v.bq = reinterpret_cast<const uint4*>(p.iq) + ((size_t)tb * G * 8 + 4 * (g & 1) + t);
-    v.pq = reinterpret_cast<const float2*>(p.iq + iq_pair_off(p.T, p.H)) + (size_t)tt * G8;
+    const int srow0 = p.T * p.k + (e - p.E) * p.T;     // first row of a shared expert
+    int rb, rt;                                         // record row of column g, pair row of token t
+    if (MODE == 0) {
+        rb = routed ? src_token(p, S, S.off[a] + ib) : ib;
+        rt = routed ? src_token(p, S, S.off[a] + it) : it;
+    } else {
+        rb = routed ? S.off[a] + ib : srow0 + ib;
+        rt = routed ? S.off[a] + it : srow0 + it;
+    }
+    const uint8_t* base = MODE == 0 ? p.iq : p.hq;
+    const size_t poff = MODE == 0 ? iq_pair_off(p.T, p.H) : iq_pair_off(p.R16, p.I);
+    // records [rows][G][2 digits][4 lanes] of 16 bytes; pairs [rows][G8]
+    v.bq = reinterpret_cast<const uint4*>(base) + ((size_t)rb * G * 8 + 4 * (g & 1) + t);
+    v.pq = reinterpret_cast<const float2*>(base + poff) + (size_t)rt * G8;
     v.o4 = S.fmt[a] == MOE_FMT_TERNARY ? 4 : 6;
     v.b = nullptr;
     v.z = nullptr;
-    v.orow[0] = t < nb ? (routed ? S.off[a] + t : p.T * p.k + (e - p.E) * p.T + t) : -1;
+    v.orow[0] = t < nb ? (routed ? S.off[a] + t : srow0 + t) : -1;
     v.orow[1] = -1;
 }
 
-// Integer-path unit end: h directly, or this K part's gate and up sums.
+// Integer-path unit end: gate/up: h directly, or this K part's gate and up sums; down:
+// this K part's output rows.  Activations outside the fp16 range are reported.
+template <int MODE>
 __device__ __forceinline__ void unit_epilogue_iq(const FfnArgs& p, const Geo& geo, const UnitPos& q,
                                                  const UnitView& v, const LaneGeo& L,
                                                  const unsigned long long (&ia)[NTL]) {
@@ -522,13 +537,16 @@ __device__ __forceinline__ void unit_epilogue_iq(const FfnArgs& p, const Geo& ge
 #pragma unroll
     for (int tl = 0; tl < NTL; ++tl) {
         const int j = NTL * q.jb + tl;
-        const float2 gu = iq::up2(ia[tl]);
-        if (geo.nkp == 1) {
-            p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(silu_f(gu.x) * gu.y);
+        const float2 r = iq::up2(ia[tl]);
+        if (MODE == 0 && geo.nkp == 1) {
+            const float hv = silu_f(r.x) * r.y;
+            if (!in_f16_range(hv)) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | kRangeDecode);
+            p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(hv);
         } else {
-            float* dst = p.gpart + ((size_t)q.kp * R + orow) * (2 * p.I) + j * 16 + L.g;
-            dst[0] = gu.x;
-            dst[8] = gu.y;
+            float* dst = MODE == 0 ? p.gpart + ((size_t)q.kp * R + orow) * (2 * p.I) + j * 16 + L.g
+                                   : p.ypart + ((size_t)q.kp * R + orow) * p.H + j * 16 + L.g;
+            dst[0] = r.x;
+            dst[8] = r.y;
         }
     }
 }
@@ -547,7 +565,9 @@ __device__ __forceinline__ void unit_epilogue(const FfnArgs& p, const Geo& geo, 
             const int orow = v.orow[cc];
             if (orow < 0) continue;
             if (MODE == 0 && geo.nkp == 1) {
-                p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(silu_f(acc[tl][cc]) * acc[tl][2 + cc]);
+                const float hv = silu_f(acc[tl][cc]) * acc[tl][2 + cc];
+                if (!in_f16_range(hv)) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | kRangeDecode);
+                p.h[(size_t)orow * p.I + j * 8 + L.g] = f32_to_f16_bits(hv);
             } else if (MODE == 0) {
                 float* dst = p.gpart + ((size_t)q.kp * R + orow) * (2 * p.I) + j * 16 + L.g;
                 dst[0] = acc[tl][cc];
@@ -581,7 +601,8 @@ __device__ inline void warm_z(const FfnArgs& p) {
         prefetch_l1(reinterpret_cast<const uint8_t*>(p.zx) + i * 128);
 }
 
-// IQ (gate/up only): ternary and 2-bit experts take the integer path (T <= kIqMaxT).
+// IQ: ternary and 2-bit experts take the integer path (T <= kIqMaxT; down: when the K-part
+// reduction formed h's records).
 template <int MODE, bool IQ>
 __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -721,14 +742,14 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
         const int hu = prod.hu[NS - 1], c = prod.hc[NS - 1];
         if (hu < 0) {                                   // nothing left (or nothing at all)
             if (unit >= 0) {
-                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, ia);
+                if (IQ && iqu) unit_epilogue_iq<MODE>(p, geo, q, v, L, ia);
                 else unit_epilogue<MODE>(p, geo, q, v, L, acc);
             }
             break;
         }
         if (hu != unit) {
             if (unit >= 0) {
-                if (IQ && iqu) unit_epilogue_iq(p, geo, q, v, L, ia);
+                if (IQ && iqu) unit_epilogue_iq<MODE>(p, geo, q, v, L, ia);
                 else unit_epilogue<MODE>(p, geo, q, v, L, acc);
             }
             unit = hu;
@@ -738,7 +759,7 @@ __global__ void __launch_bounds__(NW * 32, 1) ffn_decode_kernel(FfnArgs p) {
                 view_pass = q.pass;
                 q3 = S.fmt[q.a] == MOE_FMT_Q3;
                 iqu = IQ && !q3;
-                if (IQ && iqu) make_view_iq(p, S, q.a, L.g, L.t, v);
+                if (IQ && iqu) make_view_iq<MODE>(p, S, q.a, L.g, L.t, v);
                 else make_view<MODE>(p, S, q.a, q.pass, L.g, L.t, v);
                 if (MODE == 1) {
                     const int f = S.fmt[q.a];
@@ -826,10 +847,60 @@ __global__ void __launch_bounds__(128) finalize_gateup_kernel(FfnArgs p) {
             us.x += uv[kp].x; us.y += uv[kp].y; us.z += uv[kp].z; us.w += uv[kp].w;
         }
     }
+    const float h0 = silu_f(gs.x) * us.x, h1 = silu_f(gs.y) * us.y, h2 = silu_f(gs.z) * us.z,
+                h3 = silu_f(gs.w) * us.w;
+    if (!(in_f16_range(h0) && in_f16_range(h1) && in_f16_range(h2) && in_f16_range(h3)))
+        report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | kRangeDecode);
     uint2 o;
-    o.x = (uint32_t)f32_to_f16_bits(silu_f(gs.x) * us.x) | ((uint32_t)f32_to_f16_bits(silu_f(gs.y) * us.y) << 16);
-    o.y = (uint32_t)f32_to_f16_bits(silu_f(gs.z) * us.z) | ((uint32_t)f32_to_f16_bits(silu_f(gs.w) * us.w) << 16);
+    o.x = (uint32_t)f32_to_f16_bits(h0) | ((uint32_t)f32_to_f16_bits(h1) << 16);
+    o.y = (uint32_t)f32_to_f16_bits(h2) | ((uint32_t)f32_to_f16_bits(h3) << 16);
     *reinterpret_cast<uint2*>(p.h + row * p.I + 4 * q) = o;
+}
+
+// The same reduction when the down pass runs ternary and 2-bit experts on integer MMAs
+// (up to kIqMaxT tokens): one warp per (row, 64-column group of h), two columns per
+// lane; besides fp16 h it forms the row's integer operands from the fp32 h on a 12-bit
+// grid per group (iq_group: digit records and pairs in the hq region, pairs of the
+// padding groups zero).
+__global__ void __launch_bounds__(128) finalize_gateup_iq_kernel(FfnArgs p) {
+    griddep_launch_dependents();                        // a single small wave
+    griddep_wait();                                     // gpart comes from the gate/up pass
+    const int GI = p.I / 64, GI8 = 8 * ((GI + 7) / 8);
+    const size_t R = (size_t)p.T * (p.k + p.S);
+    const size_t w = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= R * GI8) return;                           // whole warps
+    const size_t row = w / GI8;
+    const int gq = (int)(w - row * GI8);
+    float2* pairs = reinterpret_cast<float2*>(p.hq + iq_pair_off(p.R16, p.I)) + row * GI8;
+    if (gq >= GI) {
+        if (lane == 0) pairs[gq] = make_float2(0.f, 0.f);
+        return;
+    }
+    const int c = gq * 64 + 2 * lane;                   // h columns c, c + 1 (tile c / 8, rows c % 8)
+    const float* base = p.gpart + row * (2 * p.I) + (c >> 3) * 16 + (c & 7);
+    const size_t pstride = R * (2 * p.I);
+    float2 gv[kMaxParts], uv[kMaxParts];
+#pragma unroll
+    for (int kp = 0; kp < kMaxParts; ++kp) {
+        if (kp < p.nkp_gu) {
+            gv[kp] = __ldcg(reinterpret_cast<const float2*>(base + kp * pstride));
+            uv[kp] = __ldcg(reinterpret_cast<const float2*>(base + kp * pstride + 8));
+        }
+    }
+    float2 gs = make_float2(0.f, 0.f), us = gs;
+#pragma unroll
+    for (int kp = 0; kp < kMaxParts; ++kp) {
+        if (kp < p.nkp_gu) {
+            gs.x += gv[kp].x; gs.y += gv[kp].y;
+            us.x += uv[kp].x; us.y += uv[kp].y;
+        }
+    }
+    const float h0 = silu_f(gs.x) * us.x, h1 = silu_f(gs.y) * us.y;
+    if (!(in_f16_range(h0) && in_f16_range(h1))) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | kRangeDecode);
+    *reinterpret_cast<uint32_t*>(p.h + row * p.I + c) =
+        (uint32_t)f32_to_f16_bits(h0) | ((uint32_t)f32_to_f16_bits(h1) << 16);
+    iq_group(h0, h1, lane, p.hq + (row * GI + gq) * 128, pairs + gq);
 }
 
 // y[t] = sum_j g[t,j] * ypart[inv_perm[t*k + j]] + sum_s ypart[T*k + s*T + t], in slot
@@ -986,15 +1057,22 @@ cudaError_t launch_mode(const FfnArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_gateup, cudaEvent_t ev_down) {
-    cudaError_t err = a.iq_on && a.iq ? launch_mode<0, true>(a, s) : launch_mode<0, false>(a, s);
+    const bool iq_gu = a.iq_on && a.iq;
+    // the down pass on the integer path when the K-part reduction can form h's records
+    const bool iq_dn = iq_gu && a.nkp_gu > 1 && a.hq && (long long)a.T * (a.k + a.S) <= a.R16;
+    cudaError_t err = iq_gu ? launch_mode<0, true>(a, s) : launch_mode<0, false>(a, s);
     if (err != cudaSuccess) return err;
-    if (a.nkp_gu > 1) {
+    if (iq_dn) {
+        const long long n = (long long)a.T * (a.k + a.S) * (8 * ((a.I / 64 + 7) / 8)) * 32;   // threads
+        err = launch_pdl(finalize_gateup_iq_kernel, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, s, a);
+        if (err != cudaSuccess) return err;
+    } else if (a.nkp_gu > 1) {
         const long long n = (long long)a.T * (a.k + a.S) * (a.I / 4);
         err = launch_pdl(finalize_gateup_kernel, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, s, a);
         if (err != cudaSuccess) return err;
     }
     if (ev_gateup && (err = record_event(ev_gateup, s)) != cudaSuccess) return err;
-    err = launch_mode<1, false>(a, s);
+    err = iq_dn ? launch_mode<1, true>(a, s) : launch_mode<1, false>(a, s);
     if (err != cudaSuccess) return err;
     if (ev_down && (err = record_event(ev_down, s)) != cudaSuccess) return err;
     return launch_combine(a, s);

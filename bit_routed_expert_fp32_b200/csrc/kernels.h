@@ -59,7 +59,8 @@ struct FfnArgs {
     FusedCtl* fc;            // ws: counters of the fused decode kernel
     uint32_t* dn_done;       // ws [H/16]: down tiles finished per 16-row slice of y (fused kernel)
     float* hf;               // ws fp32 [R16][I]: h of ternary / 2-bit experts (fused kernel)
-    uint8_t* hq;             // ws integer operands of those h rows (iq_size(R16, I))
+    uint8_t* hq;             // ws integer operands of those h rows (iq_size(R16, I)); also the
+                             // separate down launch's up to kIqMaxT tokens (the K-part reduction's)
     int R16;                 // rows those two regions hold: min(T, kFusedMaxT) (k + S)
     float* gsh;              // ws fp32 pairs [max(pg, pr)][gsh_rows][I] x {gate, up}: gate/up
                              // K-part sums (fused kernel; in the ypart region)
@@ -84,10 +85,10 @@ struct Ws {
 constexpr int kFusedMaxT = 16;
 // token counts for which MOE_PATH_AUTO / MOE_PATH_DECODE take the fused decode kernel,
 // from the per-step times on the full-size layer, separate launches against the fused
-// kernel: one token 92.7 against 101.7 us, two 125.7 against 147.2, three 150.5 against
-// 151.2, four 188.5 against 183.4, eight 331.9 against 308.9, sixteen 525 against 535
+// kernel: one token 90.3 against 101.7 us, two 121.0 against 147.2, three 144.2 against
+// 152.4, four 182.4 against 184.3, eight 331.9 against 308.9, sixteen 525 against 535
 // (451 against 562 with mixed formats and skewed routing)
-constexpr int kFusedAutoMinT = 3, kFusedAutoMaxT = 8;
+constexpr int kFusedAutoMinT = 5, kFusedAutoMaxT = 8;
 // token counts up to which the separate gate/up launch runs ternary and 2-bit experts on
 // integer MMAs (two signed-byte digit columns per token fill one n8 tile at four tokens)
 constexpr int kIqMaxT = 4;

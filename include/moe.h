@@ -61,7 +61,7 @@ typedef enum {
 typedef enum { MOE_FMT_TERNARY = 0, MOE_FMT_Q2 = 1, MOE_FMT_Q3 = 2, MOE_FMT_TERNARY_DENSE = 3 } moe_format;
 
 /* MOE_PATH_AUTO picks DECODE for T <= 64 and PREFILL otherwise.  DECODE runs the decode
- * kernels: for 3 <= T <= 8 the whole forward as one persistent kernel (the fused
+ * kernels: for 5 <= T <= 8 the whole forward as one persistent kernel (the fused
  * decode kernel), otherwise separate gate/up, down and combine launches (the faster
  * choice at each T on the full-size layer).  MOE_PATH_DECODE_FUSED asks for the fused
  * decode kernel at any T <= 16 (MOE_ERR_UNSUPPORTED above).  All paths compute the

@@ -61,11 +61,13 @@ def test_paths_and_launch_counts():
     # one token: the router, gate/up (K in parts), the K-part reduction, down, combine
     assert bench.path_of(c2) == "decode" and bench.decode_kparts(c2)[0] > 1
     assert bench.launches_per_step(c2) == 1 + 3 + 1
-    # 3 to 8 tokens: the router, then the whole forward as one kernel
-    for T in (3, 5, 8):
+    # 5 to 8 tokens: the router, then the whole forward as one kernel
+    for T in (5, 6, 8):
         c = dataclasses.replace(c2, T=T)
         assert bench.path_of(c) == "fused" and bench.launches_per_step(c) == 1 + 1
-    # 16 and 24 tokens: the separate decode kernels
+    # 3, 4, 16 and 24 tokens: the separate decode kernels
+    for T in (3, 4):
+        assert bench.path_of(dataclasses.replace(c2, T=T)) == "decode"
     assert bench.path_of(c3) == "decode"
     c24 = dataclasses.replace(c2, T=24)
     assert bench.path_of(c24) == "decode"

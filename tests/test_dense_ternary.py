@@ -169,10 +169,10 @@ def test_cache_expands_dense_experts_bit_exactly_and_the_layer_matches_the_oracl
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("T,path", [(1, 1), (1, 3), (4, 1), (24, 1), (96, 2)])
+@pytest.mark.parametrize("T,path", [(1, 1), (1, 3), (4, 1), (6, 1), (24, 1), (96, 2)])
 def test_forward_on_a_dense_buffer_is_reported(T, path):
-    """The separate decode launches (1 and 24 tokens), the fused decode kernel (1 token
-    when asked for, 4 tokens by default) and prefill (96): MOE_DETAIL_FORMAT, nothing
+    """The separate decode launches (1, 4 and 24 tokens), the fused decode kernel (1 token
+    when asked for, 6 tokens by default) and prefill (96): MOE_DETAIL_FORMAT, nothing
     computed, the workspace still usable."""
     import torch
     import bit_routed_expert_fp32_b200 as moe

@@ -97,9 +97,9 @@ def test_outlier_tokens_all_q2_integer_path():
     torch.cuda.empty_cache()
 
 
-def _small_layer(T=8, seed=31):
+def _small_layer(T=8, seed=31, hidden=256):
     import bit_routed_expert_fp32_b200 as moe
-    cfg = synth.micro(T=T, H=256, E=8, k=2, I=128, S=1, formats="mixed", seed=seed)
+    cfg = synth.micro(T=T, H=hidden, E=8, k=2, I=128, S=1, formats="mixed", seed=seed)
     case = H.make_case(cfg)
     packed = H.pack(case)
     return cfg, case, packed, moe.MoeLayer(cfg, packed, case.layer.router_w, case.layer.router_b, 96)
@@ -129,12 +129,18 @@ def test_token_outside_fp16_range_is_reported(path):
     H.check_outputs(y2, H.oracle_outputs(case, list(range(cfg.T))))
 
 
-@pytest.mark.parametrize("path", ["decode", "prefill"])
-def test_activation_outside_fp16_range_is_reported(path):
-    """Tokens inside the fp16 range whose activations h are not: every element 3000."""
+@pytest.mark.parametrize("path,T,hidden", [("decode", 8, 256), ("decode", 1, 256), ("decode", 1, 1024),
+                                          ("decode", 2, 1024), ("decode", 24, 256), ("decode", 24, 1024),
+                                          ("prefill", 8, 256)])
+def test_activation_outside_fp16_range_is_reported(path, T, hidden):
+    """Tokens inside the fp16 range whose activations h are not: every element 3000.  The
+    decode cases reach every place h is formed: the fused kernel (8 tokens), the separate
+    gate/up epilogue on the integer path (1 token, hidden 256: K in one part) and on the
+    bf16 path (24 tokens), and the K-part reductions (hidden 1024: K in two parts; at one
+    and two tokens the one that also forms the integer down pass's operands)."""
     import torch
     import bit_routed_expert_fp32_b200 as moe
-    cfg, case, packed, layer = _small_layer()
+    cfg, case, packed, layer = _small_layer(T=T, hidden=hidden)
     x_np = np.full((cfg.T, cfg.H), synth.f32_to_bf16_bits(np.array([3000.0], np.float32))[0], np.uint16)
     x = moe.bf16_to_device(x_np)
     y = torch.zeros((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
