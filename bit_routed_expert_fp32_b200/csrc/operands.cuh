@@ -1,6 +1,7 @@
 // Per-token operands of the decode-path gate/up kernels, formed from the bf16 tokens:
 // the Z tables of the bf16 dequantiser's offset correction and the integer path's
-// token digits, factors and offset planes (used by route.cu and decode_fused.cu).
+// token digits, factors and offset planes (used by route.cu, decode_fused.cu and, for the
+// integer records of h, decode_ffn.cu).
 #pragma once
 #include "kernels.h"
 
@@ -70,7 +71,7 @@ __device__ inline void compute_z(const OperandArgs& p, int t, int Gi, int lane) 
     }
 }
 
-// Integer operands of one row and 64-group for the fused decode kernel's integer MMAs
+// Integer operands of one row and 64-group for the decode kernels' integer MMAs
 // (ternary and 2-bit experts): the group's values v (two per lane: elements 2 lane and
 // 2 lane + 1) go on a 12-bit grid, e = 11 - floor(log2 max |v|), q = rint(v 2^e) (exact
 // for every v above 2^-4 of the group maximum).  The kernel masks each code word into

@@ -1,5 +1,5 @@
-"""Bounds the integer MMA path of the fused decode kernel relies on (host-side
-arithmetic, no GPU).
+"""Bounds the integer MMA path of the decode kernels relies on (the fused kernel; the
+separate gate/up and down launches up to four tokens; host-side arithmetic, no GPU).
 
 The path puts each 64-group of a row (a token, or an h row) on a 12-bit grid,
 q = rint(v 2^e) with e = 11 - floor(log2 max|v|), stores B = 4q or q as two signed
