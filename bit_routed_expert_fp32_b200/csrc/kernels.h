@@ -117,7 +117,9 @@ moe_status check_forward_args(const moe_shape* shape, int32_t T, const void* d_p
 // experts are active and their 32-row blocks are fewer than the warps of the GPU, so
 // K is split (into whole 8-group chunks) until there are about three units per warp
 // of a reference 148-SM part; the warps take units at run time, which balances the
-// SMs (finer splits measured no faster).  Only for T <= kSmallT; 1 otherwise.
+// SMs.  At one token on the full-size layer that is gate/up in 7 parts: 89.8 us per
+// step, against 93.0 with 5 parts (two units per warp) and 90.5 with 14 (four).  Only
+// for T <= kSmallT; 1 otherwise.
 inline void decode_kparts(const moe_shape* s, int64_t T, int* nkp_gu, int* nkp_dn) {
     *nkp_gu = *nkp_dn = 1;
     if (T < 1 || T > kSmallT) return;
