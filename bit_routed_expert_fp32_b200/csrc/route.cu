@@ -156,14 +156,21 @@ __device__ void warp_scan_counts(const int* s_cnt, int* s_off, int E, int lane) 
 // s_run[e]; writes perm / inv_perm.  One warp; pair order = (token, slot) order.
 // An id outside [0, E) (only possible with caller-given routing, which reports it) takes
 // no position; its pair's inv_perm entry is set to 0 so that readers stay in bounds.
+// dedup_k > 0 (caller-given routing, k = dedup_k): an id that an earlier slot of the same
+// token already holds is left out as an invalid one is (the range starts on a token).
 __device__ void warp_scatter(const int32_t* ids, int pair0, int n, int* s_run, int32_t* perm, int32_t* inv_perm,
-                             int lane, int E) {
+                             int lane, int E, int dedup_k = 0) {
     const unsigned lt = (1u << lane) - 1u;
     for (int base = 0; base < n; base += 32) {
         int i = base + lane;
         int e = i < n ? ids[i] : -1;
-        if (i < n && (e < 0 || e >= E)) inv_perm[pair0 + i] = 0;
         bool valid = i < n && e >= 0 && e < E;
+        if (valid && dedup_k > 1) {
+            const int sl = (pair0 + i) % dedup_k;
+            for (int j = 0; j < sl; ++j)
+                if (ids[i - sl + j] == e) valid = false;
+        }
+        if (i < n && !valid) inv_perm[pair0 + i] = 0;
         if (!valid) e = -1 - lane;
         unsigned mask = __match_any_sync(0xffffffffu, e);
         int rank = __popc(mask & lt);
@@ -563,15 +570,18 @@ __global__ void __launch_bounds__(256) route_topk_kernel(RouteArgs p) {
     const int tend = min(p.T, (c + 1) * kChunk);
     for (int t = c * kChunk + warp; t < tend; t += 8) {
         if (p.fixed_ids) {
-            // caller-given routing: copied; an id outside [0, E) is reported and counted
-            // nowhere (its pair is left out of the permutation's expert ranges)
+            // caller-given routing: copied; an id outside [0, E), or one an earlier slot of
+            // the token holds already, is reported and counted nowhere (its pair is left out
+            // of the permutation's expert ranges), so no expert has more than T rows
+            const size_t i = (size_t)t * p.k + lane;
+            const int id = lane < p.k ? __ldg(p.fixed_ids + i) : -1 - lane;
+            const unsigned same = __match_any_sync(0xffffffffu, id);
             if (lane < p.k) {
-                const size_t i = (size_t)t * p.k + lane;
-                const int id = __ldg(p.fixed_ids + i);
                 p.r.topk_ids[i] = id;
                 p.r.topk_w[i] = __ldg(p.fixed_w + i);
-                if (id >= 0 && id < p.E) atomicAdd(&s_cnt[id], 1);
-                else report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 2);
+                if (id < 0 || id >= p.E) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 2);
+                else if (same & ((1u << lane) - 1u)) report_error(p.ctrl, MOE_ERR_DEVICE_CHECK, kDetRange | 5);
+                else atomicAdd(&s_cnt[id], 1);
             }
             continue;
         }
@@ -639,7 +649,7 @@ __global__ void __launch_bounds__(32) route_scatter_kernel(RouteArgs p) {
     __syncwarp();
     const int t0 = c * kChunk, t1 = min(p.T, t0 + kChunk);
     warp_scatter(p.r.topk_ids + (size_t)t0 * p.k, t0 * p.k, (t1 - t0) * p.k, s_run, p.r.perm, p.r.inv_perm, lane,
-                 p.E);
+                 p.E, p.fixed_ids ? p.k : 0);
 }
 
 }  // namespace

@@ -258,7 +258,10 @@ moe_status moe_route(const moe_shape* shape, int32_t T, const uint16_t* d_x,
  * offsets, perm, inv_perm computed as moe_route does) and the schedule in d_ws that
  * moe_forward reads.  Same argument rules and errors as moe_route; d_ids and d_gates
  * are device pointers.  An id outside [0, E) is recorded as MOE_ERR_DEVICE_CHECK
- * (MOE_DETAIL_RANGE | 2) and its pair is left out of every expert's rows. */
+ * (MOE_DETAIL_RANGE | 2) and its pair is left out of every expert's rows; so is an id
+ * that an earlier slot of the same token holds (MOE_DETAIL_RANGE | 5): a token's k ids
+ * must be distinct, as moe_route's top-k makes them.  Outputs of a call with such a
+ * pair are unspecified. */
 moe_status moe_route_fixed(const moe_shape* shape, int32_t T, const uint16_t* d_x, const int32_t* d_ids,
                            const float* d_gates, const moe_routing* out, void* d_ws, size_t ws_bytes,
                            void* stream);

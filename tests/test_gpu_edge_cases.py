@@ -194,6 +194,38 @@ def test_wait_that_runs_out_is_reported_and_the_next_call_is_correct(T, path):
         H.check_outputs(y2, H.oracle_outputs(case, list(range(T))))
 
 
+@pytest.mark.parametrize("kind,T", [("repeated", 1), ("repeated", 2), ("repeated", 24), ("outside", 2)])
+def test_caller_routing_with_a_repeated_or_invalid_id_is_reported(kind, T):
+    """moe_route_fixed with token 0's ids [1, 1, 3, 5] (the second 1 repeats the first
+    slot's expert) or [1, 9, 3, 5] (9 >= E): MOE_DETAIL_RANGE with low byte 5 or 2, the
+    pair counted nowhere (no expert gets more rows than tokens, which the decode kernels'
+    integer path relies on), the forward runs, and the workspace then serves a normal
+    call that matches the oracle."""
+    import torch
+    import bit_routed_expert_fp32_b200 as moe
+    cfg, case, packed, layer = _small_layer(T=T, hidden=1024)
+    ids = np.array([[(3 * t + j) % cfg.E for j in range(cfg.k)] for t in range(T)], np.int32)
+    ids[0] = [1, 1] if kind == "repeated" else [1, 9]
+    if cfg.k != 2:
+        raise AssertionError("the case is written for top-2")
+    x = moe.bf16_to_device(case.x)
+    d_ids = torch.from_numpy(ids).cuda()
+    gates = torch.full((T, cfg.k), 0.5, dtype=torch.float32, device="cuda")
+    y = torch.zeros((T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    moe.moe_route_fixed(cfg, T, x, d_ids, gates, layer.rt, layer.ws)
+    layer.forward(x, y, T=T, path=PATHS["decode"])
+    st, det = _status(moe, layer.ws)
+    assert st == "MOE_ERR_DEVICE_CHECK" and det == moe.DETAIL["RANGE"] | (5 if kind == "repeated" else 2), (st, hex(det))
+    counts = layer.rt["counts"].cpu().numpy()
+    want = np.bincount(ids[1:].ravel(), minlength=cfg.E)
+    want[1] += 1                                     # token 0's first slot only
+    np.testing.assert_array_equal(counts, want)
+    assert counts.max() <= T
+    rt, y2 = H.run_gpu(case, None, path=PATHS["decode"], gpu_layer=layer)
+    H.check_routing(case, rt)
+    H.check_outputs(y2, H.oracle_outputs(case, list(range(T))))
+
+
 def test_two_host_threads_on_one_device():
     """Two host threads, each with its own workspace, routing buffers and stream, run the
     layer concurrently; every output equals the single-threaded result bit for bit."""
