@@ -62,48 +62,28 @@ PATHS = {
 }
 
 
-FUSED_AUTO_T = (5, 8)  # token counts for which the library's decode choice is the fused kernel
+def forward_plan(cfg) -> dict:
+    """The library's own plan for moe_route + moe_forward(MOE_PATH_AUTO) on this workload
+    (moe_forward_plan, host-only): which kernels run, how many launches, the K parts."""
+    import bit_routed_expert_fp32_b200 as moe
+    return moe.moe_forward_plan(cfg, cfg.T, moe.PATH_AUTO)
 
 
 def path_of(cfg) -> str:
-    """The path moe_forward(MOE_PATH_AUTO) takes for this workload."""
-    tc_ok = cfg.H % 128 == 0 and (2 * cfg.I) % 128 == 0
-    if cfg.T > 64 and tc_ok:
-        return "prefill"
-    return "fused" if FUSED_AUTO_T[0] <= cfg.T <= FUSED_AUTO_T[1] and cfg.E + cfg.S <= 272 else "decode"
+    """The kernels moe_forward(MOE_PATH_AUTO) runs for this workload: "decode" (separate
+    launches), "fused" (the fused decode kernel) or "prefill"."""
+    return forward_plan(cfg)["path"]
 
 
 def decode_kparts(cfg):
-    """K parts of the decode gate/up and down passes: the library's split rule (kernels.h,
-    decode_kparts) restated, so that the launch count below is exact."""
-    if cfg.T < 1 or cfg.T > 64:
-        return 1, 1
-    active = min(cfg.T * cfg.k, cfg.E) + cfg.S
-    target = 3 * 148 * 16
-
-    def pick(K, rows):
-        nc = (K // 64 + 7) // 8
-        base = active * (rows // 32)
-        for n in range(1, nc + 1):
-            cpk = (nc + n - 1) // n
-            eff = (nc + cpk - 1) // cpk
-            if base * eff >= target or n == nc:
-                return eff
-        return 1
-
-    return pick(cfg.H, 2 * cfg.I), pick(cfg.I, cfg.H)
+    """K parts of the separate decode gate/up and down passes (1, 1 on the other paths)."""
+    p = forward_plan(cfg)
+    return p["kparts_gu"], p["kparts_dn"]
 
 
 def launches_per_step(cfg) -> int:
-    """Kernels one step launches: routing (one fused kernel up to 64 tokens, else three)
-    plus gate/up, down and combine, plus the token gather on the prefill path and the
-    K-part reduction of gate/up on the decode path when K is split."""
-    route = 1 if cfg.T <= 64 else 3
-    if path_of(cfg) == "prefill":
-        return route + 4
-    if path_of(cfg) == "fused":
-        return route + 1
-    return route + 3 + (1 if decode_kparts(cfg)[0] > 1 else 0)
+    """Kernels one step (moe_route + moe_forward) launches."""
+    return forward_plan(cfg)["launches"]
 
 
 def max_over_ranks(x: float, world: int, device) -> float:

@@ -28,7 +28,7 @@ EXPORTS = ["moe_packed_size", "moe_pack_experts", "moe_requantize_q3_to_q2", "mo
            "moe_forward", "moe_forward_timed", "moe_get_error", "moe_decode_static", "moe_decode_static_get_error",
            "moe_workspace_set_test_stall", "moe_event_record", "moe_status_string", "moe_abi_version",
            "moe_route_fixed", "moe_gather_rows", "moe_combine_pairs", "moe_cache_size", "moe_cache_init",
-           "moe_cache_load"]
+           "moe_cache_load", "moe_forward_plan"]
 # detail codes beside MOE_ERR_TIMEOUT / MOE_ERR_DEVICE_CHECK (high bits: what; low byte: where)
 DETAIL = {"WAIT_FULL": 0x100, "WAIT_EMPTY": 0x200, "DRAIN": 0x300, "HEADER": 0x400, "ROUTED_T": 0x500,
           "RANGE": 0x600, "TEST_STALL": 0x700, "LOOP_CAP": 0x800, "FORMAT": 0x900}
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.moe_pack_experts.argtypes = [sh, vp, i32, i32, ctypes.POINTER(MatrixSrc), vp, sz]
         L.moe_requantize_q3_to_q2.argtypes = [i32, i32, ctypes.POINTER(MatrixSrc), vp, vp]
         L.moe_workspace_size.argtypes = [sh, i32, ctypes.POINTER(sz)]
+        L.moe_forward_plan.argtypes = [sh, i32, i32, vp]
         L.moe_workspace_init.argtypes = [vp, sz, vp]
         L.moe_route.argtypes = [sh, i32, vp, vp, vp, ctypes.POINTER(Routing), vp, sz, vp]
         L.moe_forward.argtypes = [sh, i32, vp, vp, ctypes.POINTER(Routing), vp, ctypes.c_int, vp, sz, vp]
@@ -192,6 +193,16 @@ def moe_workspace_size(cfg, max_tokens: int) -> int:
     out = ctypes.c_size_t(0)
     _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(_shape(cfg)), max_tokens, ctypes.byref(out)))
     return out.value
+
+
+def moe_forward_plan(cfg, T: int, path=PATH_AUTO) -> dict:
+    """The library's plan for moe_route + moe_forward (host-only): which kernels run
+    ("decode", "prefill" or "fused"), how many launches, and the K parts of the separate
+    decode passes."""
+    out = np.zeros(4, np.int32)
+    _check("moe_forward_plan", lib().moe_forward_plan(ctypes.byref(_shape(cfg)), T, path, out.ctypes.data))
+    kind = {PATH_DECODE: "decode", PATH_PREFILL: "prefill", PATH_DECODE_FUSED: "fused"}[int(out[0])]
+    return {"path": kind, "launches": int(out[1]), "kparts_gu": int(out[2]), "kparts_dn": int(out[3])}
 
 
 def moe_workspace_init(ws, stream=None) -> None:

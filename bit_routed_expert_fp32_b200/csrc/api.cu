@@ -105,6 +105,14 @@ bool routing_ok(const moe_routing* r) {
     return r && r->topk_ids && r->topk_w && r->counts && r->offsets && r->perm && r->inv_perm;
 }
 
+moe_status check_path(moe_path path, int32_t T) {
+    const int base = (int)path & ~MOE_OUT_F32;
+    if (base != MOE_PATH_AUTO && base != MOE_PATH_DECODE && base != MOE_PATH_PREFILL && base != MOE_PATH_DECODE_FUSED)
+        return MOE_ERR_INVALID_ARG;
+    if (base == MOE_PATH_DECODE_FUSED && T > kFusedMaxT) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
 moe_status check_common(const moe_shape* shape, int32_t T, const void* d_ws, size_t ws_bytes) {
     if (!shape_ok(shape) || T < 0) return MOE_ERR_INVALID_ARG;
     if ((int64_t)T * shape->top_k > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
@@ -132,10 +140,28 @@ moe_status check_forward_args(const moe_shape* shape, int32_t T, const void* d_p
     if (st != MOE_OK) return st;
     if (!d_packed || !d_x || !d_y || !routing_ok(r)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(d_packed) || !aligned16(d_x) || !aligned16(d_y) || !aligned16(d_ws)) return MOE_ERR_INVALID_ARG;
-    const int base = (int)path & ~MOE_OUT_F32;
-    if (base != MOE_PATH_AUTO && base != MOE_PATH_DECODE && base != MOE_PATH_PREFILL && base != MOE_PATH_DECODE_FUSED)
-        return MOE_ERR_INVALID_ARG;
-    if (base == MOE_PATH_DECODE_FUSED && T > kFusedMaxT) return MOE_ERR_UNSUPPORTED;
+    return check_path(path, T);
+}
+
+// Which kernels moe_forward runs for T tokens on `path` (its base value, without
+// MOE_OUT_F32): the tcgen05 prefill kernels, the fused decode kernel (from
+// kFusedAutoMinT to kFusedAutoMaxT tokens, where it measured faster on the full-size
+// layer, or when asked for), or the separate decode launches with their K parts.
+moe_status plan_forward(const moe_shape* shape, int64_t T, moe_path path, ForwardPlan* fp) {
+    // The prefill kernels tile the gate/up rows and the hidden rows by 128.
+    const bool tc_ok = shape->hidden % 128 == 0 && (2 * shape->inter) % 128 == 0;
+    if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
+    fp->prefill = path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kSmallT && tc_ok);
+    fp->fused = !fp->prefill && T <= kFusedMaxT && shape->n_experts + shape->n_shared <= kMaxSlots &&
+                (path == MOE_PATH_DECODE_FUSED || (T >= kFusedAutoMinT && T <= kFusedAutoMaxT));
+    fp->nkp_gu = fp->nkp_dn = 1;
+    if (!fp->prefill && !fp->fused) decode_kparts(shape, T, &fp->nkp_gu, &fp->nkp_dn);
+    // moe_route: one kernel up to kSmallT tokens, else logits, top-k, scatter; moe_forward:
+    // the fused kernel; or gather, gate/up, down, combine; or (decode operands above
+    // kSmallT tokens,) gate/up, (K-part reduction,) down, combine
+    const int route = T <= kSmallT ? 1 : 3;
+    const int fwd = fp->fused ? 1 : fp->prefill ? 4 : (T > kSmallT ? 1 : 0) + 3 + (fp->nkp_gu > 1 ? 1 : 0);
+    fp->launches = T > 0 ? route + fwd : 0;
     return MOE_OK;
 }
 
@@ -321,19 +347,15 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
     a.y = d_y;
     a.y_f32 = ((int)path & MOE_OUT_F32) != 0;
     path = (moe_path)((int)path & ~MOE_OUT_F32);
+    ForwardPlan fp;
+    const moe_status pst = plan_forward(shape, T, path, &fp);
+    if (pst != MOE_OK) return pst;
     a.num_ctas = sm_count();
     cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
     if (events)
         for (int i = 0; i < 4; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
     if (ev[0] && record_event(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
-    // The prefill kernels tile the gate/up rows and the hidden rows by 128.
-    const bool tc_ok = a.H % 128 == 0 && (2 * a.I) % 128 == 0;
-    if (path == MOE_PATH_PREFILL && !tc_ok) return MOE_ERR_UNSUPPORTED;
-    const bool prefill = path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kSmallT && tc_ok);
-    // the fused decode kernel where it is the faster decode choice (kFusedAutoMinT ..
-    // kFusedAutoMaxT tokens, measured on the full-size layer), or when asked for
-    const bool fused = !prefill && T <= kFusedMaxT && a.E + a.S <= kMaxSlots &&
-                       (path == MOE_PATH_DECODE_FUSED || (T >= kFusedAutoMinT && T <= kFusedAutoMaxT));
+    const bool prefill = fp.prefill, fused = fp.fused;
     cudaError_t err;
     if (fused) {
         // one kernel: the per-kernel events all follow it
@@ -352,12 +374,28 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
             ra.ops = 1;
             if (launch_decode_operands(ra, s) != cudaSuccess) return MOE_ERR_CUDA;
         }
-        if (!prefill) decode_kparts(shape, T, &a.nkp_gu, &a.nkp_dn);
+        a.nkp_gu = fp.nkp_gu;
+        a.nkp_dn = fp.nkp_dn;
         err = prefill ? launch_ffn_prefill(a, reinterpret_cast<uint16_t*>(ws + w.ypart), s, ev[1], ev[2])
                       : launch_ffn_decode(a, s, ev[1], ev[2]);
     }
     if (err != cudaSuccess) return err == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
     if (ev[3] && record_event(ev[3], s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_forward_plan(const moe_shape* shape, int32_t T, moe_path path, int32_t* plan) {
+    if (!shape_ok(shape) || T < 0 || !plan) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)T * shape->top_k > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    const moe_status st = check_path(path, T);
+    if (st != MOE_OK) return st;
+    ForwardPlan fp;
+    const moe_status pst = plan_forward(shape, T, (moe_path)((int)path & ~MOE_OUT_F32), &fp);
+    if (pst != MOE_OK) return pst;
+    plan[0] = fp.prefill ? MOE_PATH_PREFILL : fp.fused ? MOE_PATH_DECODE_FUSED : MOE_PATH_DECODE;
+    plan[1] = fp.launches;
+    plan[2] = fp.nkp_gu;
+    plan[3] = fp.nkp_dn;
     return MOE_OK;
 }
 

@@ -109,6 +109,12 @@ Ws ws_layout(const moe_shape* s, int64_t T);
 bool shape_ok(const moe_shape* s);
 moe_status check_route_args(const moe_shape* shape, int32_t T, const uint16_t* d_x, const float* d_router_w,
                             const moe_routing* out, const void* d_ws, size_t ws_bytes);
+struct ForwardPlan {
+    bool prefill, fused;     // the tcgen05 kernels; the fused decode kernel; else the decode launches
+    int nkp_gu, nkp_dn;      // K parts of the separate decode passes (1 otherwise)
+    int launches;            // kernels of moe_route + moe_forward
+};
+moe_status plan_forward(const moe_shape* shape, int64_t T, moe_path path, ForwardPlan* fp);
 moe_status check_forward_args(const moe_shape* shape, int32_t T, const void* d_packed, const uint16_t* d_x,
                               const moe_routing* r, const uint16_t* d_y, moe_path path, const void* d_ws,
                               size_t ws_bytes);

@@ -347,6 +347,18 @@ moe_status moe_forward_timed(const moe_shape* shape, int32_t T, const void* d_pa
                              moe_path path, void* d_ws, size_t ws_bytes, void* stream,
                              void* const* events, int32_t n_events);
 
+/* The kernels that moe_route followed by moe_forward(shape, T, path) launch; host-only
+ * (no device work, no CUDA call).  plan is a caller array of 4 int32:
+ *   plan[0]  the kernels moe_forward runs: MOE_PATH_DECODE (separate gate/up, down and
+ *            combine launches), MOE_PATH_PREFILL (the tcgen05 kernels) or
+ *            MOE_PATH_DECODE_FUSED (the fused decode kernel)
+ *   plan[1]  kernels launched by the two calls together (0 for T = 0)
+ *   plan[2], plan[3]  K parts of the separate decode gate/up and down passes (1 on the
+ *            other paths); gate/up in more than one part adds its reduction launch
+ * Errors: those of moe_forward's argument checks on shape, T and path
+ * (MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED); a null plan is MOE_ERR_INVALID_ARG. */
+moe_status moe_forward_plan(const moe_shape* shape, int32_t T, moe_path path, int32_t* plan);
+
 /* Synchronises the stream, reads the device error word from d_ws and clears it.
  * Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK; *detail (if not NULL)
  * receives a kernel-specific code. For tests and diagnostics; not for hot loops. */

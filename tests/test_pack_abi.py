@@ -96,6 +96,43 @@ def test_static_entry_point_checks_everything_before_any_cuda_call():
     assert L.moe_workspace_set_test_stall(None, 1 << 20, 100, None) == 1
 
 
+def test_forward_plan_names_the_kernels_and_launches():
+    """moe_forward_plan (host-only): the path choice, the launch count of moe_route +
+    moe_forward and the K parts, with moe_forward's argument errors."""
+    import dataclasses
+    L = moe.lib()
+    plan = np.zeros(4, np.int32)
+    sh = _shape(H=256, I=128, E=8, k=2, S=1)
+    assert L.moe_forward_plan(ctypes.byref(sh), 4, 0, None) == 1
+    assert L.moe_forward_plan(None, 4, 0, plan.ctypes.data) == 1
+    assert L.moe_forward_plan(ctypes.byref(sh), -1, 0, plan.ctypes.data) == 1
+    assert L.moe_forward_plan(ctypes.byref(sh), 4, 7, plan.ctypes.data) == 1                 # no such path
+    assert L.moe_forward_plan(ctypes.byref(sh), 17, moe.PATH_DECODE_FUSED, plan.ctypes.data) == 2
+    odd = _shape(H=192, I=128, E=8, k=2, S=1)                                               # H not a multiple of 128
+    assert L.moe_forward_plan(ctypes.byref(odd), 100, moe.PATH_PREFILL, plan.ctypes.data) == 2
+    cfg = synth.micro(T=1, H=256, E=8, k=2, I=128, S=1)
+    assert moe.moe_forward_plan(cfg, 0) == {"path": "decode", "launches": 0, "kparts_gu": 1, "kparts_dn": 1}
+    # decode above 64 tokens when the tcgen05 kernels cannot run: the router's three
+    # kernels, the decode operands, gate/up, down, combine
+    cfg_odd = synth.micro(T=100, H=192, E=8, k=2, I=128, S=1)
+    assert moe.moe_forward_plan(cfg_odd, 100) == {"path": "decode", "launches": 3 + 1 + 3, "kparts_gu": 1,
+                                                  "kparts_dn": 1}
+    assert moe.moe_forward_plan(cfg, 4, moe.PATH_PREFILL)["launches"] == 1 + 4
+    assert moe.moe_forward_plan(cfg, 1, moe.PATH_DECODE_FUSED) == {"path": "fused", "launches": 2, "kparts_gu": 1,
+                                                                     "kparts_dn": 1}
+    assert moe.moe_forward_plan(cfg, 1, moe.PATH_AUTO | moe.OUT_F32) == moe.moe_forward_plan(cfg, 1)   # fp32 y: same kernels
+    # the full-size layer: one token splits K (gate/up in 7 parts, which adds the
+    # reduction launch), 5-8 tokens take the fused kernel, above 64 the tcgen05 kernels
+    full = synth.CONFIGS[2]
+    assert moe.moe_forward_plan(full, 1) == {"path": "decode", "launches": 5, "kparts_gu": 7, "kparts_dn": 4}
+    for T in range(1, 97):
+        p = moe.moe_forward_plan(dataclasses.replace(full, T=T), T)
+        want = "prefill" if T > 64 else "fused" if 5 <= T <= 8 else "decode"
+        assert p["path"] == want, (T, p)
+        if want == "decode":
+            assert p["launches"] == 1 + 3 + (p["kparts_gu"] > 1)
+
+
 def test_workspace_size_never_shrinks_as_tokens_grow():
     # A workspace sized for max_tokens must serve every smaller T: the K-part split
     # of the decode passes and the few-token integer operands must not make a smaller
